@@ -1,0 +1,138 @@
+/*
+ * ssd.h -- C ABI of libssd.so: the selective state-space (Mamba-2 SSD) scan
+ * forward and the single-token decode state update, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (sources: "5.3 Tensor Parallelism support and large-cluster
+ * training", sections 2.1, 3.1, 3.2, 4.3; "Scaling State-Space Models on
+ * Multiple GPUs with Tensor Parallelism", abstract):
+ *
+ *   d_t  = softplus(dt_t + dt_bias_h)                    (per token, head)
+ *   h_t  = exp(d_t * A_h) * h_{t-1} + d_t * B_t x_t^T    (N x P state per head;
+ *                                                         A_t = a_t I, sec. 3.1)
+ *   y_t  = C_t^T h_t + D_h * x_t
+ *
+ * ssd_chunk_scan_fwd evaluates it over whole sequences in the block-decomposed
+ * (chunked) form of section 3.2: a quadratic form inside each chunk, N x P
+ * states handed from chunk to chunk.  ssd_state_update applies one step to a
+ * cached state (prefill -> decode state cache, second page's abstract).
+ *
+ * Conventions for every entry point:
+ *   - All tensor arguments are DEVICE pointers to caller-owned, contiguous,
+ *     row-major memory on the current CUDA device.  The library never frees or
+ *     keeps them.  Scalar-per-head arrays (dt_bias, A, D) are float32.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream and do not synchronise, except when
+ *     the environment variable SSD_DEBUG_CHECK=1 is set (then each call waits
+ *     for its kernels and reports device-side errors).
+ *   - Argument errors are detected on the host, before anything is launched,
+ *     and returned as an ssd_status; no exception crosses the ABI.
+ *   - The library is stateless between calls and reentrant.  Temporary device
+ *     memory is taken with cudaMallocAsync / cudaFreeAsync on `stream`.
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of x, dt, B, C and y.  A, D, dt_bias and all states are float32
+ * in both modes; accumulation is float32. */
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_NULL = 1,        /* a required pointer is NULL                          */
+    SSD_ERR_SHAPE = 2,       /* sizes out of the supported range or inconsistent    */
+    SSD_ERR_DTYPE = 3,       /* dtype is not an ssd_dtype value                     */
+    SSD_ERR_CHUNK = 4,       /* chunk is not a power of two in [16, 256]            */
+    SSD_ERR_UNSUPPORTED = 5, /* valid request this build does not implement         */
+    SSD_ERR_CUDA = 6,        /* a CUDA call failed; see ssd_last_error()            */
+    SSD_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up (debug check)     */
+    SSD_ERR_SEQIDX = 8       /* seq_idx breaks its contract (debug check only)       */
+} ssd_status;
+
+/* Problem sizes.  b = batch, L = seqlen, H = nheads, P = headdim, N = dstate,
+ * G = ngroups (head h uses group h / (H / G)), nseqs = number of packed
+ * sequences when seq_idx is given (ignored otherwise). */
+typedef struct {
+    int64_t batch, seqlen, nheads, headdim, dstate, ngroups, nseqs;
+    int32_t dtype; /* ssd_dtype */
+} ssd_dims;
+
+/*
+ * ssd_chunk_scan_fwd -- whole-sequence scan, chunked (SSD block decomposition,
+ * "5.3 Tensor Parallelism ...", section 3.2).
+ *
+ *   x          (b, L, H, P)   dtype            required
+ *   dt         (b, L, H)      dtype            required; raw, before softplus
+ *   dt_bias    (H)            float32          NULL = 0
+ *   A          (H)            float32          required; the per-head scalar a of A = a I
+ *   B, C       (b, L, G, N)   dtype            required
+ *   D          (H)            float32          NULL = no skip term
+ *   init_state (S, H, N, P)   float32          NULL = zero initial state
+ *   seq_idx    (L)            int32            NULL = each batch row is one sequence.
+ *              Otherwise batch must be 1 and the row packs nseqs sequences:
+ *              seq_idx is non-decreasing, starts at 0, moves in steps of 0 or
+ *              +1 and ends at nseqs - 1.  The state is reset at the first token
+ *              of every sequence ("A_t = 0" at sequence ends, section 4.3) and
+ *              restarted from init_state[s].  A seq_idx that breaks the contract
+ *              gives unspecified values but never an out-of-bounds access; with
+ *              SSD_DEBUG_CHECK=1 it is reported as SSD_ERR_SEQIDX.
+ *   chunk      power of two in [16, 256]: the block length Q of the
+ *              decomposition.  Results do not depend on it beyond rounding.
+ *   y          (b, L, H, P)   dtype            required; must not alias an input
+ *   final_state(S, H, N, P)   float32          NULL = not written; may alias
+ *              init_state exactly (in-place continuation)
+ *   S = nseqs when seq_idx is given, else b.
+ *
+ * Supported sizes: P and N multiples of 16 with 16 <= P, N <= 256; H % G == 0;
+ * b, L >= 0 (empty inputs are a no-op apart from final_state = init_state).
+ * Returns an ssd_status.
+ */
+SSD_API int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
+                       const float* A, const void* B, const void* C, const float* D,
+                       const float* init_state, const int32_t* seq_idx, int chunk, void* y,
+                       float* final_state, void* stream);
+
+/*
+ * ssd_state_update -- one decode step on a cached state, in place (the
+ * prefill -> decode state cache of "Scaling State-Space Models on Multiple GPUs
+ * with Tensor Parallelism", abstract; same recurrence as above for one token).
+ *
+ *   state   (b, H, N, P)  float32   in/out, required
+ *   x       (b, H, P)     dtype     required
+ *   dt      (b, H)        dtype     required; raw, same meaning as in the scan
+ *   A       (H)           float32   required
+ *   B, C    (b, G, N)     dtype     required
+ *   D       (H)           float32   NULL = no skip term
+ *   y       (b, H, P)     dtype     required
+ *   dt_bias (H)           float32   NULL = 0.  Last so that the leading
+ *           arguments keep the order of the problem statement; it must be the
+ *           same bias the prefill scan used for the continuation to be exact.
+ * Uses dims->batch, nheads, headdim, dstate, ngroups, dtype (seqlen, nseqs ignored).
+ */
+SSD_API int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const void* dt,
+                     const float* A, const void* B, const void* C, const float* D, void* y,
+                     void* stream, const float* dt_bias);
+
+/* Static English text for an ssd_status value (never NULL). */
+SSD_API const char* ssd_status_string(int status);
+
+/* Detail of the last failure on the calling host thread (e.g. the CUDA error
+ * text behind SSD_ERR_CUDA, or which argument was rejected); "" if none. */
+SSD_API const char* ssd_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H_ */

@@ -1,0 +1,60 @@
+"""ctypes loader for libssd.so (the C ABI declared in include/ssd.h).
+
+The library is built in-tree by ``state_space_model_07_b200.build``.  There is
+no fallback: if it is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
+
+SSD_F32, SSD_BF16 = 0, 1
+STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE", 4: "SSD_ERR_CHUNK",
+          5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA", 7: "SSD_ERR_TIMEOUT", 8: "SSD_ERR_SEQIDX"}
+# Every function include/ssd.h declares.
+EXPORTS = ("ssd_chunk_scan_fwd", "ssd_state_update", "ssd_status_string", "ssd_last_error")
+
+
+class SsdDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+                ("nseqs", ctypes.c_int64), ("dtype", ctypes.c_int32)]
+
+
+class SsdError(RuntimeError):
+    def __init__(self, code: int, detail: str = ""):
+        self.code = code
+        name = STATUS.get(code, str(code))
+        super().__init__(f"{name}: {detail}" if detail else name)
+
+
+_lib = None
+_VP = ctypes.c_void_p
+
+
+def lib():
+    """Loads libssd.so once; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(PATH):
+            raise RuntimeError(f"CUDA library missing: {PATH}; build it with "
+                               "`python -m state_space_model_07_b200.build`")
+        L = ctypes.CDLL(PATH)
+        dims = ctypes.POINTER(SsdDims)
+        L.ssd_chunk_scan_fwd.restype = ctypes.c_int
+        L.ssd_chunk_scan_fwd.argtypes = [dims] + [_VP] * 9 + [ctypes.c_int, _VP, _VP, _VP]
+        L.ssd_state_update.restype = ctypes.c_int
+        L.ssd_state_update.argtypes = [dims] + [_VP] * 10
+        L.ssd_status_string.restype = ctypes.c_char_p
+        L.ssd_status_string.argtypes = [ctypes.c_int]
+        L.ssd_last_error.restype = ctypes.c_char_p
+        L.ssd_last_error.argtypes = []
+        _lib = L
+    return _lib
+
+
+def check(rc: int):
+    if rc != 0:
+        raise SsdError(rc, lib().ssd_last_error().decode())

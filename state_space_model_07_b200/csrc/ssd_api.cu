@@ -1,0 +1,245 @@
+// ssd_api.cu -- the extern "C" boundary of libssd.so (declared in include/ssd.h).
+//
+// Host side only: argument validation (no device reads), path selection,
+// stream-ordered temporary memory, launches, error reporting.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "ssd.h"
+#include "ssd_common.cuh"
+#include "ssd_internal.h"
+#include "ssd_tc.h"
+
+namespace {
+
+thread_local char g_last_error[512];
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+bool debug_check() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("SSD_DEBUG_CHECK");
+        v = (e && e[0] == '1') ? 1 : 0;
+    }
+    return v == 1;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+int check_sizes(const ssd_dims* d) {
+    if (d->dtype != SSD_F32 && d->dtype != SSD_BF16)
+        return fail(SSD_ERR_DTYPE, "dtype %d is not SSD_F32 or SSD_BF16", (int)d->dtype);
+    if (d->nheads < 1 || d->ngroups < 1 || d->nheads % d->ngroups != 0)
+        return fail(SSD_ERR_SHAPE, "nheads (%lld) must be a positive multiple of ngroups (%lld)",
+                    (long long)d->nheads, (long long)d->ngroups);
+    if (d->headdim < 16 || d->headdim > 256 || d->headdim % 16 != 0)
+        return fail(SSD_ERR_SHAPE, "headdim %lld must be a multiple of 16 in [16, 256]",
+                    (long long)d->headdim);
+    if (d->dstate < 16 || d->dstate > 256 || d->dstate % 16 != 0)
+        return fail(SSD_ERR_SHAPE, "dstate %lld must be a multiple of 16 in [16, 256]",
+                    (long long)d->dstate);
+    if (d->batch < 0) return fail(SSD_ERR_SHAPE, "batch %lld < 0", (long long)d->batch);
+    if (d->nheads > 65535) return fail(SSD_ERR_SHAPE, "nheads %lld > 65535", (long long)d->nheads);
+    return SSD_OK;
+}
+
+// Sub-allocator over one cudaMallocAsync block (256-byte aligned pieces).
+struct Carve {
+    char* base = nullptr;
+    size_t off = 0;
+    void* take(size_t bytes) {
+        void* p = base + off;
+        off += (bytes + 255) & ~(size_t)255;
+        return p;
+    }
+    static size_t round(size_t bytes) { return (bytes + 255) & ~(size_t)255; }
+};
+
+int cuda_fail(const char* what, cudaError_t e) {
+    return fail(SSD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Waits for the stream and reports device-side status (debug mode only).
+int debug_sync(cudaStream_t st, const int32_t* status_dev) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail("kernel execution", e);
+    if (status_dev) {
+        int32_t s = 0;
+        e = cudaMemcpy(&s, status_dev, sizeof(s), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail("status read", e);
+        if (s == ssd::kStatusSeqIdx) return fail(SSD_ERR_SEQIDX, "seq_idx breaks its contract");
+        if (s == ssd::kStatusTimeout) return fail(SSD_ERR_TIMEOUT, "a bounded device wait gave up");
+    }
+    return SSD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssd_status_string(int s) {
+    switch (s) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_NULL: return "a required pointer is NULL";
+        case SSD_ERR_SHAPE: return "sizes out of range, inconsistent, overlapping or misaligned buffers";
+        case SSD_ERR_DTYPE: return "unknown dtype";
+        case SSD_ERR_CHUNK: return "chunk must be a power of two in [16, 256]";
+        case SSD_ERR_UNSUPPORTED: return "request not supported by this build";
+        case SSD_ERR_CUDA: return "CUDA error";
+        case SSD_ERR_TIMEOUT: return "bounded device wait timed out";
+        case SSD_ERR_SEQIDX: return "seq_idx breaks its contract";
+        default: return "unknown status";
+    }
+}
+
+const char* ssd_last_error(void) { return g_last_error; }
+
+int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
+                       const float* A, const void* B, const void* C, const float* D,
+                       const float* init_state, const int32_t* seq_idx, int chunk, void* y,
+                       float* final_state, void* stream) {
+    g_last_error[0] = 0;
+    if (!dims) return fail(SSD_ERR_NULL, "dims is NULL");
+    int rc = check_sizes(dims);
+    if (rc) return rc;
+    if (chunk < 16 || chunk > 256 || (chunk & (chunk - 1)) != 0)
+        return fail(SSD_ERR_CHUNK, "chunk %d is not a power of two in [16, 256]", chunk);
+    const int64_t b = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim;
+    const int64_t N = dims->dstate, G = dims->ngroups;
+    if (L < 0) return fail(SSD_ERR_SHAPE, "seqlen %lld < 0", (long long)L);
+    if (!A) return fail(SSD_ERR_NULL, "A is NULL");
+    int64_t S = b;
+    if (seq_idx) {
+        if (b != 1 && b * L != 0)
+            return fail(SSD_ERR_SHAPE, "seq_idx requires batch == 1 (got %lld)", (long long)b);
+        if (L >= ((int64_t)1 << 31)) return fail(SSD_ERR_SHAPE, "packed seqlen must be < 2^31");
+        S = dims->nseqs;
+        if (S < 0 || (L > 0 && (S < 1 || S > L)))
+            return fail(SSD_ERR_SHAPE, "nseqs %lld must be in [1, seqlen] for packed input",
+                        (long long)S);
+    }
+    const int64_t ntok = b * L;
+    const size_t es = dims->dtype == SSD_BF16 ? 2 : 4;
+    if (ntok > 0) {
+        if (!x || !dt || !B || !C || !y) return fail(SSD_ERR_NULL, "x, dt, B, C and y are required");
+        if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y))
+            return fail(SSD_ERR_SHAPE, "x, B, C and y must be 16-byte aligned");
+        const size_t nx = (size_t)ntok * H * P * es, nbc = (size_t)ntok * G * N * es;
+        const size_t ndt = (size_t)ntok * H * es;
+        if (overlaps(y, nx, x, nx) || overlaps(y, nx, B, nbc) || overlaps(y, nx, C, nbc) ||
+            overlaps(y, nx, dt, ndt))
+            return fail(SSD_ERR_SHAPE, "y overlaps an input");
+    }
+    const size_t nstate = (size_t)S * H * N * P * sizeof(float);
+    if ((init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)))
+        return fail(SSD_ERR_SHAPE, "init_state and final_state must be 16-byte aligned");
+    if (init_state && final_state && init_state != final_state &&
+        overlaps(init_state, nstate, final_state, nstate))
+        return fail(SSD_ERR_SHAPE, "final_state partially overlaps init_state");
+
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();  // clear a stale error so it is not blamed on this call
+
+    if (ntok == 0 || S == 0) {
+        if (final_state && S > 0) {
+            cudaError_t e = init_state
+                ? (init_state == final_state ? cudaSuccess
+                                             : cudaMemcpyAsync(final_state, init_state, nstate,
+                                                               cudaMemcpyDeviceToDevice, st))
+                : cudaMemsetAsync(final_state, 0, nstate, st);
+            if (e != cudaSuccess) return cuda_fail("empty-input state copy", e);
+        }
+        return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
+    }
+
+    ssd::ScanArgs a;
+    a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G; a.S = S;
+    a.dtype = dims->dtype; a.Q = chunk;
+    a.x = x; a.dt = dt; a.B = B; a.C = C;
+    a.dt_bias = dt_bias; a.A = A; a.D = D; a.init_state = init_state; a.seq_idx = seq_idx;
+    a.y = y; a.final_state = final_state;
+
+    const int64_t max_chunks = seq_idx ? (L + chunk - 1) / chunk + S : b * ((L + chunk - 1) / chunk);
+    const bool use_tc = ssd::tc_supported(a);
+    const size_t ws_path = use_tc ? ssd::tc_workspace_bytes(a, max_chunks)
+                                  : ssd::simt_workspace_bytes(a, max_chunks);
+    const bool dbg = debug_check();
+    size_t ws_bytes = Carve::round(ws_path) + Carve::round(sizeof(int32_t));
+    if (seq_idx) ws_bytes += 3 * Carve::round(sizeof(int32_t) * (S + 1));
+
+    Carve cv;
+    cudaError_t e = cudaMallocAsync((void**)&cv.base, ws_bytes, st);
+    if (e != cudaSuccess) return cuda_fail("cudaMallocAsync(workspace)", e);
+    void* ws_main = cv.take(ws_path);
+    int32_t* status = (int32_t*)cv.take(sizeof(int32_t));
+    ssd::SeqInfo si;
+    si.L = L; si.S = (int32_t)S; si.Q = chunk; si.packed = seq_idx ? 1 : 0;
+    si.nc_row = (int32_t)((L + chunk - 1) / chunk);
+    si.start = si.end = si.chunk_off = nullptr;
+    if (dbg) cudaMemsetAsync(status, 0, sizeof(int32_t), st);
+    if (seq_idx) {
+        int32_t* start = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
+        int32_t* end = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
+        int32_t* off = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
+        ssd::launch_seq_table(seq_idx, L, (int32_t)S, chunk, start, end, off, dbg ? status : nullptr, st);
+        si.start = start; si.end = end; si.chunk_off = off;
+    }
+    if (use_tc)
+        rc = ssd::launch_tc_scan(a, si, max_chunks, ws_main, dbg ? status : nullptr, st);
+    else
+        ssd::launch_simt_scan(a, si, max_chunks, ws_main, st);
+    e = cudaGetLastError();
+    if (rc == SSD_OK && e != cudaSuccess) rc = cuda_fail("kernel launch", e);
+    if (rc == SSD_OK && dbg) rc = debug_sync(st, status);
+    cudaError_t ef = cudaFreeAsync(cv.base, st);
+    if (rc == SSD_OK && ef != cudaSuccess) rc = cuda_fail("cudaFreeAsync(workspace)", ef);
+    return rc;
+}
+
+int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const void* dt,
+                     const float* A, const void* B, const void* C, const float* D, void* y,
+                     void* stream, const float* dt_bias) {
+    g_last_error[0] = 0;
+    if (!dims) return fail(SSD_ERR_NULL, "dims is NULL");
+    int rc = check_sizes(dims);
+    if (rc) return rc;
+    const int64_t b = dims->batch, H = dims->nheads, P = dims->headdim, N = dims->dstate;
+    if (b == 0) return SSD_OK;
+    if (!state || !x || !dt || !A || !B || !C || !y)
+        return fail(SSD_ERR_NULL, "state, x, dt, A, B, C and y are required");
+    if (!aligned16(state)) return fail(SSD_ERR_SHAPE, "state must be 16-byte aligned");
+    const size_t es = dims->dtype == SSD_BF16 ? 2 : 4;
+    if (overlaps(y, (size_t)b * H * P * es, state, (size_t)b * H * N * P * 4) ||
+        overlaps(y, (size_t)b * H * P * es, x, (size_t)b * H * P * es))
+        return fail(SSD_ERR_SHAPE, "y overlaps state or x");
+    if (b * H > 0x7fffffffLL) return fail(SSD_ERR_SHAPE, "batch * nheads too large");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    ssd::UpdateArgs a;
+    a.b = b; a.H = H; a.P = P; a.N = N; a.G = dims->ngroups; a.dtype = dims->dtype;
+    a.state = state; a.x = x; a.dt = dt; a.B = B; a.C = C; a.A = A; a.D = D; a.dt_bias = dt_bias;
+    a.y = y;
+    ssd::launch_state_update(a, st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("kernel launch", e);
+    if (debug_check()) return debug_sync(st, nullptr);
+    return SSD_OK;
+}
+
+}  // extern "C"

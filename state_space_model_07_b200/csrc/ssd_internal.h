@@ -1,0 +1,44 @@
+// ssd_internal.h -- host-side interfaces between ssd_api.cu and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssd {
+
+struct SeqInfo;
+
+// Validated arguments of one ssd_chunk_scan_fwd call.
+struct ScanArgs {
+    int64_t b, L, H, P, N, G, S;
+    int dtype;  // 0 = float32, 1 = bfloat16
+    int Q;
+    const void *x, *dt, *B, *C;
+    const float *dt_bias, *A, *D, *init_state;
+    const int32_t* seq_idx;
+    void* y;
+    float* final_state;
+};
+
+// Packed-sequence table: spans and chunk offsets computed on the device.
+void launch_seq_table(const int32_t* seq_idx, int64_t L, int32_t S, int32_t Q, int32_t* start,
+                      int32_t* end, int32_t* chunk_off, int32_t* status, cudaStream_t st);
+
+// CUDA-core path (any supported shape, float32 or bfloat16).
+size_t simt_workspace_bytes(const ScanArgs& a, int64_t max_chunks);
+void launch_simt_scan(const ScanArgs& a, const SeqInfo& si, int64_t max_chunks, void* ws,
+                      cudaStream_t st);
+
+// Decode state update.
+struct UpdateArgs {
+    int64_t b, H, P, N, G;
+    int dtype;
+    float* state;
+    const void *x, *dt, *B, *C;
+    const float *A, *D, *dt_bias;
+    void* y;
+};
+void launch_state_update(const UpdateArgs& a, cudaStream_t st);
+
+}  // namespace ssd
