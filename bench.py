@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""SSD chunked-scan forward throughput on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+ssd_chunk_scan_fwd over the workload (decay cumsum, intra-chunk quadratic
+block, chunk states, state passing, state-to-output + D skip), then one
+ssd_state_update continuing from the scan's final state with fresh
+single-token inputs.  `value` counts the scan's tokens (batch x seqlen) per
+second over all ranks.  Inputs already sit in HBM when the timed region
+starts; x and y alone (671 MB for the default workload) exceed the 126 MB L2,
+so no flush is needed between steps.
+
+Multi-GPU: the path has no exchange step on one node's data-parallel axis, so
+N ranks run N independent replicas (weak scaling), timed on the device and
+reduced with max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on this host's cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSD scan fwd tokens/s on 1 B200 + % of roofline (HBM GB/s, tensor-pipe util)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="mamba2_2.7b_layer")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --- algorithmic work per kernel launch -------------------------------------------------
+
+def workload_bytes(w, S, L_tot, es):
+    """Minimum HBM bytes of one scan: inputs read once, y written once, states."""
+    H, P, N, G = w.nheads, w.headdim, w.dstate, w.ngroups
+    ntok = L_tot
+    b = ntok * (2 * H * P * es + H * es + 2 * G * N * es)       # x + y, dt, B + C
+    b += S * H * N * P * 4 * (2 if w.init_state else 1)          # final (+ init) state
+    if w.packed_nseqs:
+        b += ntok * 4                                            # seq_idx
+    return b
+
+
+def workload_flops(w, L_tot, Q):
+    """Causal algorithmic flops of the chunked form (CB once per group)."""
+    H, P, N, G = w.nheads, w.headdim, w.dstate, w.ngroups
+    per_tok_head = 2 * ((Q + 1) / 2) * P + 2 * N * P + 2 * N * P + 2 * N * P / Q
+    per_tok_group = 2 * ((Q + 1) / 2) * N
+    return L_tot * (H * per_tok_head + G * per_tok_group)
+
+
+def decode_bytes(b, H, P, N, G, es):
+    return b * H * N * P * 4 * 2 + b * H * (2 * P * es + es) + b * G * N * 2 * es
+
+
+# --- clocks -----------------------------------------------------------------------------
+
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+           0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+           0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    def __init__(self, torch_device, period_s=0.002):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            props = torch.cuda.get_device_properties(torch_device)
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM),
+                                     self._reasons()))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        busy = [s for s in self.samples if not (s[1] & 0x1)] or self.samples
+        mask = 0
+        for _, r in busy:
+            mask |= r
+        return {"sm_mhz": statistics.median([s[0] for s in busy]) if busy else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": [n for bit, n in REASONS.items() if mask & bit and bit != 0x1]}
+
+
+# --- the oracle on a bounded sample (reference arm / cpu baseline) ----------------------
+
+_CPU_INPUTS = {}
+
+
+def oracle_sample(w, heads, rows=None):
+    """Runs the fp64 oracle on `heads` heads (all tokens) of the workload's
+    first `rows` batch rows; returns (seconds, token-equivalents, threads)."""
+    import oracle
+    from state_space_model_07_b200 import inputs
+    if w.name not in _CPU_INPUTS:
+        _CPU_INPUTS[w.name] = inputs.make_inputs(w, "cpu")
+    d = _CPU_INPUTS[w.name]
+    H, G = w.nheads, w.ngroups
+    hs = list(range(heads))
+    gs = [h // (H // G) for h in hs]
+    rows = rows or d["x"].shape[0]
+    sl = slice(0, rows)
+    sub = dict(x=d["x"][sl][:, :, hs], dt=d["dt"][sl][:, :, hs], A=d["A"][hs], B=d["B"][sl][:, :, gs],
+               C=d["C"][sl][:, :, gs], dt_bias=d["dt_bias"][hs], D=d["D"][hs],
+               init_state=None if d["init_state"] is None else d["init_state"][:, hs])
+    if d["seq_idx"] is None and sub["init_state"] is not None:
+        sub["init_state"] = sub["init_state"][sl]
+    threads = oracle.default_threads()
+    args = dict(sub)
+    t0 = time.perf_counter()
+    oracle.ssd_scan(args["x"], args["dt"], args["A"], args["B"], args["C"], dt_bias=args["dt_bias"],
+                    D=args["D"], init_state=args["init_state"], seq_idx=d["seq_idx"], nseqs=d["nseqs"],
+                    nthreads=threads)
+    dt = time.perf_counter() - t0
+    ntok = rows * d["x"].shape[1]
+    return dt, ntok * heads / H, threads
+
+
+def cpu_baseline(w, target_s=8.0):
+    heads = 1
+    while True:
+        secs, toks, threads = oracle_sample(w, heads)
+        if secs >= target_s or heads >= w.nheads:
+            break
+        heads = min(w.nheads, max(heads * 2, int(heads * target_s / max(secs, 1e-3))))
+    return {"value": toks / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{heads} of {w.nheads} heads, all tokens of every sequence, fp64 token loop; "
+                      f"{secs:.1f} s wall; value = tokens x (sampled heads / all heads) / s"}
+
+
+# --- distributed plumbing ----------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from state_space_model_07_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    # Each step: the oracle on 2 heads of every sequence (a bounded sample).
+    heads = max(1, min(w.nheads, 2))
+    for _ in range(args.warmup):
+        oracle_sample(w, heads)
+    secs, toks, threads = [], 0.0, 1
+    for _ in range(args.steps):
+        s, t, threads = oracle_sample(w, heads)
+        secs.append(s)
+        toks = t
+    total = sum(secs)
+    value = toks * args.steps / total
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": config_of(w),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{heads} of {w.nheads} heads per step, all tokens; fp64 token loop"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w):
+    c = {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads, "headdim": w.headdim,
+         "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk, "input_dtype": w.dtype,
+         "state_dtype": "f32", "parallelism": "replicas",
+         "step": "ssd_chunk_scan_fwd over the workload + 1 ssd_state_update from its final state",
+         "l2": "no flush: x and y alone exceed the 126 MB L2"}
+    if w.packed_nseqs:
+        c["packed_nseqs"] = w.packed_nseqs
+    return c
+
+
+def kernel_source_sha(name):
+    src = {"tc_scan": "ssd_tc.cu", "tc_prep": "ssd_tc.cu", "simt_chunk_out": "ssd_simt.cu",
+           "state_update": "ssd_decode.cu"}.get(name)
+    if not src:
+        return None
+    p = os.path.join(ROOT, "state_space_model_07_b200", "csrc", src)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_for(name, units_per_launch):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the kernel as it stands (same source hash); else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f).get(name)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_sha") != kernel_source_sha(name):
+        return None
+    return rec["dram_bytes"] * units_per_launch / rec["units"]
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import state_space_model_07_b200 as ssd
+    from state_space_model_07_b200 import _lib, inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    w = inputs.WORKLOADS[args.workload]
+    d = inputs.make_inputs(w, dev)
+    b, L, H, P = d["x"].shape
+    N, G, S = w.dstate, w.ngroups, d["nseqs"]
+    es = d["x"].element_size()
+    y = torch.empty_like(d["x"])
+    fs = torch.empty((S, H, N, P), dtype=torch.float32, device=dev)
+    dec = [inputs.make_decode_inputs(w, k, S if w.packed_nseqs else b, dev) for k in range(4)]
+    dec_y = torch.empty_like(dec[0]["x"])
+    stream = torch.cuda.current_stream(dev)
+
+    def step(k, xs=None):
+        src = xs or d
+        ssd.chunk_scan_fwd(src["x"], src["dt"], d["A"], src["B"], src["C"], dt_bias=d["dt_bias"], D=d["D"],
+                           init_state=d["init_state"], seq_idx=d["seq_idx"], nseqs=S, chunk=w.chunk,
+                           y=y, final_state=fs)
+        dd = dec[k % len(dec)]
+        ssd.state_update(fs, dd["x"], dd["dt"], d["A"], dd["B"], dd["C"], D=d["D"], dt_bias=d["dt_bias"],
+                         y=dec_y)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for k in range(args.warmup):
+        step(k)
+    barrier()
+    _lib.profile_read(reset=True)
+    _lib.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        barrier()
+        e0.record(stream)
+        for k in range(args.steps):
+            step(k)
+        e1.record(stream)
+        barrier()
+    _lib.profile_enable(False)
+    stats = _lib.profile_read(reset=True)
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = ms / args.steps
+    tokens = b * L if not w.packed_nseqs else L
+    value = tokens * world * args.steps / (ms * 1e-3)
+    launches = sum(v[0] for v in stats.values())
+
+    pk, pk_src = peaks()
+    # dominant kernel
+    dom = max(stats.items(), key=lambda kv: kv[1][2])
+    name, (nl, nt, tot_ms) = dom
+    avg_ms = tot_ms / max(nt, 1)
+    scan_bytes = workload_bytes(w, S, tokens, es)
+    if name in ("tc_scan", "simt_chunk_out"):
+        alg_bytes = scan_bytes
+        units = tokens
+    elif name == "state_update":
+        alg_bytes = decode_bytes(S, H, P, N, G, es)
+        units = S * H
+    else:
+        alg_bytes, units = scan_bytes, tokens
+    roof = {"kernel": name, "bound": "hbm", "achieved": alg_bytes / (avg_ms * 1e-3) / 1e9,
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_source": pk_src,
+            "avg_launch_ms": avg_ms, "launches": nl, "algorithmic_bytes_per_launch": alg_bytes,
+            "traffic": traffic_for(name, units)}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    flops = workload_flops(w, tokens, w.chunk)
+    roof["tensor_equiv"] = {"algorithmic_flops": flops, "achieved_tflops": flops / (avg_ms * 1e-3) / 1e12,
+                            "peak_tflops": pk["bf16_tflops"]}
+    per_kernel = {k: {"launches": v[0], "avg_ms": v[2] / max(v[1], 1)} for k, v in stats.items()}
+    # decode kernel on its own (part of the step)
+    if "state_update" in stats:
+        su = stats["state_update"]
+        su_ms = su[2] / max(su[1], 1)
+        per_kernel["state_update"]["achieved_gbs"] = decode_bytes(S, H, P, N, G, es) / (su_ms * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        host = {k: d[k].cpu().pin_memory() for k in ("x", "dt", "B", "C")}
+        dev_in = {k: torch.empty_like(d[k]) for k in host}
+        y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        n_e2e = max(1, min(args.steps, 20))
+        step(0, dev_in)
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for k in range(n_e2e):
+            for kk in host:
+                dev_in[kk].copy_(host[kk], non_blocking=True)
+            step(k, dev_in)
+            y_host.copy_(y, non_blocking=True)
+        f1.record(stream)
+        barrier()
+        e_ms = max_over_ranks(f0.elapsed_time(f1))
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        e2e = {"value": tokens * world * n_e2e / (e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": y.numel() * y.element_size(),
+               "steps": n_e2e, "path": "pinned host -> device copies, ssd_chunk_scan_fwd + ssd_state_update "
+                                       "through the C ABI, y copied back, all on one stream"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if es == 2 else "f32", "data": "synthetic",
+            "config": config_of(w), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "kernels": per_kernel, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -131,6 +131,30 @@ SSD_API const char* ssd_status_string(int status);
  * text behind SSD_ERR_CUDA, or which argument was rejected); "" if none. */
 SSD_API const char* ssd_last_error(void);
 
+/*
+ * Instrumentation.  No counterpart in the pages: these calls exist so that a
+ * benchmark can time the library's own kernels on the stream they run on.
+ *
+ * Every kernel launch is counted.  While profiling is enabled, each launch is
+ * also bracketed by two CUDA events recorded on its stream (recording adds no
+ * device work, but costs a few microseconds of host time per launch).
+ */
+typedef struct {
+    char name[48];      /* kernel name                                   */
+    int64_t launches;   /* launches since the last reset                 */
+    int64_t timed;      /* launches with a measured duration             */
+    double total_ms;    /* summed event-measured duration of the timed   */
+} ssd_kernel_stat;
+
+/* on != 0 turns event timing on, 0 off.  Returns the previous setting. */
+SSD_API int ssd_profile_enable(int on);
+
+/* Waits for the recorded events, folds them into the per-kernel totals and
+ * copies up to max_entries entries (kernels launched at least once) into
+ * out.  reset != 0 clears all counters afterwards.  Returns the number of
+ * entries written, or -SSD_ERR_CUDA if an event could not be read. */
+SSD_API int ssd_profile_read(ssd_kernel_stat* out, int max_entries, int reset);
+
 #ifdef __cplusplus
 }
 #endif

@@ -14,13 +14,19 @@ SSD_F32, SSD_BF16 = 0, 1
 STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE", 4: "SSD_ERR_CHUNK",
           5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA", 7: "SSD_ERR_TIMEOUT", 8: "SSD_ERR_SEQIDX"}
 # Every function include/ssd.h declares.
-EXPORTS = ("ssd_chunk_scan_fwd", "ssd_state_update", "ssd_status_string", "ssd_last_error")
+EXPORTS = ("ssd_chunk_scan_fwd", "ssd_state_update", "ssd_status_string", "ssd_last_error",
+           "ssd_profile_enable", "ssd_profile_read")
 
 
 class SsdDims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
                 ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64),
                 ("nseqs", ctypes.c_int64), ("dtype", ctypes.c_int32)]
+
+
+class SsdKernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int64), ("timed", ctypes.c_int64),
+                ("total_ms", ctypes.c_double)]
 
 
 class SsdError(RuntimeError):
@@ -51,6 +57,10 @@ def lib():
         L.ssd_status_string.argtypes = [ctypes.c_int]
         L.ssd_last_error.restype = ctypes.c_char_p
         L.ssd_last_error.argtypes = []
+        L.ssd_profile_enable.restype = ctypes.c_int
+        L.ssd_profile_enable.argtypes = [ctypes.c_int]
+        L.ssd_profile_read.restype = ctypes.c_int
+        L.ssd_profile_read.argtypes = [ctypes.POINTER(SsdKernelStat), ctypes.c_int, ctypes.c_int]
         _lib = L
     return _lib
 
@@ -58,3 +68,17 @@ def lib():
 def check(rc: int):
     if rc != 0:
         raise SsdError(rc, lib().ssd_last_error().decode())
+
+
+def profile_enable(on: bool) -> bool:
+    """Turns CUDA-event timing of every library kernel launch on or off."""
+    return bool(lib().ssd_profile_enable(1 if on else 0))
+
+
+def profile_read(reset: bool = True) -> dict:
+    """{kernel name: (launches, timed launches, total ms)} since the last reset."""
+    buf = (SsdKernelStat * 32)()
+    n = lib().ssd_profile_read(buf, 32, 1 if reset else 0)
+    if n < 0:
+        raise SsdError(-n, "profile_read")
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].timed, buf[i].total_ms) for i in range(n)}

@@ -13,6 +13,7 @@
 // per-column output is reduced across the block in shared memory.
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
+#include "ssd_prof.h"
 
 namespace ssd {
 
@@ -99,6 +100,7 @@ k_state_update(float* __restrict__ state, const T* __restrict__ x, const T* __re
 void launch_state_update(const UpdateArgs& a, cudaStream_t st) {
     const size_t smem = sizeof(float) * 2 * a.N + sizeof(float4) * kDecThreads;
     const unsigned grid = (unsigned)(a.b * a.H);
+    ProfScope ps(K_STATE_UPDATE, st);
     if (a.dtype == 0)
         k_state_update<float><<<grid, kDecThreads, smem, st>>>(
             a.state, (const float*)a.x, (const float*)a.dt, a.dt_bias, a.A, (const float*)a.B,

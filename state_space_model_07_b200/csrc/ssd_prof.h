@@ -1,0 +1,35 @@
+// ssd_prof.h -- launch counting and optional CUDA-event timing of each kernel.
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace ssd {
+
+enum KernelId : int {
+    K_SEQ_BOUNDS = 0,
+    K_SEQ_TABLE,
+    K_SIMT_CHUNK_STATE,
+    K_SIMT_STATE_PASS,
+    K_SIMT_CHUNK_OUT,
+    K_STATE_UPDATE,
+    K_TC_PREP,
+    K_TC_SCAN,
+    K_COUNT
+};
+
+// Brackets one kernel launch: counts it and, while profiling is enabled,
+// records a CUDA event pair on `st` around it.
+class ProfScope {
+  public:
+    ProfScope(KernelId id, cudaStream_t st);
+    ~ProfScope();
+    ProfScope(const ProfScope&) = delete;
+    ProfScope& operator=(const ProfScope&) = delete;
+
+  private:
+    KernelId id_;
+    cudaStream_t st_;
+    cudaEvent_t e0_ = nullptr, e1_ = nullptr;
+};
+
+}  // namespace ssd

@@ -21,6 +21,7 @@
 // is structural and needs no masking arithmetic.
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
+#include "ssd_prof.h"
 
 namespace ssd {
 
@@ -314,8 +315,14 @@ void launch_seq_table(const int32_t* seq_idx, int64_t L, int32_t S, int32_t Q, i
     int64_t blocks = (L + 255) / 256;
     if (blocks > 1184) blocks = 1184;
     if (blocks < 1) blocks = 1;
-    k_seq_bounds<<<(unsigned)blocks, 256, 0, st>>>(seq_idx, L, S, start, status);
-    k_seq_table<<<1, 32, 0, st>>>(L, S, Q, start, end, chunk_off);
+    {
+        ProfScope ps(K_SEQ_BOUNDS, st);
+        k_seq_bounds<<<(unsigned)blocks, 256, 0, st>>>(seq_idx, L, S, start, status);
+    }
+    {
+        ProfScope ps(K_SEQ_TABLE, st);
+        k_seq_table<<<1, 32, 0, st>>>(L, S, Q, start, end, chunk_off);
+    }
 }
 
 template <typename T>
@@ -324,17 +331,27 @@ static void launch_simt_t(const ScanArgs& a, const SeqInfo& si, int64_t max_chun
     const int H = (int)a.H, P = (int)a.P, N = (int)a.N, G = (int)a.G;
     const int ntn = N >= 64 ? 64 : N, ntp = P >= 64 ? 64 : P;
     dim3 g1((unsigned)max_chunks, H, (N / ntn) * (P / ntp));
-    k_simt_chunk_state<T><<<g1, kThreads, 0, st>>>(si, (const T*)a.x, (const T*)a.dt, a.dt_bias, a.A,
-                                                   (const T*)a.B, H, P, N, G, ws_states, ws_cs);
+    {
+        ProfScope ps(K_SIMT_CHUNK_STATE, st);
+        k_simt_chunk_state<T><<<g1, kThreads, 0, st>>>(si, (const T*)a.x, (const T*)a.dt, a.dt_bias,
+                                                       a.A, (const T*)a.B, H, P, N, G, ws_states, ws_cs);
+    }
     const int64_t NP = (int64_t)N * P;
     dim3 g2((unsigned)si.S, H, (unsigned)((NP / 4 + kThreads - 1) / kThreads));
-    k_simt_state_pass<<<g2, kThreads, 0, st>>>(si, a.init_state, ws_states, ws_cs, a.final_state, H, NP);
+    {
+        ProfScope ps(K_SIMT_STATE_PASS, st);
+        k_simt_state_pass<<<g2, kThreads, 0, st>>>(si, a.init_state, ws_states, ws_cs, a.final_state,
+                                                   H, NP);
+    }
     const size_t smem = sizeof(float) * (2 * kThreads + 2 * 32 * (N + 1) + 32 * 33 + 2 * 32 * 64);
     cudaFuncSetAttribute(k_simt_chunk_out<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 g3((unsigned)max_chunks, H, P / ntp);
-    k_simt_chunk_out<T><<<g3, kThreads, smem, st>>>(si, (const T*)a.x, (const T*)a.dt, a.dt_bias, a.A,
-                                                    (const T*)a.B, (const T*)a.C, a.D, ws_states,
-                                                    (T*)a.y, H, P, N, G);
+    {
+        ProfScope ps(K_SIMT_CHUNK_OUT, st);
+        k_simt_chunk_out<T><<<g3, kThreads, smem, st>>>(si, (const T*)a.x, (const T*)a.dt, a.dt_bias,
+                                                        a.A, (const T*)a.B, (const T*)a.C, a.D,
+                                                        ws_states, (T*)a.y, H, P, N, G);
+    }
 }
 
 size_t simt_workspace_bytes(const ScanArgs& a, int64_t max_chunks) {
