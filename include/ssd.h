@@ -124,6 +124,41 @@ SSD_API int ssd_state_update(const ssd_dims* dims, float* state, const void* x, 
                      const float* A, const void* B, const void* C, const float* D, void* y,
                      void* stream, const float* dt_bias);
 
+/*
+ * ssd_chunk_scan_fwd_noalloc -- the same scan, for callers that cannot let the
+ * library allocate device memory (for example a serving engine that has
+ * already given nearly all of HBM to its own pool, or a caller that forbids
+ * allocation after start-up).  The pages have no counterpart to this call; it
+ * is a deployment variant of ssd_chunk_scan_fwd.
+ *
+ * Arguments, layouts, ownership and validation are those of
+ * ssd_chunk_scan_fwd; the caller still passes all inputs and outputs.  It
+ * always runs the CUDA-core scan, whose scratch (per-chunk states, chunk
+ * decays, packed-sequence table) lives in one fixed 32 MiB device array
+ * inside the library instead of a cudaMallocAsync block:
+ *   - needed scratch = 4 * (chunks * H * (N * P + 1)) bytes plus a few KiB,
+ *     rounded to 256-byte pieces, with chunks = b * ceil(L / chunk), or
+ *     ceil(L / chunk) + nseqs when packed.  Larger calls are rejected with
+ *     SSD_ERR_UNSUPPORTED before anything is launched (ssd_last_error() says
+ *     how much was needed);
+ *   - the array is held by every GPU that uses this call, from its first use
+ *     until the process exits;
+ *   - the first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture;
+ *   - every call shares the one array, which keeps the previous call's
+ *     contents.  Everything a call reads from it is written earlier by the
+ *     same call, so stale contents do no harm; but calls that overlap on the
+ *     GPU (concurrent streams, several host threads) race on it and must be
+ *     serialised by the caller.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+SSD_API int ssd_chunk_scan_fwd_noalloc(const ssd_dims* dims, const void* x, const void* dt,
+                                       const float* dt_bias, const float* A, const void* B,
+                                       const void* C, const float* D, const float* init_state,
+                                       const int32_t* seq_idx, int chunk, void* y,
+                                       float* final_state, void* stream);
+
 /* Static English text for an ssd_status value (never NULL). */
 SSD_API const char* ssd_status_string(int status);
 

@@ -15,7 +15,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE"
           5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA", 7: "SSD_ERR_TIMEOUT", 8: "SSD_ERR_SEQIDX"}
 # Every function include/ssd.h declares.
 EXPORTS = ("ssd_chunk_scan_fwd", "ssd_state_update", "ssd_status_string", "ssd_last_error",
-           "ssd_profile_enable", "ssd_profile_read")
+           "ssd_profile_enable", "ssd_profile_read", "ssd_chunk_scan_fwd_noalloc")
 
 
 class SsdDims(ctypes.Structure):
@@ -51,6 +51,8 @@ def lib():
         dims = ctypes.POINTER(SsdDims)
         L.ssd_chunk_scan_fwd.restype = ctypes.c_int
         L.ssd_chunk_scan_fwd.argtypes = [dims] + [_VP] * 9 + [ctypes.c_int, _VP, _VP, _VP]
+        L.ssd_chunk_scan_fwd_noalloc.restype = ctypes.c_int
+        L.ssd_chunk_scan_fwd_noalloc.argtypes = [dims] + [_VP] * 9 + [ctypes.c_int, _VP, _VP, _VP]
         L.ssd_state_update.restype = ctypes.c_int
         L.ssd_state_update.argtypes = [dims] + [_VP] * 10
         L.ssd_status_string.restype = ctypes.c_char_p

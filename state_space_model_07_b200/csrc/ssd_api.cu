@@ -8,6 +8,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "ssd.h"
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
@@ -243,3 +245,149 @@ int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const vo
 }
 
 }  // extern "C"
+
+// ---- Scan without any device allocation ---------------------------------------------
+//
+// Some callers cannot let a library allocate device memory: a serving engine
+// that has already handed nearly all of HBM to its own pool (so a
+// cudaMallocAsync inside the call fails or forces the pool to give memory
+// back), or a caller that forbids allocation after start-up to keep latency
+// predictable.  ssd_chunk_scan_fwd_noalloc serves them: it runs the CUDA-core
+// scan with its scratch (per-chunk states, chunk decays, packed-sequence
+// table, status word) placed in the fixed-size array below instead of a
+// stream-ordered allocation.
+
+// Scratch limit of the no-allocation scan, in bytes (32 MiB).  The array is
+// part of the library's device image: every GPU that uses the entry point
+// holds it from its first use until the process exits.
+static constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= kMaxDevices) return fail(SSD_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(no-alloc scratch)", e);
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return SSD_OK;
+}
+
+}  // namespace
+
+extern "C" int ssd_chunk_scan_fwd_noalloc(const ssd_dims* dims, const void* x, const void* dt,
+                                          const float* dt_bias, const float* A, const void* B,
+                                          const void* C, const float* D, const float* init_state,
+                                          const int32_t* seq_idx, int chunk, void* y,
+                                          float* final_state, void* stream) {
+    g_last_error[0] = 0;
+    if (!dims) return fail(SSD_ERR_NULL, "dims is NULL");
+    int rc = check_sizes(dims);
+    if (rc) return rc;
+    if (chunk < 16 || chunk > 256 || (chunk & (chunk - 1)) != 0)
+        return fail(SSD_ERR_CHUNK, "chunk %d is not a power of two in [16, 256]", chunk);
+    const int64_t b = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim;
+    const int64_t N = dims->dstate, G = dims->ngroups;
+    if (L < 0) return fail(SSD_ERR_SHAPE, "seqlen %lld < 0", (long long)L);
+    if (!A) return fail(SSD_ERR_NULL, "A is NULL");
+    int64_t S = b;
+    if (seq_idx) {
+        if (b != 1 && b * L != 0)
+            return fail(SSD_ERR_SHAPE, "seq_idx requires batch == 1 (got %lld)", (long long)b);
+        if (L >= ((int64_t)1 << 31)) return fail(SSD_ERR_SHAPE, "packed seqlen must be < 2^31");
+        S = dims->nseqs;
+        if (S < 0 || (L > 0 && (S < 1 || S > L)))
+            return fail(SSD_ERR_SHAPE, "nseqs %lld must be in [1, seqlen] for packed input",
+                        (long long)S);
+    }
+    const int64_t ntok = b * L;
+    const size_t es = dims->dtype == SSD_BF16 ? 2 : 4;
+    if (ntok > 0) {
+        if (!x || !dt || !B || !C || !y) return fail(SSD_ERR_NULL, "x, dt, B, C and y are required");
+        if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y))
+            return fail(SSD_ERR_SHAPE, "x, B, C and y must be 16-byte aligned");
+        const size_t nx = (size_t)ntok * H * P * es, nbc = (size_t)ntok * G * N * es;
+        const size_t ndt = (size_t)ntok * H * es;
+        if (overlaps(y, nx, x, nx) || overlaps(y, nx, B, nbc) || overlaps(y, nx, C, nbc) ||
+            overlaps(y, nx, dt, ndt))
+            return fail(SSD_ERR_SHAPE, "y overlaps an input");
+    }
+    const size_t nstate = (size_t)S * H * N * P * sizeof(float);
+    if ((init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)))
+        return fail(SSD_ERR_SHAPE, "init_state and final_state must be 16-byte aligned");
+    if (init_state && final_state && init_state != final_state &&
+        overlaps(init_state, nstate, final_state, nstate))
+        return fail(SSD_ERR_SHAPE, "final_state partially overlaps init_state");
+
+    cudaStream_t st = (cudaStream_t)stream;
+    if (ntok == 0 || S == 0) {
+        cudaGetLastError();
+        if (final_state && S > 0) {
+            cudaError_t e = init_state
+                ? (init_state == final_state ? cudaSuccess
+                                             : cudaMemcpyAsync(final_state, init_state, nstate,
+                                                               cudaMemcpyDeviceToDevice, st))
+                : cudaMemsetAsync(final_state, 0, nstate, st);
+            if (e != cudaSuccess) return cuda_fail("empty-input state copy", e);
+        }
+        return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
+    }
+
+    ssd::ScanArgs a;
+    a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G; a.S = S;
+    a.dtype = dims->dtype; a.Q = chunk;
+    a.x = x; a.dt = dt; a.B = B; a.C = C;
+    a.dt_bias = dt_bias; a.A = A; a.D = D; a.init_state = init_state; a.seq_idx = seq_idx;
+    a.y = y; a.final_state = final_state;
+    const int64_t max_chunks = seq_idx ? (L + chunk - 1) / chunk + S : b * ((L + chunk - 1) / chunk);
+    const size_t ws_path = ssd::simt_workspace_bytes(a, max_chunks);
+    size_t need = Carve::round(ws_path) + Carve::round(sizeof(int32_t));
+    if (seq_idx) need += 3 * Carve::round(sizeof(int32_t) * (S + 1));
+    if (need > kNoAllocScratchBytes)
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "this call needs %zu bytes of scratch; the no-allocation scan is limited to %zu "
+                    "bytes (32 MiB): use ssd_chunk_scan_fwd",
+                    need, kNoAllocScratchBytes);
+
+    void* scratch = nullptr;
+    rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+    cudaGetLastError();
+    Carve cv;
+    cv.base = (char*)scratch;
+    void* ws_main = cv.take(ws_path);
+    int32_t* status = (int32_t*)cv.take(sizeof(int32_t));
+    const bool dbg = debug_check();
+    if (dbg) cudaMemsetAsync(status, 0, sizeof(int32_t), st);
+    ssd::SeqInfo si;
+    si.L = L; si.S = (int32_t)S; si.Q = chunk; si.packed = seq_idx ? 1 : 0;
+    si.nc_row = (int32_t)((L + chunk - 1) / chunk);
+    si.start = si.end = si.chunk_off = nullptr;
+    if (seq_idx) {
+        int32_t* start = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
+        int32_t* end = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
+        int32_t* off = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
+        ssd::launch_seq_table(seq_idx, L, (int32_t)S, chunk, start, end, off, dbg ? status : nullptr, st);
+        si.start = start; si.end = end; si.chunk_off = off;
+    }
+    ssd::launch_simt_scan(a, si, max_chunks, ws_main, st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("kernel launch", e);
+    if (dbg) return debug_sync(st, status);
+    return SSD_OK;
+}

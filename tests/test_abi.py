@@ -126,3 +126,14 @@ def test_python_wrapper_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(RuntimeError, match="CUDA library missing"):
         _lib.lib()
+
+
+def test_noalloc_scan_refuses_oversized_calls_on_the_host(L):
+    # Refused before any device work: the fake pointers are never touched.
+    d = dims(batch=8, seqlen=4096, nheads=80, headdim=64, dstate=128, ngroups=1)
+    v = ctypes.c_void_p
+    rc = L.ssd_chunk_scan_fwd_noalloc(ctypes.byref(d), v(FAKE), v(FAKE * 2), None, v(FAKE * 3),
+                                      v(FAKE * 40000), v(FAKE * 80000), None, None, None, 256,
+                                      v(FAKE * 120000), None, None)
+    assert rc == 5
+    assert "32 MiB" in L.ssd_last_error().decode()
