@@ -151,9 +151,10 @@ def test_causality_bitwise():
     assert not torch.equal(y1[:, t:], y2[:, t:])
 
 
-def test_packed_isolation_bitwise():
+@pytest.mark.parametrize("dstate", [128, 256])
+def test_packed_isolation_bitwise(dstate):
     """Changing one sequence's inputs leaves every other sequence unchanged, bit for bit."""
-    w = inputs.scaled(W["packed_varlen"], nheads=8)
+    w = inputs.scaled(W["packed_varlen"], nheads=8, dstate=dstate)
     lens = [300, 17, 129, 128, 600, 1]
     d = inputs.make_inputs(w, "cuda", lengths=lens)
     y1, f1 = gpu_scan(d)
@@ -222,3 +223,21 @@ def test_prefill_then_decode_equals_longer_scan():
     yr, fr = oracle_scan(to_cpu(long))
     assert_close(torch.stack(ys, 1), yr[:, w.seqlen:], 1e-2, "decode outputs")
     assert_close(st, fr, 1e-2, "decode final state")
+
+
+def test_tensor_core_path_runs_for_bf16_p64_n128():
+    """bf16, P = 64, N = 128, chunk 128/256 calls launch the tcgen05 kernel (and
+    fp32 calls the CUDA-core kernels): no silent fallback between the two."""
+    from state_space_model_07_b200 import _lib
+    w = inputs.scaled(W["mamba2_2.7b_layer"], batch=1, seqlen=300, nheads=2)
+    d = inputs.make_inputs(w, "cuda")
+    _lib.profile_read(reset=True)
+    gpu_scan(d)
+    torch.cuda.synchronize()
+    launched = _lib.profile_read(reset=True)
+    assert launched.get("tc_scan", (0,))[0] == 1 and "simt_chunk_out" not in launched
+    d32 = inputs.make_inputs(inputs.scaled(w, dtype="f32"), "cuda")
+    gpu_scan(d32)
+    torch.cuda.synchronize()
+    launched = _lib.profile_read(reset=True)
+    assert launched.get("simt_chunk_out", (0,))[0] == 1 and "tc_scan" not in launched
