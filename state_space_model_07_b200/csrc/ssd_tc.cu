@@ -22,9 +22,10 @@
 //     shared memory.  C B^T on those fp16 copies is exact for normal-range
 //     bf16 values.
 //
-// Warp roles (160 threads): warps 0-3 are the math warpgroup (thread j owns
-// token / state row j of the tile, TMEM lane j); warp 4 lane 0 issues the TMA
-// loads (two-stage ring) and every tcgen05.mma.  All waits are bounded: on a
+// Warp roles (288 threads): warps 0-7 are two math warpgroups (thread j of
+// each owns token / state row j of the tile, TMEM lane j, and one half of the
+// row's columns); warp 8 lane 0 issues the TMA loads (two-stage ring) and
+// every tcgen05.mma.  All waits are bounded: on a
 // timeout the kernel records SSD_ERR_TIMEOUT in the status word and returns
 // after freeing its TMEM.
 #include <cuda.h>
@@ -45,8 +46,8 @@ using namespace ptx;
 constexpr int kT = 128;           // tokens per tile
 constexpr int kP = 64;            // headdim handled by this kernel
 constexpr int kN = 128;           // dstate handled by this kernel
-constexpr int kMathThreads = 128;
-constexpr int kThreads = 160;
+constexpr int kMathThreads = 256;
+constexpr int kThreads = 288;
 constexpr uint32_t kTmemCols = 512;
 // TMEM column map
 constexpr uint32_t kColCB = 0, kColS = 128, kColYd = 192, kColYo = 256, kColSc = 320;
@@ -61,10 +62,10 @@ struct __align__(1024) TcSmem {
     uint8_t c[2][2][kHalfBytes];      // C tile (fp16)
     uint8_t wx[kTileBytesX];          // (w o x) fp16, token rows
     uint8_t hs[kN * kP * 2];          // h_prev fp16, state rows
-    float cs[kT];
+    float cs[kT];          // tile-local cumulative decay, base-2 exponent
     float d[kT];
     float colfac[kT];
-    float wtot[4];
+    float wtot[2][4];
     uint64_t full[2];
     uint64_t cb_done, os_done, yd_done, ops_ready, s_ready, epi_done;
     uint32_t tmem_base;
@@ -84,7 +85,7 @@ struct TcParams {
     int H, G;
 };
 
-__device__ __forceinline__ void math_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void math_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ void set_abort(TcSmem& s, int32_t* status) {
     s.abort = 1;
@@ -136,7 +137,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
     tc_fence_after();
     const uint32_t tmem = s.tmem_base;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------------ control
         if (lane == 0 && nt > 0) {
             tma_prefetch_desc(&tm_x);
@@ -221,87 +222,101 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
         }
     } else {
         // -------------------------------------------------------------- math
-        const int j = tid;                       // token row / state row / TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const float Ah = p.A[h];
+        // Thread (quarter, ch, lane): token / state row j = 32 quarter + lane
+        // (TMEM lane j), columns [32 ch, 32 ch + 32) of its row.
+        const int quarter = warp & 3, ch = warp >> 2;
+        const int j = 32 * quarter + lane;
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        const float kLog2e = 1.4426950408889634f;
+        const float A2 = p.A[h] * kLog2e;     // decays are kept as base-2 exponents
         const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
         const float Dh = p.D ? p.D[h] : 0.f;
-        float hreg[kP];
+        float hreg[32];
         {
-            const float* src = p.init_state ? p.init_state + (((int64_t)seq * H + h) * kN + j) * kP : nullptr;
+            const float* src = p.init_state
+                ? p.init_state + (((int64_t)seq * H + h) * kN + j) * kP + 32 * ch : nullptr;
 #pragma unroll
-            for (int c = 0; c < kP; c += 4) {
+            for (int c = 0; c < 32; c += 4) {
                 float4 v = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
                 hreg[c] = v.x; hreg[c + 1] = v.y; hreg[c + 2] = v.z; hreg[c + 3] = v.w;
             }
         }
-        float cs_last_prev = 0.f;
+        float cs2_last_prev = 0.f;
         bool ok = true;
+        // dt of this thread's token in the next tile, loaded one tile ahead
+        float dt_next = 0.f;
+        if (nt > 0 && j < len) dt_next = __bfloat162float(p.dt[(tok0 + j) * H + h]);
         for (int t = 0; t < nt; ++t) {
             const int st = t & 1;
             const int q = (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT);
             const int64_t tok = tok0 + (int64_t)t * kT + j;
-            // (1) step sizes and the tile-local cumulative log-decay
+            // (1) step sizes and the tile-local cumulative log2-decay (both warpgroups
+            //     compute it; warpgroup 0 publishes it)
             float dj = 0.f, a = 0.f;
             if (j < q) {
-                const float z = __bfloat162float(p.dt[tok * H + h]) + bias;
-                dj = softplus_f(z);
-                a = dj * Ah;
+                dj = softplus_f(dt_next + bias);
+                a = dj * A2;
             }
+            if (t + 1 < nt && (int64_t)(t + 1) * kT + j < len)
+                dt_next = __bfloat162float(p.dt[(tok + kT) * H + h]);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float u = __shfl_up_sync(0xffffffffu, a, o);
                 if (lane >= o) a += u;
             }
-            if (lane == 31) s.wtot[warp] = a;
+            if (lane == 31) s.wtot[ch][quarter] = a;
             math_bar();
-            for (int w = 0; w < warp; ++w) a += s.wtot[w];
-            const float csj = a;
-            // column factor of the rank-1 split exp(cs_j - cs_i) = exp(cs_j - cs_m) exp(cs_m - cs_i)
-            // with pivot m = last token of i's 32-token block (lane 31 of this warp)
-            const float cs_pivot = __shfl_sync(0xffffffffu, csj, 31);
-            s.cs[j] = csj;
-            s.d[j] = dj;
-            s.colfac[j] = expf(cs_pivot - csj) * dj;
+            for (int w = 0; w < quarter; ++w) a += s.wtot[ch][w];
+            const float cs2j = a;
+            // column factor of the rank-1 split 2^(cs_j - cs_i) = 2^(cs_j - cs_m) 2^(cs_m - cs_i),
+            // pivot m = last token of i's 32-token block (lane 31 of this warp)
+            const float cs2_pivot = __shfl_sync(0xffffffffu, cs2j, 31);
+            if (ch == 0) {
+                s.cs[j] = cs2j;
+                s.d[j] = dj;
+                s.colfac[j] = ex2(cs2_pivot - cs2j) * dj;
+            }
             math_bar();
-            const float cs_last = s.cs[q - 1];
+            const float cs2_last = s.cs[q - 1];
 
             // (2) state entering this tile -> fp16 operand of Yo = C h_prev
             if (t > 0) {
                 if (!(ok = wait_bar(s, &s.os_done, (t - 1) & 1, p.status))) break;
                 tc_fence_after();
-                const float e = expf(cs_last_prev);
+                const float e = ex2(cs2_last_prev);
+                uint32_t r0[16], r1[16];
+                tmem_ld16(tmem + lane_base + kColSc + 32 * ch, r0);
+                tmem_ld16(tmem + lane_base + kColSc + 32 * ch + 16, r1);
+                tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < kP; c += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(tmem + lane_base + kColSc + c, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) hreg[c + k] = e * hreg[c + k] + __uint_as_float(r[k]);
+                for (int k = 0; k < 16; ++k) {
+                    hreg[k] = e * hreg[k] + __uint_as_float(r0[k]);
+                    hreg[16 + k] = e * hreg[16 + k] + __uint_as_float(r1[k]);
                 }
             }
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int m = 0; m < 4; ++m) {
                 uint4 v;
-                v.x = pack_f16x2(hreg[8 * c + 0], hreg[8 * c + 1]);
-                v.y = pack_f16x2(hreg[8 * c + 2], hreg[8 * c + 3]);
-                v.z = pack_f16x2(hreg[8 * c + 4], hreg[8 * c + 5]);
-                v.w = pack_f16x2(hreg[8 * c + 6], hreg[8 * c + 7]);
-                *reinterpret_cast<uint4*>(s.hs + sw128_off(j, c)) = v;
+                v.x = pack_f16x2(hreg[8 * m + 0], hreg[8 * m + 1]);
+                v.y = pack_f16x2(hreg[8 * m + 2], hreg[8 * m + 3]);
+                v.z = pack_f16x2(hreg[8 * m + 4], hreg[8 * m + 5]);
+                v.w = pack_f16x2(hreg[8 * m + 6], hreg[8 * m + 7]);
+                *reinterpret_cast<uint4*>(s.hs + sw128_off(j, 4 * ch + m)) = v;
             }
 
             // (3) x -> fp16 in place, w o x, rows past the sequence end zeroed
             if (!(ok = wait_bar(s, &s.full[st], (t >> 1) & 1, p.status))) break;
             if (!(ok = wait_bar(s, &s.cb_done, t & 1, p.status))) break;
-            uint32_t xr[32];
+            uint32_t xr[16];
             {
-                const float w = dj * expf(cs_last - csj);
+                const float w = dj * ex2(cs2_last - cs2j);
                 uint8_t* xt = s.x[st];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4 v = *reinterpret_cast<const uint4*>(xt + sw128_off(j, c));
+                for (int m = 0; m < 4; ++m) {
+                    const uint32_t off = sw128_off(j, 4 * ch + m);
+                    uint4 v = *reinterpret_cast<const uint4*>(xt + off);
                     if (j >= q) v = make_uint4(0u, 0u, 0u, 0u);
-                    xr[4 * c] = v.x; xr[4 * c + 1] = v.y; xr[4 * c + 2] = v.z; xr[4 * c + 3] = v.w;
+                    xr[4 * m] = v.x; xr[4 * m + 1] = v.y; xr[4 * m + 2] = v.z; xr[4 * m + 3] = v.w;
                     uint4 xf, wf;
                     xf.x = pack_f16x2(bf16lo(v.x), bf16hi(v.x));
                     xf.y = pack_f16x2(bf16lo(v.y), bf16hi(v.y));
@@ -311,57 +326,62 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                     wf.y = pack_f16x2(w * bf16lo(v.y), w * bf16hi(v.y));
                     wf.z = pack_f16x2(w * bf16lo(v.z), w * bf16hi(v.z));
                     wf.w = pack_f16x2(w * bf16lo(v.w), w * bf16hi(v.w));
-                    *reinterpret_cast<uint4*>(xt + sw128_off(j, c)) = xf;
-                    *reinterpret_cast<uint4*>(s.wx + sw128_off(j, c)) = wf;
+                    *reinterpret_cast<uint4*>(xt + off) = xf;
+                    *reinterpret_cast<uint4*>(s.wx + off) = wf;
                 }
                 if (j >= q) {
                     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        *reinterpret_cast<uint4*>(s.b[st][0] + sw128_off(j, c)) = z;
-                        *reinterpret_cast<uint4*>(s.b[st][1] + sw128_off(j, c)) = z;
-                    }
+                    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(s.b[st][ch] + sw128_off(j, c)) = z;
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&s.ops_ready);
 
-            // (4) S = CB o decay o d, causal, written to TMEM as the A operand of Yd
+            // (4) S = CB o decay o d, causal, into TMEM as the A operand of Yd.
+            //     This thread covers CB columns [32 bi + 16 ch, + 16) of each 32-block bi.
             tc_fence_after();
             {
                 const int bj = j >> 5;
 #pragma unroll
-                for (int bi = 0; bi < 4; ++bi) {
-                    uint32_t sv[16];
-                    if (bi > bj) {
+                for (int pair = 0; pair < 2; ++pair) {
+                    uint32_t r[2][16];
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) sv[k] = 0u;
-                    } else {
-                        uint32_t r0[16], r1[16];
-                        tmem_ld16(tmem + lane_base + kColCB + 32 * bi, r0);
-                        tmem_ld16(tmem + lane_base + kColCB + 32 * bi + 16, r1);
-                        tmem_ld_wait();
-                        float v[32];
-                        if (bi < bj) {
-                            const float rf = expf(csj - s.cs[32 * bi + 31]);
+                    for (int u = 0; u < 2; ++u)
+                        if (2 * pair + u <= bj)
+                            tmem_ld16(tmem + lane_base + kColCB + 32 * (2 * pair + u) + 16 * ch, r[u]);
+                    tmem_ld_wait();
 #pragma unroll
-                            for (int k = 0; k < 16; ++k) {
-                                v[k] = __uint_as_float(r0[k]) * s.colfac[32 * bi + k] * rf;
-                                v[k + 16] = __uint_as_float(r1[k]) * s.colfac[32 * bi + 16 + k] * rf;
+                    for (int u = 0; u < 2; ++u) {
+                        const int bi = 2 * pair + u;
+                        uint32_t sv[8];
+                        const int i0 = 32 * bi + 16 * ch;
+                        if (bi > bj) {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) sv[k] = 0u;
+                        } else if (bi < bj) {
+                            const float rf = ex2(cs2j - s.cs[32 * bi + 31]);
+#pragma unroll
+                            for (int k = 0; k < 16; k += 4) {
+                                const float4 cf = *reinterpret_cast<const float4*>(&s.colfac[i0 + k]);
+                                sv[k / 2] = pack_f16x2(__uint_as_float(r[u][k]) * cf.x * rf,
+                                                       __uint_as_float(r[u][k + 1]) * cf.y * rf);
+                                sv[k / 2 + 1] = pack_f16x2(__uint_as_float(r[u][k + 2]) * cf.z * rf,
+                                                           __uint_as_float(r[u][k + 3]) * cf.w * rf);
                             }
                         } else {
 #pragma unroll
-                            for (int k = 0; k < 32; ++k) {
-                                const int i = 32 * bi + k;
-                                const float cb = __uint_as_float(k < 16 ? r0[k] : r1[k - 16]);
-                                v[k] = i <= j ? cb * expf(csj - s.cs[i]) * s.d[i] : 0.f;
+                            for (int k = 0; k < 16; k += 2) {
+                                const int i = i0 + k;
+                                const float e0 = ex2(cs2j - s.cs[i]) * s.d[i];
+                                const float e1 = ex2(cs2j - s.cs[i + 1]) * s.d[i + 1];
+                                sv[k / 2] = pack_f16x2(i <= j ? __uint_as_float(r[u][k]) * e0 : 0.f,
+                                                       i + 1 <= j ? __uint_as_float(r[u][k + 1]) * e1 : 0.f);
                             }
                         }
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) sv[k] = pack_f16x2(v[2 * k], v[2 * k + 1]);
+                        tmem_st8(tmem + lane_base + kColS + 16 * bi + 8 * ch, sv);
                     }
-                    tmem_st16(tmem + lane_base + kColS + 16 * bi, sv);
                 }
                 tmem_st_wait();
             }
@@ -372,53 +392,55 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             if (!(ok = wait_bar(s, &s.yd_done, t & 1, p.status))) break;
             tc_fence_after();
             {
-                const float ej = expf(csj);
-                __nv_bfloat16* yrow = p.y + tok * H * kP + (int64_t)h * kP;
+                const float ej = ex2(cs2j);
+                __nv_bfloat16* yrow = p.y + tok * H * kP + (int64_t)h * kP + 32 * ch;
 #pragma unroll
-                for (int c = 0; c < kP; c += 16) {
+                for (int half = 0; half < 2; ++half) {
                     uint32_t rd[16], ro[16];
-                    tmem_ld16(tmem + lane_base + kColYd + c, rd);
-                    tmem_ld16(tmem + lane_base + kColYo + c, ro);
+                    tmem_ld16(tmem + lane_base + kColYd + 32 * ch + 16 * half, rd);
+                    tmem_ld16(tmem + lane_base + kColYo + 32 * ch + 16 * half, ro);
                     tmem_ld_wait();
+                    if (half == 1) {
+                        tc_fence_before();
+                        mbar_arrive(&s.epi_done);
+                    }
                     uint32_t out[8];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
-                        const uint32_t xv = xr[(c >> 1) + k];
-                        const float y0 = __uint_as_float(rd[2 * k]) + ej * __uint_as_float(ro[2 * k]) +
-                                         Dh * bf16lo(xv);
-                        const float y1 = __uint_as_float(rd[2 * k + 1]) +
-                                         ej * __uint_as_float(ro[2 * k + 1]) + Dh * bf16hi(xv);
-                        out[k] = pack_bf16x2(y0, y1);
+                        const uint32_t xv = xr[8 * half + k];
+                        out[k] = pack_bf16x2(
+                            __uint_as_float(rd[2 * k]) + ej * __uint_as_float(ro[2 * k]) + Dh * bf16lo(xv),
+                            __uint_as_float(rd[2 * k + 1]) + ej * __uint_as_float(ro[2 * k + 1]) +
+                                Dh * bf16hi(xv));
                     }
                     if (j < q) {
-                        *reinterpret_cast<uint4*>(yrow + c) = make_uint4(out[0], out[1], out[2], out[3]);
-                        *reinterpret_cast<uint4*>(yrow + c + 8) = make_uint4(out[4], out[5], out[6], out[7]);
+                        *reinterpret_cast<uint4*>(yrow + 16 * half) = make_uint4(out[0], out[1], out[2], out[3]);
+                        *reinterpret_cast<uint4*>(yrow + 16 * half + 8) = make_uint4(out[4], out[5], out[6], out[7]);
                     }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&s.epi_done);
-            cs_last_prev = cs_last;
+            cs2_last_prev = cs2_last;
         }
         // final state after the last tile
         if (ok && nt > 0) {
             if (wait_bar(s, &s.os_done, (nt - 1) & 1, p.status)) {
                 tc_fence_after();
-                const float e = expf(cs_last_prev);
+                const float e = ex2(cs2_last_prev);
+                uint32_t r0[16], r1[16];
+                tmem_ld16(tmem + lane_base + kColSc + 32 * ch, r0);
+                tmem_ld16(tmem + lane_base + kColSc + 32 * ch + 16, r1);
+                tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < kP; c += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(tmem + lane_base + kColSc + c, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) hreg[c + k] = e * hreg[c + k] + __uint_as_float(r[k]);
+                for (int k = 0; k < 16; ++k) {
+                    hreg[k] = e * hreg[k] + __uint_as_float(r0[k]);
+                    hreg[16 + k] = e * hreg[16 + k] + __uint_as_float(r1[k]);
                 }
             }
         }
         if (p.final_state && !s.abort) {
-            float* dst = p.final_state + (((int64_t)seq * H + h) * kN + j) * kP;
+            float* dst = p.final_state + (((int64_t)seq * H + h) * kN + j) * kP + 32 * ch;
 #pragma unroll
-            for (int c = 0; c < kP; c += 4)
+            for (int c = 0; c < 32; c += 4)
                 *reinterpret_cast<float4*>(dst + c) = make_float4(hreg[c], hreg[c + 1], hreg[c + 2], hreg[c + 3]);
         }
     }

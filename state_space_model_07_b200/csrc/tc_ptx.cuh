@@ -191,7 +191,14 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                    "r"(r[13]), "r"(r[14]), "r"(r[15])                                                \
                  : "memory")
 
+#define SSD_TMEM_ST8(taddr, r)                                                                       \
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"             \
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),     \
+                   "r"(r[6]), "r"(r[7])                                                              \
+                 : "memory")
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) { SSD_TMEM_LD16(taddr, r); }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) { SSD_TMEM_ST8(taddr, r); }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     SSD_TMEM_ST16(taddr, r);
 }
@@ -202,6 +209,14 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 // tile of 128-byte rows whose 8-row groups are 1024 bytes apart. ------------------------------
 __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {
     return r * 128u + ((c ^ (r & 7u)) << 4);
+}
+
+// 2^x on the MUFU unit (relative error about 2^-22; -inf and large negative
+// arguments give +0).
+__device__ __forceinline__ float ex2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
 // ---- packing -------------------------------------------------------------------------------------
