@@ -58,16 +58,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// `limit_ns` of wall time (returns false) so that a lost arrival can never
-// hang the GPU; callers turn that into an error status.
+// `limit_cycles` SM clock cycles (about two seconds by default; returns false)
+// so that a lost arrival can never hang the GPU; callers turn that into an
+// error status.  The clock is the SM's own cycle counter, which is cheap to
+// read on every poll.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          uint64_t limit_ns = 2000000000ull) {
+                                          long long limit_cycles = 4000000000ll) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > limit_ns) return false;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > limit_cycles) return false;
     }
+    return true;
 }
 
 // ---- proxies and fences ------------------------------------------------------------
@@ -197,7 +199,14 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                    "r"(r[6]), "r"(r[7])                                                              \
                  : "memory")
 
+#define SSD_TMEM_LD8(taddr, r)                                                                       \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"              \
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),           \
+                   "=r"(r[6]), "=r"(r[7])                                                            \
+                 : "r"(taddr))
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) { SSD_TMEM_LD16(taddr, r); }
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) { SSD_TMEM_LD8(taddr, r); }
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) { SSD_TMEM_ST8(taddr, r); }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     SSD_TMEM_ST16(taddr, r);
