@@ -331,49 +331,44 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             // handles the 32-column blocks pr <= quarter of its parity.  Blocks strictly
             // below the diagonal use the rank-1 split; the block holding the diagonal uses
             // the full exponential in every lane (exact there too), so no lane diverges.
+#pragma unroll 1
+            for (int b = 2 * half; b <= 2 * quarter + 1; b += (b & 1) ? 3 : 1) {
+                // 16-column block b (pairs pr = b / 2 of this warp's parity)
+                const int pr = b >> 1;
+                const int i0 = 16 * b;
+                uint32_t r[16];
+                tmem_ld16(tmem + lane_base + kColCB + i0, r);
+                float f[16];
+                if (pr < quarter) {
+                    const float rf = ex2(cs2j - s.cs[buf][i0 + 15]);
 #pragma unroll
-            for (int pr = 0; pr < 4; ++pr) {
-                if (pr > quarter || (pr & 1) != half) continue;
-                uint32_t r[2][16];
-                tmem_ld16(tmem + lane_base + kColCB + 32 * pr, r[0]);
-                tmem_ld16(tmem + lane_base + kColCB + 32 * pr + 16, r[1]);
-                tmem_ld_wait();
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int i0 = 32 * pr + 16 * u;
-                    float f[16];
-                    if (pr < quarter) {
-                        const float rf = ex2(cs2j - s.cs[buf][i0 + 15]);
-#pragma unroll
-                        for (int k = 0; k < 16; k += 4) {
-                            const float4 cf = *reinterpret_cast<const float4*>(&s.colfac[buf][i0 + k]);
-                            f[k] = cf.x * rf; f[k + 1] = cf.y * rf; f[k + 2] = cf.z * rf; f[k + 3] = cf.w * rf;
-                        }
-                    } else {
-                        float c[16], dd[16];
-#pragma unroll
-                        for (int k = 0; k < 16; k += 4) {
-                            const float4 cv = *reinterpret_cast<const float4*>(&s.cs[buf][i0 + k]);
-                            const float4 dv = *reinterpret_cast<const float4*>(&s.d[buf][i0 + k]);
-                            c[k] = cv.x; c[k + 1] = cv.y; c[k + 2] = cv.z; c[k + 3] = cv.w;
-                            dd[k] = dv.x; dd[k + 1] = dv.y; dd[k + 2] = dv.z; dd[k + 3] = dv.w;
-                        }
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) f[k] = i0 + k <= j ? ex2(cs2j - c[k]) * dd[k] : 0.f;
+                    for (int k = 0; k < 16; k += 4) {
+                        const float4 cf = *reinterpret_cast<const float4*>(&s.colfac[buf][i0 + k]);
+                        f[k] = cf.x * rf; f[k + 1] = cf.y * rf; f[k + 2] = cf.z * rf; f[k + 3] = cf.w * rf;
                     }
-                    uint32_t sv[8];
+                } else {
+                    float c[16], dd[16];
 #pragma unroll
-                    for (int k = 0; k < 16; k += 2) {
-                        float v0 = __uint_as_float(r[u][k]) * f[k];
-                        float v1 = __uint_as_float(r[u][k + 1]) * f[k + 1];
-                        if (pr == quarter) {
-                            if (i0 + k == j) v0 += Dh;
-                            if (i0 + k + 1 == j) v1 += Dh;
-                        }
-                        sv[k / 2] = pack_f16x2(v0, v1);
+                    for (int k = 0; k < 16; k += 4) {
+                        const float4 cv = *reinterpret_cast<const float4*>(&s.cs[buf][i0 + k]);
+                        const float4 dv = *reinterpret_cast<const float4*>(&s.d[buf][i0 + k]);
+                        c[k] = cv.x; c[k + 1] = cv.y; c[k + 2] = cv.z; c[k + 3] = cv.w;
+                        dd[k] = dv.x; dd[k + 1] = dv.y; dd[k + 2] = dv.z; dd[k + 3] = dv.w;
                     }
-                    tmem_st8(tmem + lane_base + kColS + 8 * (2 * pr + u), sv);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) f[k] = i0 + k <= j ? ex2(cs2j - c[k]) * dd[k] : 0.f;
                 }
+                tmem_ld_wait();
+                uint32_t sv[8];
+#pragma unroll
+                for (int k = 0; k < 16; k += 2) {
+                    float v0 = __uint_as_float(r[k]) * f[k];
+                    float v1 = __uint_as_float(r[k + 1]) * f[k + 1];
+                    if (i0 + k == j) v0 += Dh;
+                    if (i0 + k + 1 == j) v1 += Dh;
+                    sv[k / 2] = pack_f16x2(v0, v1);
+                }
+                tmem_st8(tmem + lane_base + kColS + 8 * b, sv);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -459,16 +454,21 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             mbar_arrive(&s.x_ready);
             return true;
         };
-        bool ok = nt == 0 || prepare(0, true);
-        for (int t = 0; ok && t < nt; ++t) {
-            const int st = t & 1;
-            const int q = (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT);
-            if (t + 1 < nt) {
-                // the state entering tile t + 1 is complete once B^T (w o x) of tile t has been added
-                if (!(ok = wait_role<2>(s, &s.sc_done, t & 1, p.status, warp == 8, &s.e_flag))) break;
-                tc_fence_after();
-                if (!(ok = prepare(t + 1, false))) break;
+        // Step k prepares tile k (once the state entering it is complete) and then
+        // writes the output of tile k - 1.
+        bool ok = true;
+        for (int k = 0; ok && k <= nt; ++k) {
+            if (k < nt) {
+                // the state entering tile k is complete once B^T (w o x) of tile k - 1 has been added
+                if (k > 0) {
+                    if (!(ok = wait_role<2>(s, &s.sc_done, (k - 1) & 1, p.status, warp == 8, &s.e_flag))) break;
+                    tc_fence_after();
+                }
+                if (!(ok = prepare(k, k == 0))) break;
             }
+            if (k == 0) continue;
+            const int t = k - 1, st = t & 1;
+            const int q = (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT);
             // epilogue of tile t: y = Yd + 2^cs_j Yo   (D x is inside Yd)
             if (!(ok = wait_role<2>(s, &s.yd_par[st], (t >> 1) & 1, p.status, warp == 8, &s.e_flag))) break;
             tc_fence_after();
@@ -484,9 +484,9 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                     tmem_ld_wait();
                     uint32_t out[8];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        out[k] = pack_bf16x2(__uint_as_float(rd[2 * k]) + ej * __uint_as_float(ro[2 * k]),
-                                             __uint_as_float(rd[2 * k + 1]) + ej * __uint_as_float(ro[2 * k + 1]));
+                    for (int k2 = 0; k2 < 8; ++k2)
+                        out[k2] = pack_bf16x2(__uint_as_float(rd[2 * k2]) + ej * __uint_as_float(ro[2 * k2]),
+                                              __uint_as_float(rd[2 * k2 + 1]) + ej * __uint_as_float(ro[2 * k2 + 1]));
                     if (j < q) {
                         *reinterpret_cast<uint4*>(yrow + c) = make_uint4(out[0], out[1], out[2], out[3]);
                         *reinterpret_cast<uint4*>(yrow + c + 8) = make_uint4(out[4], out[5], out[6], out[7]);
