@@ -62,14 +62,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // so that a lost arrival can never hang the GPU; callers turn that into an
 // error status.  The clock is the SM's own cycle counter, which is cheap to
 // read on every poll.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          long long limit_cycles = 4000000000ll) {
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long long limit_cycles) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (clock64() - t0 > limit_cycles) return false;
     }
     return true;
+}
+
+// The first test is inlined; the polling loop is shared out of line to keep
+// the kernels' code (and instruction-cache footprint) small.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          long long limit_cycles = 4000000000ll) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, limit_cycles);
 }
 
 // ---- proxies and fences ------------------------------------------------------------
