@@ -2,7 +2,7 @@
 """SSD chunked-scan forward throughput on B200, one JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--batch B] [--no-e2e] [--no-cpu-baseline]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
 ssd_chunk_scan_fwd over the workload (decay cumsum, intra-chunk quadratic
@@ -49,7 +49,17 @@ def parse():
     ap.add_argument("--workload", default="mamba2_2.7b_layer")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (small cases for profiling; not a bench line)")
     return ap.parse_args()
+
+
+def workload_of(args):
+    from state_space_model_07_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    if args.batch is not None and not w.packed_nseqs:
+        w = inputs.scaled(w, batch=args.batch)
+    return w
 
 
 def peaks():
@@ -164,9 +174,9 @@ def oracle_sample(w, heads, rows=None):
     first `rows` batch rows; returns (seconds, token-equivalents, threads)."""
     import oracle
     from state_space_model_07_b200 import inputs
-    if w.name not in _CPU_INPUTS:
-        _CPU_INPUTS[w.name] = inputs.make_inputs(w, "cpu")
-    d = _CPU_INPUTS[w.name]
+    if (w.name, w.batch) not in _CPU_INPUTS:
+        _CPU_INPUTS[(w.name, w.batch)] = inputs.make_inputs(w, "cpu")
+    d = _CPU_INPUTS[(w.name, w.batch)]
     H, G = w.nheads, w.ngroups
     hs = list(range(heads))
     gs = [h // (H // G) for h in hs]
@@ -211,8 +221,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    from state_space_model_07_b200 import inputs
-    w = inputs.WORKLOADS[args.workload]
+    w = workload_of(args)
     # Each step: the oracle on 2 heads of every sequence (a bounded sample).
     heads = max(1, min(w.nheads, 2))
     for _ in range(args.warmup):
@@ -284,7 +293,7 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    w = inputs.WORKLOADS[args.workload]
+    w = workload_of(args)
     d = inputs.make_inputs(w, dev)
     b, L, H, P = d["x"].shape
     N, G, S = w.dstate, w.ngroups, d["nseqs"]
