@@ -54,40 +54,63 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kT = 128;           // tokens per tile
-constexpr int kP = 64;            // headdim handled by this kernel
-constexpr int kN = 128;           // dstate handled by this kernel
+constexpr int kT = 128;             // tokens per tile
+constexpr int kP = 64;              // headdim handled by this kernel
 constexpr int kRoleThreads = 256;   // P and E: two warps per TMEM lane quarter
 constexpr int kThreads = 576;
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: C B^T, S (fp16 pairs), Yd[2], Yo[2], running state H
-constexpr uint32_t kColCB = 0, kColS = 128, kColYd = 192, kColYo = 320, kColH = 448;
+constexpr uint32_t kTileBytesX = kT * kP * 2;     // 16 KB
+constexpr uint32_t kBoxBytes = kT * 64 * 2;       // one 64-column box of a B or C tile: 16 KB
 
-constexpr uint32_t kTileBytesX = kT * kP * 2;        // 16 KB
-constexpr uint32_t kHalfBytes = kT * 64 * 2;         // one 64-column half of a B or C tile: 16 KB
-constexpr uint32_t kStageBytes = kTileBytesX + 4 * kHalfBytes;
+// Layout constants for dstate N (128 or 256).
+//   N = 128: B and C tiles double-buffered; Yd, Yo double-buffered.
+//   N = 256: B and C tiles (64 KB each) single-buffered, reloaded once the
+//            tile's C h_prev and B^T (w o x) MMAs are done; Yd single-buffered
+//            (its MMA waits for the previous epilogue), Yo double-buffered; the
+//            state takes two 128-lane TMEM blocks.
+template <int N>
+struct Cfg {
+    static constexpr int kBoxes = N / 64;                   // 64-column boxes per B / C tile
+    static constexpr int kBCStages = N == 128 ? 2 : 1;
+    static constexpr int kYdBufs = N == 128 ? 2 : 1;
+    static constexpr int kHBlocks = N / 128;                // 128-row blocks of the state
+    // TMEM columns: C B^T | S (fp16 pairs) | Yd[kYdBufs] | Yo[2] | H[kHBlocks]
+    static constexpr uint32_t kColCB = 0, kColS = 128, kColYd = 192;
+    static constexpr uint32_t kColYo = kColYd + 64 * kYdBufs;
+    static constexpr uint32_t kColH = kColYo + 128;
+    static_assert(kColH + 64 * kHBlocks <= kTmemCols, "TMEM columns");
+    static constexpr uint32_t kBCBytes = 2 * kBoxes * kBoxBytes;  // B and C of one tile
+};
 
+struct TcCtl {
+    int abort;
+    int p_flag, e_flag;    // leader-wait results handed to the rest of a role
+};
+
+template <int N>
 struct __align__(1024) TcSmem {
-    uint8_t x[2][kTileBytesX];        // x tile per stage (bf16 from TMA, fp16 after conversion)
-    uint8_t b[2][2][kHalfBytes];      // B tile (fp16) per stage: n in [0,64) and [64,128)
-    uint8_t c[2][2][kHalfBytes];      // C tile (fp16)
-    uint8_t wx[2][kTileBytesX];       // (w o x) fp16, token rows, by tile parity
-    uint8_t hs[kN * kP * 2];          // h_prev fp16, state rows
+    uint8_t x[2][kTileBytesX];                         // x per stage (bf16 from TMA, fp16 after conversion)
+    uint8_t b[Cfg<N>::kBCStages][Cfg<N>::kBoxes][kBoxBytes];  // B (fp16), 64-column boxes
+    uint8_t c[Cfg<N>::kBCStages][Cfg<N>::kBoxes][kBoxBytes];  // C (fp16)
+    uint8_t wx[kTileBytesX];                           // (w o x) fp16, token rows
+    uint8_t hs[N * kP * 2];                            // h_prev fp16, state rows
     float cs[2][kT];       // tile-local cumulative decay (base-2 exponent), by tile parity
     float d[2][kT];
     float colfac[2][kT];   // 2^(cs_m - cs_i) d_i with pivot m = last token of i's 16-block
     float wtot[2][4];
-    uint64_t full[2];         // TMA -> E, W8            (per stage)
-    uint64_t scan_done[2];    // P -> E                  (per tile parity)
-    uint64_t e_done[2];       // E -> P                  (per tile parity)
-    uint64_t yd_par[2];       // W9 commit -> E, P, W8   (per tile parity)
-    uint64_t cb_done;         // W8 commit -> P
-    uint64_t s_ready;         // P -> W8, W9
-    uint64_t x_ready;         // E -> W9
-    uint64_t sc_done;         // W9 commit -> E
+    // Every barrier's next phase depends on an action its waiters take after
+    // waiting, so no waiter can ever see a barrier two phases ahead.
+    uint64_t xfull[2];        // TMA x -> E, W17          (per x stage)
+    uint64_t bcfull[2];       // TMA B, C -> W16          (per B/C stage)
+    uint64_t scan_done[2];    // P -> E                   (per tile parity)
+    uint64_t e_done[2];       // E -> P (and W17 at N = 256)  (per tile parity)
+    uint64_t yd_par[2];       // W17 commit -> E, P, W16  (per tile parity)
+    uint64_t cb_done;         // W16 commit -> P
+    uint64_t s_ready;         // P -> W16, W17
+    uint64_t x_ready;         // E -> W17
+    uint64_t sc_done;         // W17 commit -> E (and W16 at N = 256)
     uint32_t tmem_base;
-    int abort;
-    int p_flag, e_flag;    // leader-wait results handed to the rest of a role
+    TcCtl ctl;
 };
 
 struct TcParams {
@@ -108,16 +131,12 @@ __device__ __forceinline__ void p_bar() { asm volatile("bar.sync 1, 256;" ::: "m
 __device__ __forceinline__ __half2 u2h(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
 __device__ __forceinline__ uint32_t h2u(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
-__device__ __forceinline__ void set_abort(TcSmem& s, int32_t* status) {
-    s.abort = 1;
-    if (status) atomicExch(status, kStatusTimeout);
-}
-
 // Bounded wait of a single issuing thread; false once the CTA has given up.
-__device__ __forceinline__ bool wait_bar(TcSmem& s, uint64_t* bar, uint32_t parity, int32_t* status) {
-    if (*(volatile int*)&s.abort) return false;
+__device__ __forceinline__ bool wait_bar(TcCtl& c, uint64_t* bar, uint32_t parity, int32_t* status) {
+    if (*(volatile int*)&c.abort) return false;
     if (!mbar_wait(bar, parity)) {
-        set_abort(s, status);
+        c.abort = 1;
+        if (status) atomicExch(status, kStatusTimeout);
         return false;
     }
     return true;
@@ -126,8 +145,8 @@ __device__ __forceinline__ bool wait_bar(TcSmem& s, uint64_t* bar, uint32_t pari
 // Bounded wait of a whole warp; the result is the same in every lane, so the
 // warp-collective TMEM instructions that follow stay uniform even on the
 // error path.
-__device__ __forceinline__ bool wait_bar_w(TcSmem& s, uint64_t* bar, uint32_t parity, int32_t* status) {
-    return __all_sync(0xffffffffu, wait_bar(s, bar, parity, status));
+__device__ __forceinline__ bool wait_bar_w(TcCtl& c, uint64_t* bar, uint32_t parity, int32_t* status) {
+    return __all_sync(0xffffffffu, wait_bar(c, bar, parity, status));
 }
 
 // Bounded wait of a whole 8-warp role: only the role's first warp polls the
@@ -135,24 +154,27 @@ __device__ __forceinline__ bool wait_bar_w(TcSmem& s, uint64_t* bar, uint32_t pa
 // warps take no issue slots from the warps doing work.  `flag` carries the
 // leader's result (false once the CTA has given up) to the others.
 template <int kBarId>
-__device__ __forceinline__ bool wait_role(TcSmem& s, uint64_t* bar, uint32_t parity, int32_t* status,
+__device__ __forceinline__ bool wait_role(TcCtl& c, uint64_t* bar, uint32_t parity, int32_t* status,
                                           bool leader, int* flag) {
     if (leader) {
-        const bool ok = wait_bar_w(s, bar, parity, status);
+        const bool ok = wait_bar_w(c, bar, parity, status);
         if ((threadIdx.x & 31) == 0) *(volatile int*)flag = ok ? 1 : 0;
     }
     asm volatile("bar.sync %0, 256;" ::"n"(kBarId) : "memory");
     return *(volatile int*)flag != 0;
 }
 
+template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
 k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
           const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
+    using C = Cfg<N>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // Align to 1024 bytes (128-byte swizzle atoms) by pointer arithmetic on the
     // shared array, so that the compiler keeps every access in the shared state
     // space (a round trip through an integer would turn them into generic ones).
-    TcSmem& s = *reinterpret_cast<TcSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    TcSmem<N>& s = *reinterpret_cast<TcSmem<N>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    TcCtl& ctl = s.ctl;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, G = p.G;
     const int h = blockIdx.x % H;
@@ -167,7 +189,8 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.full[i], 1);
+            mbar_init(&s.xfull[i], 1);
+            mbar_init(&s.bcfull[i], 1);
             mbar_init(&s.scan_done[i], kRoleThreads);
             mbar_init(&s.e_done[i], kRoleThreads);
             mbar_init(&s.yd_par[i], 1);
@@ -176,7 +199,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
         mbar_init(&s.s_ready, kRoleThreads);
         mbar_init(&s.x_ready, kRoleThreads);
         mbar_init(&s.sc_done, 1);
-        s.abort = 0;
+        ctl.abort = 0;
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(&s.tmem_base, kTmemCols);
@@ -192,43 +215,64 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
             tma_prefetch_desc(&tm_c);
-            int loads_issued = 0;
-            auto issue_loads = [&](int t) {
+            int x_issued = 0, bc_issued = 0;
+            auto load_x = [&](int t) {
                 const int st = t & 1;
+                mbar_expect_tx(&s.xfull[st], kTileBytesX);
+                tma_load_3d(s.x[st], &tm_x, &s.xfull[st], 0, h, (int)(tok0 + (int64_t)t * kT));
+                ++x_issued;
+            };
+            auto load_bc = [&](int t) {
+                const int st = t % C::kBCStages;
                 const int tok = (int)(tok0 + (int64_t)t * kT);
-                mbar_expect_tx(&s.full[st], kStageBytes);
-                tma_load_3d(s.x[st], &tm_x, &s.full[st], 0, h, tok);
-                for (int k = 0; k < 2; ++k) {
-                    tma_load_3d(s.b[st][k], &tm_b, &s.full[st], 64 * k, g, tok);
-                    tma_load_3d(s.c[st][k], &tm_c, &s.full[st], 64 * k, g, tok);
+                mbar_expect_tx(&s.bcfull[st], C::kBCBytes);
+                for (int k = 0; k < C::kBoxes; ++k) {
+                    tma_load_3d(s.b[st][k], &tm_b, &s.bcfull[st], 64 * k, g, tok);
+                    tma_load_3d(s.c[st][k], &tm_c, &s.bcfull[st], 64 * k, g, tok);
                 }
-                ++loads_issued;
+                ++bc_issued;
             };
             const uint32_t id_cb = idesc_f16(128, 128, 0, 0);
-            issue_loads(0);
-            if (nt > 1) issue_loads(1);
+            load_x(0);
+            load_bc(0);
+            if (nt > 1) {
+                load_x(1);
+                if (C::kBCStages == 2) load_bc(1);
+            }
             bool ok = true;
             for (int t = 0; t < nt; ++t) {
-                const int st = t & 1;
-                if (!(ok = wait_bar(s, &s.full[st], (t >> 1) & 1, p.status))) break;
+                const int bst = t % C::kBCStages;
+                const uint32_t bpar = (uint32_t)((t / C::kBCStages) & 1);
+                if (!(ok = wait_bar(ctl, &s.bcfull[bst], bpar, p.status))) break;
                 // P has finished reading C B^T of the previous tile
-                if (t > 0 && !(ok = wait_bar(s, &s.s_ready, (t - 1) & 1, p.status))) break;
+                if (t > 0 && !(ok = wait_bar(ctl, &s.s_ready, (t - 1) & 1, p.status))) break;
                 tc_fence_after();
-                const uint32_t cb = smem_u32(s.c[st][0]), bb = smem_u32(s.b[st][0]);
-                for (int k = 0; k < kN / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
-                    mma_ss(tmem + kColCB, sdesc_sw128(cb + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024),
+                const uint32_t cb = smem_u32(s.c[bst][0]), bb = smem_u32(s.b[bst][0]);
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
+                    mma_ss(tmem + C::kColCB, sdesc_sw128(cb + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024),
                            id_cb, k > 0);
                 }
                 mma_commit(&s.cb_done);
-                // stage (t + 1) & 1 is free once every MMA of tile t - 1 has completed
                 if (t >= 1 && t + 1 < nt) {
-                    if (!(ok = wait_bar(s, &s.yd_par[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status))) break;
-                    issue_loads(t + 1);
+                    // x stage (t + 1) & 1 (and, double-buffered, that B/C stage) is free once
+                    // every MMA of tile t - 1 has completed
+                    if (!(ok = wait_bar(ctl, &s.yd_par[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status))) break;
+                    load_x(t + 1);
+                    if (C::kBCStages == 2) load_bc(t + 1);
+                }
+                if (C::kBCStages == 1 && t + 1 < nt) {
+                    // the single B/C stage is free once C h_prev and B^T (w o x) of tile t are done
+                    if (!(ok = wait_bar(ctl, &s.sc_done, t & 1, p.status))) break;
+                    load_bc(t + 1);
                 }
             }
-            if (!ok)
-                for (int t = 0; t < loads_issued; ++t) mbar_wait(&s.full[t & 1], (t >> 1) & 1, 400000000ll);
+            if (!ok) {
+                // Give up: let the copies already in flight land before the CTA exits.
+                for (int t = 0; t < x_issued; ++t) mbar_wait(&s.xfull[t & 1], (t >> 1) & 1, 400000000ll);
+                for (int t = 0; t < bc_issued; ++t)
+                    mbar_wait(&s.bcfull[t % C::kBCStages], (t / C::kBCStages) & 1, 400000000ll);
+            }
         }
     } else if (warp == 17) {
         // ----------------------------------- W17: C h_prev, B^T (w o x), S x
@@ -236,28 +280,35 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             const uint32_t id_pn = idesc_f16(128, 64, 0, 1);   // K-major A, MN-major B
             const uint32_t id_mn = idesc_f16(128, 64, 1, 1);   // MN-major A and B
             for (int t = 0; t < nt; ++t) {
-                const int st = t & 1;
-                if (!wait_bar(s, &s.x_ready, t & 1, p.status)) break;
+                const int st = t & 1, bst = t % C::kBCStages;
+                if (!wait_bar(ctl, &s.x_ready, t & 1, p.status)) break;
                 tc_fence_after();
-                const uint32_t cb = smem_u32(s.c[st][0]), bb = smem_u32(s.b[st][0]);
-                const uint32_t hsb = smem_u32(s.hs), wxb = smem_u32(s.wx[st]), xb = smem_u32(s.x[st]);
+                const uint32_t cb = smem_u32(s.c[bst][0]), bb = smem_u32(s.b[bst][0]);
+                const uint32_t hsb = smem_u32(s.hs), wxb = smem_u32(s.wx), xb = smem_u32(s.x[st]);
                 // Yo = C h_prev
-                for (int k = 0; k < kN / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
-                    mma_ss(tmem + kColYo + 64 * st, sdesc_sw128(cb + off, 16, 1024),
-                           sdesc_sw128(hsb + k * 2048, kHalfBytes, 1024), id_pn, k > 0);
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
+                    mma_ss(tmem + C::kColYo + 64 * st, sdesc_sw128(cb + off, 16, 1024),
+                           sdesc_sw128(hsb + k * 2048, kBoxBytes, 1024), id_pn, k > 0);
                 }
-                // H += B^T (w o x): needs the B rows past the sequence end zeroed by P
-                if (!wait_bar(s, &s.s_ready, t & 1, p.status)) break;
+                // H += B^T (w o x), one 128-row block of the state at a time: needs the B rows
+                // past the sequence end zeroed by P
+                if (!wait_bar(ctl, &s.s_ready, t & 1, p.status)) break;
                 tc_fence_after();
-                for (int k = 0; k < kT / 16; ++k)
-                    mma_ss(tmem + kColH, sdesc_sw128(bb + k * 2048, kHalfBytes, 1024),
-                           sdesc_sw128(wxb + k * 2048, kHalfBytes, 1024), id_mn, 1);
+                for (int mb = 0; mb < C::kHBlocks; ++mb)
+                    for (int k = 0; k < kT / 16; ++k)
+                        mma_ss(tmem + C::kColH + 64 * mb,
+                               sdesc_sw128(bb + 2 * mb * kBoxBytes + k * 2048, kBoxBytes, 1024),
+                               sdesc_sw128(wxb + k * 2048, kBoxBytes, 1024), id_mn, 1);
                 mma_commit(&s.sc_done);
-                // Yd = S x  (S carries D on its diagonal)
+                // Yd = S x  (S carries D on its diagonal); a single Yd buffer must first be
+                // read out by the previous epilogue
+                if (C::kYdBufs == 1 && t > 0 &&
+                    !wait_bar(ctl, &s.e_done[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status))
+                    break;
+                const uint32_t yd = tmem + C::kColYd + 64 * (C::kYdBufs == 2 ? st : 0);
                 for (int k = 0; k < kT / 16; ++k)
-                    mma_ts(tmem + kColYd + 64 * st, tmem + kColS + k * 8,
-                           sdesc_sw128(xb + k * 2048, kHalfBytes, 1024), id_pn, k > 0);
+                    mma_ts(yd, tmem + C::kColS + k * 8, sdesc_sw128(xb + k * 2048, kBoxBytes, 1024), id_pn, k > 0);
                 mma_commit(&s.yd_par[st]);
             }
         }
@@ -276,18 +327,19 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 #pragma unroll
             for (int pr = 0; pr < 4; ++pr)
                 if (pr > quarter && (pr & 1) == half) {
-                    tmem_st8(tmem + lane_base + kColS + 16 * pr, z);
-                    tmem_st8(tmem + lane_base + kColS + 16 * pr + 8, z);
+                    tmem_st8(tmem + lane_base + C::kColS + 16 * pr, z);
+                    tmem_st8(tmem + lane_base + C::kColS + 16 * pr + 8, z);
                 }
             tmem_st_wait();
         }
         float dt_next = 0.f;
         if (nt > 0 && j < len) dt_next = __bfloat162float(p.dt[(tok0 + j) * H + h]);
         for (int t = 0; t < nt; ++t) {
-            const int buf = t & 1;
+            const int buf = t & 1, bst = t % C::kBCStages;
             const int q = (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT);
             // E is done with tile t - 2, whose decay arrays share this parity
-            if (t >= 2 && !wait_role<1>(s, &s.e_done[buf], ((t - 2) >> 1) & 1, p.status, warp == 0, &s.p_flag)) break;
+            if (t >= 2 && !wait_role<1>(ctl, &s.e_done[buf], ((t - 2) >> 1) & 1, p.status, warp == 0, &ctl.p_flag))
+                break;
             // both warps of a quarter compute the scan; the first one publishes it
             float dj = 0.f, a = 0.f;
             if (j < q) {
@@ -315,29 +367,32 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             }
             mbar_arrive(&s.scan_done[buf]);
             p_bar();
-            if (!wait_role<1>(s, &s.cb_done, t & 1, p.status, warp == 0, &s.p_flag)) break;
+            if (!wait_role<1>(ctl, &s.cb_done, t & 1, p.status, warp == 0, &ctl.p_flag)) break;
             if (j >= q) {
                 // C B^T has read this tile's B: zero the rows past the sequence end
                 // so that B^T (w o x) sees exact zeros there (even for non-finite data)
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                for (int bx = half; bx < C::kBoxes; bx += 2)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(s.b[buf][half] + sw128_off(j, c)) = z;
+                    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(s.b[bst][bx] + sw128_off(j, c)) = z;
                 fence_proxy_async_smem();
             }
             // S of the previous tile has been consumed by its S x
-            if (t > 0 && !wait_role<1>(s, &s.yd_par[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status, warp == 0, &s.p_flag)) break;
+            if (t > 0 &&
+                !wait_role<1>(ctl, &s.yd_par[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status, warp == 0, &ctl.p_flag))
+                break;
             tc_fence_after();
             // S = C B^T o 2^(cs_j - cs_i) d_i for i <= j, plus D on the diagonal.  This warp
-            // handles the 32-column blocks pr <= quarter of its parity.  Blocks strictly
-            // below the diagonal use the rank-1 split; the block holding the diagonal uses
-            // the full exponential in every lane (exact there too), so no lane diverges.
+            // handles the 32-column blocks pr <= quarter of its parity, 16 columns at a time.
+            // Blocks strictly below the diagonal use the rank-1 split; the block holding the
+            // diagonal uses the full exponential in every lane (exact there too), so no lane
+            // diverges.
 #pragma unroll 1
             for (int b = 2 * half; b <= 2 * quarter + 1; b += (b & 1) ? 3 : 1) {
-                // 16-column block b (pairs pr = b / 2 of this warp's parity)
                 const int pr = b >> 1;
                 const int i0 = 16 * b;
                 uint32_t r[16];
-                tmem_ld16(tmem + lane_base + kColCB + i0, r);
+                tmem_ld16(tmem + lane_base + C::kColCB + i0, r);
                 float f[16];
                 if (pr < quarter) {
                     const float rf = ex2(cs2j - s.cs[buf][i0 + 15]);
@@ -368,7 +423,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                     if (i0 + k + 1 == j) v1 += Dh;
                     sv[k / 2] = pack_f16x2(v0, v1);
                 }
-                tmem_st8(tmem + lane_base + kColS + 8 * b, sv);
+                tmem_st8(tmem + lane_base + C::kColS + 8 * b, sv);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -380,52 +435,59 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
         const int j = 32 * quarter + lane;
         const int col0 = 32 * half;           // this warp's 32 of the 64 state / x / y columns
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-        const float* init_row = p.init_state ? p.init_state + (((int64_t)seq * H + h) * kN + j) * kP : nullptr;
+        const float* init_base = p.init_state ? p.init_state + ((int64_t)seq * H + h) * N * kP : nullptr;
         // Tile u's operands: fp16 copy of the state entering it (hs), the state in
         // TMEM pre-scaled by the tile's total decay (B^T (w o x) is then added by
-        // the MMA), x in fp16 and (w o x).
+        // the MMA), x in fp16 and (w o x).  State row n = 128 hb + j lives in TMEM
+        // block hb.
         auto prepare = [&](int u, bool first) -> bool {
             const int st = u & 1;
             const int qu = (int)(len - (int64_t)u * kT < kT ? len - (int64_t)u * kT : kT);
-            if (!wait_role<2>(s, &s.scan_done[st], (u >> 1) & 1, p.status, warp == 8, &s.e_flag)) return false;
+            if (!wait_role<2>(ctl, &s.scan_done[st], (u >> 1) & 1, p.status, warp == 8, &ctl.e_flag)) return false;
             const float cs2j = s.cs[st][j], dj = s.d[st][j], cs2_last = s.cs[st][qu - 1];
             const float e = ex2(cs2_last);
-            uint32_t hv[2][16];
-            if (first) {
+#pragma unroll 1
+            for (int hb = 0; hb < C::kHBlocks; ++hb) {
+                const int n = 128 * hb + j;
+                const uint32_t hcol = tmem + lane_base + C::kColH + 64 * hb + col0;
+                uint32_t hv[2][16];
+                if (first) {
+                    const float* src = init_base ? init_base + (int64_t)n * kP + col0 : nullptr;
 #pragma unroll
-                for (int m = 0; m < 2; ++m)
+                    for (int m = 0; m < 2; ++m)
 #pragma unroll
-                    for (int k = 0; k < 16; k += 4) {
-                        const float4 v = init_row ? *reinterpret_cast<const float4*>(init_row + col0 + 16 * m + k)
-                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-                        hv[m][k] = __float_as_uint(v.x); hv[m][k + 1] = __float_as_uint(v.y);
-                        hv[m][k + 2] = __float_as_uint(v.z); hv[m][k + 3] = __float_as_uint(v.w);
-                    }
-            } else {
-                tmem_ld16(tmem + lane_base + kColH + col0, hv[0]);
-                tmem_ld16(tmem + lane_base + kColH + col0 + 16, hv[1]);
-                tmem_ld_wait();
-            }
+                        for (int k = 0; k < 16; k += 4) {
+                            const float4 v = src ? *reinterpret_cast<const float4*>(src + 16 * m + k)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                            hv[m][k] = __float_as_uint(v.x); hv[m][k + 1] = __float_as_uint(v.y);
+                            hv[m][k + 2] = __float_as_uint(v.z); hv[m][k + 3] = __float_as_uint(v.w);
+                        }
+                } else {
+                    tmem_ld16(hcol, hv[0]);
+                    tmem_ld16(hcol + 16, hv[1]);
+                    tmem_ld_wait();
+                }
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                uint4 v0, v1;
-                v0.x = pack_f16x2(__uint_as_float(hv[m][0]), __uint_as_float(hv[m][1]));
-                v0.y = pack_f16x2(__uint_as_float(hv[m][2]), __uint_as_float(hv[m][3]));
-                v0.z = pack_f16x2(__uint_as_float(hv[m][4]), __uint_as_float(hv[m][5]));
-                v0.w = pack_f16x2(__uint_as_float(hv[m][6]), __uint_as_float(hv[m][7]));
-                v1.x = pack_f16x2(__uint_as_float(hv[m][8]), __uint_as_float(hv[m][9]));
-                v1.y = pack_f16x2(__uint_as_float(hv[m][10]), __uint_as_float(hv[m][11]));
-                v1.z = pack_f16x2(__uint_as_float(hv[m][12]), __uint_as_float(hv[m][13]));
-                v1.w = pack_f16x2(__uint_as_float(hv[m][14]), __uint_as_float(hv[m][15]));
-                const int c = col0 + 16 * m;
-                *reinterpret_cast<uint4*>(s.hs + sw128_off(j, c / 8)) = v0;
-                *reinterpret_cast<uint4*>(s.hs + sw128_off(j, c / 8 + 1)) = v1;
+                for (int m = 0; m < 2; ++m) {
+                    uint4 v0, v1;
+                    v0.x = pack_f16x2(__uint_as_float(hv[m][0]), __uint_as_float(hv[m][1]));
+                    v0.y = pack_f16x2(__uint_as_float(hv[m][2]), __uint_as_float(hv[m][3]));
+                    v0.z = pack_f16x2(__uint_as_float(hv[m][4]), __uint_as_float(hv[m][5]));
+                    v0.w = pack_f16x2(__uint_as_float(hv[m][6]), __uint_as_float(hv[m][7]));
+                    v1.x = pack_f16x2(__uint_as_float(hv[m][8]), __uint_as_float(hv[m][9]));
+                    v1.y = pack_f16x2(__uint_as_float(hv[m][10]), __uint_as_float(hv[m][11]));
+                    v1.z = pack_f16x2(__uint_as_float(hv[m][12]), __uint_as_float(hv[m][13]));
+                    v1.w = pack_f16x2(__uint_as_float(hv[m][14]), __uint_as_float(hv[m][15]));
+                    const int c = col0 + 16 * m;
+                    *reinterpret_cast<uint4*>(s.hs + sw128_off(n, c / 8)) = v0;
+                    *reinterpret_cast<uint4*>(s.hs + sw128_off(n, c / 8 + 1)) = v1;
 #pragma unroll
-                for (int k = 0; k < 16; ++k) hv[m][k] = __float_as_uint(e * __uint_as_float(hv[m][k]));
-                tmem_st16(tmem + lane_base + kColH + c, hv[m]);
+                    for (int k = 0; k < 16; ++k) hv[m][k] = __float_as_uint(e * __uint_as_float(hv[m][k]));
+                    tmem_st16(hcol + 16 * m, hv[m]);
+                }
             }
             tmem_st_wait();
-            if (!wait_role<2>(s, &s.full[st], (u >> 1) & 1, p.status, warp == 8, &s.e_flag)) return false;
+            if (!wait_role<2>(ctl, &s.xfull[st], (u >> 1) & 1, p.status, warp == 8, &ctl.e_flag)) return false;
             const __half2 w2 = __float2half2_rn(dj * ex2(cs2_last - cs2j));
             uint8_t* xt = s.x[st];
             uint4 v[4];
@@ -447,7 +509,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 wf.w = h2u(__hmul2(u2h(xf.w), w2));
                 const uint32_t off = sw128_off(j, col0 / 8 + m);
                 *reinterpret_cast<uint4*>(xt + off) = xf;
-                *reinterpret_cast<uint4*>(s.wx[st] + off) = wf;
+                *reinterpret_cast<uint4*>(s.wx + off) = wf;
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -459,9 +521,10 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
         bool ok = true;
         for (int k = 0; ok && k <= nt; ++k) {
             if (k < nt) {
-                // the state entering tile k is complete once B^T (w o x) of tile k - 1 has been added
+                // the state entering tile k is complete once B^T (w o x) of tile k - 1 has been
+                // added; that also frees hs and (w o x) for tile k
                 if (k > 0) {
-                    if (!(ok = wait_role<2>(s, &s.sc_done, (k - 1) & 1, p.status, warp == 8, &s.e_flag))) break;
+                    if (!(ok = wait_role<2>(ctl, &s.sc_done, (k - 1) & 1, p.status, warp == 8, &ctl.e_flag))) break;
                     tc_fence_after();
                 }
                 if (!(ok = prepare(k, k == 0))) break;
@@ -470,17 +533,19 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             const int t = k - 1, st = t & 1;
             const int q = (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT);
             // epilogue of tile t: y = Yd + 2^cs_j Yo   (D x is inside Yd)
-            if (!(ok = wait_role<2>(s, &s.yd_par[st], (t >> 1) & 1, p.status, warp == 8, &s.e_flag))) break;
+            if (!(ok = wait_role<2>(ctl, &s.yd_par[st], (t >> 1) & 1, p.status, warp == 8, &ctl.e_flag))) break;
             tc_fence_after();
             {
                 const float ej = ex2(s.cs[st][j]);
                 __nv_bfloat16* yrow = p.y + (tok0 + (int64_t)t * kT + j) * H * kP + (int64_t)h * kP;
+                const uint32_t yd = tmem + lane_base + C::kColYd + 64 * (C::kYdBufs == 2 ? st : 0);
+                const uint32_t yo = tmem + lane_base + C::kColYo + 64 * st;
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
                     const int c = col0 + 16 * m;
                     uint32_t rd[16], ro[16];
-                    tmem_ld16(tmem + lane_base + kColYd + 64 * st + c, rd);
-                    tmem_ld16(tmem + lane_base + kColYo + 64 * st + c, ro);
+                    tmem_ld16(yd + c, rd);
+                    tmem_ld16(yo + c, ro);
                     tmem_ld_wait();
                     uint32_t out[8];
 #pragma unroll
@@ -498,24 +563,29 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
         }
         // final state: H after the last tile's B^T (w o x) (or init_state for an empty sequence)
         if (p.final_state) {
-            float* dst = p.final_state + (((int64_t)seq * H + h) * kN + j) * kP;
-            if (nt == 0) {
+#pragma unroll 1
+            for (int hb = 0; hb < C::kHBlocks; ++hb) {
+                const int n = 128 * hb + j;
+                float* dst = p.final_state + (((int64_t)seq * H + h) * N + n) * kP + col0;
+                if (nt == 0) {
+                    const float* src = init_base ? init_base + (int64_t)n * kP + col0 : nullptr;
 #pragma unroll
-                for (int c = col0; c < col0 + 32; c += 4)
-                    *reinterpret_cast<float4*>(dst + c) =
-                        init_row ? *reinterpret_cast<const float4*>(init_row + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-            } else if (ok) {
-                tc_fence_after();
+                    for (int c = 0; c < 32; c += 4)
+                        *reinterpret_cast<float4*>(dst + c) =
+                            src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                } else if (ok) {
+                    tc_fence_after();
 #pragma unroll
-                for (int c = col0; c < col0 + 32; c += 16) {
-                    uint32_t hv[16];
-                    tmem_ld16(tmem + lane_base + kColH + c, hv);
-                    tmem_ld_wait();
+                    for (int c = 0; c < 32; c += 16) {
+                        uint32_t hv[16];
+                        tmem_ld16(tmem + lane_base + C::kColH + 64 * hb + col0 + c, hv);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int k = 0; k < 16; k += 4)
-                        *reinterpret_cast<float4*>(dst + c + k) =
-                            make_float4(__uint_as_float(hv[k]), __uint_as_float(hv[k + 1]),
-                                        __uint_as_float(hv[k + 2]), __uint_as_float(hv[k + 3]));
+                        for (int k = 0; k < 16; k += 4)
+                            *reinterpret_cast<float4*>(dst + c + k) =
+                                make_float4(__uint_as_float(hv[k]), __uint_as_float(hv[k + 1]),
+                                            __uint_as_float(hv[k + 2]), __uint_as_float(hv[k + 3]));
+                    }
                 }
             }
         }
@@ -573,7 +643,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType ty, const void* base, uint64_t
 }  // namespace
 
 bool tc_supported(const ScanArgs& a) {
-    return a.dtype == 1 && a.P == kP && a.N == kN && (a.Q == 128 || a.Q == 256) &&
+    return a.dtype == 1 && a.P == kP && (a.N == 128 || a.N == 256) && (a.Q == 128 || a.Q == 256) &&
            a.b * a.L < ((int64_t)1 << 31) && a.S * a.H < ((int64_t)1 << 31) && get_encode() != nullptr;
 }
 
@@ -610,10 +680,16 @@ int launch_tc_scan(const ScanArgs& a, const SeqInfo& si, int64_t, void* ws, int3
     p.status = status;
     p.H = (int)a.H;
     p.G = (int)a.G;
-    const size_t smem = sizeof(TcSmem) + 1024;
-    cudaFuncSetAttribute(k_tc_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     ProfScope ps(K_TC_SCAN, st);
-    k_tc_scan<<<(unsigned)(a.S * a.H), kThreads, smem, st>>>(tm_x, tm_b, tm_c, p);
+    if (a.N == 128) {
+        const size_t smem = sizeof(TcSmem<128>) + 1024;
+        cudaFuncSetAttribute(k_tc_scan<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_tc_scan<128><<<(unsigned)(a.S * a.H), kThreads, smem, st>>>(tm_x, tm_b, tm_c, p);
+    } else {
+        const size_t smem = sizeof(TcSmem<256>) + 1024;
+        cudaFuncSetAttribute(k_tc_scan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_tc_scan<256><<<(unsigned)(a.S * a.H), kThreads, smem, st>>>(tm_x, tm_b, tm_c, p);
+    }
     return 0;
 }
 

@@ -225,11 +225,13 @@ def test_prefill_then_decode_equals_longer_scan():
     assert_close(st, fr, 1e-2, "decode final state")
 
 
-def test_tensor_core_path_runs_for_bf16_p64_n128():
-    """bf16, P = 64, N = 128, chunk 128/256 calls launch the tcgen05 kernel (and
-    fp32 calls the CUDA-core kernels): no silent fallback between the two."""
+@pytest.mark.parametrize("dstate", [128, 256])
+def test_tensor_core_path_runs_for_bf16_p64(dstate):
+    """bf16, P = 64, N = 128 or 256, chunk 128/256 calls launch the tcgen05
+    kernel (and fp32 calls the CUDA-core kernels): no silent fallback between
+    the two."""
     from state_space_model_07_b200 import _lib
-    w = inputs.scaled(W["mamba2_2.7b_layer"], batch=1, seqlen=300, nheads=2)
+    w = inputs.scaled(W["mamba2_2.7b_layer"], batch=1, seqlen=300, nheads=2, dstate=dstate)
     d = inputs.make_inputs(w, "cuda")
     _lib.profile_read(reset=True)
     gpu_scan(d)
