@@ -596,6 +596,476 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Decoupled-state kernel (N = 128).
+//
+// The state recurrence leaves the tensor core's critical path: per tile the
+// MMA computes the tile's own state contribution s = B_w^T x (B_w = rows of B
+// scaled by w_i = d_i 2^(cs_last - cs_i)) into a fresh TMEM buffer, and the E
+// warps keep h in fp32 registers, h <- 2^cs_last h + s.  The output of a tile
+// is one accumulator, Y = C' h_prev + S x, with C' = rows of C scaled by
+// 2^cs_j, so the epilogue is a plain copy-out.  B_w and C' are made in place
+// in shared memory once C B^T has consumed B and C.
+//
+// Roles (608 threads):
+//   P   (warps 0-7):  C', B_w scaling; the causal mask S; the decay scan of
+//                     the next tile.  Two warps per TMEM lane quarter split
+//                     the 16-column blocks of a row by parity.
+//   E   (warps 8-15): x -> fp16 in place; h update and fp16 copy of it for
+//                     the next tile's C' h_prev; epilogue.  Two warps per
+//                     lane quarter split the 64 columns.
+//   W16 (lane 0):     TMA loads, two stages.
+//   W17 (lane 0):     s, C' h_prev and S x MMAs.
+//   W18 (lane 0):     C B^T MMAs (two TMEM buffers, so P can start tile t + 1
+//                     while S x of tile t is still waiting).
+// Every per-tile barrier exists per tile parity, and every barrier's next
+// phase (tile t + 2) depends on an action its waiters take after waiting for
+// tile t, so no waiter can see a barrier two phases ahead.
+namespace v2 {
+
+constexpr int kThreads2 = 608;
+constexpr int kRoleWarps = 8;       // P and E arrive once per warp
+
+// One arrival per warp: the warp's lanes synchronise first (ordering their
+// shared-memory and TMEM writes before the release of the arrival), so the
+// barrier counts warps, not threads.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+constexpr uint32_t kColCB = 0;      // two 128-column fp32 buffers
+constexpr uint32_t kColS = 256;     // S, fp16 pairs (64 columns)
+constexpr uint32_t kColSt = 320;    // s, fp32 128 x 64
+constexpr uint32_t kColY = 384;     // two 64-column fp32 buffers
+
+struct __align__(1024) Smem {
+    uint8_t x[2][kTileBytesX];        // x (bf16 from TMA, fp16 after conversion)
+    uint8_t b[2][2][kBoxBytes];       // B -> B_w (fp16), two 64-column boxes per stage
+    uint8_t c[2][2][kBoxBytes];       // C -> C' (fp16)
+    uint8_t hs[2][kTileBytesX];       // state entering tile t (fp16), buffer t & 1
+    float cs[2][kT];                  // tile-local cumulative decay (base-2 exponent)
+    float d[2][kT];
+    float colfac[2][kT];              // 2^(cs_m - cs_i) d_i, pivot m = last token of i's 16-block
+    float wtot[2][2][4];
+    uint64_t xfull[2], bcfull[2];     // TMA -> E, W18
+    uint64_t cb_full[2];              // W18 commit -> P
+    uint64_t cb_free[2];              // P -> W18
+    uint64_t bc_ready[2];             // P (B_w, C' written) -> W17
+    uint64_t s_ready[2];              // P (S in TMEM) -> W17
+    uint64_t scan_done[2];            // P -> E
+    uint64_t x_ready[2];              // E -> W17
+    uint64_t hs_ready[2];             // E -> W17
+    uint64_t e_done[2];               // E (Y read) -> W17
+    uint64_t s_done[2];               // W17 commit -> E
+    uint64_t y_full[2];               // W17 commit -> E, P, W16
+    uint64_t fin[2];                  // W17, W18: own MMAs drained before exit
+    uint32_t tmem_base;
+    TcCtl ctl;
+};
+
+__global__ void __launch_bounds__(kThreads2, 1)
+k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+           const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
+    constexpr int N = 128;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    TcCtl& ctl = s.ctl;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.H, G = p.G;
+    const int h = blockIdx.x % H;
+    const int seq = blockIdx.x / H;
+    const int g = h / (H / G);
+
+    int64_t row, t0, t1;
+    seq_span(p.si, seq, row, t0, t1);
+    const int64_t len = t1 > t0 ? t1 - t0 : 0;
+    const int nt = (int)((len + kT - 1) / kT);
+    const int64_t tok0 = row * p.si.L + t0;
+    auto tile_len = [&](int t) { return (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT); };
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.xfull[i], 1);
+            mbar_init(&s.bcfull[i], 1);
+            mbar_init(&s.cb_full[i], 1);
+            mbar_init(&s.cb_free[i], kRoleWarps);
+            mbar_init(&s.bc_ready[i], kRoleWarps);
+            mbar_init(&s.s_ready[i], kRoleWarps);
+            mbar_init(&s.scan_done[i], kRoleWarps);
+            mbar_init(&s.x_ready[i], kRoleWarps);
+            mbar_init(&s.hs_ready[i], kRoleWarps);
+            mbar_init(&s.e_done[i], kRoleWarps);
+            mbar_init(&s.s_done[i], 1);
+            mbar_init(&s.y_full[i], 1);
+            mbar_init(&s.fin[i], 1);
+        }
+        ctl.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(&s.tmem_base, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+    const float kLog2e = 1.4426950408889634f;
+
+    if (warp == 16) {
+        // ------------------------------------------------------------ W16: TMA
+        if (lane == 0 && nt > 0) {
+            tma_prefetch_desc(&tm_x);
+            tma_prefetch_desc(&tm_b);
+            tma_prefetch_desc(&tm_c);
+            int issued = 0;
+            for (int u = 0; u < nt; ++u) {
+                const int st = u & 1;
+                // stage st is free once every MMA of tile u - 2 has completed
+                if (u >= 2 && !wait_bar(ctl, &s.y_full[st], ((u - 2) >> 1) & 1, p.status)) break;
+                const int tok = (int)(tok0 + (int64_t)u * kT);
+                mbar_expect_tx(&s.xfull[st], kTileBytesX);
+                tma_load_3d(s.x[st], &tm_x, &s.xfull[st], 0, h, tok);
+                mbar_expect_tx(&s.bcfull[st], 4 * kBoxBytes);
+                for (int k = 0; k < 2; ++k) {
+                    tma_load_3d(s.b[st][k], &tm_b, &s.bcfull[st], 64 * k, g, tok);
+                    tma_load_3d(s.c[st][k], &tm_c, &s.bcfull[st], 64 * k, g, tok);
+                }
+                ++issued;
+            }
+            if (*(volatile int*)&ctl.abort) {
+                // let the copies already in flight land before the CTA exits
+                for (int u = 0; u < issued; ++u) {
+                    mbar_wait(&s.xfull[u & 1], (u >> 1) & 1, 400000000ll);
+                    mbar_wait(&s.bcfull[u & 1], (u >> 1) & 1, 400000000ll);
+                }
+            }
+        }
+    } else if (warp == 18) {
+        // -------------------------------------------------------- W18: C B^T
+        if (lane == 0 && nt > 0) {
+            const uint32_t id_cb = idesc_f16(128, 128, 0, 0);
+            for (int t = 0; t < nt; ++t) {
+                const int st = t & 1;
+                if (!wait_bar(ctl, &s.bcfull[st], (t >> 1) & 1, p.status)) break;
+                // P has read C B^T of tile t - 2 out of this buffer
+                if (t >= 2 && !wait_bar(ctl, &s.cb_free[st], ((t - 2) >> 1) & 1, p.status)) break;
+                tc_fence_after();
+                const uint32_t cb = smem_u32(s.c[st][0]), bb = smem_u32(s.b[st][0]);
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
+                    mma_ss(tmem + kColCB + 128 * st, sdesc_sw128(cb + off, 16, 1024),
+                           sdesc_sw128(bb + off, 16, 1024), id_cb, k > 0);
+                }
+                mma_commit(&s.cb_full[st]);
+            }
+            mma_commit(&s.fin[0]);
+            mbar_wait(&s.fin[0], 0, 400000000ll);
+        }
+    } else if (warp == 17) {
+        // ------------------------------------------- W17: s, C' h_prev, S x
+        if (lane == 0 && nt > 0) {
+            const uint32_t id_st = idesc_f16(128, 64, 1, 1);   // MN-major A (B_w^T) and B (x)
+            const uint32_t id_y = idesc_f16(128, 64, 0, 1);    // K-major A, MN-major B
+            for (int t = 0; t < nt; ++t) {
+                const int st = t & 1;
+                const uint32_t par = (t >> 1) & 1;
+                const uint32_t bb = smem_u32(s.b[st][0]), cb = smem_u32(s.c[st][0]);
+                const uint32_t xb = smem_u32(s.x[st]), hsb = smem_u32(s.hs[st]);
+                // s = B_w^T x  (state rows 0..127 = TMEM lanes)
+                if (!wait_bar(ctl, &s.x_ready[st], par, p.status)) break;
+                if (!wait_bar(ctl, &s.bc_ready[st], par, p.status)) break;
+                tc_fence_after();
+                for (int k = 0; k < kT / 16; ++k)
+                    mma_ss(tmem + kColSt, sdesc_sw128(bb + k * 2048, kBoxBytes, 1024),
+                           sdesc_sw128(xb + k * 2048, kBoxBytes, 1024), id_st, k > 0);
+                mma_commit(&s.s_done[st]);
+                // Y = C' h_prev: needs the state entering tile t and a free Y buffer
+                if (!wait_bar(ctl, &s.hs_ready[st], par, p.status)) break;
+                if (t >= 2 && !wait_bar(ctl, &s.e_done[st], ((t - 2) >> 1) & 1, p.status)) break;
+                tc_fence_after();
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
+                    mma_ss(tmem + kColY + 64 * st, sdesc_sw128(cb + off, 16, 1024),
+                           sdesc_sw128(hsb + k * 2048, kBoxBytes, 1024), id_y, k > 0);
+                }
+                // Y += S x
+                if (!wait_bar(ctl, &s.s_ready[st], par, p.status)) break;
+                tc_fence_after();
+                for (int k = 0; k < kT / 16; ++k)
+                    mma_ts(tmem + kColY + 64 * st, tmem + kColS + k * 8,
+                           sdesc_sw128(xb + k * 2048, kBoxBytes, 1024), id_y, 1);
+                mma_commit(&s.y_full[st]);
+            }
+            mma_commit(&s.fin[1]);
+            mbar_wait(&s.fin[1], 0, 400000000ll);
+        }
+    } else if (warp < 8) {
+        // ------------------------------- P: scaling, decay mask, decay scan
+        const int quarter = warp & 3, half = warp >> 2;
+        const int j = 32 * quarter + lane;
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        const bool leader = warp == 4;
+        const float A2 = p.A[h] * kLog2e;
+        const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+        const float Dh = p.D ? p.D[h] : 0.f;
+        // S blocks right of this quarter's diagonal stay zero: write them once.
+        {
+            const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            for (int b = 2 * quarter + 2 + half; b < 8; b += 2) tmem_st8(tmem + lane_base + kColS + 8 * b, z);
+            tmem_st_wait();
+        }
+        // decay scan of tile u into the arrays of parity u & 1
+        float dt_next = 0.f;
+        auto scan = [&](int u) {
+            const int buf = u & 1, qu = tile_len(u);
+            float dj = 0.f, a = 0.f;
+            if (j < qu) {
+                dj = softplus_f(dt_next + bias);
+                a = dj * A2;
+            }
+            if ((int64_t)(u + 1) * kT + j < len) dt_next = __bfloat162float(p.dt[(tok0 + (int64_t)(u + 1) * kT + j) * H + h]);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, a, o);
+                if (lane >= o) a += v;
+            }
+            if (lane == 31) s.wtot[buf][half][quarter] = a;
+            p_bar();
+            for (int w = 0; w < quarter; ++w) a += s.wtot[buf][half][w];
+            const float cs_pivot = __shfl_sync(0xffffffffu, a, lane | 15);
+            if (half == 0) {
+                s.cs[buf][j] = a;
+                s.d[buf][j] = dj;
+                s.colfac[buf][j] = ex2(cs_pivot - a) * dj;
+            }
+            warp_arrive(&s.scan_done[buf]);
+        };
+        if (nt > 0) {
+            if (j < len) dt_next = __bfloat162float(p.dt[(tok0 + j) * H + h]);
+            scan(0);
+        }
+        for (int t = 0; t < nt; ++t) {
+            const int st = t & 1;
+            const uint32_t par = (t >> 1) & 1;
+            const int q = tile_len(t);
+            if (!wait_role<1>(ctl, &s.cb_full[st], par, p.status, leader, &ctl.p_flag)) break;
+            tc_fence_after();
+            const float cs2j = s.cs[st][j];
+            {
+                // C'_j = 2^cs_j C_j, B_w_j = d_j 2^(cs_last - cs_j) B_j (zero past the sequence end);
+                // this warp takes the 64-column box `half` of row j
+                const float cs_last = s.cs[st][q - 1];
+                const __half2 e2 = __float2half2_rn(ex2(cs2j));
+                const __half2 w2 = __float2half2_rn(s.d[st][j] * ex2(cs_last - cs2j));
+                uint8_t* brow = s.b[st][half];
+                uint8_t* crow = s.c[st][half];
+                // four 16-byte chunks of B and of C at a time: all loads before the stores
+#pragma unroll
+                for (int c0 = 0; c0 < 8; c0 += 4) {
+                    uint4 vb[4], vc[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        vb[c] = *reinterpret_cast<const uint4*>(brow + sw128_off(j, c0 + c));
+                        vc[c] = *reinterpret_cast<const uint4*>(crow + sw128_off(j, c0 + c));
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        vb[c].x = h2u(__hmul2(u2h(vb[c].x), w2)); vb[c].y = h2u(__hmul2(u2h(vb[c].y), w2));
+                        vb[c].z = h2u(__hmul2(u2h(vb[c].z), w2)); vb[c].w = h2u(__hmul2(u2h(vb[c].w), w2));
+                        vc[c].x = h2u(__hmul2(u2h(vc[c].x), e2)); vc[c].y = h2u(__hmul2(u2h(vc[c].y), e2));
+                        vc[c].z = h2u(__hmul2(u2h(vc[c].z), e2)); vc[c].w = h2u(__hmul2(u2h(vc[c].w), e2));
+                        if (j >= q) vb[c] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        *reinterpret_cast<uint4*>(brow + sw128_off(j, c0 + c)) = vb[c];
+                        *reinterpret_cast<uint4*>(crow + sw128_off(j, c0 + c)) = vc[c];
+                    }
+                }
+                fence_proxy_async_smem();
+                warp_arrive(&s.bc_ready[st]);
+            }
+            // S = C B^T o 2^(cs_j - cs_i) d_i (i <= j), D on the diagonal.  This warp takes the
+            // 16-column blocks b = 2m + half: m < quarter lie left of the diagonal 32-block
+            // (rank-1 split, one exponential per block), m = quarter holds the diagonal (one
+            // exponential per element, masked with a select).  All held in registers until
+            // the S buffer is free.
+            uint32_t sv[4][8];
+            const uint32_t cbuf = tmem + lane_base + kColCB + 128 * st;
+#pragma unroll
+            for (int m = 0; m < 3; ++m) {
+                if (m < quarter) {
+                    const int i0 = 16 * (2 * m + half);
+                    uint32_t r[16];
+                    tmem_ld16(cbuf + i0, r);
+                    const float rf = ex2(cs2j - s.cs[st][i0 + 15]);
+                    float f[16];
+#pragma unroll
+                    for (int k = 0; k < 16; k += 4) {
+                        const float4 cf = *reinterpret_cast<const float4*>(&s.colfac[st][i0 + k]);
+                        f[k] = cf.x * rf; f[k + 1] = cf.y * rf; f[k + 2] = cf.z * rf; f[k + 3] = cf.w * rf;
+                    }
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int k = 0; k < 16; k += 2)
+                        sv[m][k / 2] = pack_f16x2(__uint_as_float(r[k]) * f[k], __uint_as_float(r[k + 1]) * f[k + 1]);
+                }
+            }
+            {
+                const int i0 = 16 * (2 * quarter + half);
+                uint32_t r[16];
+                tmem_ld16(cbuf + i0, r);
+                float f[16];
+#pragma unroll
+                for (int k = 0; k < 16; k += 4) {
+                    const float4 cv = *reinterpret_cast<const float4*>(&s.cs[st][i0 + k]);
+                    const float4 dv = *reinterpret_cast<const float4*>(&s.d[st][i0 + k]);
+                    f[k] = ex2(cs2j - cv.x) * dv.x;
+                    f[k + 1] = ex2(cs2j - cv.y) * dv.y;
+                    f[k + 2] = ex2(cs2j - cv.z) * dv.z;
+                    f[k + 3] = ex2(cs2j - cv.w) * dv.w;
+                }
+                tmem_ld_wait();
+#pragma unroll
+                for (int k = 0; k < 16; k += 2) {
+                    float v0 = i0 + k <= j ? __uint_as_float(r[k]) * f[k] : 0.f;
+                    float v1 = i0 + k + 1 <= j ? __uint_as_float(r[k + 1]) * f[k + 1] : 0.f;
+                    if (i0 + k == j) v0 += Dh;
+                    if (i0 + k + 1 == j) v1 += Dh;
+                    sv[3][k / 2] = pack_f16x2(v0, v1);
+                }
+            }
+            tc_fence_before();
+            warp_arrive(&s.cb_free[st]);
+            // the S buffer is free once S x of tile t - 1 has completed
+            if (t > 0 && !wait_role<1>(ctl, &s.y_full[st ^ 1], ((t - 1) >> 1) & 1, p.status, leader, &ctl.p_flag))
+                break;
+            tc_fence_after();
+#pragma unroll
+            for (int m = 0; m < 3; ++m)
+                if (m < quarter) tmem_st8(tmem + lane_base + kColS + 8 * (2 * m + half), sv[m]);
+            tmem_st8(tmem + lane_base + kColS + 8 * (2 * quarter + half), sv[3]);
+            tmem_st_wait();
+            tc_fence_before();
+            warp_arrive(&s.s_ready[st]);
+            if (t + 1 < nt) scan(t + 1);
+        }
+    } else if (warp < 16) {
+        // ------------------------------------ E: x to fp16, state, epilogue
+        const int quarter = warp & 3, half = (warp >> 2) & 1;
+        const int j = 32 * quarter + lane;     // token row (x, y) and state row (s, h)
+        const int col0 = 32 * half;
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        const bool leader = warp == 8;
+        float hreg[32];
+        {
+            const float* src = p.init_state ? p.init_state + (((int64_t)seq * H + h) * N + j) * kP + col0 : nullptr;
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+                const float4 v = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                hreg[c] = v.x; hreg[c + 1] = v.y; hreg[c + 2] = v.z; hreg[c + 3] = v.w;
+            }
+        }
+        // fp16 copy of the state entering tile u, into hs[u & 1]
+        auto put_state = [&](int u) {
+            uint8_t* hsu = s.hs[u & 1];
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+                uint4 v;
+                v.x = pack_f16x2(hreg[c], hreg[c + 1]);
+                v.y = pack_f16x2(hreg[c + 2], hreg[c + 3]);
+                v.z = pack_f16x2(hreg[c + 4], hreg[c + 5]);
+                v.w = pack_f16x2(hreg[c + 6], hreg[c + 7]);
+                *reinterpret_cast<uint4*>(hsu + sw128_off(j, (col0 + c) / 8)) = v;
+            }
+            fence_proxy_async_smem();
+            warp_arrive(&s.hs_ready[u & 1]);
+        };
+        if (nt > 0) put_state(0);
+        float e_state = 1.f;   // 2^cs_last of the tile whose s is pending
+        bool ok = true;
+        for (int k = 0; ok && k <= nt; ++k) {
+            if (k >= 1) {
+                // h <- 2^cs_last h + s for tile k - 1
+                const int u = k - 1;
+                if (!(ok = wait_role<2>(ctl, &s.s_done[u & 1], (u >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                tc_fence_after();
+                {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16(tmem + lane_base + kColSt + col0, r0);
+                    tmem_ld16(tmem + lane_base + kColSt + col0 + 16, r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        hreg[i] = fmaf(e_state, hreg[i], __uint_as_float(r0[i]));
+                        hreg[16 + i] = fmaf(e_state, hreg[16 + i], __uint_as_float(r1[i]));
+                    }
+                }
+                tc_fence_before();
+                if (k < nt) put_state(k);
+            }
+            if (k < nt) {
+                // x of tile k to fp16 in place (zero past the sequence end)
+                if (!(ok = wait_role<2>(ctl, &s.scan_done[k & 1], (k >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                const int q = tile_len(k);
+                e_state = ex2(s.cs[k & 1][q - 1]);
+                if (!(ok = wait_role<2>(ctl, &s.xfull[k & 1], (k >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                uint8_t* xt = s.x[k & 1];
+                uint4 v[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) v[m] = *reinterpret_cast<const uint4*>(xt + sw128_off(j, col0 / 8 + m));
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    uint4 o;
+                    o.x = pack_f16x2(bf16lo(v[m].x), bf16hi(v[m].x));
+                    o.y = pack_f16x2(bf16lo(v[m].y), bf16hi(v[m].y));
+                    o.z = pack_f16x2(bf16lo(v[m].z), bf16hi(v[m].z));
+                    o.w = pack_f16x2(bf16lo(v[m].w), bf16hi(v[m].w));
+                    if (j >= q) o = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(xt + sw128_off(j, col0 / 8 + m)) = o;
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                warp_arrive(&s.x_ready[k & 1]);
+            }
+            if (k >= 1) {
+                // epilogue of tile k - 1: y = Y
+                const int u = k - 1, q = tile_len(u);
+                if (!(ok = wait_role<2>(ctl, &s.y_full[u & 1], (u >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                tc_fence_after();
+                __nv_bfloat16* yrow = p.y + (tok0 + (int64_t)u * kT + j) * H * kP + (int64_t)h * kP + col0;
+                {
+                    uint32_t r[32];
+                    tmem_ld16(tmem + lane_base + kColY + 64 * (u & 1) + col0, *reinterpret_cast<uint32_t(*)[16]>(r));
+                    tmem_ld16(tmem + lane_base + kColY + 64 * (u & 1) + col0 + 16,
+                              *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+                    tmem_ld_wait();
+                    uint32_t o[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                    if (j < q) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4*>(yrow + 8 * c) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                    }
+                }
+                tc_fence_before();
+                warp_arrive(&s.e_done[u & 1]);
+            }
+        }
+        if (p.final_state && (ok || nt == 0)) {
+            float* dst = p.final_state + (((int64_t)seq * H + h) * N + j) * kP + col0;
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+                *reinterpret_cast<float4*>(dst + c) = make_float4(hreg[c], hreg[c + 1], hreg[c + 2], hreg[c + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace v2
+
 // bf16 -> fp16 copies of B and C (8 elements per thread step).
 __global__ void k_tc_prep(const uint4* __restrict__ b, const uint4* __restrict__ c, uint4* __restrict__ b16,
                           uint4* __restrict__ c16, int64_t n8) {
@@ -682,9 +1152,9 @@ int launch_tc_scan(const ScanArgs& a, const SeqInfo& si, int64_t, void* ws, int3
     p.G = (int)a.G;
     ProfScope ps(K_TC_SCAN, st);
     if (a.N == 128) {
-        const size_t smem = sizeof(TcSmem<128>) + 1024;
-        cudaFuncSetAttribute(k_tc_scan<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_tc_scan<128><<<(unsigned)(a.S * a.H), kThreads, smem, st>>>(tm_x, tm_b, tm_c, p);
+        const size_t smem = sizeof(v2::Smem) + 1024;
+        cudaFuncSetAttribute(v2::k_tc_scan2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        v2::k_tc_scan2<<<(unsigned)(a.S * a.H), v2::kThreads2, smem, st>>>(tm_x, tm_b, tm_c, p);
     } else {
         const size_t smem = sizeof(TcSmem<256>) + 1024;
         cudaFuncSetAttribute(k_tc_scan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
