@@ -599,32 +599,74 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 // ---------------------------------------------------------------------------
 // Decoupled-state kernel (N = 128).
 //
-// The state recurrence leaves the tensor core's critical path: per tile the
-// MMA computes the tile's own state contribution s = B_w^T x (B_w = rows of B
-// scaled by w_i = d_i 2^(cs_last - cs_i)) into a fresh TMEM buffer, and the E
-// warps keep h in fp32 registers, h <- 2^cs_last h + s.  The output of a tile
-// is one accumulator, Y = C' h_prev + S x, with C' = rows of C scaled by
-// 2^cs_j, so the epilogue is a plain copy-out.  B_w and C' are made in place
-// in shared memory once C B^T has consumed B and C.
+// Shared-memory bandwidth (128 B per clock per SM, shared by TMA writes, the
+// MMAs' operand reads and the threads) is what bounds this kernel, so the
+// design keeps bytes out of shared memory:
+//   * C goes to TMEM once (tcgen05.cp); C B^T and C' h_prev take A from TMEM.
+//     C' = rows of C scaled by 2^cs_j is made in place in TMEM, so the output
+//     of a tile is one accumulator Y = C' h_prev + S x.
+//   * x arrives by TMA and is converted in place to fp16; the E warps also
+//     write w o x once.
+//   * The state recurrence runs on the E warps in fp32 registers,
+//     h <- 2^cs_last h + s, with s = B^T (w o x) the tile's own contribution
+//     from the tensor core; only an fp16 copy of h goes to shared memory.
+// Per 128-token tile that is ~290 KB of shared-memory traffic.
 //
-// Roles (608 threads):
-//   P   (warps 0-7):  C', B_w scaling; the causal mask S; the decay scan of
-//                     the next tile.  Two warps per TMEM lane quarter split
-//                     the 16-column blocks of a row by parity.
-//   E   (warps 8-15): x -> fp16 in place; h update and fp16 copy of it for
-//                     the next tile's C' h_prev; epilogue.  Two warps per
-//                     lane quarter split the 64 columns.
-//   W16 (lane 0):     TMA loads, two stages.
+// No role thread keeps a global load in flight across an mbarrier arrival
+// (an arrival is a release, which waits for the thread's outstanding loads):
+// global inputs come in through TMA or through the dt warp, whose own waits
+// are off the critical path.
+//
+// Roles (640 threads):
+//   P   (warps 0-7):  C' scaling, the causal mask S, the decay scan of the
+//                     next tile.  Two warps per TMEM lane quarter split the
+//                     16-column blocks of a row by parity.
+//   E   (warps 8-15): x -> fp16 operands, the state update, the epilogue.
+//                     Two warps per lane quarter split the 64 columns.
+//   W16 (lane 0):     TMA loads of x, B and C, two stages.
 //   W17 (lane 0):     s, C' h_prev and S x MMAs.
-//   W18 (lane 0):     C B^T MMAs (two TMEM buffers, so P can start tile t + 1
-//                     while S x of tile t is still waiting).
+//   W18 (lane 0):     C -> TMEM copies and the C B^T MMAs.
+//   W19:              dt of the coming tiles into a four-tile shared ring.
 // Every per-tile barrier exists per tile parity, and every barrier's next
 // phase (tile t + 2) depends on an action its waiters take after waiting for
 // tile t, so no waiter can see a barrier two phases ahead.
-namespace v2 {
+namespace v3 {
 
-constexpr int kThreads2 = 608;
+constexpr int kThreads3 = 640;
+
+// Per-tile event timestamps of CTA 0, compiled in only with -DSSD_TC_TRACE
+// (performance analysis builds); a no-op otherwise.
+#ifdef SSD_TC_TRACE
+__device__ long long g_tc_trace[48][1024];
+#define TC_TRACE(ev, t) \
+    do { if (blockIdx.x == 0 && (t) >= 0 && (t) < 1024) g_tc_trace[ev][t] = clock64(); } while (0)
+#else
+#define TC_TRACE(ev, t) do { } while (0)
+#endif
 constexpr int kRoleWarps = 8;       // P and E arrive once per warp
+constexpr uint32_t kColC = 0;       // two 64-column buffers: C, then C' (fp16 pairs)
+constexpr uint32_t kColCB = 128;    // C B^T, fp32 128 x 128
+constexpr uint32_t kColS = 256;     // S, fp16 pairs (64 columns)
+constexpr uint32_t kColSt = 320;    // s, fp32 128 x 64
+constexpr uint32_t kColY = 384;     // two 64-column fp32 buffers
+
+// softplus(z) = max(z, 0) + log(1 + e), e = exp(-|z|) in (0, 1], with the
+// hardware base-2 exponential and logarithm; for e < 2^-7 the logarithm is
+// replaced by its Taylor series e - e^2/2 + e^3/3 (truncation < e^4/4 < 2^-30,
+// and no cancellation in 1 + e).  Relative error ~1e-6, which the decay and
+// the update d B x^T pass through unamplified.
+__device__ __forceinline__ float softplus_fast(float z) {
+    const float e = ex2(-fabsf(z) * 1.4426950408889634f);
+    float l;
+    if (e < 0.0078125f) {
+        l = e * fmaf(e, fmaf(e, 0.333333343f, -0.5f), 1.f);
+    } else {
+        float lg;
+        asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(1.f + e));
+        l = lg * 0.693147182f;
+    }
+    return fmaxf(z, 0.f) + l;
+}
 
 // One arrival per warp: the warp's lanes synchronise first (ordering their
 // shared-memory and TMEM writes before the release of the arrival), so the
@@ -633,38 +675,38 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
-constexpr uint32_t kColCB = 0;      // two 128-column fp32 buffers
-constexpr uint32_t kColS = 256;     // S, fp16 pairs (64 columns)
-constexpr uint32_t kColSt = 320;    // s, fp32 128 x 64
-constexpr uint32_t kColY = 384;     // two 64-column fp32 buffers
 
 struct __align__(1024) Smem {
-    uint8_t x[2][kTileBytesX];        // x (bf16 from TMA, fp16 after conversion)
-    uint8_t b[2][2][kBoxBytes];       // B -> B_w (fp16), two 64-column boxes per stage
-    uint8_t c[2][2][kBoxBytes];       // C -> C' (fp16)
+    uint8_t b[2][2][kBoxBytes];       // B (fp16), two 64-column boxes per stage
+    uint8_t c[2][2][kBoxBytes];       // C (fp16)
+    uint8_t x[2][kTileBytesX];        // x (bf16 from TMA, fp16 after conversion), per stage
+    uint8_t wx[kTileBytesX];          // w o x (fp16)
     uint8_t hs[2][kTileBytesX];       // state entering tile t (fp16), buffer t & 1
     float cs[2][kT];                  // tile-local cumulative decay (base-2 exponent)
     float d[2][kT];
     float colfac[2][kT];              // 2^(cs_m - cs_i) d_i, pivot m = last token of i's 16-block
     float wtot[2][2][4];
-    uint64_t xfull[2], bcfull[2];     // TMA -> E, W18
-    uint64_t cb_full[2];              // W18 commit -> P
-    uint64_t cb_free[2];              // P -> W18
-    uint64_t bc_ready[2];             // P (B_w, C' written) -> W17
+    float dts[4][kT];                 // raw dt of tile u in slot u & 3
+    uint64_t full[2];                 // TMA x, B, C -> W18, W17, E
+    uint64_t dt_full[4];              // W19 -> P
+    uint64_t dt_free[4];              // P -> W19
+    uint64_t cb_full[2];              // W18 commit (C in TMEM, C B^T) -> P
+    uint64_t cb_free[2];              // P (C B^T read) -> W18
+    uint64_t c_scaled[2];             // P (C' in TMEM) -> W17
     uint64_t s_ready[2];              // P (S in TMEM) -> W17
     uint64_t scan_done[2];            // P -> E
-    uint64_t x_ready[2];              // E -> W17
+    uint64_t x_ready[2];              // E (x, w o x written) -> W17
     uint64_t hs_ready[2];             // E -> W17
     uint64_t e_done[2];               // E (Y read) -> W17
     uint64_t s_done[2];               // W17 commit -> E
-    uint64_t y_full[2];               // W17 commit -> E, P, W16
-    uint64_t fin[2];                  // W17, W18: own MMAs drained before exit
+    uint64_t y_full[2];               // W17 commit -> E, P, W16, W18
+    uint64_t fin[2];                  // W17, W18: own tcgen05 work drained before exit
     uint32_t tmem_base;
     TcCtl ctl;
 };
 
-__global__ void __launch_bounds__(kThreads2, 1)
-k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+__global__ void __launch_bounds__(kThreads3, 1)
+k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
            const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
     constexpr int N = 128;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -684,12 +726,15 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     auto tile_len = [&](int t) { return (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT); };
 
     if (tid == 0) {
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&s.dt_full[i], 1);
+            mbar_init(&s.dt_free[i], kRoleWarps);
+        }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.xfull[i], 1);
-            mbar_init(&s.bcfull[i], 1);
+            mbar_init(&s.full[i], 1);
             mbar_init(&s.cb_full[i], 1);
             mbar_init(&s.cb_free[i], kRoleWarps);
-            mbar_init(&s.bc_ready[i], kRoleWarps);
+            mbar_init(&s.c_scaled[i], kRoleWarps);
             mbar_init(&s.s_ready[i], kRoleWarps);
             mbar_init(&s.scan_done[i], kRoleWarps);
             mbar_init(&s.x_ready[i], kRoleWarps);
@@ -709,8 +754,37 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     const uint32_t tmem = s.tmem_base;
     const float kLog2e = 1.4426950408889634f;
 
-    if (warp == 16) {
-        // ------------------------------------------------------------ W16: TMA
+#ifdef SSD_TC_TRACE
+    if (warp == 16 && lane == 1) {
+        // observer: timestamps of MMA completions
+        if (blockIdx.x == 0) {
+            int tc = 0, ts = 0, ty = 0;
+            const long long t_start = clock64();
+            while ((tc < nt || ts < nt || ty < nt) && clock64() - t_start < 2000000000ll) {
+                if (tc < nt && mbar_test_wait(&s.cb_full[tc & 1], (tc >> 1) & 1)) { TC_TRACE(25, tc); ++tc; }
+                if (ts < nt && mbar_test_wait(&s.s_done[ts & 1], (ts >> 1) & 1)) { TC_TRACE(26, ts); ++ts; }
+                if (ty < nt && mbar_test_wait(&s.y_full[ty & 1], (ty >> 1) & 1)) { TC_TRACE(27, ty); ++ty; }
+            }
+        }
+    } else
+#endif
+    if (warp == 19) {
+        // ------------------------------------------- W19: dt into the shared ring
+        for (int u = 0; u < nt; ++u) {
+            const int sl = u & 3;
+            // P has read slot sl for tile u - 4
+            if (u >= 4 && !wait_bar_w(ctl, &s.dt_free[sl], ((u - 4) >> 2) & 1, p.status)) break;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = 32 * i + lane;
+                s.dts[sl][r] = (int64_t)u * kT + r < len
+                                   ? __bfloat162float(p.dt[(tok0 + (int64_t)u * kT + r) * H + h]) : 0.f;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.dt_full[sl]);
+        }
+    } else if (warp == 16) {
+        // ------------------------------------------------- W16: TMA x, B, C
         if (lane == 0 && nt > 0) {
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
@@ -721,84 +795,98 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 // stage st is free once every MMA of tile u - 2 has completed
                 if (u >= 2 && !wait_bar(ctl, &s.y_full[st], ((u - 2) >> 1) & 1, p.status)) break;
                 const int tok = (int)(tok0 + (int64_t)u * kT);
-                mbar_expect_tx(&s.xfull[st], kTileBytesX);
-                tma_load_3d(s.x[st], &tm_x, &s.xfull[st], 0, h, tok);
-                mbar_expect_tx(&s.bcfull[st], 4 * kBoxBytes);
+                mbar_expect_tx(&s.full[st], kTileBytesX + 4 * kBoxBytes);
+                tma_load_3d(s.x[st], &tm_x, &s.full[st], 0, h, tok);
                 for (int k = 0; k < 2; ++k) {
-                    tma_load_3d(s.b[st][k], &tm_b, &s.bcfull[st], 64 * k, g, tok);
-                    tma_load_3d(s.c[st][k], &tm_c, &s.bcfull[st], 64 * k, g, tok);
+                    tma_load_3d(s.b[st][k], &tm_b, &s.full[st], 64 * k, g, tok);
+                    tma_load_3d(s.c[st][k], &tm_c, &s.full[st], 64 * k, g, tok);
                 }
                 ++issued;
+                TC_TRACE(0, u);
             }
             if (*(volatile int*)&ctl.abort) {
                 // let the copies already in flight land before the CTA exits
-                for (int u = 0; u < issued; ++u) {
-                    mbar_wait(&s.xfull[u & 1], (u >> 1) & 1, 400000000ll);
-                    mbar_wait(&s.bcfull[u & 1], (u >> 1) & 1, 400000000ll);
-                }
+                for (int u = 0; u < issued; ++u) mbar_wait(&s.full[u & 1], (u >> 1) & 1, 400000000ll);
             }
         }
     } else if (warp == 18) {
-        // -------------------------------------------------------- W18: C B^T
+        // ------------------------------------------- W18: C -> TMEM, C B^T
         if (lane == 0 && nt > 0) {
             const uint32_t id_cb = idesc_f16(128, 128, 0, 0);
             for (int t = 0; t < nt; ++t) {
                 const int st = t & 1;
-                if (!wait_bar(ctl, &s.bcfull[st], (t >> 1) & 1, p.status)) break;
-                // P has read C B^T of tile t - 2 out of this buffer
-                if (t >= 2 && !wait_bar(ctl, &s.cb_free[st], ((t - 2) >> 1) & 1, p.status)) break;
+                if (!wait_bar(ctl, &s.full[st], (t >> 1) & 1, p.status)) break;
+                // TMEM C buffer st is free once C' h_prev of tile t - 2 has completed
+                if (t >= 2 && !wait_bar(ctl, &s.y_full[st], ((t - 2) >> 1) & 1, p.status)) break;
                 tc_fence_after();
-                const uint32_t cb = smem_u32(s.c[st][0]), bb = smem_u32(s.b[st][0]);
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
-                    mma_ss(tmem + kColCB + 128 * st, sdesc_sw128(cb + off, 16, 1024),
-                           sdesc_sw128(bb + off, 16, 1024), id_cb, k > 0);
-                }
+                // descriptors differ per K step only in the start address (low bits, in 16-byte units)
+                const uint64_t dc = sdesc_sw128(smem_u32(s.c[st][0]), 16, 1024);
+                const uint64_t db = sdesc_sw128(smem_u32(s.b[st][0]), 16, 1024);
+                const uint32_t ct = tmem + kColC + 64 * st;
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k)
+                    tmem_cp_128x256b(ct + 8 * k, dc + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4));
+                TC_TRACE(1, t);
+                // P has read C B^T of tile t - 1
+                if (t >= 1 && !wait_bar(ctl, &s.cb_free[st ^ 1], ((t - 1) >> 1) & 1, p.status)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k)
+                    mma_ts(tmem + kColCB, ct + 8 * k, db + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4), id_cb,
+                           k > 0);
                 mma_commit(&s.cb_full[st]);
+                TC_TRACE(2, t);
             }
             mma_commit(&s.fin[0]);
             mbar_wait(&s.fin[0], 0, 400000000ll);
         }
     } else if (warp == 17) {
-        // ------------------------------------------- W17: s, C' h_prev, S x
+        // ------------------------------------------ W17: s, C' h_prev, S x
         if (lane == 0 && nt > 0) {
-            const uint32_t id_st = idesc_f16(128, 64, 1, 1);   // MN-major A (B_w^T) and B (x)
-            const uint32_t id_y = idesc_f16(128, 64, 0, 1);    // K-major A, MN-major B
+            const uint32_t id_st = idesc_f16(128, 64, 1, 1);   // MN-major A (B^T) and B (w o x)
+            const uint32_t id_y = idesc_f16(128, 64, 0, 1);    // A from TMEM, MN-major B
             for (int t = 0; t < nt; ++t) {
                 const int st = t & 1;
                 const uint32_t par = (t >> 1) & 1;
-                const uint32_t bb = smem_u32(s.b[st][0]), cb = smem_u32(s.c[st][0]);
-                const uint32_t xb = smem_u32(s.x[st]), hsb = smem_u32(s.hs[st]);
-                // s = B_w^T x  (state rows 0..127 = TMEM lanes)
+                const uint64_t db = sdesc_sw128(smem_u32(s.b[st][0]), kBoxBytes, 1024);
+                const uint64_t dwx = sdesc_sw128(smem_u32(s.wx), kBoxBytes, 1024);
+                const uint64_t dx = sdesc_sw128(smem_u32(s.x[st]), kBoxBytes, 1024);
+                const uint64_t dhs = sdesc_sw128(smem_u32(s.hs[st]), kBoxBytes, 1024);
+                // s = B^T (w o x)  (state rows 0..127 = TMEM lanes)
                 if (!wait_bar(ctl, &s.x_ready[st], par, p.status)) break;
-                if (!wait_bar(ctl, &s.bc_ready[st], par, p.status)) break;
+                if (!wait_bar(ctl, &s.full[st], par, p.status)) break;
+                TC_TRACE(3, t);
                 tc_fence_after();
+#pragma unroll
                 for (int k = 0; k < kT / 16; ++k)
-                    mma_ss(tmem + kColSt, sdesc_sw128(bb + k * 2048, kBoxBytes, 1024),
-                           sdesc_sw128(xb + k * 2048, kBoxBytes, 1024), id_st, k > 0);
+                    mma_ss(tmem + kColSt, db + (uint64_t)(k * 128), dwx + (uint64_t)(k * 128), id_st, k > 0);
                 mma_commit(&s.s_done[st]);
-                // Y = C' h_prev: needs the state entering tile t and a free Y buffer
+                TC_TRACE(4, t);
+                // Y = C' h_prev: needs the state entering tile t, C' and a free Y buffer
                 if (!wait_bar(ctl, &s.hs_ready[st], par, p.status)) break;
+                if (!wait_bar(ctl, &s.c_scaled[st], par, p.status)) break;
                 if (t >= 2 && !wait_bar(ctl, &s.e_done[st], ((t - 2) >> 1) & 1, p.status)) break;
+                TC_TRACE(5, t);
                 tc_fence_after();
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
-                    mma_ss(tmem + kColY + 64 * st, sdesc_sw128(cb + off, 16, 1024),
-                           sdesc_sw128(hsb + k * 2048, kBoxBytes, 1024), id_y, k > 0);
-                }
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k)
+                    mma_ts(tmem + kColY + 64 * st, tmem + kColC + 64 * st + 8 * k, dhs + (uint64_t)(k * 128), id_y, k > 0);
+                TC_TRACE(6, t);
                 // Y += S x
                 if (!wait_bar(ctl, &s.s_ready[st], par, p.status)) break;
+                TC_TRACE(7, t);
                 tc_fence_after();
+#pragma unroll
                 for (int k = 0; k < kT / 16; ++k)
-                    mma_ts(tmem + kColY + 64 * st, tmem + kColS + k * 8,
-                           sdesc_sw128(xb + k * 2048, kBoxBytes, 1024), id_y, 1);
+                    mma_ts(tmem + kColY + 64 * st, tmem + kColS + k * 8, dx + (uint64_t)(k * 128), id_y, 1);
                 mma_commit(&s.y_full[st]);
+                TC_TRACE(8, t);
             }
             mma_commit(&s.fin[1]);
             mbar_wait(&s.fin[1], 0, 400000000ll);
         }
     } else if (warp < 8) {
-        // ------------------------------- P: scaling, decay mask, decay scan
+        // -------------------------------------- P: C', decay mask, decay scan
         const int quarter = warp & 3, half = warp >> 2;
         const int j = 32 * quarter + lane;
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
@@ -813,22 +901,29 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             tmem_st_wait();
         }
         // decay scan of tile u into the arrays of parity u & 1
-        float dt_next = 0.f;
-        auto scan = [&](int u) {
+        auto scan = [&](int u) -> bool {
             const int buf = u & 1, qu = tile_len(u);
+            if (tid == 128) TC_TRACE(30, u);
+            if (!wait_role<1>(ctl, &s.dt_full[u & 3], (u >> 2) & 1, p.status, leader, &ctl.p_flag)) return false;
+            if (tid == 128) TC_TRACE(31, u);
+            const float dtj = s.dts[u & 3][j];
+            warp_arrive(&s.dt_free[u & 3]);
+            if (tid == 128) TC_TRACE(32, u);
             float dj = 0.f, a = 0.f;
             if (j < qu) {
-                dj = softplus_f(dt_next + bias);
+                dj = softplus_fast(dtj + bias);
                 a = dj * A2;
             }
-            if ((int64_t)(u + 1) * kT + j < len) dt_next = __bfloat162float(p.dt[(tok0 + (int64_t)(u + 1) * kT + j) * H + h]);
+            if (tid == 128) TC_TRACE(33, u);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float v = __shfl_up_sync(0xffffffffu, a, o);
                 if (lane >= o) a += v;
             }
             if (lane == 31) s.wtot[buf][half][quarter] = a;
+            if (tid == 128) TC_TRACE(34, u);
             p_bar();
+            if (tid == 128) TC_TRACE(35, u);
             for (int w = 0; w < quarter; ++w) a += s.wtot[buf][half][w];
             const float cs_pivot = __shfl_sync(0xffffffffu, a, lane | 15);
             if (half == 0) {
@@ -836,52 +931,38 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 s.d[buf][j] = dj;
                 s.colfac[buf][j] = ex2(cs_pivot - a) * dj;
             }
+            if (tid == 128) TC_TRACE(36, u);
             warp_arrive(&s.scan_done[buf]);
+            if (tid == 128) TC_TRACE(37, u);
+            return true;
         };
-        if (nt > 0) {
-            if (j < len) dt_next = __bfloat162float(p.dt[(tok0 + j) * H + h]);
-            scan(0);
-        }
+        if (nt > 0) scan(0);
         for (int t = 0; t < nt; ++t) {
             const int st = t & 1;
             const uint32_t par = (t >> 1) & 1;
-            const int q = tile_len(t);
             if (!wait_role<1>(ctl, &s.cb_full[st], par, p.status, leader, &ctl.p_flag)) break;
+            if (tid == 128) TC_TRACE(9, t);
             tc_fence_after();
             const float cs2j = s.cs[st][j];
             {
-                // C'_j = 2^cs_j C_j, B_w_j = d_j 2^(cs_last - cs_j) B_j (zero past the sequence end);
-                // this warp takes the 64-column box `half` of row j
-                const float cs_last = s.cs[st][q - 1];
+                // C'_j = 2^cs_j C_j in place in TMEM (this warp: 32 of the 64 columns)
                 const __half2 e2 = __float2half2_rn(ex2(cs2j));
-                const __half2 w2 = __float2half2_rn(s.d[st][j] * ex2(cs_last - cs2j));
-                uint8_t* brow = s.b[st][half];
-                uint8_t* crow = s.c[st][half];
-                // four 16-byte chunks of B and of C at a time: all loads before the stores
+                const uint32_t ct = tmem + lane_base + kColC + 64 * st + 32 * half;
+                uint32_t r0[16], r1[16];
+                tmem_ld16(ct, r0);
+                tmem_ld16(ct + 16, r1);
+                tmem_ld_wait();
 #pragma unroll
-                for (int c0 = 0; c0 < 8; c0 += 4) {
-                    uint4 vb[4], vc[4];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        vb[c] = *reinterpret_cast<const uint4*>(brow + sw128_off(j, c0 + c));
-                        vc[c] = *reinterpret_cast<const uint4*>(crow + sw128_off(j, c0 + c));
-                    }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        vb[c].x = h2u(__hmul2(u2h(vb[c].x), w2)); vb[c].y = h2u(__hmul2(u2h(vb[c].y), w2));
-                        vb[c].z = h2u(__hmul2(u2h(vb[c].z), w2)); vb[c].w = h2u(__hmul2(u2h(vb[c].w), w2));
-                        vc[c].x = h2u(__hmul2(u2h(vc[c].x), e2)); vc[c].y = h2u(__hmul2(u2h(vc[c].y), e2));
-                        vc[c].z = h2u(__hmul2(u2h(vc[c].z), e2)); vc[c].w = h2u(__hmul2(u2h(vc[c].w), e2));
-                        if (j >= q) vb[c] = make_uint4(0u, 0u, 0u, 0u);
-                    }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        *reinterpret_cast<uint4*>(brow + sw128_off(j, c0 + c)) = vb[c];
-                        *reinterpret_cast<uint4*>(crow + sw128_off(j, c0 + c)) = vc[c];
-                    }
+                for (int i = 0; i < 16; ++i) {
+                    r0[i] = h2u(__hmul2(u2h(r0[i]), e2));
+                    r1[i] = h2u(__hmul2(u2h(r1[i]), e2));
                 }
-                fence_proxy_async_smem();
-                warp_arrive(&s.bc_ready[st]);
+                tmem_st16(ct, r0);
+                tmem_st16(ct + 16, r1);
+                tmem_st_wait();
+                tc_fence_before();
+                warp_arrive(&s.c_scaled[st]);
+                if (tid == 128) TC_TRACE(10, t);
             }
             // S = C B^T o 2^(cs_j - cs_i) d_i (i <= j), D on the diagonal.  This warp takes the
             // 16-column blocks b = 2m + half: m < quarter lie left of the diagonal 32-block
@@ -889,7 +970,7 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             // exponential per element, masked with a select).  All held in registers until
             // the S buffer is free.
             uint32_t sv[4][8];
-            const uint32_t cbuf = tmem + lane_base + kColCB + 128 * st;
+            const uint32_t cbuf = tmem + lane_base + kColCB;
 #pragma unroll
             for (int m = 0; m < 3; ++m) {
                 if (m < quarter) {
@@ -935,9 +1016,12 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
             tc_fence_before();
             warp_arrive(&s.cb_free[st]);
+            if (tid == 128) TC_TRACE(11, t);
+            if (tid == 96) TC_TRACE(15, t);
             // the S buffer is free once S x of tile t - 1 has completed
             if (t > 0 && !wait_role<1>(ctl, &s.y_full[st ^ 1], ((t - 1) >> 1) & 1, p.status, leader, &ctl.p_flag))
                 break;
+            if (tid == 128) TC_TRACE(12, t);
             tc_fence_after();
 #pragma unroll
             for (int m = 0; m < 3; ++m)
@@ -946,10 +1030,13 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             tmem_st_wait();
             tc_fence_before();
             warp_arrive(&s.s_ready[st]);
-            if (t + 1 < nt) scan(t + 1);
+            if (tid == 128) TC_TRACE(13, t);
+            if (tid == 96) TC_TRACE(16, t);
+            if (t + 1 < nt && !scan(t + 1)) break;
+            if (tid == 128) TC_TRACE(14, t);
         }
     } else if (warp < 16) {
-        // ------------------------------------ E: x to fp16, state, epilogue
+        // -------------------------------- E: x operands, state, epilogue
         const int quarter = warp & 3, half = (warp >> 2) & 1;
         const int j = 32 * quarter + lane;     // token row (x, y) and state row (s, h)
         const int col0 = 32 * half;
@@ -987,6 +1074,7 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 // h <- 2^cs_last h + s for tile k - 1
                 const int u = k - 1;
                 if (!(ok = wait_role<2>(ctl, &s.s_done[u & 1], (u >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                if (tid == 256) TC_TRACE(17, u);
                 tc_fence_after();
                 {
                     uint32_t r0[16], r1[16];
@@ -999,56 +1087,91 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                         hreg[16 + i] = fmaf(e_state, hreg[16 + i], __uint_as_float(r1[i]));
                     }
                 }
+                if (tid == 256) TC_TRACE(38, u);
                 tc_fence_before();
                 if (k < nt) put_state(k);
+                if (tid == 256) TC_TRACE(18, u);
             }
             if (k < nt) {
-                // x of tile k to fp16 in place (zero past the sequence end)
+                // x of tile k to the fp16 operands x and w o x (zero past the sequence end)
                 if (!(ok = wait_role<2>(ctl, &s.scan_done[k & 1], (k >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                if (tid == 256) TC_TRACE(19, k);
                 const int q = tile_len(k);
-                e_state = ex2(s.cs[k & 1][q - 1]);
-                if (!(ok = wait_role<2>(ctl, &s.xfull[k & 1], (k >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                const float cs_last = s.cs[k & 1][q - 1];
+                e_state = ex2(cs_last);
+                const __half2 w2 = __float2half2_rn(s.d[k & 1][j] * ex2(cs_last - s.cs[k & 1][j]));
+                if (tid == 256) TC_TRACE(39, k);
+                if (!(ok = wait_role<2>(ctl, &s.full[k & 1], (k >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                if (tid == 256) TC_TRACE(40, k);
                 uint8_t* xt = s.x[k & 1];
-                uint4 v[4];
+                uint4 xv[4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) v[m] = *reinterpret_cast<const uint4*>(xt + sw128_off(j, col0 / 8 + m));
+                for (int m = 0; m < 4; ++m) xv[m] = *reinterpret_cast<const uint4*>(xt + sw128_off(j, col0 / 8 + m));
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
-                    uint4 o;
-                    o.x = pack_f16x2(bf16lo(v[m].x), bf16hi(v[m].x));
-                    o.y = pack_f16x2(bf16lo(v[m].y), bf16hi(v[m].y));
-                    o.z = pack_f16x2(bf16lo(v[m].z), bf16hi(v[m].z));
-                    o.w = pack_f16x2(bf16lo(v[m].w), bf16hi(v[m].w));
+                    uint4 o, w;
+                    o.x = pack_f16x2(bf16lo(xv[m].x), bf16hi(xv[m].x));
+                    o.y = pack_f16x2(bf16lo(xv[m].y), bf16hi(xv[m].y));
+                    o.z = pack_f16x2(bf16lo(xv[m].z), bf16hi(xv[m].z));
+                    o.w = pack_f16x2(bf16lo(xv[m].w), bf16hi(xv[m].w));
                     if (j >= q) o = make_uint4(0u, 0u, 0u, 0u);
-                    *reinterpret_cast<uint4*>(xt + sw128_off(j, col0 / 8 + m)) = o;
+                    w.x = h2u(__hmul2(u2h(o.x), w2));
+                    w.y = h2u(__hmul2(u2h(o.y), w2));
+                    w.z = h2u(__hmul2(u2h(o.z), w2));
+                    w.w = h2u(__hmul2(u2h(o.w), w2));
+                    const uint32_t off = sw128_off(j, col0 / 8 + m);
+                    *reinterpret_cast<uint4*>(xt + off) = o;
+                    *reinterpret_cast<uint4*>(s.wx + off) = w;
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 warp_arrive(&s.x_ready[k & 1]);
+                if (tid == 256) TC_TRACE(20, k);
+                if (tid == 480) TC_TRACE(23, k);
             }
             if (k >= 1) {
                 // epilogue of tile k - 1: y = Y
                 const int u = k - 1, q = tile_len(u);
                 if (!(ok = wait_role<2>(ctl, &s.y_full[u & 1], (u >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                if (tid == 256) TC_TRACE(21, u);
                 tc_fence_after();
-                __nv_bfloat16* yrow = p.y + (tok0 + (int64_t)u * kT + j) * H * kP + (int64_t)h * kP + col0;
-                {
-                    uint32_t r[32];
-                    tmem_ld16(tmem + lane_base + kColY + 64 * (u & 1) + col0, *reinterpret_cast<uint32_t(*)[16]>(r));
-                    tmem_ld16(tmem + lane_base + kColY + 64 * (u & 1) + col0 + 16,
-                              *reinterpret_cast<uint32_t(*)[16]>(r + 16));
-                    tmem_ld_wait();
-                    uint32_t o[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) o[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                    if (j < q) {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            *reinterpret_cast<uint4*>(yrow + 8 * c) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-                    }
-                }
+                uint32_t r[32];
+                tmem_ld16(tmem + lane_base + kColY + 64 * (u & 1) + col0, *reinterpret_cast<uint32_t(*)[16]>(r));
+                tmem_ld16(tmem + lane_base + kColY + 64 * (u & 1) + col0 + 16,
+                          *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+                tmem_ld_wait();
+                // Y is in registers: release the buffer before the global stores
                 tc_fence_before();
                 warp_arrive(&s.e_done[u & 1]);
+                if (tid == 256) TC_TRACE(22, u);
+                if (tid == 480) TC_TRACE(24, u);
+                if (tid == 256) TC_TRACE(41, u);
+                {
+                    // Through this warp's 2 KB of hs[u & 1] (free: C' h_prev of tile u has
+                    // completed; rewritten only after the next role barrier): rows of 64 bytes
+                    // with 16-byte chunks XOR-swizzled by row pairs (no bank conflicts either
+                    // way), then 8 rows x 64 bytes per store instruction instead of 32 rows.
+                    uint8_t* stg = s.hs[u & 1] + (warp - 8) * 2048;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (c ^ ((lane >> 1) & 3))) = make_uint4(
+                            pack_bf16x2(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
+                            pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
+                            pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
+                            pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+                    __syncwarp();
+                    const int cc = lane >> 3;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int rl = 8 * i + (lane & 7);
+                        const uint4 val = *reinterpret_cast<const uint4*>(stg + rl * 64 + 16 * (cc ^ ((rl >> 1) & 3)));
+                        const int row = 32 * quarter + rl;
+                        if (row < q)
+                            *reinterpret_cast<uint4*>(p.y + (tok0 + (int64_t)u * kT + row) * H * kP + (int64_t)h * kP +
+                                                      col0 + 8 * cc) = val;
+                    }
+                }
+                if (tid == 256) TC_TRACE(42, u);
             }
         }
         if (p.final_state && (ok || nt == 0)) {
@@ -1064,7 +1187,7 @@ k_tc_scan2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-}  // namespace v2
+}  // namespace v3
 
 // bf16 -> fp16 copies of B and C (8 elements per thread step).
 __global__ void k_tc_prep(const uint4* __restrict__ b, const uint4* __restrict__ c, uint4* __restrict__ b16,
@@ -1112,6 +1235,12 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType ty, const void* base, uint64_t
 
 }  // namespace
 
+#ifdef SSD_TC_TRACE
+extern "C" __attribute__((visibility("default"))) int ssd_tc_trace_read(long long* out) {
+    return (int)cudaMemcpyFromSymbol(out, v3::g_tc_trace, sizeof(v3::g_tc_trace));
+}
+#endif
+
 bool tc_supported(const ScanArgs& a) {
     return a.dtype == 1 && a.P == kP && (a.N == 128 || a.N == 256) && (a.Q == 128 || a.Q == 256) &&
            a.b * a.L < ((int64_t)1 << 31) && a.S * a.H < ((int64_t)1 << 31) && get_encode() != nullptr;
@@ -1152,9 +1281,9 @@ int launch_tc_scan(const ScanArgs& a, const SeqInfo& si, int64_t, void* ws, int3
     p.G = (int)a.G;
     ProfScope ps(K_TC_SCAN, st);
     if (a.N == 128) {
-        const size_t smem = sizeof(v2::Smem) + 1024;
-        cudaFuncSetAttribute(v2::k_tc_scan2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        v2::k_tc_scan2<<<(unsigned)(a.S * a.H), v2::kThreads2, smem, st>>>(tm_x, tm_b, tm_c, p);
+        const size_t smem = sizeof(v3::Smem) + 1024;
+        cudaFuncSetAttribute(v3::k_tc_scan3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        v3::k_tc_scan3<<<(unsigned)(a.S * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, p);
     } else {
         const size_t smem = sizeof(TcSmem<256>) + 1024;
         cudaFuncSetAttribute(k_tc_scan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -57,6 +57,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+#ifdef SSD_MBAR_HINT
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"((uint32_t)SSD_MBAR_HINT)
+        : "memory");
+    return ok != 0;
+}
+#endif
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // `limit_cycles` SM clock cycles (about two seconds by default; returns false)
 // so that a lost arrival can never hang the GPU; callers turn that into an
@@ -64,7 +91,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // read on every poll.
 __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long long limit_cycles) {
     const long long t0 = clock64();
+#if defined(SSD_MBAR_SPIN)
+    while (!mbar_test_wait(bar, parity)) {
+#elif defined(SSD_MBAR_HINT)
+    while (!mbar_try_wait_hint(bar, parity)) {
+#else
     while (!mbar_try_wait(bar, parity)) {
+#endif
         if (clock64() - t0 > limit_cycles) return false;
     }
     return true;
@@ -173,6 +206,15 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
         ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// TMEM[lanes 0..127, 8 columns from taddr] = a 128-row x 32-byte matrix read
+// from shared memory through `sdesc` (the layout an MMA would read for one
+// K = 16 step of an fp16 A operand), row r -> lane r, bytes in column order.
+// Asynchronous; ordered with the MMAs this thread issues and covered by
+// tcgen05.commit like they are.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Arrives on `bar` once every MMA this thread issued before has completed.
