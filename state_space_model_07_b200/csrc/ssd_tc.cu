@@ -617,12 +617,14 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 // global inputs come in through TMA or through the dt warp, whose own waits
 // are off the critical path.
 //
-// Roles (640 threads):
+// Roles (768 threads):
 //   P   (warps 0-7):  C' scaling, the causal mask S, the decay scan of the
 //                     next tile.  Two warps per TMEM lane quarter split the
 //                     16-column blocks of a row by parity.
-//   E   (warps 8-15): x -> fp16 operands, the state update, the epilogue.
-//                     Two warps per lane quarter split the 64 columns.
+//   E   (warps 8-15): x -> fp16 operands and the state update.  Two warps
+//                     per lane quarter split the 64 columns.
+//   Y   (warps 20-23): the epilogue, Y (TMEM) -> bf16 -> y, one warp per
+//                     lane quarter.
 //   W16 (lane 0):     TMA loads of x, B and C, two stages.
 //   W17 (lane 0):     s, C' h_prev and S x MMAs.
 //   W18 (lane 0):     C -> TMEM copies and the C B^T MMAs.
@@ -632,7 +634,8 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 // tile t, so no waiter can see a barrier two phases ahead.
 namespace v3 {
 
-constexpr int kThreads3 = 640;
+constexpr int kThreads3 = 768;
+constexpr int kYWarps = 4;          // epilogue warps, one per TMEM lane quarter
 
 // Per-tile event timestamps of CTA 0, compiled in only with -DSSD_TC_TRACE
 // (performance analysis builds); a no-op otherwise.
@@ -739,7 +742,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             mbar_init(&s.scan_done[i], kRoleWarps);
             mbar_init(&s.x_ready[i], kRoleWarps);
             mbar_init(&s.hs_ready[i], kRoleWarps);
-            mbar_init(&s.e_done[i], kRoleWarps);
+            mbar_init(&s.e_done[i], kYWarps);
             mbar_init(&s.s_done[i], 1);
             mbar_init(&s.y_full[i], 1);
             mbar_init(&s.fin[i], 1);
@@ -1035,8 +1038,43 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (t + 1 < nt && !scan(t + 1)) break;
             if (tid == 128) TC_TRACE(14, t);
         }
+    } else if (warp >= 20) {
+        // ---------------------------------------------- Y: epilogue, y = Y
+        const int quarter = warp & 3;
+        const int j = 32 * quarter + lane;
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        for (int u = 0; u < nt; ++u) {
+            const int q = tile_len(u);
+            if (!wait_bar_w(ctl, &s.y_full[u & 1], (u >> 1) & 1, p.status)) break;
+            tc_fence_after();
+            __nv_bfloat16* yrow = p.y + (tok0 + (int64_t)u * kT + j) * H * kP + (int64_t)h * kP;
+            const uint32_t ya = tmem + lane_base + kColY + 64 * (u & 1);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t r[32];
+                tmem_ld16(ya + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(r));
+                tmem_ld16(ya + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+                tmem_ld_wait();
+                if (half == 1) {
+                    // Y is in registers: release the buffer before the global stores
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.e_done[u & 1]);
+                }
+                if (j < q) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(yrow + 32 * half + 8 * c) = make_uint4(
+                            pack_bf16x2(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
+                            pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
+                            pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
+                            pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+                }
+            }
+            if (lane == 0 && warp == 20) TC_TRACE(22, u);
+        }
     } else if (warp < 16) {
-        // -------------------------------- E: x operands, state, epilogue
+        // ------------------------------------------- E: x operands, state
         const int quarter = warp & 3, half = (warp >> 2) & 1;
         const int j = 32 * quarter + lane;     // token row (x, y) and state row (s, h)
         const int col0 = 32 * half;
@@ -1128,50 +1166,6 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 warp_arrive(&s.x_ready[k & 1]);
                 if (tid == 256) TC_TRACE(20, k);
                 if (tid == 480) TC_TRACE(23, k);
-            }
-            if (k >= 1) {
-                // epilogue of tile k - 1: y = Y
-                const int u = k - 1, q = tile_len(u);
-                if (!(ok = wait_role<2>(ctl, &s.y_full[u & 1], (u >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
-                if (tid == 256) TC_TRACE(21, u);
-                tc_fence_after();
-                uint32_t r[32];
-                tmem_ld16(tmem + lane_base + kColY + 64 * (u & 1) + col0, *reinterpret_cast<uint32_t(*)[16]>(r));
-                tmem_ld16(tmem + lane_base + kColY + 64 * (u & 1) + col0 + 16,
-                          *reinterpret_cast<uint32_t(*)[16]>(r + 16));
-                tmem_ld_wait();
-                // Y is in registers: release the buffer before the global stores
-                tc_fence_before();
-                warp_arrive(&s.e_done[u & 1]);
-                if (tid == 256) TC_TRACE(22, u);
-                if (tid == 480) TC_TRACE(24, u);
-                if (tid == 256) TC_TRACE(41, u);
-                {
-                    // Through this warp's 2 KB of hs[u & 1] (free: C' h_prev of tile u has
-                    // completed; rewritten only after the next role barrier): rows of 64 bytes
-                    // with 16-byte chunks XOR-swizzled by row pairs (no bank conflicts either
-                    // way), then 8 rows x 64 bytes per store instruction instead of 32 rows.
-                    uint8_t* stg = s.hs[u & 1] + (warp - 8) * 2048;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (c ^ ((lane >> 1) & 3))) = make_uint4(
-                            pack_bf16x2(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
-                            pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
-                            pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
-                            pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
-                    __syncwarp();
-                    const int cc = lane >> 3;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int rl = 8 * i + (lane & 7);
-                        const uint4 val = *reinterpret_cast<const uint4*>(stg + rl * 64 + 16 * (cc ^ ((rl >> 1) & 3)));
-                        const int row = 32 * quarter + rl;
-                        if (row < q)
-                            *reinterpret_cast<uint4*>(p.y + (tok0 + (int64_t)u * kT + row) * H * kP + (int64_t)h * kP +
-                                                      col0 + 8 * cc) = val;
-                    }
-                }
-                if (tid == 256) TC_TRACE(42, u);
             }
         }
         if (p.final_state && (ok || nt == 0)) {
