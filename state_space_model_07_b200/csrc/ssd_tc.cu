@@ -84,7 +84,7 @@ struct Cfg {
 
 struct TcCtl {
     int abort;
-    int p_flag, e_flag;    // leader-wait results handed to the rest of a role
+    int p_flag, e_flag, y_flag;    // leader-wait results handed to the rest of a role
 };
 
 template <int N>
@@ -643,6 +643,7 @@ constexpr int kYWarps = 4;          // epilogue warps, one per TMEM lane quarter
 __device__ long long g_tc_trace[48][1024];
 #define TC_TRACE(ev, t) \
     do { if (blockIdx.x == 0 && (t) >= 0 && (t) < 1024) g_tc_trace[ev][t] = clock64(); } while (0)
+__device__ unsigned long long g_cta_span[8192][3];   // start, end (global ns), SM id
 #else
 #define TC_TRACE(ev, t) do { } while (0)
 #endif
@@ -700,7 +701,8 @@ struct __align__(1024) Smem {
     uint64_t scan_done[2];            // P -> E
     uint64_t x_ready[2];              // E (x, w o x written) -> W17
     uint64_t hs_ready[2];             // E -> W17
-    uint64_t e_done[2];               // E (Y read) -> W17
+    uint64_t e_done[2];               // Y (Y read from TMEM) -> W17
+    uint64_t stg_free[2];             // Y (y staged in hs[t & 1] has been stored) -> E
     uint64_t s_done[2];               // W17 commit -> E
     uint64_t y_full[2];               // W17 commit -> E, P, W16, W18
     uint64_t fin[2];                  // W17, W18: own tcgen05 work drained before exit
@@ -710,7 +712,7 @@ struct __align__(1024) Smem {
 
 __global__ void __launch_bounds__(kThreads3, 1)
 k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-           const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
+           const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const TcParams p) {
     constexpr int N = 128;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -743,6 +745,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             mbar_init(&s.x_ready[i], kRoleWarps);
             mbar_init(&s.hs_ready[i], kRoleWarps);
             mbar_init(&s.e_done[i], kYWarps);
+            mbar_init(&s.stg_free[i], 1);
             mbar_init(&s.s_done[i], 1);
             mbar_init(&s.y_full[i], 1);
             mbar_init(&s.fin[i], 1);
@@ -756,6 +759,14 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = s.tmem_base;
     const float kLog2e = 1.4426950408889634f;
+#ifdef SSD_TC_TRACE
+    if (tid == 0 && blockIdx.x < 8192) {
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        g_cta_span[blockIdx.x][0] = globaltimer_ns();
+        g_cta_span[blockIdx.x][2] = smid;
+    }
+#endif
 
 #ifdef SSD_TC_TRACE
     if (warp == 16 && lane == 1) {
@@ -981,16 +992,21 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     uint32_t r[16];
                     tmem_ld16(cbuf + i0, r);
                     const float rf = ex2(cs2j - s.cs[st][i0 + 15]);
-                    float f[16];
+                    const uint64_t rf2 = f2pack(rf, rf);
+                    uint64_t f[8];
 #pragma unroll
-                    for (int k = 0; k < 16; k += 4) {
-                        const float4 cf = *reinterpret_cast<const float4*>(&s.colfac[st][i0 + k]);
-                        f[k] = cf.x * rf; f[k + 1] = cf.y * rf; f[k + 2] = cf.z * rf; f[k + 3] = cf.w * rf;
+                    for (int k = 0; k < 8; k += 2) {
+                        const float4 cf = *reinterpret_cast<const float4*>(&s.colfac[st][i0 + 2 * k]);
+                        f[k] = f2mul(f2pack(cf.x, cf.y), rf2);
+                        f[k + 1] = f2mul(f2pack(cf.z, cf.w), rf2);
                     }
                     tmem_ld_wait();
 #pragma unroll
-                    for (int k = 0; k < 16; k += 2)
-                        sv[m][k / 2] = pack_f16x2(__uint_as_float(r[k]) * f[k], __uint_as_float(r[k + 1]) * f[k + 1]);
+                    for (int k = 0; k < 8; ++k) {
+                        float lo, hi;
+                        f2unpack(f2mul(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), f[k]), lo, hi);
+                        sv[m][k] = pack_f16x2(lo, hi);
+                    }
                 }
             }
             {
@@ -1040,39 +1056,68 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         }
     } else if (warp >= 20) {
         // ---------------------------------------------- Y: epilogue, y = Y
+        // A full tile is staged (bf16, 128-byte swizzled rows) in hs[u & 1], free once C' h_prev
+        // of tile u has completed and until E writes the state entering tile u + 2 there, and
+        // leaves by one TMA store; a partial tile (the end of a sequence) is stored row by row,
+        // since the rows past its end belong to the next sequence.
         const int quarter = warp & 3;
         const int j = 32 * quarter + lane;
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        const bool issuer = warp == 20 && lane == 0;
+        bool stored = false;
+        if (issuer) tma_prefetch_desc(&tm_y);
         for (int u = 0; u < nt; ++u) {
             const int q = tile_len(u);
-            if (!wait_bar_w(ctl, &s.y_full[u & 1], (u >> 1) & 1, p.status)) break;
+            // one warp polls, the four decide together (they meet at named barrier 3 below)
+            if (warp == 20) {
+                const bool okw = wait_bar_w(ctl, &s.y_full[u & 1], (u >> 1) & 1, p.status);
+                if (lane == 0) *(volatile int*)&ctl.y_flag = okw ? 1 : 0;
+            }
+            asm volatile("bar.sync 3, 128;" ::: "memory");
+            if (!*(volatile int*)&ctl.y_flag) break;
             tc_fence_after();
-            __nv_bfloat16* yrow = p.y + (tok0 + (int64_t)u * kT + j) * H * kP + (int64_t)h * kP;
             const uint32_t ya = tmem + lane_base + kColY + 64 * (u & 1);
+            uint8_t* stg = s.hs[u & 1];
+            __nv_bfloat16* yrow = p.y + (tok0 + (int64_t)u * kT + j) * H * kP + (int64_t)h * kP;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            for (int hh = 0; hh < 2; ++hh) {
                 uint32_t r[32];
-                tmem_ld16(ya + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(r));
-                tmem_ld16(ya + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+                tmem_ld16(ya + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(r));
+                tmem_ld16(ya + 32 * hh + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
                 tmem_ld_wait();
-                if (half == 1) {
-                    // Y is in registers: release the buffer before the global stores
+                if (hh == 1) {
+                    // Y is in registers: release the buffer before storing
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&s.e_done[u & 1]);
                 }
-                if (j < q) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4*>(yrow + 32 * half + 8 * c) = make_uint4(
-                            pack_bf16x2(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
-                            pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
-                            pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
-                            pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 val = make_uint4(
+                        pack_bf16x2(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
+                        pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
+                        pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
+                        pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+                    if (q == kT)
+                        *reinterpret_cast<uint4*>(stg + sw128_off(j, 4 * hh + c)) = val;
+                    else if (j < q)
+                        *reinterpret_cast<uint4*>(yrow + 32 * hh + 8 * c) = val;
                 }
+            }
+            if (q == kT) fence_proxy_async_smem();
+            asm volatile("bar.sync 3, 128;" ::: "memory");
+            if (issuer) {
+                if (q == kT) {
+                    tma_store_3d(&tm_y, stg, 0, h, (int)(tok0 + (int64_t)u * kT));
+                    bulk_commit();
+                    bulk_wait_read0();
+                    stored = true;
+                }
+                mbar_arrive(&s.stg_free[u & 1]);
             }
             if (lane == 0 && warp == 20) TC_TRACE(22, u);
         }
+        if (issuer && stored) bulk_wait0();
     } else if (warp < 16) {
         // ------------------------------------------- E: x operands, state
         const int quarter = warp & 3, half = (warp >> 2) & 1;
@@ -1119,14 +1164,24 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     tmem_ld16(tmem + lane_base + kColSt + col0, r0);
                     tmem_ld16(tmem + lane_base + kColSt + col0 + 16, r1);
                     tmem_ld_wait();
+                    const uint64_t e2 = f2pack(e_state, e_state);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        hreg[i] = fmaf(e_state, hreg[i], __uint_as_float(r0[i]));
-                        hreg[16 + i] = fmaf(e_state, hreg[16 + i], __uint_as_float(r1[i]));
+                    for (int i = 0; i < 16; i += 2) {
+                        float lo, hi;
+                        f2unpack(f2fma(e2, f2pack(hreg[i], hreg[i + 1]),
+                                       f2pack(__uint_as_float(r0[i]), __uint_as_float(r0[i + 1]))), lo, hi);
+                        hreg[i] = lo; hreg[i + 1] = hi;
+                        f2unpack(f2fma(e2, f2pack(hreg[16 + i], hreg[17 + i]),
+                                       f2pack(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1]))), lo, hi);
+                        hreg[16 + i] = lo; hreg[17 + i] = hi;
                     }
                 }
                 if (tid == 256) TC_TRACE(38, u);
                 tc_fence_before();
+                // hs[k & 1] held y of tile k - 2 on its way out
+                if (k < nt && k >= 2 &&
+                    !(ok = wait_role<2>(ctl, &s.stg_free[k & 1], ((k - 2) >> 1) & 1, p.status, leader, &ctl.e_flag)))
+                    break;
                 if (k < nt) put_state(k);
                 if (tid == 256) TC_TRACE(18, u);
             }
@@ -1178,6 +1233,9 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+#ifdef SSD_TC_TRACE
+    if (tid == 0 && blockIdx.x < 8192) g_cta_span[blockIdx.x][1] = globaltimer_ns();
+#endif
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
@@ -1233,6 +1291,13 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType ty, const void* base, uint64_t
 extern "C" __attribute__((visibility("default"))) int ssd_tc_trace_read(long long* out) {
     return (int)cudaMemcpyFromSymbol(out, v3::g_tc_trace, sizeof(v3::g_tc_trace));
 }
+extern "C" __attribute__((visibility("default"))) int ssd_tc_span_read(unsigned long long* out) {
+    return (int)cudaMemcpyFromSymbol(out, v3::g_cta_span, sizeof(v3::g_cta_span));
+}
+extern "C" __attribute__((visibility("default"))) int ssd_tc_poll_read(unsigned long long* out) {
+    cudaMemcpyFromSymbol(out, ptx::g_poll_iters, sizeof(ptx::g_poll_iters));
+    return (int)cudaMemcpyFromSymbol(out + 32, ptx::g_poll_calls, sizeof(ptx::g_poll_calls));
+}
 #endif
 
 bool tc_supported(const ScanArgs& a) {
@@ -1261,6 +1326,9 @@ int launch_tc_scan(const ScanArgs& a, const SeqInfo& si, int64_t, void* ws, int3
         !make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, b16, (uint64_t)a.N, (uint64_t)a.G, (uint64_t)ntok) ||
         !make_map(&tm_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c16, (uint64_t)a.N, (uint64_t)a.G, (uint64_t)ntok))
         return 6;  // SSD_ERR_CUDA
+    CUtensorMap tm_y;
+    if (!make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, (uint64_t)a.P, (uint64_t)a.H, (uint64_t)ntok))
+        return 6;
     TcParams p;
     p.si = si;
     p.dt = (const __nv_bfloat16*)a.dt;
@@ -1277,7 +1345,7 @@ int launch_tc_scan(const ScanArgs& a, const SeqInfo& si, int64_t, void* ws, int3
     if (a.N == 128) {
         const size_t smem = sizeof(v3::Smem) + 1024;
         cudaFuncSetAttribute(v3::k_tc_scan3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        v3::k_tc_scan3<<<(unsigned)(a.S * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, p);
+        v3::k_tc_scan3<<<(unsigned)(a.S * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, tm_y, p);
     } else {
         const size_t smem = sizeof(TcSmem<256>) + 1024;
         cudaFuncSetAttribute(k_tc_scan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

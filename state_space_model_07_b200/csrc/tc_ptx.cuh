@@ -89,8 +89,15 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
 // so that a lost arrival can never hang the GPU; callers turn that into an
 // error status.  The clock is the SM's own cycle counter, which is cheap to
 // read on every poll.
+#ifdef SSD_TC_TRACE
+__device__ unsigned long long g_poll_iters[32];
+__device__ unsigned long long g_poll_calls[32];
+#endif
 __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long long limit_cycles) {
     const long long t0 = clock64();
+#ifdef SSD_TC_TRACE
+    unsigned long long iters = 0;
+#endif
 #if defined(SSD_MBAR_SPIN)
     while (!mbar_test_wait(bar, parity)) {
 #elif defined(SSD_MBAR_HINT)
@@ -98,8 +105,20 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long
 #else
     while (!mbar_try_wait(bar, parity)) {
 #endif
+#ifdef SSD_TC_TRACE
+        ++iters;
+#endif
+#ifdef SSD_MBAR_BACKOFF_NS
+        __nanosleep(SSD_MBAR_BACKOFF_NS);
+#endif
         if (clock64() - t0 > limit_cycles) return false;
     }
+#ifdef SSD_TC_TRACE
+    if (blockIdx.x == 0 && (threadIdx.x & 31) == 0) {
+        atomicAdd(&g_poll_iters[threadIdx.x >> 5], iters);
+        atomicAdd(&g_poll_calls[threadIdx.x >> 5], 1ull);
+    }
+#endif
     return true;
 }
 
@@ -143,6 +162,21 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
           "r"(c2)
         : "memory");
 }
+
+// Shared -> global tile store through the tensor map (coordinates must be
+// non-negative; rows past the tensor's outer extent are not written).
+// Completion is tracked per thread with the bulk async-group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* src, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until the source shared memory of every committed bulk store may be reused.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until every committed bulk store has completed.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---- tcgen05: tensor memory ------------------------------------------------------------
 
@@ -291,6 +325,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // bf16 pair (low half = element 0) -> two floats, exactly.
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction per two lanes of work).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
