@@ -217,6 +217,23 @@ def dist_env():
         int(os.environ.get("LOCAL_RANK", 0))
 
 
+def max_over_ranks(v, world, device):
+    """Max of a per-rank float over all ranks (device-timed numbers are
+    reported as the slowest rank's)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(tokens_per_rank, world, steps, ms):
+    """Whole-job tokens/s: every rank processes its own replica of the workload."""
+    return tokens_per_rank * world * steps / (ms * 1e-3)
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -318,13 +335,6 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for k in range(args.warmup):
         step(k)
     barrier()
@@ -340,10 +350,10 @@ def run_ours(args):
         barrier()
     _lib.profile_enable(False)
     stats = _lib.profile_read(reset=True)
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_step = ms / args.steps
     tokens = b * L if not w.packed_nseqs else L
-    value = tokens * world * args.steps / (ms * 1e-3)
+    value = throughput(tokens, world, args.steps, ms)
     launches = sum(v[0] for v in stats.values())
 
     pk, pk_src = peaks()
@@ -392,9 +402,9 @@ def run_ours(args):
             y_host.copy_(y, non_blocking=True)
         f1.record(stream)
         barrier()
-        e_ms = max_over_ranks(f0.elapsed_time(f1))
+        e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev)
         h2d = sum(t.numel() * t.element_size() for t in host.values())
-        e2e = {"value": tokens * world * n_e2e / (e_ms * 1e-3), "unit": "tokens/s",
+        e2e = {"value": throughput(tokens, world, n_e2e, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": y.numel() * y.element_size(),
                "steps": n_e2e, "path": "pinned host -> device copies, ssd_chunk_scan_fwd + ssd_state_update "
                                        "through the C ABI, y copied back, all on one stream"}
