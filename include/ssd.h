@@ -26,8 +26,12 @@
  *     for its kernels and reports device-side errors).
  *   - Argument errors are detected on the host, before anything is launched,
  *     and returned as an ssd_status; no exception crosses the ABI.
- *   - The library is stateless between calls and reentrant.  Temporary device
- *     memory is taken with cudaMallocAsync / cudaFreeAsync on `stream`.
+ *   - The library keeps no data between calls and is reentrant.  Temporary
+ *     device memory is taken stream-ordered on `stream` (cudaMallocFromPoolAsync
+ *     / cudaFreeAsync) from a memory pool the library creates per device on
+ *     first use.  The pool keeps freed workspace mapped for later calls (it
+ *     holds at most the largest workspace in flight, until the process exits)
+ *     so that a call after a synchronisation does not map it again.
  */
 #ifndef SSD_H_
 #define SSD_H_
@@ -135,7 +139,7 @@ SSD_API int ssd_state_update(const ssd_dims* dims, float* state, const void* x, 
  * ssd_chunk_scan_fwd; the caller still passes all inputs and outputs.  It
  * always runs the CUDA-core scan, whose scratch (per-chunk states, chunk
  * decays, packed-sequence table) lives in one fixed 32 MiB device array
- * inside the library instead of a cudaMallocAsync block:
+ * inside the library instead of a stream-ordered pool block:
  *   - needed scratch = 4 * (chunks * H * (N * P + 1)) bytes plus a few KiB,
  *     rounded to 256-byte pieces, with chunks = b * ceil(L / chunk), or
  *     ceil(L / chunk) + nseqs when packed.  Larger calls are rejected with

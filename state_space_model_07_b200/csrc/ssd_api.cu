@@ -1,7 +1,8 @@
 // ssd_api.cu -- the extern "C" boundary of libssd.so (declared in include/ssd.h).
 //
 // Host side only: argument validation (no device reads), path selection,
-// stream-ordered temporary memory, launches, error reporting.
+// stream-ordered temporary memory (from a library-owned pool), launches, error
+// reporting.
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -61,7 +62,7 @@ int check_sizes(const ssd_dims* d) {
     return SSD_OK;
 }
 
-// Sub-allocator over one cudaMallocAsync block (256-byte aligned pieces).
+// Sub-allocator over one stream-ordered block (256-byte aligned pieces).
 struct Carve {
     char* base = nullptr;
     size_t off = 0;
@@ -75,6 +76,37 @@ struct Carve {
 
 int cuda_fail(const char* what, cudaError_t e) {
     return fail(SSD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// The library's own stream-ordered memory pool, one per device, created on
+// first use with that device current.  Its release threshold is unlimited: a
+// workspace freed at the end of a call stays mapped in the pool for the next
+// call instead of going back to the OS at the next synchronisation (which made
+// each call after a sync map the workspace again, occasionally for
+// milliseconds).  The pool holds at most the largest workspace in flight at a
+// time; the caller's own allocations (torch's, the default pool's) are left
+// alone.  Returns nullptr if the pool cannot be made.
+cudaMemPool_t workspace_pool() {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+        uint64_t keep = ~(uint64_t)0;
+        if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+            cudaMemPoolDestroy(pool);
+            return nullptr;
+        }
+        pools[dev] = pool;
+    }
+    return pools[dev];
 }
 
 // Waits for the stream and reports device-side status (debug mode only).
@@ -186,8 +218,10 @@ int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, cons
     if (seq_idx) ws_bytes += 3 * Carve::round(sizeof(int32_t) * (S + 1));
 
     Carve cv;
-    cudaError_t e = cudaMallocAsync((void**)&cv.base, ws_bytes, st);
-    if (e != cudaSuccess) return cuda_fail("cudaMallocAsync(workspace)", e);
+    cudaMemPool_t pool = workspace_pool();
+    if (!pool) return fail(SSD_ERR_CUDA, "could not create the workspace memory pool");
+    cudaError_t e = cudaMallocFromPoolAsync((void**)&cv.base, ws_bytes, pool, st);
+    if (e != cudaSuccess) return cuda_fail("cudaMallocFromPoolAsync(workspace)", e);
     void* ws_main = cv.take(ws_path);
     int32_t* status = (int32_t*)cv.take(sizeof(int32_t));
     ssd::SeqInfo si;
@@ -250,8 +284,8 @@ int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const vo
 //
 // Some callers cannot let a library allocate device memory: a serving engine
 // that has already handed nearly all of HBM to its own pool (so a
-// cudaMallocAsync inside the call fails or forces the pool to give memory
-// back), or a caller that forbids allocation after start-up to keep latency
+// stream-ordered allocation inside the call fails or forces memory back out
+// of that pool), or a caller that forbids allocation after start-up to keep latency
 // predictable.  ssd_chunk_scan_fwd_noalloc serves them: it runs the CUDA-core
 // scan with its scratch (per-chunk states, chunk decays, packed-sequence
 // table, status word) placed in the fixed-size array below instead of a

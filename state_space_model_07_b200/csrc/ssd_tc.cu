@@ -602,8 +602,9 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 // Shared-memory bandwidth (128 B per clock per SM, shared by TMA writes, the
 // MMAs' operand reads and the threads) is what bounds this kernel, so the
 // design keeps bytes out of shared memory:
-//   * C B^T and C h_prev read B and C from the same shared-memory stage; the
-//     epilogue combines y = S x + 2^cs_j C h_prev from two TMEM accumulators.
+//   * C goes to TMEM once (tcgen05.cp); C B^T and C' h_prev take A from TMEM.
+//     C' = rows of C scaled by 2^cs_j is made in place in TMEM, so the output
+//     of a tile is one accumulator Y = C' h_prev + S x.
 //   * x arrives by TMA and is converted in place to fp16; the E warps also
 //     write w o x once.
 //   * The state recurrence runs on the E warps in fp32 registers,
@@ -617,7 +618,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 // four tiles ahead.
 //
 // Roles (768 threads):
-//   P   (warps 0-7):  the causal mask S.  Two warps per TMEM
+//   P   (warps 0-7):  C' scaling and the causal mask S.  Two warps per TMEM
 //                     lane quarter split the 16-column blocks of a row by
 //                     parity.
 //   E   (warps 8-15): x -> fp16 operands and the state update.  Two warps
@@ -625,8 +626,8 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 //   Y   (warps 20-23): the epilogue, Y (TMEM) -> bf16 -> y, one warp per
 //                     lane quarter.
 //   W16 (lane 0):     TMA loads of x, B and C, two stages.
-//   W17 (lane 0):     C h_prev, s and S x MMAs.
-//   W18 (lane 0):     the C B^T MMAs.
+//   W17 (lane 0):     s, C' h_prev and S x MMAs.
+//   W18 (lane 0):     C -> TMEM copies and the C B^T MMAs.
 //   W19:              the decay scan (softplus, cumulative sum, mask column
 //                     factors) of the coming tiles into a four-slot ring.
 // Every per-tile barrier exists per tile parity, and every barrier's next
@@ -648,10 +649,11 @@ __device__ unsigned long long g_cta_span[8192][3];   // start, end (global ns), 
 #define TC_TRACE(ev, t) do { } while (0)
 #endif
 constexpr int kRoleWarps = 8;       // P and E arrive once per warp
-constexpr uint32_t kColCB = 0;      // C B^T, fp32 128 x 128
-constexpr uint32_t kColS = 128;     // S, fp16 pairs (64 columns)
-constexpr uint32_t kColSt = 192;    // s, fp32 128 x 64
-constexpr uint32_t kColY = 256;     // two buffers of S x (64 columns) and C h_prev (64 columns)
+constexpr uint32_t kColC = 0;       // two 64-column buffers: C, then C' (fp16 pairs)
+constexpr uint32_t kColCB = 128;    // C B^T, fp32 128 x 128
+constexpr uint32_t kColS = 256;     // S, fp16 pairs (64 columns)
+constexpr uint32_t kColSt = 320;    // s, fp32 128 x 64
+constexpr uint32_t kColY = 384;     // two 64-column fp32 buffers
 
 // softplus(z) = max(z, 0) + log(1 + e), e = exp(-|z|) in (0, 1], with the
 // hardware base-2 exponential and logarithm; for e < 2^-7 the logarithm is
@@ -688,18 +690,18 @@ struct __align__(1024) Smem {
     float cs[4][kT];                  // tile-local cumulative decay (base-2 exponent), slot u & 3
     float d[4][kT];
     float colfac[4][kT];              // 2^(cs_m - cs_i) d_i, pivot m = last token of i's 16-block
-    uint64_t xfull[2];                // TMA x -> E, W17
-    uint64_t bcfull[2];               // TMA B, C -> W18, W17
+    uint64_t full[2];                 // TMA x, B, C -> W18, W17, E
     uint64_t scan_done[4];            // W19 (decay scan of tile u in slot u & 3) -> P, E
-    uint64_t scan_free[4];            // P, E, Y (slot read) -> W19
-    uint64_t cb_full[2];              // W18 commit (C B^T) -> P, W16
+    uint64_t scan_free[4];            // P, E (slot read) -> W19
+    uint64_t cb_full[2];              // W18 commit (C in TMEM, C B^T) -> P
     uint64_t cb_free[2];              // P (C B^T read) -> W18
+    uint64_t c_scaled[2];             // P (C' in TMEM) -> W17
     uint64_t s_ready[2];              // P (S in TMEM) -> W17
     uint64_t x_ready[2];              // E (x, w o x written) -> W17
     uint64_t hs_ready[2];             // E -> W17
     uint64_t e_done[2];               // Y (Y read from TMEM) -> W17
     uint64_t stg_free[2];             // Y (y staged in hs[t & 1] has been stored) -> E
-    uint64_t s_done[2];               // W17 commit (C h_prev, s) -> E, W16
+    uint64_t s_done[2];               // W17 commit -> E
     uint64_t y_full[2];               // W17 commit -> E, P, W16, W18
     uint64_t fin[2];                  // W17, W18: own tcgen05 work drained before exit
     uint32_t tmem_base;
@@ -729,13 +731,13 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     if (tid == 0) {
         for (int i = 0; i < 4; ++i) {
             mbar_init(&s.scan_done[i], 1);
-            mbar_init(&s.scan_free[i], 2 * kRoleWarps + kYWarps);
+            mbar_init(&s.scan_free[i], 2 * kRoleWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.xfull[i], 1);
-            mbar_init(&s.bcfull[i], 1);
+            mbar_init(&s.full[i], 1);
             mbar_init(&s.cb_full[i], 1);
             mbar_init(&s.cb_free[i], kRoleWarps);
+            mbar_init(&s.c_scaled[i], kRoleWarps);
             mbar_init(&s.s_ready[i], kRoleWarps);
             mbar_init(&s.x_ready[i], kRoleWarps);
             mbar_init(&s.hs_ready[i], kRoleWarps);
@@ -798,16 +800,13 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         for (int u = 0; u < nt; ++u) {
             const int sl = u & 3, qu = tile_len(u);
             // P and E have read slot sl for tile u - 4
-            if (lane == 0) TC_TRACE(43, u);
             if (u >= 4 && !wait_bar_w(ctl, &s.scan_free[sl], ((u - 4) >> 2) & 1, p.status)) break;
-            if (lane == 0) TC_TRACE(44, u);
             float dd[4], cs[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 dd[i] = 4 * lane + i < qu ? softplus_fast(dtn[i] + bias) : 0.f;
                 cs[i] = (i ? cs[i - 1] : 0.f) + dd[i] * A2;
             }
-            if (lane == 0) TC_TRACE(45, u);
             float incl = cs[3];
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -828,7 +827,6 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             *reinterpret_cast<float4*>(&s.colfac[sl][4 * lane]) = make_float4(cf[0], cf[1], cf[2], cf[3]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.scan_done[sl]);
-            if (lane == 0) TC_TRACE(46, u);
             if (u + 1 < nt) load_dt(u + 1);
         }
     } else if (warp == 16) {
@@ -837,54 +835,51 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
             tma_prefetch_desc(&tm_c);
-            int issued_bc = 0, issued_x = 0;
+            int issued = 0;
             for (int u = 0; u < nt; ++u) {
                 const int st = u & 1;
-                const uint32_t pp = ((u - 2) >> 1) & 1;
+                // stage st is free once every MMA of tile u - 2 has completed
+                if (u >= 2 && !wait_bar(ctl, &s.y_full[st], ((u - 2) >> 1) & 1, p.status)) break;
                 const int tok = (int)(tok0 + (int64_t)u * kT);
-                // B, C stage st is free once C B^T (cb_full) and C h_prev, B^T (w o x) (s_done)
-                // of tile u - 2 have completed
-                if (u >= 2 && !(wait_bar(ctl, &s.cb_full[st], pp, p.status) &&
-                                wait_bar(ctl, &s.s_done[st], pp, p.status)))
-                    break;
-                mbar_expect_tx(&s.bcfull[st], 4 * kBoxBytes);
+                mbar_expect_tx(&s.full[st], kTileBytesX + 4 * kBoxBytes);
+                tma_load_3d(s.x[st], &tm_x, &s.full[st], 0, h, tok);
                 for (int k = 0; k < 2; ++k) {
-                    tma_load_3d(s.b[st][k], &tm_b, &s.bcfull[st], 64 * k, g, tok);
-                    tma_load_3d(s.c[st][k], &tm_c, &s.bcfull[st], 64 * k, g, tok);
+                    tma_load_3d(s.b[st][k], &tm_b, &s.full[st], 64 * k, g, tok);
+                    tma_load_3d(s.c[st][k], &tm_c, &s.full[st], 64 * k, g, tok);
                 }
-                ++issued_bc;
-                // x stage st is free once S x of tile u - 2 has completed
-                if (u >= 2 && !wait_bar(ctl, &s.y_full[st], pp, p.status)) break;
-                mbar_expect_tx(&s.xfull[st], kTileBytesX);
-                tma_load_3d(s.x[st], &tm_x, &s.xfull[st], 0, h, tok);
-                ++issued_x;
+                ++issued;
                 TC_TRACE(0, u);
             }
             if (*(volatile int*)&ctl.abort) {
                 // let the copies already in flight land before the CTA exits
-                for (int u = 0; u < issued_bc; ++u) mbar_wait(&s.bcfull[u & 1], (u >> 1) & 1, 400000000ll);
-                for (int u = 0; u < issued_x; ++u) mbar_wait(&s.xfull[u & 1], (u >> 1) & 1, 400000000ll);
+                for (int u = 0; u < issued; ++u) mbar_wait(&s.full[u & 1], (u >> 1) & 1, 400000000ll);
             }
         }
     } else if (warp == 18) {
-        // ------------------------------------------------------- W18: C B^T
+        // ------------------------------------------- W18: C -> TMEM, C B^T
         if (lane == 0 && nt > 0) {
             const uint32_t id_cb = idesc_f16(128, 128, 0, 0);
             for (int t = 0; t < nt; ++t) {
                 const int st = t & 1;
-                if (!wait_bar(ctl, &s.bcfull[st], (t >> 1) & 1, p.status)) break;
-                TC_TRACE(1, t);
-                // P has read C B^T of tile t - 1
-                if (t >= 1 && !wait_bar(ctl, &s.cb_free[st ^ 1], ((t - 1) >> 1) & 1, p.status)) break;
+                if (!wait_bar(ctl, &s.full[st], (t >> 1) & 1, p.status)) break;
+                // TMEM C buffer st is free once C' h_prev of tile t - 2 has completed
+                if (t >= 2 && !wait_bar(ctl, &s.y_full[st], ((t - 2) >> 1) & 1, p.status)) break;
                 tc_fence_after();
                 // descriptors differ per K step only in the start address (low bits, in 16-byte units)
                 const uint64_t dc = sdesc_sw128(smem_u32(s.c[st][0]), 16, 1024);
                 const uint64_t db = sdesc_sw128(smem_u32(s.b[st][0]), 16, 1024);
+                const uint32_t ct = tmem + kColC + 64 * st;
 #pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint64_t off = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
-                    mma_ss(tmem + kColCB, dc + off, db + off, id_cb, k > 0);
-                }
+                for (int k = 0; k < N / 16; ++k)
+                    tmem_cp_128x256b(ct + 8 * k, dc + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4));
+                TC_TRACE(1, t);
+                // P has read C B^T of tile t - 1
+                if (t >= 1 && !wait_bar(ctl, &s.cb_free[st ^ 1], ((t - 1) >> 1) & 1, p.status)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k)
+                    mma_ts(tmem + kColCB, ct + 8 * k, db + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4), id_cb,
+                           k > 0);
                 mma_commit(&s.cb_full[st]);
                 TC_TRACE(2, t);
             }
@@ -892,33 +887,20 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             mbar_wait(&s.fin[0], 0, 400000000ll);
         }
     } else if (warp == 17) {
-        // ------------------------------------------ W17: C h_prev, s, S x
+        // ------------------------------------------ W17: s, C' h_prev, S x
         if (lane == 0 && nt > 0) {
             const uint32_t id_st = idesc_f16(128, 64, 1, 1);   // MN-major A (B^T) and B (w o x)
-            const uint32_t id_yo = idesc_f16(128, 64, 0, 1);   // K-major A (C), MN-major B (h_prev)
-            const uint32_t id_yd = idesc_f16(128, 64, 0, 1);   // A (S) from TMEM, MN-major B (x)
+            const uint32_t id_y = idesc_f16(128, 64, 0, 1);    // A from TMEM, MN-major B
             for (int t = 0; t < nt; ++t) {
                 const int st = t & 1;
                 const uint32_t par = (t >> 1) & 1;
-                const uint64_t dc = sdesc_sw128(smem_u32(s.c[st][0]), 16, 1024);
                 const uint64_t db = sdesc_sw128(smem_u32(s.b[st][0]), kBoxBytes, 1024);
                 const uint64_t dwx = sdesc_sw128(smem_u32(s.wx), kBoxBytes, 1024);
                 const uint64_t dx = sdesc_sw128(smem_u32(s.x[st]), kBoxBytes, 1024);
                 const uint64_t dhs = sdesc_sw128(smem_u32(s.hs[st]), kBoxBytes, 1024);
-                const uint32_t yd = tmem + kColY + 128 * st, yo = yd + 64;
-                // Yo = C h_prev: needs B, C, the state entering tile t and a free Y buffer
-                if (!wait_bar(ctl, &s.bcfull[st], par, p.status)) break;
-                if (!wait_bar(ctl, &s.hs_ready[st], par, p.status)) break;
-                if (t >= 2 && !wait_bar(ctl, &s.e_done[st], ((t - 2) >> 1) & 1, p.status)) break;
-                TC_TRACE(5, t);
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < N / 16; ++k)
-                    mma_ss(yo, dc + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4), dhs + (uint64_t)(k * 128),
-                           id_yo, k > 0);
-                TC_TRACE(6, t);
                 // s = B^T (w o x)  (state rows 0..127 = TMEM lanes)
                 if (!wait_bar(ctl, &s.x_ready[st], par, p.status)) break;
+                if (!wait_bar(ctl, &s.full[st], par, p.status)) break;
                 TC_TRACE(3, t);
                 tc_fence_after();
 #pragma unroll
@@ -926,12 +908,23 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     mma_ss(tmem + kColSt, db + (uint64_t)(k * 128), dwx + (uint64_t)(k * 128), id_st, k > 0);
                 mma_commit(&s.s_done[st]);
                 TC_TRACE(4, t);
-                // Yd = S x
+                // Y = C' h_prev: needs the state entering tile t, C' and a free Y buffer
+                if (!wait_bar(ctl, &s.hs_ready[st], par, p.status)) break;
+                if (!wait_bar(ctl, &s.c_scaled[st], par, p.status)) break;
+                if (t >= 2 && !wait_bar(ctl, &s.e_done[st], ((t - 2) >> 1) & 1, p.status)) break;
+                TC_TRACE(5, t);
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k)
+                    mma_ts(tmem + kColY + 64 * st, tmem + kColC + 64 * st + 8 * k, dhs + (uint64_t)(k * 128), id_y, k > 0);
+                TC_TRACE(6, t);
+                // Y += S x
                 if (!wait_bar(ctl, &s.s_ready[st], par, p.status)) break;
                 TC_TRACE(7, t);
                 tc_fence_after();
 #pragma unroll
-                for (int k = 0; k < kT / 16; ++k) mma_ts(yd, tmem + kColS + k * 8, dx + (uint64_t)(k * 128), id_yd, k > 0);
+                for (int k = 0; k < kT / 16; ++k)
+                    mma_ts(tmem + kColY + 64 * st, tmem + kColS + k * 8, dx + (uint64_t)(k * 128), id_y, 1);
                 mma_commit(&s.y_full[st]);
                 TC_TRACE(8, t);
             }
@@ -939,7 +932,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             mbar_wait(&s.fin[1], 0, 400000000ll);
         }
     } else if (warp < 8) {
-        // ------------------------------------------------ P: C', decay mask
+        // -------------------------------------- P: C', decay mask, decay scan
         const int quarter = warp & 3, half = warp >> 2;
         const int j = 32 * quarter + lane;
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
@@ -960,7 +953,26 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (tid == 128) TC_TRACE(9, t);
             tc_fence_after();
             const float cs2j = s.cs[sl][j];
-            if (tid == 128) TC_TRACE(10, t);
+            {
+                // C'_j = 2^cs_j C_j in place in TMEM (this warp: 32 of the 64 columns)
+                const __half2 e2 = __float2half2_rn(ex2(cs2j));
+                const uint32_t ct = tmem + lane_base + kColC + 64 * st + 32 * half;
+                uint32_t r0[16], r1[16];
+                tmem_ld16(ct, r0);
+                tmem_ld16(ct + 16, r1);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    r0[i] = h2u(__hmul2(u2h(r0[i]), e2));
+                    r1[i] = h2u(__hmul2(u2h(r1[i]), e2));
+                }
+                tmem_st16(ct, r0);
+                tmem_st16(ct + 16, r1);
+                tmem_st_wait();
+                tc_fence_before();
+                warp_arrive(&s.c_scaled[st]);
+                if (tid == 128) TC_TRACE(10, t);
+            }
             // S = C B^T o 2^(cs_j - cs_i) d_i (i <= j), D on the diagonal.  This warp takes the
             // 16-column blocks b = 2m + half: m < quarter lie left of the diagonal 32-block
             // (rank-1 split, one exponential per block), m = quarter holds the diagonal (one
@@ -1035,6 +1047,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             warp_arrive(&s.s_ready[st]);
             if (tid == 128) TC_TRACE(13, t);
             if (tid == 96) TC_TRACE(16, t);
+
             if (tid == 128) TC_TRACE(14, t);
         }
     } else if (warp >= 20) {
@@ -1053,27 +1066,20 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             const int q = tile_len(u);
             // one warp polls, the four decide together (they meet at named barrier 3 below)
             if (warp == 20) {
-                const bool okw = wait_bar_w(ctl, &s.scan_done[u & 3], (u >> 2) & 1, p.status) &&
-                                 wait_bar_w(ctl, &s.y_full[u & 1], (u >> 1) & 1, p.status);
+                const bool okw = wait_bar_w(ctl, &s.y_full[u & 1], (u >> 1) & 1, p.status);
                 if (lane == 0) *(volatile int*)&ctl.y_flag = okw ? 1 : 0;
             }
             asm volatile("bar.sync 3, 128;" ::: "memory");
             if (!*(volatile int*)&ctl.y_flag) break;
             tc_fence_after();
-            // the decay factor 2^cs_j of row j's C h_prev term (slot u & 3 is held until read)
-            const float ej = ex2(s.cs[u & 3][j]);
-            warp_arrive(&s.scan_free[u & 3]);
-            const uint64_t ej2 = f2pack(ej, ej);
-            const uint32_t ya = tmem + lane_base + kColY + 128 * (u & 1);
+            const uint32_t ya = tmem + lane_base + kColY + 64 * (u & 1);
             uint8_t* stg = s.hs[u & 1];
             __nv_bfloat16* yrow = p.y + (tok0 + (int64_t)u * kT + j) * H * kP + (int64_t)h * kP;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                uint32_t rd[32], ro[32];
-                tmem_ld16(ya + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(rd));
-                tmem_ld16(ya + 32 * hh + 16, *reinterpret_cast<uint32_t(*)[16]>(rd + 16));
-                tmem_ld16(ya + 64 + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(ro));
-                tmem_ld16(ya + 64 + 32 * hh + 16, *reinterpret_cast<uint32_t(*)[16]>(ro + 16));
+                uint32_t r[32];
+                tmem_ld16(ya + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(r));
+                tmem_ld16(ya + 32 * hh + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
                 tmem_ld_wait();
                 if (hh == 1) {
                     // Y is in registers: release the buffer before storing
@@ -1081,17 +1087,13 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&s.e_done[u & 1]);
                 }
-                // y = S x + 2^cs_j C h_prev
-                float r[32];
-#pragma unroll
-                for (int i = 0; i < 32; i += 2)
-                    f2unpack(f2fma(ej2, f2pack(__uint_as_float(ro[i]), __uint_as_float(ro[i + 1])),
-                                   f2pack(__uint_as_float(rd[i]), __uint_as_float(rd[i + 1]))), r[i], r[i + 1]);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const uint4 val = make_uint4(
-                        pack_bf16x2(r[8 * c], r[8 * c + 1]), pack_bf16x2(r[8 * c + 2], r[8 * c + 3]),
-                        pack_bf16x2(r[8 * c + 4], r[8 * c + 5]), pack_bf16x2(r[8 * c + 6], r[8 * c + 7]));
+                        pack_bf16x2(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
+                        pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
+                        pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
+                        pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
                     if (q == kT)
                         *reinterpret_cast<uint4*>(stg + sw128_off(j, 4 * hh + c)) = val;
                     else if (j < q)
@@ -1189,7 +1191,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 const __half2 w2 = __float2half2_rn(s.d[k & 3][j] * ex2(cs_last - s.cs[k & 3][j]));
                 warp_arrive(&s.scan_free[k & 3]);
                 if (tid == 256) TC_TRACE(39, k);
-                if (!(ok = wait_role<2>(ctl, &s.xfull[k & 1], (k >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                if (!(ok = wait_role<2>(ctl, &s.full[k & 1], (k >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
                 if (tid == 256) TC_TRACE(40, k);
                 uint8_t* xt = s.x[k & 1];
                 uint4 xv[4];

@@ -45,17 +45,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                  ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
 
 // Non-blocking probe of the phase with the given parity.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
@@ -70,19 +59,21 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-#ifdef SSD_MBAR_HINT
-__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity) {
+// Potentially blocking test with a suspend-time hint: a thread whose phase is
+// not complete may sleep, but for at most about `ns` nanoseconds before it
+// tests again.  Without the hint the sleep limit is system-dependent, and
+// waits were measured to overrun by up to tens of milliseconds.
+__device__ __forceinline__ bool mbar_try_wait_ns(uint64_t* bar, uint32_t parity, uint32_t ns) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"((uint32_t)SSD_MBAR_HINT)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
         : "memory");
     return ok != 0;
 }
-#endif
 
 // Waits for the phase with the given parity to complete.  Gives up after
 // `limit_cycles` SM clock cycles (about two seconds by default; returns false)
@@ -98,18 +89,9 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long
 #ifdef SSD_TC_TRACE
     unsigned long long iters = 0;
 #endif
-#if defined(SSD_MBAR_SPIN)
-    while (!mbar_test_wait(bar, parity)) {
-#elif defined(SSD_MBAR_HINT)
-    while (!mbar_try_wait_hint(bar, parity)) {
-#else
-    while (!mbar_try_wait(bar, parity)) {
-#endif
+    while (!mbar_try_wait_ns(bar, parity, 500)) {
 #ifdef SSD_TC_TRACE
         ++iters;
-#endif
-#ifdef SSD_MBAR_BACKOFF_NS
-        __nanosleep(SSD_MBAR_BACKOFF_NS);
 #endif
         if (clock64() - t0 > limit_cycles) return false;
     }
@@ -122,11 +104,11 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long
     return true;
 }
 
-// The first test is inlined; the polling loop is shared out of line to keep
-// the kernels' code (and instruction-cache footprint) small.
+// The first, non-blocking test is inlined; the polling loop is shared out of
+// line to keep the kernels' code (and instruction-cache footprint) small.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           long long limit_cycles = 4000000000ll) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     return mbar_wait_slow(bar, parity, limit_cycles);
 }
 
