@@ -869,14 +869,14 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 const uint64_t dc = sdesc_sw128(smem_u32(s.c[st][0]), 16, 1024);
                 const uint64_t db = sdesc_sw128(smem_u32(s.b[st][0]), 16, 1024);
                 const uint32_t ct = tmem + kColC + 64 * st;
-#pragma unroll
+#pragma unroll 1
                 for (int k = 0; k < N / 16; ++k)
                     tmem_cp_128x256b(ct + 8 * k, dc + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4));
                 TC_TRACE(1, t);
                 // P has read C B^T of tile t - 1
                 if (t >= 1 && !wait_bar(ctl, &s.cb_free[st ^ 1], ((t - 1) >> 1) & 1, p.status)) break;
                 tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                 for (int k = 0; k < N / 16; ++k)
                     mma_ts(tmem + kColCB, ct + 8 * k, db + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4), id_cb,
                            k > 0);
@@ -903,7 +903,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 if (!wait_bar(ctl, &s.full[st], par, p.status)) break;
                 TC_TRACE(3, t);
                 tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                 for (int k = 0; k < kT / 16; ++k)
                     mma_ss(tmem + kColSt, db + (uint64_t)(k * 128), dwx + (uint64_t)(k * 128), id_st, k > 0);
                 mma_commit(&s.s_done[st]);
@@ -914,7 +914,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 if (t >= 2 && !wait_bar(ctl, &s.e_done[st], ((t - 2) >> 1) & 1, p.status)) break;
                 TC_TRACE(5, t);
                 tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                 for (int k = 0; k < N / 16; ++k)
                     mma_ts(tmem + kColY + 64 * st, tmem + kColC + 64 * st + 8 * k, dhs + (uint64_t)(k * 128), id_y, k > 0);
                 TC_TRACE(6, t);
@@ -922,7 +922,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 if (!wait_bar(ctl, &s.s_ready[st], par, p.status)) break;
                 TC_TRACE(7, t);
                 tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                 for (int k = 0; k < kT / 16; ++k)
                     mma_ts(tmem + kColY + 64 * st, tmem + kColS + k * 8, dx + (uint64_t)(k * 128), id_y, 1);
                 mma_commit(&s.y_full[st]);
@@ -1075,7 +1075,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             const uint32_t ya = tmem + lane_base + kColY + 64 * (u & 1);
             uint8_t* stg = s.hs[u & 1];
             __nv_bfloat16* yrow = p.y + (tok0 + (int64_t)u * kT + j) * H * kP + (int64_t)h * kP;
-#pragma unroll
+#pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t r[32];
                 tmem_ld16(ya + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(r));
@@ -1194,16 +1194,14 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 if (!(ok = wait_role<2>(ctl, &s.full[k & 1], (k >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
                 if (tid == 256) TC_TRACE(40, k);
                 uint8_t* xt = s.x[k & 1];
-                uint4 xv[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) xv[m] = *reinterpret_cast<const uint4*>(xt + sw128_off(j, col0 / 8 + m));
-#pragma unroll
+#pragma unroll 1
                 for (int m = 0; m < 4; ++m) {
+                    const uint4 xv = *reinterpret_cast<const uint4*>(xt + sw128_off(j, col0 / 8 + m));
                     uint4 o, w;
-                    o.x = pack_f16x2(bf16lo(xv[m].x), bf16hi(xv[m].x));
-                    o.y = pack_f16x2(bf16lo(xv[m].y), bf16hi(xv[m].y));
-                    o.z = pack_f16x2(bf16lo(xv[m].z), bf16hi(xv[m].z));
-                    o.w = pack_f16x2(bf16lo(xv[m].w), bf16hi(xv[m].w));
+                    o.x = pack_f16x2(bf16lo(xv.x), bf16hi(xv.x));
+                    o.y = pack_f16x2(bf16lo(xv.y), bf16hi(xv.y));
+                    o.z = pack_f16x2(bf16lo(xv.z), bf16hi(xv.z));
+                    o.w = pack_f16x2(bf16lo(xv.w), bf16hi(xv.w));
                     if (j >= q) o = make_uint4(0u, 0u, 0u, 0u);
                     w.x = h2u(__hmul2(u2h(o.x), w2));
                     w.y = h2u(__hmul2(u2h(o.y), w2));
