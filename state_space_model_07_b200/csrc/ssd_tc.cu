@@ -164,6 +164,19 @@ __device__ __forceinline__ bool wait_role(TcCtl& c, uint64_t* bar, uint32_t pari
     return *(volatile int*)flag != 0;
 }
 
+// The same for two barriers at once (one named-barrier round for both);
+// `bar2` may be null.
+template <int kBarId>
+__device__ __forceinline__ bool wait_role2(TcCtl& c, uint64_t* bar1, uint32_t par1, uint64_t* bar2, uint32_t par2,
+                                           int32_t* status, bool leader, int* flag) {
+    if (leader) {
+        const bool ok = wait_bar_w(c, bar1, par1, status) && (!bar2 || wait_bar_w(c, bar2, par2, status));
+        if ((threadIdx.x & 31) == 0) *(volatile int*)flag = ok ? 1 : 0;
+    }
+    asm volatile("bar.sync %0, 256;" ::"n"(kBarId) : "memory");
+    return *(volatile int*)flag != 0;
+}
+
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
 k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
@@ -948,8 +961,8 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             const int st = t & 1;
             const uint32_t par = (t >> 1) & 1;
             const int sl = t & 3;
-            if (!wait_role<1>(ctl, &s.scan_done[sl], (t >> 2) & 1, p.status, leader, &ctl.p_flag)) break;
-            if (!wait_role<1>(ctl, &s.cb_full[st], par, p.status, leader, &ctl.p_flag)) break;
+            if (!wait_role2<1>(ctl, &s.scan_done[sl], (t >> 2) & 1, &s.cb_full[st], par, p.status, leader, &ctl.p_flag))
+                break;
             if (tid == 128) TC_TRACE(9, t);
             tc_fence_after();
             const float cs2j = s.cs[sl][j];
@@ -1152,7 +1165,11 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (k >= 1) {
                 // h <- 2^cs_last h + s for tile k - 1
                 const int u = k - 1;
-                if (!(ok = wait_role<2>(ctl, &s.s_done[u & 1], (u >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
+                // (and hs[k & 1] free again: it held y of tile k - 2 on its way out)
+                if (!(ok = wait_role2<2>(ctl, &s.s_done[u & 1], (u >> 1) & 1,
+                                         (k >= 2 && k < nt) ? &s.stg_free[k & 1] : nullptr, ((k - 2) >> 1) & 1,
+                                         p.status, leader, &ctl.e_flag)))
+                    break;
                 if (tid == 256) TC_TRACE(17, u);
                 tc_fence_after();
                 {
@@ -1174,16 +1191,14 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 }
                 if (tid == 256) TC_TRACE(38, u);
                 tc_fence_before();
-                // hs[k & 1] held y of tile k - 2 on its way out
-                if (k < nt && k >= 2 &&
-                    !(ok = wait_role<2>(ctl, &s.stg_free[k & 1], ((k - 2) >> 1) & 1, p.status, leader, &ctl.e_flag)))
-                    break;
                 if (k < nt) put_state(k);
                 if (tid == 256) TC_TRACE(18, u);
             }
             if (k < nt) {
                 // x of tile k to the fp16 operands x and w o x (zero past the sequence end)
-                if (!(ok = wait_role<2>(ctl, &s.scan_done[k & 3], (k >> 2) & 1, p.status, leader, &ctl.e_flag))) break;
+                if (!(ok = wait_role2<2>(ctl, &s.scan_done[k & 3], (k >> 2) & 1, &s.full[k & 1], (k >> 1) & 1, p.status,
+                                         leader, &ctl.e_flag)))
+                    break;
                 if (tid == 256) TC_TRACE(19, k);
                 const int q = tile_len(k);
                 const float cs_last = s.cs[k & 3][q - 1];
@@ -1191,8 +1206,6 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 const __half2 w2 = __float2half2_rn(s.d[k & 3][j] * ex2(cs_last - s.cs[k & 3][j]));
                 warp_arrive(&s.scan_free[k & 3]);
                 if (tid == 256) TC_TRACE(39, k);
-                if (!(ok = wait_role<2>(ctl, &s.full[k & 1], (k >> 1) & 1, p.status, leader, &ctl.e_flag))) break;
-                if (tid == 256) TC_TRACE(40, k);
                 uint8_t* xt = s.x[k & 1];
 #pragma unroll 1
                 for (int m = 0; m < 4; ++m) {
