@@ -274,13 +274,21 @@ def config_of(w):
 
 
 def kernel_source_sha(name):
+    """Hash of the kernel's source with comments and blank lines removed, so
+    that a recorded DRAM capture stays attached to the code it measured and
+    drops off as soon as the code (not its comments) changes."""
+    import re
     src = {"tc_scan": "ssd_tc.cu", "tc_prep": "ssd_tc.cu", "simt_chunk_out": "ssd_simt.cu",
            "state_update": "ssd_decode.cu"}.get(name)
     if not src:
         return None
     p = os.path.join(ROOT, "state_space_model_07_b200", "csrc", src)
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(p, encoding="utf-8") as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def traffic_for(name, units_per_launch):

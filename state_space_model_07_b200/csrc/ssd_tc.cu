@@ -7,38 +7,36 @@
 //     chunk of 256 tokens is two tiles joined by the same N x P state hand-over
 //     as two chunks are, so the result equals the chunked form up to rounding.
 //   * Per tile, with d = softplus(dt + dt_bias), cs = tile-local inclusive
-//     cumulative sum of d*A:
+//     cumulative sum of d*A, w_i = d_i exp(cs_last - cs_i):
 //       CB   = C B^T                               tcgen05, fp16 x fp16 -> fp32 TMEM
 //       S    = CB o exp(cs_j - cs_i) d_i (i <= j)  math warps, written back to TMEM
-//       Yd   = S x                                 tcgen05, A from TMEM
-//       Yo   = C h_prev                            tcgen05 (low-rank term of the
-//                                                  state entering the tile)
-//       Sc   = B^T (w o x), w_i = d_i exp(cs_last - cs_i)     tcgen05
-//       y    = Yd + exp(cs_j) Yo + D x             math warps -> bf16 -> HBM
-//       h    = exp(cs_last) h_prev + Sc            math warps, fp32 in registers
+//       y    = S x + exp(cs_j) C h_prev + D x      tcgen05 (+ math warps)
+//       h    = exp(cs_last) h_prev + B^T (w o x)   tcgen05 for the B^T (w o x) term
 //   * The operands the math warps produce (S, h_prev, w o x) are rounded to fp16
 //     (11-bit significand): bf16's 8 bits miss the 1e-2 (1 + |y|) accuracy bound.
 //     B and C are converted to fp16 once by k_tc_prep; x is converted in place in
 //     shared memory.  C B^T on those fp16 copies is exact for normal-range
-//     bf16 values.  The skip term D x rides on the diagonal of S, and the state
-//     is accumulated in TMEM by the MMA itself: the math warps scale it by the
-//     tile's total decay, then B^T (w o x) is added on the tensor core.
+//     bf16 values.  The skip term D x rides on the diagonal of S.
 //
-// Warp roles (576 threads), pipelined through mbarriers.  A warp can reach
-// only its quarter of the 128 TMEM lanes, so each role has two warps per lane
-// quarter (thread j of a quarter owns token / state row j = TMEM lane j):
-//   P  (warps 0-7):   decay scan and the causal mask S of tile t; the two warps
-//                     of a quarter split its 32-column blocks by parity, which
-//                     evens out the triangular work.
-//   E  (warps 8-15):  state hand-over and fp16 x, (w o x), h for tile t + 1,
-//                     then the output epilogue of tile t (Yd, Yo are double-
-//                     buffered); the two warps of a quarter split the columns.
-//   W16 (lane 0):     TMA loads (two-stage ring) and the C B^T MMAs.
-//   W17 (lane 0):     the C h_prev, B^T (w o x) and S x MMAs.
-// Every mbarrier's next phase depends on an action its waiters take after
-// waiting, so no waiter can see a barrier two phases ahead.  All waits are
-// bounded: on a timeout the kernel records SSD_ERR_TIMEOUT in the status word
-// and returns after freeing its TMEM.
+// Two kernels:
+//   * k_tc_scan3 (N = 128, below in namespace v3): the state recurrence runs on
+//     CUDA cores in fp32 registers, off the tensor core's critical path; C is
+//     copied to TMEM and scaled there by exp(cs_j), so the output is one
+//     accumulator; y leaves by TMA tensor stores.  Its own header comment has
+//     the roles and the hand-off rules.
+//   * k_tc_scan<N> (N = 256): the first design, in which the MMA accumulates
+//     the state in TMEM (the math warps scale it by the tile's total decay,
+//     then B^T (w o x) is added on the tensor core) and the epilogue combines
+//     two accumulators.  Warp roles (576 threads): P (warps 0-7) decay scan and
+//     the causal mask; E (warps 8-15) state hand-over, fp16 operands and the
+//     epilogue; W16 TMA loads and C B^T; W17 the other MMAs.
+//
+// A warp can reach only its quarter of the 128 TMEM lanes, so each math role
+// has two warps per lane quarter (thread j of a quarter owns token / state row
+// j = TMEM lane j).  Every mbarrier's next phase depends on an action its
+// waiters take after waiting, so no waiter can see a barrier two phases ahead.
+// All waits are bounded: on a timeout the kernel records SSD_ERR_TIMEOUT in the
+// status word and returns after freeing its TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
