@@ -1,0 +1,46 @@
+"""Host-side pieces of bench.py that need no GPU."""
+import json
+
+import bench
+
+
+def test_roofline_traffic_is_attached_to_the_measured_code_only(tmp_path, monkeypatch):
+    # the committed DRAM capture is reported for the kernel as it stands ...
+    rec = json.load(open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")))["tc_scan"]
+    assert rec["source_sha"] == bench.kernel_source_sha("tc_scan")
+    assert bench.traffic_for("tc_scan", rec["units"]) == rec["dram_bytes"]
+    # ... scales with the units a launch processes ...
+    assert bench.traffic_for("tc_scan", 2 * rec["units"]) == 2 * rec["dram_bytes"]
+    # ... and is dropped once the recorded hash no longer matches the code
+    bad = dict(rec, source_sha="0" * 16)
+    p = tmp_path / "profiles"
+    p.mkdir()
+    (p / "traffic.json").write_text(json.dumps({"tc_scan": bad}))
+    csrc = tmp_path / "state_space_model_07_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "ssd_tc.cu").write_text(open(bench.os.path.join(bench.ROOT, "state_space_model_07_b200", "csrc",
+                                                            "ssd_tc.cu")).read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_for("tc_scan", rec["units"]) is None
+
+
+def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    csrc = tmp_path / "state_space_model_07_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    f = csrc / "ssd_tc.cu"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f.write_text("int a = 1;  // one\n/* block */\nint b = 2;\n")
+    h0 = bench.kernel_source_sha("tc_scan")
+    f.write_text("// header\nint a = 1;\n\nint b = 2;  /* two */\n")
+    assert bench.kernel_source_sha("tc_scan") == h0
+    f.write_text("int a = 1;\nint b = 3;\n")
+    assert bench.kernel_source_sha("tc_scan") != h0
+
+
+def test_algorithmic_bytes_of_the_bench_workload():
+    from state_space_model_07_b200 import inputs
+    w = inputs.WORKLOADS["mamba2_2.7b_layer"]
+    tokens = w.batch * w.seqlen
+    # x + y (80 heads x 64 x 2 B each), dt (80 x 2 B), B + C (128 x 2 B each) per token, plus the final state
+    per_tok = 2 * 80 * 64 * 2 + 80 * 2 + 2 * 128 * 2
+    assert bench.workload_bytes(w, w.batch, tokens, 2) == tokens * per_tok + 8 * 80 * 128 * 64 * 4 == 714080256
