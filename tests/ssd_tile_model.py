@@ -1,0 +1,108 @@
+"""A numpy model of the tile algebra the tensor-core scan kernel evaluates.
+
+Written from "5.3 Tensor Parallelism support and large-cluster training",
+section 3.2 (block decomposition) and the recurrence of section 2.1, with the
+kernel's own choices spelled out so that they can be checked against the fp64
+oracle on the CPU:
+
+* 128-token tiles; decays as base-2 exponents, cs_j = sum_{k <= j in tile} d_k A log2(e);
+* the causal mask S[j, i] = (C_j . B_i) 2^(cs_j - cs_i) d_i (i <= j) split per
+  16-token column block b: blocks left of the row's 32-row lane quarter use the
+  rank-1 form 2^(cs_j - cs_m) * (2^(cs_m - cs_i) d_i) with pivot m = the block's
+  last token; the two blocks of the row's own quarter use the direct form;
+  D rides on the diagonal of S;
+* w_i = d_i 2^(cs_last - cs_i); the tile's own state term s = B^T (w o x);
+* y = S x + C' h_prev with C' = rows of C scaled by 2^cs_j;
+* h <- 2^cs_last h + s, carried in fp32 between tiles.
+
+``rounding`` chooses what the kernel rounds: None keeps everything in fp64
+(the form must then equal the oracle up to fp64 rounding); "kernel" rounds the
+tensor-core operands the way the kernel does (fp16 S, x, w o x, h_prev, B, C,
+C'; fp32 accumulation and state; bf16 y); "bf16_operands" rounds S, w o x and
+h_prev to bf16 instead, the alternative the kernel rejects.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+LOG2E = 1.4426950408889634
+T = 128
+
+
+def _round(a, kind):
+    if kind is None:
+        return a
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    dt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[kind]
+    return t.to(dt).to(torch.float64).numpy()
+
+
+def _softplus(z):
+    return np.where(z > 0, z + np.log1p(np.exp(-np.abs(z))), np.log1p(np.exp(np.minimum(z, 0))))
+
+
+def _mask(CB, cs, d, Dh, q):
+    """S for one tile, block by block as the kernel forms it (exact identities)."""
+    S = np.zeros_like(CB)
+    for j in range(T):
+        quarter = j // 32
+        for b in range(8):
+            cols = np.arange(16 * b, 16 * b + 16)
+            if b < 2 * quarter:                              # left of the row's quarter: rank-1
+                m = 16 * b + 15
+                rf = np.exp2(cs[j] - cs[m])
+                colfac = np.exp2(cs[m] - cs[cols]) * d[cols]
+                S[j, cols] = CB[j, cols] * (colfac * rf)
+            elif b <= 2 * quarter + 1:                       # the row's own quarter: direct
+                f = np.exp2(cs[j] - cs[cols]) * d[cols]
+                S[j, cols] = np.where(cols <= j, CB[j, cols] * f, 0.0)
+        S[j, j] += Dh
+    return S
+
+
+def tile_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, rounding=None):
+    """x (b,L,H,P), dt (b,L,H), B/C (b,L,G,N), A/dt_bias/D (H,), init_state (b,H,N,P).
+
+    Returns (y, final_state) as fp64 arrays."""
+    x, dt, B, C = (np.asarray(v, dtype=np.float64) for v in (x, dt, B, C))
+    A = np.asarray(A, dtype=np.float64)
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    bias = np.zeros(H) if dt_bias is None else np.asarray(dt_bias, dtype=np.float64)
+    Dv = np.zeros(H) if D is None else np.asarray(D, dtype=np.float64)
+    k16 = "f16" if rounding == "kernel" else ("bf16" if rounding == "bf16_operands" else None)
+    kop = "f16" if rounding in ("kernel", "bf16_operands") else None   # x, B, C, C' always fp16 in the kernel
+    k32 = "f32" if rounding else None
+    y = np.zeros((b, L, H, P))
+    fs = np.zeros((b, H, N, P))
+    for bb in range(b):
+        for h in range(H):
+            g = h // (H // G)
+            hst = np.zeros((N, P)) if init_state is None else np.asarray(init_state, np.float64)[bb, h].copy()
+            for t0 in range(0, L, T):
+                q = min(T, L - t0)
+                d = np.zeros(T)
+                d[:q] = _softplus(dt[bb, t0:t0 + q, h] + bias[h])
+                d = _round(d, k32)
+                cs = np.cumsum(d * A[h] * LOG2E)
+                cs = _round(cs, k32)
+                xt = np.zeros((T, P))
+                xt[:q] = x[bb, t0:t0 + q, h]
+                Bt = np.zeros((T, N))
+                Bt[:q] = B[bb, t0:t0 + q, g]
+                Ct = np.zeros((T, N))
+                Ct[:q] = C[bb, t0:t0 + q, g]
+                Bt, Ct, x16 = _round(Bt, kop), _round(Ct, kop), _round(xt, kop)
+                CB = _round(Ct @ Bt.T, k32)
+                S = _round(_mask(CB, cs, d, Dv[h], q), k16)
+                w = d * np.exp2(cs[q - 1] - cs)
+                wx = _round(w[:, None] * x16, k16)
+                s_tile = _round(Bt.T @ wx, k32)
+                Cp = _round(np.exp2(cs)[:, None] * Ct, kop)
+                Y = S @ x16 + Cp @ _round(hst, k16)
+                yt = _round(Y, "bf16") if rounding else Y
+                y[bb, t0:t0 + q, h] = yt[:q]
+                hst = _round(np.exp2(cs[q - 1]) * hst + s_tile, k32)
+            fs[bb, h] = hst
+    return y, fs
