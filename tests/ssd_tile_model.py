@@ -106,3 +106,39 @@ def tile_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, rounding=No
                 hst = _round(np.exp2(cs[q - 1]) * hst + s_tile, k32)
             fs[bb, h] = hst
     return y, fs
+
+
+def segment_split_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, segments=2):
+    """The sequence-split scheme for long sequences with few heads, in fp64.
+
+    Pass 1 runs every segment independently from a zero state (segment 0 from the
+    real initial state), giving y and each segment's final state; pass 2 chains
+    the segment states, h_in(k) = 2^(total decay of segment k-1) h_in(k-1) +
+    final(k-1); pass 3 adds 2^(cs_j) C_j h_in(k) to y of every segment k >= 1,
+    with cs_j the cumulative decay from the segment's start to token j."""
+    x, dt, B, C = (np.asarray(v, dtype=np.float64) for v in (x, dt, B, C))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    bias = np.zeros(H) if dt_bias is None else np.asarray(dt_bias, dtype=np.float64)
+    bounds = np.linspace(0, L, segments + 1).astype(int)
+    y = np.zeros((b, L, H, P))
+    h_in = np.zeros((b, H, N, P)) if init_state is None else np.asarray(init_state, np.float64).copy()
+    for k in range(segments):
+        s0, s1 = bounds[k], bounds[k + 1]
+        h0 = h_in if k == 0 else None
+        yk, fk = tile_form(x[:, s0:s1], dt[:, s0:s1], A, B[:, s0:s1], C[:, s0:s1], dt_bias, D, h0)  # pass 1
+        if k > 0:                                                                                     # pass 3
+            for bb in range(b):
+                for h in range(H):
+                    g = h // (H // G)
+                    d = _softplus(dt[bb, s0:s1, h] + bias[h])
+                    cs = np.cumsum(d * np.asarray(A, np.float64)[h] * LOG2E)
+                    yk[bb, :, h] += (np.exp2(cs)[:, None] * C[bb, s0:s1, g]) @ h_in[bb, h]
+        y[:, s0:s1] = yk
+        # pass 2: the state entering segment k + 1
+        for bb in range(b):
+            for h in range(H):
+                d = _softplus(dt[bb, s0:s1, h] + bias[h])
+                total = np.exp2(np.sum(d * np.asarray(A, np.float64)[h] * LOG2E))
+                h_in[bb, h] = fk[bb, h] + (0.0 if k == 0 else total * h_in[bb, h])
+    return y, h_in

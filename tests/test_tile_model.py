@@ -46,3 +46,14 @@ def test_kernel_roundings_stay_in_the_bf16_bound_and_bf16_operands_do_worse():
     yb, _ = tile_form(**args, rounding="bf16_operands")
     # seeded inputs: 0.0037 with the kernel's fp16 operands, 0.0134 (over the bound) with bf16 ones
     assert _rel(yb, yr) > max(1e-2, 1.5 * e16)
+
+
+def test_sequence_split_scheme_is_exact():
+    """The planned split of long sequences into segments (zero-state passes, a chain of the
+    segment states, a C h_in correction) reproduces the recurrence."""
+    from tests.ssd_tile_model import segment_split_form
+    args, yr, fr = _case("long_context", seqlen=700, nheads=2, ngroups=1)
+    for segments in (2, 3):
+        y, fs = segment_split_form(**args, segments=segments)
+        assert _rel(y, yr) < 1e-9
+        assert _rel(fs, fr) < 1e-9
