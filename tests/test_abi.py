@@ -137,3 +137,21 @@ def test_noalloc_scan_refuses_oversized_calls_on_the_host(L):
                                       v(FAKE * 120000), None, None)
     assert rc == 5
     assert "32 MiB" in L.ssd_last_error().decode()
+
+
+def test_python_wrapper_rejects_host_and_mistyped_tensors_before_any_call():
+    """The binding validates on the host and raises before reaching the library:
+    no CPU path exists, so CPU tensors are an error, as are wrong dtypes and layouts."""
+    import torch
+    import state_space_model_07_b200 as ssd
+    x = torch.zeros(1, 8, 2, 16, dtype=torch.bfloat16)
+    dt = torch.zeros(1, 8, 2, dtype=torch.bfloat16)
+    A = torch.zeros(2)
+    B = torch.zeros(1, 8, 1, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ssd.chunk_scan_fwd(x, dt, A, B, B, chunk=16)
+    with pytest.raises(TypeError):
+        ssd.chunk_scan_fwd([0], dt, A, B, B, chunk=16)
+    st = torch.zeros(1, 2, 16, 16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ssd.state_update(st, x[:, 0], dt[:, 0], A, B[:, 0], B[:, 0])
