@@ -57,3 +57,23 @@ def test_sequence_split_scheme_is_exact():
         y, fs = segment_split_form(**args, segments=segments)
         assert _rel(y, yr) < 1e-9
         assert _rel(fs, fr) < 1e-9
+
+
+def test_kernel_roundings_hold_at_dstate_256():
+    """The packed workload's sizes (N = 256, 4 groups, initial state ~ N(0, 0.1^2)) double the
+    length of every contraction over N; with the same fp16 operands the tile form stays inside
+    the bound there too (seeded: 0.0050), while bf16 thread-made operands miss it by 5x."""
+    w = inputs.scaled(inputs.WORKLOADS["packed_varlen"], nheads=8, ngroups=4)
+    d = inputs.make_inputs(w, "cpu", lengths=[400])     # one sequence: tile_form has no seq_idx
+    args = dict(x=d["x"].float().numpy(), dt=d["dt"].float().numpy(), A=d["A"].numpy(),
+                B=d["B"].float().numpy(), C=d["C"].float().numpy(), dt_bias=d["dt_bias"].numpy(),
+                D=d["D"].numpy(), init_state=d["init_state"].numpy())
+    yr, fr = oracle.ssd_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_bias=d["dt_bias"], D=d["D"],
+                             init_state=d["init_state"])
+    yr, fr = np.asarray(yr), np.asarray(fr)
+    y, fs = tile_form(**args)
+    assert _rel(y, yr) < 1e-9 and _rel(fs, fr) < 1e-9
+    y16, f16 = tile_form(**args, rounding="kernel")
+    assert _rel(y16, yr) < 1e-2 and _rel(f16, fr) < 1e-2
+    yb, _ = tile_form(**args, rounding="bf16_operands")
+    assert _rel(yb, yr) > 2e-2
