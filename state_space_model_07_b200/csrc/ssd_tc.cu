@@ -99,7 +99,7 @@ struct __align__(1024) TcSmem {
     // Every barrier's next phase depends on an action its waiters take after
     // waiting, so no waiter can ever see a barrier two phases ahead.
     uint64_t xfull[2];        // TMA x -> E, W17          (per x stage)
-    uint64_t bcfull[2];       // TMA B, C -> W16          (per B/C stage)
+    uint64_t bcfull[2];       // TMA B, C -> W16, W17     (per B/C stage)
     uint64_t scan_done[2];    // P -> E                   (per tile parity)
     uint64_t e_done[2];       // E -> P (and W17 at N = 256)  (per tile parity)
     uint64_t yd_par[2];       // W17 commit -> E, P, W16  (per tile parity)
@@ -293,6 +293,9 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             for (int t = 0; t < nt; ++t) {
                 const int st = t & 1, bst = t % C::kBCStages;
                 if (!wait_bar(ctl, &s.x_ready, t & 1, p.status)) break;
+                // C h_prev reads the C tile: its TMA load must have landed (x_ready does not
+                // imply it: E waits only for x)
+                if (!wait_bar(ctl, &s.bcfull[bst], (uint32_t)((t / C::kBCStages) & 1), p.status)) break;
                 tc_fence_after();
                 const uint32_t cb = smem_u32(s.c[bst][0]), bb = smem_u32(s.b[bst][0]);
                 const uint32_t hsb = smem_u32(s.hs), wxb = smem_u32(s.wx), xb = smem_u32(s.x[st]);

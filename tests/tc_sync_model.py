@@ -1,0 +1,550 @@
+"""A checkable model of how the tensor-core scan kernels synchronise their roles.
+
+Both kernels in ``state_space_model_07_b200/csrc/ssd_tc.cu`` split one CTA into
+warp roles that hand buffers (shared-memory stages, TMEM regions) to one another
+through mbarriers, while TMA copies and tcgen05 MMAs run asynchronously to the
+threads that issued them.  Whether that hand-off protocol is free of data races,
+deadlocks and parity aliasing is an argument about orderings, which a GPU run
+can confirm only for the schedules the hardware happened to take.  This module
+restates each role's sequence of barrier operations and buffer accesses (per
+tile, in program order, as the kernel source has them) and runs the roles
+under many random schedules, checking every one:
+
+* mbarriers follow the PTX phase rules: a phase completes when its pending
+  arrival count and its transaction count both reach zero; ``try_wait.parity``
+  passes when the phase of the given parity has completed, i.e. when the
+  number of completed phases and the parity differ in their low bit.  Each
+  wait in the model names the phase index it means; a wait that passes on any
+  other phase (a barrier two phases ahead of, or behind, its waiter) is
+  reported as aliasing.
+* async engines: each TMA load completes on its own, in any order, and then
+  counts its bytes down on its barrier; tcgen05 operations of one issuing
+  thread run in issue order, and ``tcgen05.commit`` arrives on its barrier
+  once all earlier operations of that thread are done; a TMA store's
+  shared-memory reads finish at the issuer's ``wait_group.read``.
+* happens-before is tracked with vector clocks (arrivals release, passed
+  waits acquire; an async operation inherits its issuer's clock at issue), and
+  every buffer access is checked against the conflicting accesses before it
+  (two accesses conflict when one is a write and neither happens before the
+  other).
+* at CTA exit (all roles done) no TMA copy or tensor-core operation may still
+  be in flight (the kernel frees TMEM there).
+
+A role whose warps always meet at a named barrier before each mbarrier wait
+(the kernel's leader-polls-then-``bar.sync`` waits) moves as one agent; its
+per-warp arrivals are one arrival of the role's warp count.
+"""
+from __future__ import annotations
+
+import random
+from dataclasses import dataclass, field
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+def _join(a: dict, b: dict) -> dict:
+    out = dict(a)
+    for k, v in b.items():
+        if out.get(k, 0) < v:
+            out[k] = v
+    return out
+
+
+class Barrier:
+    def __init__(self, name: str, count: int):
+        self.name, self.count = name, count
+        self.pending, self.tx, self.completed = count, 0, 0
+        self.acc: dict = {}
+        self.phase_vc: list = []
+
+    def _release(self, vc):
+        self.acc = _join(self.acc, vc)
+
+    def arrive(self, vc, weight=1, tx=0):
+        self._release(vc)
+        self.tx += tx
+        self.pending -= weight
+        if self.pending < 0:
+            raise ProtocolError(f"{self.name}: more arrivals than its count in phase {self.completed}")
+        self._maybe_complete()
+
+    def complete_tx(self, vc, nbytes=1):
+        self._release(vc)
+        self.tx -= nbytes
+        self._maybe_complete()
+
+    def _maybe_complete(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase_vc.append(self.acc)
+            self.completed += 1
+            self.pending, self.acc = self.count, {}
+
+    def try_wait(self, phase: int):
+        """(passed, vc) for a wait meant for phase index `phase` (parity phase & 1)."""
+        passed = (self.completed & 1) != (phase & 1)
+        if passed:
+            if self.completed != phase + 1:
+                raise ProtocolError(f"{self.name}: wait for phase {phase} passed with {self.completed} "
+                                    f"phases complete (parity aliasing)")
+            return True, self.phase_vc[phase]
+        if self.completed >= phase + 2:
+            raise ProtocolError(f"{self.name}: barrier ran two phases past a waiter for phase {phase}")
+        return False, None
+
+
+@dataclass
+class _Buf:
+    write: tuple | None = None                     # (component, clock, who)
+    reads: list = field(default_factory=list)
+
+
+class Machine:
+    """One CTA: barriers, buffers, role agents and async engines."""
+
+    def __init__(self):
+        self.bars: dict[str, Barrier] = {}
+        self.bufs: dict[str, _Buf] = {}
+        self.agents: dict[str, dict] = {}
+        self.tc_queues: dict[str, list] = {}       # issuer -> in-order tcgen05 ops
+        self.tc_last: dict[str, dict] = {}
+        self.bulk_queues: dict[str, list] = {}     # issuer -> in-order TMA store reads
+        self.bulk_last: dict[str, dict] = {}
+        self.tma_loads: list = []                  # independent in-flight loads
+        self.nop = 0
+
+    # ---- declarations
+    def barrier(self, name, count):
+        self.bars[name] = Barrier(name, count)
+
+    def role(self, name, gen):
+        self.agents[name] = {"gen": gen, "op": None, "done": False, "vc": {name: 1}}
+        self.tc_queues[name], self.bulk_queues[name] = [], []
+        self.tc_last[name], self.bulk_last[name] = {}, {}
+
+    # ---- accesses and happens-before
+    @staticmethod
+    def _hb(epoch, vc):
+        return vc.get(epoch[0], 0) >= epoch[1]
+
+    def _access(self, buf, kind, epoch, vc, who):
+        b = self.bufs.setdefault(buf, _Buf())
+        if b.write is not None and not self._hb(b.write, vc):
+            raise ProtocolError(f"race on {buf}: {who} {kind}s it unordered with a write by {b.write[2]}")
+        if kind == "write":
+            for r in b.reads:
+                if not self._hb(r, vc):
+                    raise ProtocolError(f"race on {buf}: {who} writes it unordered with a read by {r[2]}")
+            b.write, b.reads = epoch, []
+        else:
+            b.reads.append(epoch)
+
+    def _async_vc(self, base):
+        self.nop += 1
+        cid = ("op", self.nop)
+        vc = dict(base)
+        vc[cid] = 1
+        return vc, (cid, 1)
+
+    # ---- one step of an agent
+    def _fetch(self, a):
+        if a["op"] is None and not a["done"]:
+            try:
+                a["op"] = next(a["gen"])
+            except StopIteration:
+                a["done"] = True
+
+    def _runnable(self, name):
+        a = self.agents[name]
+        self._fetch(a)
+        if a["done"]:
+            return False
+        op = a["op"]
+        if op[0] == "wait":
+            ok, _ = self.bars[op[1]].try_wait(op[2])
+            return ok
+        if op[0] == "store_wait":
+            return not self.bulk_queues[name]
+        return True
+
+    def _tick(self, name):
+        a = self.agents[name]
+        a["vc"] = dict(a["vc"])
+        a["vc"][name] += 1
+
+    def _step_agent(self, name):
+        a = self.agents[name]
+        op, vc = a["op"], a["vc"]
+        kind = op[0]
+        if kind == "wait":
+            _, pvc = self.bars[op[1]].try_wait(op[2])
+            a["vc"] = _join(vc, pvc)
+        elif kind == "store_wait":
+            a["vc"] = _join(vc, self.bulk_last[name])
+        elif kind == "arrive":
+            self.bars[op[1]].arrive(vc, weight=op[2] if len(op) > 2 else 1)
+            self._tick(name)
+        elif kind == "arrive_tx":
+            self.bars[op[1]].arrive(vc, weight=1, tx=op[2])
+            self._tick(name)
+        elif kind in ("read", "write"):
+            for buf in op[1:]:
+                self._access(buf, kind, (name, vc[name], name), vc, name)
+        elif kind == "tma_load":
+            self.tma_loads.append((op[1], op[2], dict(vc)))
+            self._tick(name)
+        elif kind in ("mma", "commit"):
+            self.tc_queues[name].append((op, dict(vc)))
+            self._tick(name)
+        elif kind == "store":
+            self.bulk_queues[name].append((op, dict(vc)))
+            self._tick(name)
+        else:
+            raise ValueError(kind)
+        a["op"] = None
+
+    # ---- async engines
+    def _step_tma(self, i):
+        bar, buf, ivc = self.tma_loads.pop(i)
+        vc, ep = self._async_vc(ivc)
+        self._access(buf, "write", (ep[0], ep[1], f"TMA load of {buf}"), vc, f"TMA load of {buf}")
+        self.bars[bar].complete_tx(vc)
+
+    def _step_tc(self, issuer):
+        op, ivc = self.tc_queues[issuer].pop(0)
+        vc, ep = self._async_vc(_join(ivc, self.tc_last[issuer]))
+        who = f"tcgen05 op of {issuer}"
+        if op[0] == "mma":
+            reads, writes = op[1], op[2]
+            for buf in reads:
+                self._access(buf, "read", (ep[0], ep[1], who), vc, who)
+            for buf in writes:
+                self._access(buf, "write", (ep[0], ep[1], who), vc, who)
+        else:
+            self.bars[op[1]].arrive(vc)
+        self.tc_last[issuer] = vc
+
+    def _step_bulk(self, issuer):
+        op, ivc = self.bulk_queues[issuer].pop(0)
+        vc, ep = self._async_vc(_join(ivc, self.bulk_last[issuer]))
+        who = f"TMA store of {issuer}"
+        for buf in op[1]:
+            self._access(buf, "read", (ep[0], ep[1], who), vc, who)
+        self.bulk_last[issuer] = vc
+
+    # ---- schedule
+    def run(self, rng: random.Random, max_steps=1_000_000):
+        names = list(self.agents)
+        weight = {n: 10 ** rng.uniform(-2.5, 0) for n in names}
+        w_tma, w_tc, w_bulk = (10 ** rng.uniform(-2.5, 0) for _ in range(3))
+        for _ in range(max_steps):
+            choices, weights = [], []
+            for n in names:
+                if self._runnable(n):
+                    choices.append(("agent", n))
+                    weights.append(weight[n])
+            if all(a["done"] for a in self.agents.values()):
+                break                               # every role has left: the CTA frees TMEM and exits
+            for i in range(len(self.tma_loads)):
+                choices.append(("tma", i))
+                weights.append(w_tma)
+            for n, q in self.tc_queues.items():
+                if q:
+                    choices.append(("tc", n))
+                    weights.append(w_tc)
+            for n, q in self.bulk_queues.items():
+                if q:
+                    choices.append(("bulk", n))
+                    weights.append(w_bulk)
+            if not choices:
+                break
+            kind, arg = rng.choices(choices, weights)[0]
+            if kind == "agent":
+                self._step_agent(arg)
+            elif kind == "tma":
+                self._step_tma(arg)
+            elif kind == "tc":
+                self._step_tc(arg)
+            else:
+                self._step_bulk(arg)
+        else:
+            raise RuntimeError("schedule did not finish")
+        stuck = {n: a["op"] for n, a in self.agents.items() if not a["done"]}
+        if stuck:
+            raise ProtocolError(f"deadlock: {stuck}")
+        if self.tma_loads or any(self.tc_queues.values()) or any(self.bulk_queues.values()):
+            raise ProtocolError("CTA exits with TMA copies or tensor-core operations in flight")
+
+
+# ---------------------------------------------------------------------------
+# The decoupled-state kernel (k_tc_scan3, d_state 128).  `nt` tiles of 128
+# tokens; `partial` = the last tile is shorter (its y leaves by row stores,
+# not through the staging tile).  `drop` removes named protocol steps, to show
+# that the checker catches each of them.
+
+def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -> Machine:
+    m = Machine()
+    for i in range(4):
+        m.barrier(f"scan_done{i}", 1)
+        m.barrier(f"scan_free{i}", 16)
+    for i in range(2):
+        for name, count in (("full", 1), ("cb_full", 1), ("cb_free", 8), ("c_scaled", 8), ("s_ready", 8),
+                            ("x_ready", 8), ("hs_ready", 8), ("e_done", 4), ("stg_free", 1), ("s_done", 1),
+                            ("y_full", 1), ("fin", 1)):
+            m.barrier(f"{name}{i}", count)
+    full_tile = lambda u: not (partial and u == nt - 1)
+
+    def w19():      # decay scan into the four-slot ring
+        for u in range(nt):
+            sl = u & 3
+            if u >= 4 and "w19_scan_free" not in drop:
+                yield ("wait", f"scan_free{sl}", (u - 4) >> 2)
+            yield ("write", f"ring{sl}")
+            yield ("arrive", f"scan_done{sl}")
+
+    def w16():      # TMA loads of x, B, C, two stages
+        for u in range(nt):
+            st = u & 1
+            if u >= 2 and "w16_y_full" not in drop:
+                yield ("wait", f"y_full{st}", (u - 2) >> 1)
+            yield ("arrive_tx", f"full{st}", 3)
+            for buf in ("x", "b", "c"):
+                yield ("tma_load", f"full{st}", f"{buf}{st}")
+
+    def w18():      # C -> TMEM copy and C B^T
+        if nt == 0:
+            return
+        for t in range(nt):
+            st = t & 1
+            yield ("wait", f"full{st}", t >> 1)
+            if t >= 2 and "w18_y_full" not in drop:
+                yield ("wait", f"y_full{st}", (t - 2) >> 1)
+            yield ("mma", (f"c{st}",), (f"tC{st}",))                       # tcgen05.cp
+            if t >= 1 and "w18_cb_free" not in drop:
+                yield ("wait", f"cb_free{st ^ 1}", (t - 1) >> 1)
+            yield ("mma", (f"tC{st}", f"b{st}"), ("tCB",))
+            yield ("commit", f"cb_full{st}")
+        if "w18_fin" not in drop:
+            yield ("commit", "fin0")
+            yield ("wait", "fin0", 0)
+
+    def w17():      # s, C' h_prev, S x
+        if nt == 0:
+            return
+        for t in range(nt):
+            st, ph = t & 1, t >> 1
+            yield ("wait", f"x_ready{st}", ph)
+            yield ("wait", f"full{st}", ph)
+            yield ("mma", (f"b{st}", "wx"), ("tSt",))
+            yield ("commit", f"s_done{st}")
+            yield ("wait", f"hs_ready{st}", ph)
+            yield ("wait", f"c_scaled{st}", ph)
+            if t >= 2 and "w17_e_done" not in drop:
+                yield ("wait", f"e_done{st}", (t - 2) >> 1)
+            yield ("mma", (f"tC{st}", f"hs{st}"), (f"tY{st}",))
+            if "w17_s_ready" not in drop:
+                yield ("wait", f"s_ready{st}", ph)
+            yield ("mma", ("tS", f"x{st}", f"tY{st}"), (f"tY{st}",))
+            yield ("commit", f"y_full{st}")
+        if "w17_fin" not in drop:
+            yield ("commit", "fin1")
+            yield ("wait", "fin1", 0)
+
+    def p_role():   # C' scaling and the decay mask S
+        yield ("write", "tS")                       # blocks right of the diagonal, zeroed once
+        for t in range(nt):
+            st, sl = t & 1, t & 3
+            yield ("wait", f"scan_done{sl}", t >> 2)
+            yield ("wait", f"cb_full{st}", t >> 1)
+            yield ("read", f"ring{sl}", f"tC{st}")
+            yield ("write", f"tC{st}")
+            yield ("arrive", f"c_scaled{st}", 8)
+            yield ("read", "tCB", f"ring{sl}")
+            yield ("arrive", f"cb_free{st}", 8)
+            yield ("arrive", f"scan_free{sl}", 8)
+            if t > 0 and "p_y_full" not in drop:
+                yield ("wait", f"y_full{st ^ 1}", (t - 1) >> 1)
+            yield ("write", "tS")
+            yield ("arrive", f"s_ready{st}", 8)
+
+    def y_role():   # epilogue and TMA store of y
+        stored = False
+        for u in range(nt):
+            st = u & 1
+            yield ("wait", f"y_full{st}", u >> 1)
+            yield ("read", f"tY{st}")
+            if full_tile(u):
+                yield ("write", f"hs{st}")
+            yield ("arrive", f"e_done{st}", 4)
+            if full_tile(u):
+                yield ("write", f"hs{st}")
+                yield ("store", (f"hs{st}",))
+                if "y_store_wait" not in drop:
+                    yield ("store_wait",)
+                stored = True
+            yield ("arrive", f"stg_free{st}")
+        if stored:
+            yield ("store_wait",)
+
+    def e_role():   # x operands and the fp32 state
+        if nt > 0:
+            yield ("write", "hs0")
+            yield ("arrive", "hs_ready0", 8)
+        for k in range(nt + 1):
+            if k >= 1:
+                u = k - 1
+                yield ("wait", f"s_done{u & 1}", u >> 1)
+                if 2 <= k < nt and "e_stg_free" not in drop:
+                    yield ("wait", f"stg_free{k & 1}", (k - 2) >> 1)
+                yield ("read", "tSt")
+                if k < nt:
+                    yield ("write", f"hs{k & 1}")
+                    yield ("arrive", f"hs_ready{k & 1}", 8)
+            if k < nt:
+                yield ("wait", f"scan_done{k & 3}", k >> 2)
+                yield ("wait", f"full{k & 1}", k >> 1)
+                yield ("read", f"ring{k & 3}")
+                yield ("arrive", f"scan_free{k & 3}", 8)
+                yield ("read", f"x{k & 1}")
+                yield ("write", f"x{k & 1}", "wx")
+                yield ("arrive", f"x_ready{k & 1}", 8)
+
+    for name, gen in (("W19", w19()), ("W16", w16()), ("W18", w18()), ("W17", w17()), ("P", p_role()),
+                      ("Y", y_role()), ("E", e_role())):
+        m.role(name, gen)
+    return m
+
+
+# ---------------------------------------------------------------------------
+# The first-generation kernel (k_tc_scan<N>): state accumulated in TMEM.
+# n = 128: B/C double-buffered, two Yd buffers; n = 256: one B/C stage (its
+# reload waits for the tile's C h_prev and B^T (w o x)), one Yd buffer (its
+# S x waits for the previous epilogue).
+
+def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = frozenset()) -> Machine:
+    bc_stages = 2 if n == 128 else 1
+    yd_bufs = 2 if n == 128 else 1
+    m = Machine()
+    for i in range(2):
+        m.barrier(f"xfull{i}", 1)
+        m.barrier(f"bcfull{i}", 1)
+        m.barrier(f"scan_done{i}", 8)
+        m.barrier(f"e_done{i}", 8)
+        m.barrier(f"yd_par{i}", 1)
+    for name, count in (("cb_done", 1), ("s_ready", 8), ("x_ready", 8), ("sc_done", 1)):
+        m.barrier(name, count)
+    last_partial = lambda t: partial and t == nt - 1
+
+    def w16():      # TMA and C B^T
+        if nt == 0:
+            return
+
+        def load_x(t):
+            yield ("arrive_tx", f"xfull{t & 1}", 1)
+            yield ("tma_load", f"xfull{t & 1}", f"x{t & 1}")
+
+        def load_bc(t):
+            st = t % bc_stages
+            yield ("arrive_tx", f"bcfull{st}", 2)
+            yield ("tma_load", f"bcfull{st}", f"b{st}")
+            yield ("tma_load", f"bcfull{st}", f"c{st}")
+
+        yield from load_x(0)
+        yield from load_bc(0)
+        if nt > 1:
+            yield from load_x(1)
+            if bc_stages == 2:
+                yield from load_bc(1)
+        for t in range(nt):
+            bst = t % bc_stages
+            yield ("wait", f"bcfull{bst}", t // bc_stages)
+            if t > 0 and "w16_s_ready" not in drop:
+                yield ("wait", "s_ready", t - 1)
+            yield ("mma", (f"c{bst}", f"b{bst}"), ("tCB",))
+            yield ("commit", "cb_done")
+            if t >= 1 and t + 1 < nt:
+                if "w16_yd_par" not in drop:
+                    yield ("wait", f"yd_par{(t - 1) & 1}", (t - 1) >> 1)
+                yield from load_x(t + 1)
+                if bc_stages == 2:
+                    yield from load_bc(t + 1)
+            if bc_stages == 1 and t + 1 < nt:
+                if "w16_sc_done" not in drop:
+                    yield ("wait", "sc_done", t)
+                yield from load_bc(t + 1)
+        # the kernel's W16 has no drain of its own: every tcgen05 op it issued is
+        # waited on by P (cb_done) before the CTA can finish
+
+    def w17():
+        for t in range(nt):
+            st, bst = t & 1, t % bc_stages
+            yield ("wait", "x_ready", t)
+            if "w17_bcfull" not in drop:
+                yield ("wait", f"bcfull{bst}", t // bc_stages)
+            yield ("mma", (f"c{bst}", "hs"), (f"tYo{st}",))
+            yield ("wait", "s_ready", t)
+            yield ("mma", (f"b{bst}", "wx", "tH"), ("tH",))
+            yield ("commit", "sc_done")
+            if yd_bufs == 1 and t > 0 and "w17_e_done" not in drop:
+                yield ("wait", f"e_done{(t - 1) & 1}", (t - 1) >> 1)
+            yd = f"tYd{st if yd_bufs == 2 else 0}"
+            yield ("mma", ("tS", f"x{st}"), (yd,))
+            yield ("commit", f"yd_par{st}")
+
+    def p_role():
+        yield ("write", "tS")
+        for t in range(nt):
+            buf, bst = t & 1, t % bc_stages
+            if t >= 2 and "p_e_done" not in drop:
+                yield ("wait", f"e_done{buf}", (t - 2) >> 1)
+            yield ("write", f"ring{buf}")
+            yield ("arrive", f"scan_done{buf}", 8)
+            yield ("wait", "cb_done", t)
+            if last_partial(t):
+                yield ("write", f"b{bst}")          # rows past the sequence end zeroed
+            if t > 0 and "p_yd_par" not in drop:
+                yield ("wait", f"yd_par{(t - 1) & 1}", (t - 1) >> 1)
+            yield ("read", "tCB", f"ring{buf}")
+            yield ("write", "tS")
+            yield ("arrive", "s_ready", 8)
+
+    def e_role():
+        def prepare(u):
+            st = u & 1
+            yield ("wait", f"scan_done{st}", u >> 1)
+            yield ("read", f"ring{st}")
+            if u > 0:
+                yield ("read", "tH")
+            yield ("write", "hs", "tH")
+            yield ("wait", f"xfull{st}", u >> 1)
+            yield ("read", f"x{st}")
+            yield ("write", f"x{st}", "wx")
+            yield ("arrive", "x_ready", 8)
+
+        for k in range(nt + 1):
+            if k < nt:
+                if k > 0 and "e_sc_done" not in drop:
+                    yield ("wait", "sc_done", k - 1)
+                yield from prepare(k)
+            if k == 0:
+                continue
+            t = k - 1
+            st = t & 1
+            yield ("wait", f"yd_par{st}", t >> 1)
+            yield ("read", f"ring{st}", f"tYd{st if yd_bufs == 2 else 0}", f"tYo{st}")
+            yield ("arrive", f"e_done{st}", 8)
+        if nt > 0:
+            yield ("read", "tH")
+
+    for name, gen in (("W16", w16()), ("W17", w17()), ("P", p_role()), ("E", e_role())):
+        m.role(name, gen)
+    return m
+
+
+def check(build, schedules: int, seed: int, **kw) -> None:
+    """Runs `schedules` random schedules of the model `build(**kw)`; raises ProtocolError on the first
+    race, deadlock, aliasing or exit with work in flight."""
+    rng = random.Random(seed)
+    for _ in range(schedules):
+        build(**kw).run(rng)

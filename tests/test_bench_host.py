@@ -44,3 +44,22 @@ def test_algorithmic_bytes_of_the_bench_workload():
     # x + y (80 heads x 64 x 2 B each), dt (80 x 2 B), B + C (128 x 2 B each) per token, plus the final state
     per_tok = 2 * 80 * 64 * 2 + 80 * 2 + 2 * 128 * 2
     assert bench.workload_bytes(w, w.batch, tokens, 2) == tokens * per_tok + 8 * 80 * 128 * 64 * 4 == 714080256
+
+
+def test_scan_hash_covers_the_measured_kernel_not_the_d_state_256_one(tmp_path, monkeypatch):
+    src = open(bench.os.path.join(bench.ROOT, "state_space_model_07_b200", "csrc", "ssd_tc.cu")).read()
+    csrc = tmp_path / "state_space_model_07_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    f = csrc / "ssd_tc.cu"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f.write_text(src)
+    h0 = bench.kernel_source_sha("tc_scan")
+    # an edit inside the first-generation k_tc_scan<N> (another kernel) keeps the hash ...
+    sig = "k_tc_scan(const __grid_constant__"
+    i = src.index("{", src.index(sig))
+    f.write_text(src[:i + 1] + "\n    int unused_probe = 0;\n" + src[i + 1:])
+    assert bench.kernel_source_sha("tc_scan") == h0
+    # ... one inside k_tc_scan3 does not
+    j = src.index("{", src.index("k_tc_scan3(const __grid_constant__"))
+    f.write_text(src[:j + 1] + "\n    int unused_probe = 0;\n" + src[j + 1:])
+    assert bench.kernel_source_sha("tc_scan") != h0

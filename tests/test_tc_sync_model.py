@@ -1,0 +1,171 @@
+"""The role hand-off protocol of the tensor-core scan kernels, model-checked on the CPU.
+
+``tests/tc_sync_model.py`` restates, per role and tile, the mbarrier waits, arrivals,
+buffer accesses and async copies / MMAs of ``k_tc_scan3`` (d_state 128) and of the
+first-generation ``k_tc_scan<N>`` (d_state 256, and its 128 configuration), and runs
+them under random schedules with vector-clock race detection.  The tests check that
+the protocol has no race, deadlock or parity aliasing for 0 .. 9 tiles (full and
+ragged last tile), and that removing any wait the protocol needs is caught.
+"""
+import random
+
+import pytest
+
+from tests.tc_sync_model import Barrier, Machine, ProtocolError, build_scan1, build_scan3, check
+
+TILES = (0, 1, 2, 3, 4, 5, 6, 9)
+
+
+# ---- the checker itself -------------------------------------------------------------
+
+
+def test_barrier_parity_and_transaction_rules():
+    b = Barrier("b", 2)
+    assert b.try_wait(0) == (False, None)
+    b.arrive({"a": 1}, tx=3)
+    b.arrive({"c": 1})
+    assert not b.try_wait(0)[0]             # arrivals done, bytes outstanding
+    b.complete_tx({"tma": 1}, 3)
+    ok, vc = b.try_wait(0)
+    assert ok and vc == {"a": 1, "c": 1, "tma": 1}
+    b.arrive({}, weight=2)                  # phase 1 completes: a waiter for phase 0 now sees parity 0 again
+    with pytest.raises(ProtocolError, match="two phases past"):
+        b.try_wait(0)
+    b2 = Barrier("b2", 1)
+    b2.arrive({})
+    with pytest.raises(ProtocolError, match="aliasing"):
+        b2.try_wait(2)                      # a waiter two phases ahead would pass on phase 0
+    with pytest.raises(ProtocolError, match="more arrivals"):
+        Barrier("b3", 1).arrive({}, weight=2)
+
+
+def _two_roles(ordered):
+    m = Machine()
+    m.barrier("ready", 1)
+
+    def producer():
+        yield ("write", "buf")
+        yield ("arrive", "ready")
+
+    def consumer():
+        if ordered:
+            yield ("wait", "ready", 0)
+        yield ("read", "buf")
+
+    m.role("prod", producer())
+    m.role("cons", consumer())
+    return m
+
+
+def test_race_detector_needs_the_barrier_and_accepts_it():
+    found = False
+    rng = random.Random(0)
+    for _ in range(50):
+        _two_roles(True).run(rng)
+        try:
+            _two_roles(False).run(rng)
+        except ProtocolError as e:
+            found = found or "race on buf" in str(e)
+    assert found
+
+
+def test_async_mma_is_ordered_only_through_its_commit():
+    def build(wait_commit):
+        m = Machine()
+        m.barrier("done", 1)
+
+        def issuer():
+            yield ("mma", ("a",), ("acc",))
+            yield ("commit", "done")
+
+        def reader():
+            if wait_commit:
+                yield ("wait", "done", 0)
+            yield ("read", "acc")
+
+        m.role("W", issuer())
+        m.role("R", reader())
+        return m
+
+    rng = random.Random(1)
+    for _ in range(50):
+        build(True).run(rng)
+    with pytest.raises(ProtocolError):
+        for _ in range(200):
+            build(False).run(rng)
+
+
+def test_exit_with_work_in_flight_is_reported():
+    m = Machine()
+
+    def issuer():
+        yield ("mma", (), ("acc",))           # issued, never committed and waited for
+
+    m.role("W", issuer())
+    with pytest.raises(ProtocolError, match="in flight"):
+        m.run(random.Random(0))
+
+
+# ---- the kernels ----------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("partial", [False, True])
+def test_scan3_protocol_has_no_race_deadlock_or_aliasing(partial):
+    for nt in TILES:
+        check(build_scan3, 25, seed=100 + nt, nt=nt, partial=partial)
+
+
+@pytest.mark.parametrize("n", [128, 256])
+@pytest.mark.parametrize("partial", [False, True])
+def test_scan1_protocol_has_no_race_deadlock_or_aliasing(n, partial):
+    for nt in TILES:
+        check(build_scan1, 25, seed=200 + nt, nt=nt, n=n, partial=partial)
+
+
+def _caught(build, drop, **kw):
+    for nt in (3, 5, 8):
+        for partial in (False, True):
+            try:
+                check(build, 40, seed=nt, nt=nt, partial=partial, drop=frozenset([drop]), **kw)
+            except ProtocolError as e:
+                return str(e)
+    return None
+
+
+NEEDED = [
+    (build_scan3, {}, "w19_scan_free", "ring"),
+    (build_scan3, {}, "w16_y_full", "x0"),
+    (build_scan3, {}, "w18_cb_free", "tCB"),
+    (build_scan3, {}, "w17_s_ready", "tS"),
+    (build_scan3, {}, "p_y_full", "tS"),
+    (build_scan3, {}, "y_store_wait", "hs"),
+    (build_scan3, {}, "e_stg_free", "hs"),
+    (build_scan1, {"n": 128}, "w16_s_ready", "tCB"),
+    (build_scan1, {"n": 128}, "w16_yd_par", "x"),
+    (build_scan1, {"n": 256}, "w16_sc_done", "b0"),
+    (build_scan1, {"n": 256}, "w17_e_done", "tYd0"),
+    (build_scan1, {"n": 128}, "w17_bcfull", "c0"),
+    (build_scan1, {"n": 256}, "w17_bcfull", "c0"),
+    (build_scan1, {"n": 256}, "p_e_done", "ring"),
+    (build_scan1, {"n": 256}, "p_yd_par", "tS"),
+    (build_scan1, {"n": 256}, "e_sc_done", ""),
+]
+
+
+@pytest.mark.parametrize("build,kw,drop,buf", NEEDED, ids=[f"{b.__name__}-{kw.get('n', 128)}-{d}" for b, kw, d, _ in NEEDED])
+def test_removing_a_needed_wait_is_caught(build, kw, drop, buf):
+    msg = _caught(build, drop, **kw)
+    assert msg is not None and "race on " + buf in msg, msg
+
+
+def test_waits_implied_by_other_waits():
+    """Waits the kernels keep although another wait already implies them:
+    k_tc_scan3's W18 y_full wait (its full-barrier wait follows W16's y_full wait), W17's
+    e_done wait (hs_ready follows E's stg_free wait, which follows Y's read of the Y buffer),
+    and, with one B/C stage, the first-generation W16's s_ready wait (the stage's reload
+    waited for sc_done, which follows s_ready).  The tensor-core drains before exit (fin)
+    matter only on the timeout path, which the model does not take."""
+    for build, kw, drop in ((build_scan3, {}, "w18_y_full"), (build_scan3, {}, "w17_e_done"),
+                            (build_scan3, {}, "w17_fin"), (build_scan3, {}, "w18_fin"),
+                            (build_scan1, {"n": 256}, "w16_s_ready")):
+        assert _caught(build, drop, **kw) is None, drop
