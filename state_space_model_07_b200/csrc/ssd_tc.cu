@@ -624,7 +624,9 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 //   * The state recurrence runs on the E warps in fp32 registers,
 //     h <- 2^cs_last h + s, with s = B^T (w o x) the tile's own contribution
 //     from the tensor core; only an fp16 copy of h goes to shared memory.
-// Per 128-token tile that is ~290 KB of shared-memory traffic.
+// Per 128-token tile that is ~320 KB of shared-memory traffic (TMA writes of
+// x, B, C 80 KB; tcgen05.cp of C 32 KB; MMA operand reads 112 KB; the E
+// warps 64 KB; y staging and its TMA store 32 KB), ~2.5 k cycles at 128 B/clk.
 //
 // No role thread keeps a global load in flight across an mbarrier arrival
 // (an arrival is a release, which waits for the thread's outstanding loads):
