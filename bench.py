@@ -273,11 +273,12 @@ def config_of(w):
     return c
 
 
-# Definitions in a source file that compile to kernels other than the one a
+# Definitions in a source file that belong only to kernels other than the one a
 # capture measured: removed before hashing.  ssd_tc.cu also holds the
-# first-generation k_tc_scan<N> (the d_state 256 kernel), which shares no code
-# generation with the measured k_tc_scan3 beyond the helpers outside it.
-_NOT_MEASURED = {"tc_scan": ("template <int N>", "k_tc_scan(const __grid_constant__")}
+# first-generation k_tc_scan<N> (the d_state 256 kernel) and its shared-memory
+# layout TcSmem<N>, neither of which the measured k_tc_scan3 uses.
+_NOT_MEASURED = {"tc_scan": (("template <int N>", "k_tc_scan(const __grid_constant__"),
+                             ("template <int N>", "struct __align__(1024) TcSmem {"))}
 
 
 def _drop_definition(code, head, signature):
@@ -310,8 +311,8 @@ def kernel_source_sha(name):
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     text = re.sub(r"//[^\n]*", "", text)
     code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
-    if name in _NOT_MEASURED:
-        code = _drop_definition(code, *_NOT_MEASURED[name])
+    for head, signature in _NOT_MEASURED.get(name, ()):
+        code = _drop_definition(code, head, signature)
     return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 

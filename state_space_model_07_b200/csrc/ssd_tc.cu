@@ -107,6 +107,7 @@ struct __align__(1024) TcSmem {
     uint64_t s_ready;         // P -> W16, W17
     uint64_t x_ready;         // E -> W17
     uint64_t sc_done;         // W17 commit -> E (and W16 at N = 256)
+    uint64_t fin[2];          // W16, W17: own tcgen05 work drained before exit
     uint32_t tmem_base;
     TcCtl ctl;
 };
@@ -205,6 +206,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             mbar_init(&s.scan_done[i], kRoleThreads);
             mbar_init(&s.e_done[i], kRoleThreads);
             mbar_init(&s.yd_par[i], 1);
+            mbar_init(&s.fin[i], 1);
         }
         mbar_init(&s.cb_done, 1);
         mbar_init(&s.s_ready, kRoleThreads);
@@ -284,6 +286,10 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 for (int t = 0; t < bc_issued; ++t)
                     mbar_wait(&s.bcfull[t % C::kBCStages], (t / C::kBCStages) & 1, 400000000ll);
             }
+            // every C B^T issued has completed before TMEM is freed (on a timeout nobody else
+            // waits for the last ones)
+            mma_commit(&s.fin[0]);
+            mbar_wait(&s.fin[0], 0, 400000000ll);
         }
     } else if (warp == 17) {
         // ----------------------------------- W17: C h_prev, B^T (w o x), S x
@@ -324,6 +330,10 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 for (int k = 0; k < kT / 16; ++k)
                     mma_ts(yd, tmem + C::kColS + k * 8, sdesc_sw128(xb + k * 2048, kBoxBytes, 1024), id_pn, k > 0);
                 mma_commit(&s.yd_par[st]);
+            }
+            if (nt > 0) {
+                mma_commit(&s.fin[1]);
+                mbar_wait(&s.fin[1], 0, 400000000ll);
             }
         }
     } else if (warp < 8) {

@@ -29,6 +29,12 @@ under many random schedules, checking every one:
   other).
 * at CTA exit (all roles done) no TMA copy or tensor-core operation may still
   be in flight (the kernel frees TMEM there).
+* the timeout path: a run may time out one waiting role at a random step.
+  Every copy and MMA issued before then completes first, since a timeout
+  takes hundreds of milliseconds.  The CTA then gives up: later waits fail at
+  once, as the kernel's wait_bar does when the abort flag is set, and each
+  role leaves its loop the way the kernel does.  From there on only deadlock
+  and exit with work in flight are checked.
 
 A role whose warps always meet at a named barrier before each mbarrier wait
 (the kernel's leader-polls-then-``bar.sync`` waits) moves as one agent; its
@@ -81,9 +87,13 @@ class Barrier:
             self.completed += 1
             self.pending, self.acc = self.count, {}
 
-    def try_wait(self, phase: int):
-        """(passed, vc) for a wait meant for phase index `phase` (parity phase & 1)."""
+    def try_wait(self, phase: int, strict: bool = True):
+        """(passed, vc) for a wait meant for phase index `phase` (parity phase & 1).  A strict
+        wait (the protocol's own) must pass on exactly that phase; a drain on the timeout path
+        only asks whether the parity has flipped."""
         passed = (self.completed & 1) != (phase & 1)
+        if not strict:
+            return passed, (self.phase_vc[-1] if passed else None)
         if passed:
             if self.completed != phase + 1:
                 raise ProtocolError(f"{self.name}: wait for phase {phase} passed with {self.completed} "
@@ -113,13 +123,15 @@ class Machine:
         self.bulk_last: dict[str, dict] = {}
         self.tma_loads: list = []                  # independent in-flight loads
         self.nop = 0
+        self.abort = False                         # a bounded wait has timed out
+        self.races = True                          # race checks (off once the CTA is giving up)
 
     # ---- declarations
     def barrier(self, name, count):
         self.bars[name] = Barrier(name, count)
 
     def role(self, name, gen):
-        self.agents[name] = {"gen": gen, "op": None, "done": False, "vc": {name: 1}}
+        self.agents[name] = {"gen": gen, "op": None, "done": False, "vc": {name: 1}, "send": None}
         self.tc_queues[name], self.bulk_queues[name] = [], []
         self.tc_last[name], self.bulk_last[name] = {}, {}
 
@@ -129,6 +141,8 @@ class Machine:
         return vc.get(epoch[0], 0) >= epoch[1]
 
     def _access(self, buf, kind, epoch, vc, who):
+        if not self.races:
+            return
         b = self.bufs.setdefault(buf, _Buf())
         if b.write is not None and not self._hb(b.write, vc):
             raise ProtocolError(f"race on {buf}: {who} {kind}s it unordered with a write by {b.write[2]}")
@@ -151,9 +165,15 @@ class Machine:
     def _fetch(self, a):
         if a["op"] is None and not a["done"]:
             try:
-                a["op"] = next(a["gen"])
+                a["op"] = a["gen"].send(a["send"])
             except StopIteration:
                 a["done"] = True
+            a["send"] = None
+
+    def _progress_possible(self, bar):
+        """Whether async work in flight can still complete a phase of `bar`."""
+        return (any(ld[0] == bar for ld in self.tma_loads)
+                or any(op[0] == "commit" and op[1] == bar for q in self.tc_queues.values() for op, _ in q))
 
     def _runnable(self, name):
         a = self.agents[name]
@@ -162,10 +182,39 @@ class Machine:
             return False
         op = a["op"]
         if op[0] == "wait":
-            ok, _ = self.bars[op[1]].try_wait(op[2])
-            return ok
+            # the kernel's wait_bar gives up at once when the CTA is aborting
+            return self.abort or self.bars[op[1]].try_wait(op[2])[0]
+        if op[0] == "bwait":
+            # a bounded wait that ignores the abort flag: passes on the parity, or times out
+            # once nothing in flight can complete the phase
+            return self.bars[op[1]].try_wait(op[2], strict=False)[0] or not self._progress_possible(op[1])
         if op[0] == "store_wait":
             return not self.bulk_queues[name]
+        return True
+
+    def _drain_async(self):
+        """A timeout takes hundreds of milliseconds, which every copy and MMA issued before it
+        outlasts: they all complete first."""
+        while self.tma_loads:
+            self._step_tma(0)
+        for n in self.tc_queues:
+            while self.tc_queues[n]:
+                self._step_tc(n)
+        for n in self.bulk_queues:
+            while self.bulk_queues[n]:
+                self._step_bulk(n)
+
+    def _fault(self, rng):
+        """Times out one role that is waiting; the CTA starts giving up."""
+        waiting = [n for n, a in self.agents.items() if not a["done"] and a["op"] is not None
+                   and a["op"][0] == "wait"]
+        if not waiting:
+            return False
+        self._drain_async()
+        name = rng.choice(waiting)
+        self.abort, self.races = True, False
+        a = self.agents[name]
+        a["op"], a["send"] = None, False
         return True
 
     def _tick(self, name):
@@ -178,8 +227,17 @@ class Machine:
         op, vc = a["op"], a["vc"]
         kind = op[0]
         if kind == "wait":
-            _, pvc = self.bars[op[1]].try_wait(op[2])
-            a["vc"] = _join(vc, pvc)
+            ok, pvc = self.bars[op[1]].try_wait(op[2], strict=not self.abort)
+            if self.abort:
+                ok = False           # wait_bar checks the abort flag before it polls
+            if ok:
+                a["vc"] = _join(vc, pvc)
+            a["send"] = ok
+        elif kind == "bwait":
+            ok, pvc = self.bars[op[1]].try_wait(op[2], strict=False)
+            if ok:
+                a["vc"] = _join(vc, pvc)
+            a["send"] = ok
         elif kind == "store_wait":
             a["vc"] = _join(vc, self.bulk_last[name])
         elif kind == "arrive":
@@ -234,11 +292,17 @@ class Machine:
         self.bulk_last[issuer] = vc
 
     # ---- schedule
-    def run(self, rng: random.Random, max_steps=1_000_000):
+    def run(self, rng: random.Random, max_steps=1_000_000, fault_at=None):
+        """One random schedule.  `fault_at`: the step at which a waiting role times out (the
+        first step from there on at which some role waits), None for none."""
         names = list(self.agents)
         weight = {n: 10 ** rng.uniform(-2.5, 0) for n in names}
         w_tma, w_tc, w_bulk = (10 ** rng.uniform(-2.5, 0) for _ in range(3))
-        for _ in range(max_steps):
+        for step in range(max_steps):
+            if fault_at is not None and step >= fault_at and not self.abort:
+                for n in names:
+                    self._fetch(self.agents[n])
+                self._fault(rng)
             choices, weights = [], []
             for n in names:
                 if self._runnable(n):
@@ -278,10 +342,16 @@ class Machine:
 
 
 # ---------------------------------------------------------------------------
+# Role scripts.  Each yields the operations of one role in program order; a
+# wait evaluates to True when it passed and False when it gave up (the
+# kernel's bounded waits), after which the role leaves its loop as the kernel
+# does.  `drop` removes named protocol steps, to show that the checker
+# catches each of them.
+
+
 # The decoupled-state kernel (k_tc_scan3, d_state 128).  `nt` tiles of 128
 # tokens; `partial` = the last tile is shorter (its y leaves by row stores,
-# not through the staging tile).  `drop` removes named protocol steps, to show
-# that the checker catches each of them.
+# not through the staging tile).
 
 def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -> Machine:
     m = Machine()
@@ -299,64 +369,77 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -
         for u in range(nt):
             sl = u & 3
             if u >= 4 and "w19_scan_free" not in drop:
-                yield ("wait", f"scan_free{sl}", (u - 4) >> 2)
+                if not (yield ("wait", f"scan_free{sl}", (u - 4) >> 2)):
+                    break
             yield ("write", f"ring{sl}")
             yield ("arrive", f"scan_done{sl}")
 
     def w16():      # TMA loads of x, B, C, two stages
+        issued = 0
         for u in range(nt):
             st = u & 1
             if u >= 2 and "w16_y_full" not in drop:
-                yield ("wait", f"y_full{st}", (u - 2) >> 1)
+                if not (yield ("wait", f"y_full{st}", (u - 2) >> 1)):
+                    break
             yield ("arrive_tx", f"full{st}", 3)
             for buf in ("x", "b", "c"):
                 yield ("tma_load", f"full{st}", f"{buf}{st}")
+            issued += 1
+        if m.abort and "w16_drain" not in drop:
+            # let the copies in flight land before the CTA exits
+            for u in range(issued):
+                yield ("bwait", f"full{u & 1}", u >> 1)
 
     def w18():      # C -> TMEM copy and C B^T
         if nt == 0:
             return
         for t in range(nt):
             st = t & 1
-            yield ("wait", f"full{st}", t >> 1)
+            if not (yield ("wait", f"full{st}", t >> 1)):
+                break
             if t >= 2 and "w18_y_full" not in drop:
-                yield ("wait", f"y_full{st}", (t - 2) >> 1)
+                if not (yield ("wait", f"y_full{st}", (t - 2) >> 1)):
+                    break
             yield ("mma", (f"c{st}",), (f"tC{st}",))                       # tcgen05.cp
             if t >= 1 and "w18_cb_free" not in drop:
-                yield ("wait", f"cb_free{st ^ 1}", (t - 1) >> 1)
+                if not (yield ("wait", f"cb_free{st ^ 1}", (t - 1) >> 1)):
+                    break
             yield ("mma", (f"tC{st}", f"b{st}"), ("tCB",))
             yield ("commit", f"cb_full{st}")
         if "w18_fin" not in drop:
             yield ("commit", "fin0")
-            yield ("wait", "fin0", 0)
+            yield ("bwait", "fin0", 0)
 
     def w17():      # s, C' h_prev, S x
         if nt == 0:
             return
         for t in range(nt):
             st, ph = t & 1, t >> 1
-            yield ("wait", f"x_ready{st}", ph)
-            yield ("wait", f"full{st}", ph)
+            if not (yield ("wait", f"x_ready{st}", ph)) or not (yield ("wait", f"full{st}", ph)):
+                break
             yield ("mma", (f"b{st}", "wx"), ("tSt",))
             yield ("commit", f"s_done{st}")
-            yield ("wait", f"hs_ready{st}", ph)
-            yield ("wait", f"c_scaled{st}", ph)
+            if not (yield ("wait", f"hs_ready{st}", ph)) or not (yield ("wait", f"c_scaled{st}", ph)):
+                break
             if t >= 2 and "w17_e_done" not in drop:
-                yield ("wait", f"e_done{st}", (t - 2) >> 1)
+                if not (yield ("wait", f"e_done{st}", (t - 2) >> 1)):
+                    break
             yield ("mma", (f"tC{st}", f"hs{st}"), (f"tY{st}",))
             if "w17_s_ready" not in drop:
-                yield ("wait", f"s_ready{st}", ph)
+                if not (yield ("wait", f"s_ready{st}", ph)):
+                    break
             yield ("mma", ("tS", f"x{st}", f"tY{st}"), (f"tY{st}",))
             yield ("commit", f"y_full{st}")
         if "w17_fin" not in drop:
             yield ("commit", "fin1")
-            yield ("wait", "fin1", 0)
+            yield ("bwait", "fin1", 0)
 
     def p_role():   # C' scaling and the decay mask S
         yield ("write", "tS")                       # blocks right of the diagonal, zeroed once
         for t in range(nt):
             st, sl = t & 1, t & 3
-            yield ("wait", f"scan_done{sl}", t >> 2)
-            yield ("wait", f"cb_full{st}", t >> 1)
+            if not (yield ("wait", f"scan_done{sl}", t >> 2)) or not (yield ("wait", f"cb_full{st}", t >> 1)):
+                break
             yield ("read", f"ring{sl}", f"tC{st}")
             yield ("write", f"tC{st}")
             yield ("arrive", f"c_scaled{st}", 8)
@@ -364,7 +447,8 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -
             yield ("arrive", f"cb_free{st}", 8)
             yield ("arrive", f"scan_free{sl}", 8)
             if t > 0 and "p_y_full" not in drop:
-                yield ("wait", f"y_full{st ^ 1}", (t - 1) >> 1)
+                if not (yield ("wait", f"y_full{st ^ 1}", (t - 1) >> 1)):
+                    break
             yield ("write", "tS")
             yield ("arrive", f"s_ready{st}", 8)
 
@@ -372,7 +456,8 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -
         stored = False
         for u in range(nt):
             st = u & 1
-            yield ("wait", f"y_full{st}", u >> 1)
+            if not (yield ("wait", f"y_full{st}", u >> 1)):
+                break
             yield ("read", f"tY{st}")
             if full_tile(u):
                 yield ("write", f"hs{st}")
@@ -394,16 +479,18 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -
         for k in range(nt + 1):
             if k >= 1:
                 u = k - 1
-                yield ("wait", f"s_done{u & 1}", u >> 1)
+                if not (yield ("wait", f"s_done{u & 1}", u >> 1)):
+                    break
                 if 2 <= k < nt and "e_stg_free" not in drop:
-                    yield ("wait", f"stg_free{k & 1}", (k - 2) >> 1)
+                    if not (yield ("wait", f"stg_free{k & 1}", (k - 2) >> 1)):
+                        break
                 yield ("read", "tSt")
                 if k < nt:
                     yield ("write", f"hs{k & 1}")
                     yield ("arrive", f"hs_ready{k & 1}", 8)
             if k < nt:
-                yield ("wait", f"scan_done{k & 3}", k >> 2)
-                yield ("wait", f"full{k & 1}", k >> 1)
+                if not (yield ("wait", f"scan_done{k & 3}", k >> 2)) or not (yield ("wait", f"full{k & 1}", k >> 1)):
+                    break
                 yield ("read", f"ring{k & 3}")
                 yield ("arrive", f"scan_free{k & 3}", 8)
                 yield ("read", f"x{k & 1}")
@@ -416,13 +503,14 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -
     return m
 
 
-# ---------------------------------------------------------------------------
 # The first-generation kernel (k_tc_scan<N>): state accumulated in TMEM.
 # n = 128: B/C double-buffered, two Yd buffers; n = 256: one B/C stage (its
 # reload waits for the tile's C h_prev and B^T (w o x)), one Yd buffer (its
-# S x waits for the previous epilogue).
+# S x waits for the previous epilogue).  `fin`: the two MMA-issuing threads
+# drain their tensor-core work before the CTA exits.
 
-def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = frozenset()) -> Machine:
+def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = frozenset(),
+                fin: bool = True) -> Machine:
     bc_stages = 2 if n == 128 else 1
     yd_bufs = 2 if n == 128 else 1
     m = Machine()
@@ -432,6 +520,7 @@ def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = 
         m.barrier(f"scan_done{i}", 8)
         m.barrier(f"e_done{i}", 8)
         m.barrier(f"yd_par{i}", 1)
+        m.barrier(f"fin{i}", 1)
     for name, count in (("cb_done", 1), ("s_ready", 8), ("x_ready", 8), ("sc_done", 1)):
         m.barrier(name, count)
     last_partial = lambda t: partial and t == nt - 1
@@ -439,16 +528,19 @@ def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = 
     def w16():      # TMA and C B^T
         if nt == 0:
             return
+        issued = {"x": 0, "bc": 0}
 
         def load_x(t):
             yield ("arrive_tx", f"xfull{t & 1}", 1)
             yield ("tma_load", f"xfull{t & 1}", f"x{t & 1}")
+            issued["x"] += 1
 
         def load_bc(t):
             st = t % bc_stages
             yield ("arrive_tx", f"bcfull{st}", 2)
             yield ("tma_load", f"bcfull{st}", f"b{st}")
             yield ("tma_load", f"bcfull{st}", f"c{st}")
+            issued["bc"] += 1
 
         yield from load_x(0)
         yield from load_bc(0)
@@ -456,55 +548,76 @@ def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = 
             yield from load_x(1)
             if bc_stages == 2:
                 yield from load_bc(1)
+        ok = True
         for t in range(nt):
             bst = t % bc_stages
-            yield ("wait", f"bcfull{bst}", t // bc_stages)
+            if not (ok := (yield ("wait", f"bcfull{bst}", t // bc_stages))):
+                break
             if t > 0 and "w16_s_ready" not in drop:
-                yield ("wait", "s_ready", t - 1)
+                if not (ok := (yield ("wait", "s_ready", t - 1))):
+                    break
             yield ("mma", (f"c{bst}", f"b{bst}"), ("tCB",))
             yield ("commit", "cb_done")
             if t >= 1 and t + 1 < nt:
                 if "w16_yd_par" not in drop:
-                    yield ("wait", f"yd_par{(t - 1) & 1}", (t - 1) >> 1)
+                    if not (ok := (yield ("wait", f"yd_par{(t - 1) & 1}", (t - 1) >> 1))):
+                        break
                 yield from load_x(t + 1)
                 if bc_stages == 2:
                     yield from load_bc(t + 1)
             if bc_stages == 1 and t + 1 < nt:
                 if "w16_sc_done" not in drop:
-                    yield ("wait", "sc_done", t)
+                    if not (ok := (yield ("wait", "sc_done", t))):
+                        break
                 yield from load_bc(t + 1)
-        # the kernel's W16 has no drain of its own: every tcgen05 op it issued is
-        # waited on by P (cb_done) before the CTA can finish
+        if not ok:
+            for t in range(issued["x"]):
+                yield ("bwait", f"xfull{t & 1}", t >> 1)
+            for t in range(issued["bc"]):
+                yield ("bwait", f"bcfull{t % bc_stages}", t // bc_stages)
+        if fin:
+            yield ("commit", "fin0")
+            yield ("bwait", "fin0", 0)
 
     def w17():
         for t in range(nt):
             st, bst = t & 1, t % bc_stages
-            yield ("wait", "x_ready", t)
+            if not (yield ("wait", "x_ready", t)):
+                break
             if "w17_bcfull" not in drop:
-                yield ("wait", f"bcfull{bst}", t // bc_stages)
+                if not (yield ("wait", f"bcfull{bst}", t // bc_stages)):
+                    break
             yield ("mma", (f"c{bst}", "hs"), (f"tYo{st}",))
-            yield ("wait", "s_ready", t)
+            if not (yield ("wait", "s_ready", t)):
+                break
             yield ("mma", (f"b{bst}", "wx", "tH"), ("tH",))
             yield ("commit", "sc_done")
             if yd_bufs == 1 and t > 0 and "w17_e_done" not in drop:
-                yield ("wait", f"e_done{(t - 1) & 1}", (t - 1) >> 1)
+                if not (yield ("wait", f"e_done{(t - 1) & 1}", (t - 1) >> 1)):
+                    break
             yd = f"tYd{st if yd_bufs == 2 else 0}"
             yield ("mma", ("tS", f"x{st}"), (yd,))
             yield ("commit", f"yd_par{st}")
+        if fin and nt > 0:
+            yield ("commit", "fin1")
+            yield ("bwait", "fin1", 0)
 
     def p_role():
         yield ("write", "tS")
         for t in range(nt):
             buf, bst = t & 1, t % bc_stages
             if t >= 2 and "p_e_done" not in drop:
-                yield ("wait", f"e_done{buf}", (t - 2) >> 1)
+                if not (yield ("wait", f"e_done{buf}", (t - 2) >> 1)):
+                    break
             yield ("write", f"ring{buf}")
             yield ("arrive", f"scan_done{buf}", 8)
-            yield ("wait", "cb_done", t)
+            if not (yield ("wait", "cb_done", t)):
+                break
             if last_partial(t):
                 yield ("write", f"b{bst}")          # rows past the sequence end zeroed
             if t > 0 and "p_yd_par" not in drop:
-                yield ("wait", f"yd_par{(t - 1) & 1}", (t - 1) >> 1)
+                if not (yield ("wait", f"yd_par{(t - 1) & 1}", (t - 1) >> 1)):
+                    break
             yield ("read", "tCB", f"ring{buf}")
             yield ("write", "tS")
             yield ("arrive", "s_ready", 8)
@@ -512,29 +625,36 @@ def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = 
     def e_role():
         def prepare(u):
             st = u & 1
-            yield ("wait", f"scan_done{st}", u >> 1)
+            if not (yield ("wait", f"scan_done{st}", u >> 1)):
+                return False
             yield ("read", f"ring{st}")
             if u > 0:
                 yield ("read", "tH")
             yield ("write", "hs", "tH")
-            yield ("wait", f"xfull{st}", u >> 1)
+            if not (yield ("wait", f"xfull{st}", u >> 1)):
+                return False
             yield ("read", f"x{st}")
             yield ("write", f"x{st}", "wx")
             yield ("arrive", "x_ready", 8)
+            return True
 
+        ok = True
         for k in range(nt + 1):
             if k < nt:
                 if k > 0 and "e_sc_done" not in drop:
-                    yield ("wait", "sc_done", k - 1)
-                yield from prepare(k)
+                    if not (ok := (yield ("wait", "sc_done", k - 1))):
+                        break
+                if not (ok := (yield from prepare(k))):
+                    break
             if k == 0:
                 continue
             t = k - 1
             st = t & 1
-            yield ("wait", f"yd_par{st}", t >> 1)
+            if not (ok := (yield ("wait", f"yd_par{st}", t >> 1))):
+                break
             yield ("read", f"ring{st}", f"tYd{st if yd_bufs == 2 else 0}", f"tYo{st}")
             yield ("arrive", f"e_done{st}", 8)
-        if nt > 0:
+        if nt > 0 and ok:
             yield ("read", "tH")
 
     for name, gen in (("W16", w16()), ("W17", w17()), ("P", p_role()), ("E", e_role())):
@@ -542,9 +662,12 @@ def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = 
     return m
 
 
-def check(build, schedules: int, seed: int, **kw) -> None:
+def check(build, schedules: int, seed: int, faults: bool = False, **kw) -> None:
     """Runs `schedules` random schedules of the model `build(**kw)`; raises ProtocolError on the first
-    race, deadlock, aliasing or exit with work in flight."""
+    race, deadlock, aliasing or exit with work in flight.  With `faults`, each schedule also times
+    out one waiting role at a random step (the timeout path: only deadlock and exit with work in
+    flight are checked from there on)."""
     rng = random.Random(seed)
     for _ in range(schedules):
-        build(**kw).run(rng)
+        m = build(**kw)
+        m.run(rng, fault_at=rng.randrange(0, 40 * (kw.get("nt", 1) + 1)) if faults else None)

@@ -164,8 +164,41 @@ def test_waits_implied_by_other_waits():
     e_done wait (hs_ready follows E's stg_free wait, which follows Y's read of the Y buffer),
     and, with one B/C stage, the first-generation W16's s_ready wait (the stage's reload
     waited for sc_done, which follows s_ready).  The tensor-core drains before exit (fin)
-    matter only on the timeout path, which the model does not take."""
+    matter only on the timeout path (tested below)."""
     for build, kw, drop in ((build_scan3, {}, "w18_y_full"), (build_scan3, {}, "w17_e_done"),
                             (build_scan3, {}, "w17_fin"), (build_scan3, {}, "w18_fin"),
                             (build_scan1, {"n": 256}, "w16_s_ready")):
         assert _caught(build, drop, **kw) is None, drop
+
+
+# ---- the timeout path -------------------------------------------------------------------
+# A bounded wait that gives up sets the CTA's abort flag; every later wait gives up at
+# once, each role leaves its loop, and before the CTA frees TMEM and exits every TMA copy
+# and tcgen05 operation it issued must have completed.
+
+
+def _faults(build, drop=frozenset(), **kw):
+    try:
+        for nt in (1, 2, 3, 5, 7):
+            for partial in (False, True):
+                check(build, 60, seed=300 + nt, faults=True, nt=nt, partial=partial, drop=drop, **kw)
+    except ProtocolError as e:
+        return str(e)
+    return None
+
+
+def test_scan3_timeout_path_exits_with_nothing_in_flight():
+    assert _faults(build_scan3) is None
+
+
+@pytest.mark.parametrize("drain", ["w16_drain", "w17_fin", "w18_fin"])
+def test_scan3_needs_each_of_its_drains(drain):
+    assert "in flight" in (_faults(build_scan3, frozenset([drain])) or "")
+
+
+@pytest.mark.parametrize("n", [128, 256])
+def test_scan1_timeout_path_needs_its_mma_drains(n):
+    """The first-generation kernel's MMA-issuing threads drain their tensor-core work before
+    exit; without that, a timeout can leave MMAs writing TMEM after it is freed."""
+    assert _faults(build_scan1, n=n) is None
+    assert "in flight" in (_faults(build_scan1, n=n, fin=False) or "")
