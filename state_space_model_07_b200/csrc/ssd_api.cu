@@ -123,32 +123,14 @@ int debug_sync(cudaStream_t st, const int32_t* status_dev) {
     return SSD_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* ssd_status_string(int s) {
-    switch (s) {
-        case SSD_OK: return "ok";
-        case SSD_ERR_NULL: return "a required pointer is NULL";
-        case SSD_ERR_SHAPE: return "sizes out of range, inconsistent, overlapping or misaligned buffers";
-        case SSD_ERR_DTYPE: return "unknown dtype";
-        case SSD_ERR_CHUNK: return "chunk must be a power of two in [16, 256]";
-        case SSD_ERR_UNSUPPORTED: return "request not supported by this build";
-        case SSD_ERR_CUDA: return "CUDA error";
-        case SSD_ERR_TIMEOUT: return "bounded device wait timed out";
-        case SSD_ERR_SEQIDX: return "seq_idx breaks its contract";
-        default: return "unknown status";
-    }
-}
-
-const char* ssd_last_error(void) { return g_last_error; }
-
-int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
-                       const float* A, const void* B, const void* C, const float* D,
-                       const float* init_state, const int32_t* seq_idx, int chunk, void* y,
-                       float* final_state, void* stream) {
-    g_last_error[0] = 0;
+// Host-side validation shared by both scan entry points; touches no device
+// memory.  On SSD_OK, `a` holds the launch arguments, `max_chunks` the number
+// of chunks the scan may visit (packed input: one partial chunk more per
+// sequence) and `nstate` the bytes of one (S, H, N, P) float32 state array.
+int prepare_scan(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
+                 const float* A, const void* B, const void* C, const float* D,
+                 const float* init_state, const int32_t* seq_idx, int chunk, void* y,
+                 float* final_state, ssd::ScanArgs& a, int64_t& max_chunks, size_t& nstate) {
     if (!dims) return fail(SSD_ERR_NULL, "dims is NULL");
     int rc = check_sizes(dims);
     if (rc) return rc;
@@ -180,42 +162,104 @@ int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, cons
             overlaps(y, nx, dt, ndt))
             return fail(SSD_ERR_SHAPE, "y overlaps an input");
     }
-    const size_t nstate = (size_t)S * H * N * P * sizeof(float);
+    nstate = (size_t)S * H * N * P * sizeof(float);
     if ((init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)))
         return fail(SSD_ERR_SHAPE, "init_state and final_state must be 16-byte aligned");
     if (init_state && final_state && init_state != final_state &&
         overlaps(init_state, nstate, final_state, nstate))
         return fail(SSD_ERR_SHAPE, "final_state partially overlaps init_state");
 
-    cudaStream_t st = (cudaStream_t)stream;
-    cudaGetLastError();  // clear a stale error so it is not blamed on this call
-
-    if (ntok == 0 || S == 0) {
-        if (final_state && S > 0) {
-            cudaError_t e = init_state
-                ? (init_state == final_state ? cudaSuccess
-                                             : cudaMemcpyAsync(final_state, init_state, nstate,
-                                                               cudaMemcpyDeviceToDevice, st))
-                : cudaMemsetAsync(final_state, 0, nstate, st);
-            if (e != cudaSuccess) return cuda_fail("empty-input state copy", e);
-        }
-        return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
-    }
-
-    ssd::ScanArgs a;
     a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G; a.S = S;
     a.dtype = dims->dtype; a.Q = chunk;
     a.x = x; a.dt = dt; a.B = B; a.C = C;
     a.dt_bias = dt_bias; a.A = A; a.D = D; a.init_state = init_state; a.seq_idx = seq_idx;
     a.y = y; a.final_state = final_state;
+    max_chunks = seq_idx ? (L + chunk - 1) / chunk + S : b * ((L + chunk - 1) / chunk);
+    return SSD_OK;
+}
 
-    const int64_t max_chunks = seq_idx ? (L + chunk - 1) / chunk + S : b * ((L + chunk - 1) / chunk);
+// A scan with no tokens (or no sequences): final_state = init_state (or zero).
+int empty_scan(const ssd::ScanArgs& a, size_t nstate, cudaStream_t st) {
+    if (a.final_state && a.S > 0) {
+        cudaError_t e = a.init_state
+            ? (a.init_state == a.final_state ? cudaSuccess
+                                             : cudaMemcpyAsync(a.final_state, a.init_state, nstate,
+                                                               cudaMemcpyDeviceToDevice, st))
+            : cudaMemsetAsync(a.final_state, 0, nstate, st);
+        if (e != cudaSuccess) return cuda_fail("empty-input state copy", e);
+    }
+    return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
+}
+
+// Bytes of scratch a scan needs besides its path's own workspace: the status
+// word and, for packed input, the sequence table (start, end, chunk offsets).
+size_t scan_table_bytes(const ssd::ScanArgs& a) {
+    size_t n = Carve::round(sizeof(int32_t));
+    if (a.seq_idx) n += 3 * Carve::round(sizeof(int32_t) * (a.S + 1));
+    return n;
+}
+
+// Carves the status word and the sequence table out of `cv` (after the path's
+// workspace), fills the sequence description and, for packed input, launches
+// the kernels that build the table.
+ssd::SeqInfo scan_tables(const ssd::ScanArgs& a, Carve& cv, bool dbg, int32_t** status, cudaStream_t st) {
+    *status = (int32_t*)cv.take(sizeof(int32_t));
+    if (dbg) cudaMemsetAsync(*status, 0, sizeof(int32_t), st);
+    ssd::SeqInfo si;
+    si.L = a.L; si.S = (int32_t)a.S; si.Q = a.Q; si.packed = a.seq_idx ? 1 : 0;
+    si.nc_row = (int32_t)((a.L + a.Q - 1) / a.Q);
+    si.start = si.end = si.chunk_off = nullptr;
+    if (a.seq_idx) {
+        int32_t* start = (int32_t*)cv.take(sizeof(int32_t) * (a.S + 1));
+        int32_t* end = (int32_t*)cv.take(sizeof(int32_t) * (a.S + 1));
+        int32_t* off = (int32_t*)cv.take(sizeof(int32_t) * (a.S + 1));
+        ssd::launch_seq_table(a.seq_idx, a.L, (int32_t)a.S, a.Q, start, end, off, dbg ? *status : nullptr, st);
+        si.start = start; si.end = end; si.chunk_off = off;
+    }
+    return si;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssd_status_string(int s) {
+    switch (s) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_NULL: return "a required pointer is NULL";
+        case SSD_ERR_SHAPE: return "sizes out of range, inconsistent, overlapping or misaligned buffers";
+        case SSD_ERR_DTYPE: return "unknown dtype";
+        case SSD_ERR_CHUNK: return "chunk must be a power of two in [16, 256]";
+        case SSD_ERR_UNSUPPORTED: return "request not supported by this build";
+        case SSD_ERR_CUDA: return "CUDA error";
+        case SSD_ERR_TIMEOUT: return "bounded device wait timed out";
+        case SSD_ERR_SEQIDX: return "seq_idx breaks its contract";
+        default: return "unknown status";
+    }
+}
+
+const char* ssd_last_error(void) { return g_last_error; }
+
+int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
+                       const float* A, const void* B, const void* C, const float* D,
+                       const float* init_state, const int32_t* seq_idx, int chunk, void* y,
+                       float* final_state, void* stream) {
+    g_last_error[0] = 0;
+    ssd::ScanArgs a;
+    int64_t max_chunks = 0;
+    size_t nstate = 0;
+    int rc = prepare_scan(dims, x, dt, dt_bias, A, B, C, D, init_state, seq_idx, chunk, y, final_state, a,
+                          max_chunks, nstate);
+    if (rc) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();  // clear a stale error so it is not blamed on this call
+    if (a.b * a.L == 0 || a.S == 0) return empty_scan(a, nstate, st);
+
     const bool use_tc = ssd::tc_supported(a);
     const size_t ws_path = use_tc ? ssd::tc_workspace_bytes(a, max_chunks)
                                   : ssd::simt_workspace_bytes(a, max_chunks);
     const bool dbg = debug_check();
-    size_t ws_bytes = Carve::round(ws_path) + Carve::round(sizeof(int32_t));
-    if (seq_idx) ws_bytes += 3 * Carve::round(sizeof(int32_t) * (S + 1));
+    const size_t ws_bytes = Carve::round(ws_path) + scan_table_bytes(a);
 
     Carve cv;
     cudaMemPool_t pool = workspace_pool();
@@ -223,19 +267,8 @@ int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, cons
     cudaError_t e = cudaMallocFromPoolAsync((void**)&cv.base, ws_bytes, pool, st);
     if (e != cudaSuccess) return cuda_fail("cudaMallocFromPoolAsync(workspace)", e);
     void* ws_main = cv.take(ws_path);
-    int32_t* status = (int32_t*)cv.take(sizeof(int32_t));
-    ssd::SeqInfo si;
-    si.L = L; si.S = (int32_t)S; si.Q = chunk; si.packed = seq_idx ? 1 : 0;
-    si.nc_row = (int32_t)((L + chunk - 1) / chunk);
-    si.start = si.end = si.chunk_off = nullptr;
-    if (dbg) cudaMemsetAsync(status, 0, sizeof(int32_t), st);
-    if (seq_idx) {
-        int32_t* start = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
-        int32_t* end = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
-        int32_t* off = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
-        ssd::launch_seq_table(seq_idx, L, (int32_t)S, chunk, start, end, off, dbg ? status : nullptr, st);
-        si.start = start; si.end = end; si.chunk_off = off;
-    }
+    int32_t* status = nullptr;
+    const ssd::SeqInfo si = scan_tables(a, cv, dbg, &status, st);
     if (use_tc)
         rc = ssd::launch_tc_scan(a, si, max_chunks, ws_main, dbg ? status : nullptr, st);
     else
@@ -330,68 +363,18 @@ extern "C" int ssd_chunk_scan_fwd_noalloc(const ssd_dims* dims, const void* x, c
                                           const int32_t* seq_idx, int chunk, void* y,
                                           float* final_state, void* stream) {
     g_last_error[0] = 0;
-    if (!dims) return fail(SSD_ERR_NULL, "dims is NULL");
-    int rc = check_sizes(dims);
-    if (rc) return rc;
-    if (chunk < 16 || chunk > 256 || (chunk & (chunk - 1)) != 0)
-        return fail(SSD_ERR_CHUNK, "chunk %d is not a power of two in [16, 256]", chunk);
-    const int64_t b = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim;
-    const int64_t N = dims->dstate, G = dims->ngroups;
-    if (L < 0) return fail(SSD_ERR_SHAPE, "seqlen %lld < 0", (long long)L);
-    if (!A) return fail(SSD_ERR_NULL, "A is NULL");
-    int64_t S = b;
-    if (seq_idx) {
-        if (b != 1 && b * L != 0)
-            return fail(SSD_ERR_SHAPE, "seq_idx requires batch == 1 (got %lld)", (long long)b);
-        if (L >= ((int64_t)1 << 31)) return fail(SSD_ERR_SHAPE, "packed seqlen must be < 2^31");
-        S = dims->nseqs;
-        if (S < 0 || (L > 0 && (S < 1 || S > L)))
-            return fail(SSD_ERR_SHAPE, "nseqs %lld must be in [1, seqlen] for packed input",
-                        (long long)S);
-    }
-    const int64_t ntok = b * L;
-    const size_t es = dims->dtype == SSD_BF16 ? 2 : 4;
-    if (ntok > 0) {
-        if (!x || !dt || !B || !C || !y) return fail(SSD_ERR_NULL, "x, dt, B, C and y are required");
-        if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y))
-            return fail(SSD_ERR_SHAPE, "x, B, C and y must be 16-byte aligned");
-        const size_t nx = (size_t)ntok * H * P * es, nbc = (size_t)ntok * G * N * es;
-        const size_t ndt = (size_t)ntok * H * es;
-        if (overlaps(y, nx, x, nx) || overlaps(y, nx, B, nbc) || overlaps(y, nx, C, nbc) ||
-            overlaps(y, nx, dt, ndt))
-            return fail(SSD_ERR_SHAPE, "y overlaps an input");
-    }
-    const size_t nstate = (size_t)S * H * N * P * sizeof(float);
-    if ((init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)))
-        return fail(SSD_ERR_SHAPE, "init_state and final_state must be 16-byte aligned");
-    if (init_state && final_state && init_state != final_state &&
-        overlaps(init_state, nstate, final_state, nstate))
-        return fail(SSD_ERR_SHAPE, "final_state partially overlaps init_state");
-
-    cudaStream_t st = (cudaStream_t)stream;
-    if (ntok == 0 || S == 0) {
-        cudaGetLastError();
-        if (final_state && S > 0) {
-            cudaError_t e = init_state
-                ? (init_state == final_state ? cudaSuccess
-                                             : cudaMemcpyAsync(final_state, init_state, nstate,
-                                                               cudaMemcpyDeviceToDevice, st))
-                : cudaMemsetAsync(final_state, 0, nstate, st);
-            if (e != cudaSuccess) return cuda_fail("empty-input state copy", e);
-        }
-        return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
-    }
-
     ssd::ScanArgs a;
-    a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G; a.S = S;
-    a.dtype = dims->dtype; a.Q = chunk;
-    a.x = x; a.dt = dt; a.B = B; a.C = C;
-    a.dt_bias = dt_bias; a.A = A; a.D = D; a.init_state = init_state; a.seq_idx = seq_idx;
-    a.y = y; a.final_state = final_state;
-    const int64_t max_chunks = seq_idx ? (L + chunk - 1) / chunk + S : b * ((L + chunk - 1) / chunk);
+    int64_t max_chunks = 0;
+    size_t nstate = 0;
+    int rc = prepare_scan(dims, x, dt, dt_bias, A, B, C, D, init_state, seq_idx, chunk, y, final_state, a,
+                          max_chunks, nstate);
+    if (rc) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    if (a.b * a.L == 0 || a.S == 0) return empty_scan(a, nstate, st);
+
     const size_t ws_path = ssd::simt_workspace_bytes(a, max_chunks);
-    size_t need = Carve::round(ws_path) + Carve::round(sizeof(int32_t));
-    if (seq_idx) need += 3 * Carve::round(sizeof(int32_t) * (S + 1));
+    const size_t need = Carve::round(ws_path) + scan_table_bytes(a);
     if (need > kNoAllocScratchBytes)
         return fail(SSD_ERR_UNSUPPORTED,
                     "this call needs %zu bytes of scratch; the no-allocation scan is limited to %zu "
@@ -405,20 +388,9 @@ extern "C" int ssd_chunk_scan_fwd_noalloc(const ssd_dims* dims, const void* x, c
     Carve cv;
     cv.base = (char*)scratch;
     void* ws_main = cv.take(ws_path);
-    int32_t* status = (int32_t*)cv.take(sizeof(int32_t));
     const bool dbg = debug_check();
-    if (dbg) cudaMemsetAsync(status, 0, sizeof(int32_t), st);
-    ssd::SeqInfo si;
-    si.L = L; si.S = (int32_t)S; si.Q = chunk; si.packed = seq_idx ? 1 : 0;
-    si.nc_row = (int32_t)((L + chunk - 1) / chunk);
-    si.start = si.end = si.chunk_off = nullptr;
-    if (seq_idx) {
-        int32_t* start = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
-        int32_t* end = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
-        int32_t* off = (int32_t*)cv.take(sizeof(int32_t) * (S + 1));
-        ssd::launch_seq_table(seq_idx, L, (int32_t)S, chunk, start, end, off, dbg ? status : nullptr, st);
-        si.start = start; si.end = end; si.chunk_off = off;
-    }
+    int32_t* status = nullptr;
+    const ssd::SeqInfo si = scan_tables(a, cv, dbg, &status, st);
     ssd::launch_simt_scan(a, si, max_chunks, ws_main, st);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("kernel launch", e);

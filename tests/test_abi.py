@@ -58,14 +58,17 @@ def dims(**kw):
     return _lib.SsdDims(**base)
 
 
-def scan(L, d, chunk=128, **ptrs):
+def scan(L, d, chunk=128, entry="ssd_chunk_scan_fwd", **ptrs):
     p = dict(x=FAKE, dt=FAKE * 2, dt_bias=None, A=FAKE * 3, B=FAKE * 40, C=FAKE * 80, D=None,
              init_state=None, seq_idx=None, y=FAKE * 120, final_state=None)
     p.update(ptrs)
     v = lambda k: None if p[k] is None else ctypes.c_void_p(p[k])
-    return L.ssd_chunk_scan_fwd(ctypes.byref(d) if d is not None else None, v("x"), v("dt"), v("dt_bias"),
-                                v("A"), v("B"), v("C"), v("D"), v("init_state"), v("seq_idx"), chunk,
-                                v("y"), v("final_state"), None)
+    return getattr(L, entry)(ctypes.byref(d) if d is not None else None, v("x"), v("dt"), v("dt_bias"),
+                             v("A"), v("B"), v("C"), v("D"), v("init_state"), v("seq_idx"), chunk,
+                             v("y"), v("final_state"), None)
+
+
+ENTRIES = ["ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc"]
 
 
 @pytest.mark.parametrize("kw,chunk,ptrs,code", [
@@ -86,13 +89,22 @@ def scan(L, d, chunk=128, **ptrs):
     ({"batch": 1, "nseqs": 65}, 128, {"seq_idx": FAKE * 200}, 2),
     ({}, 128, {"init_state": FAKE * 300, "final_state": FAKE * 300 + 64}, 2),  # partial overlap
 ])
-def test_scan_rejects_bad_arguments(L, kw, chunk, ptrs, code):
-    assert scan(L, dims(**kw), chunk, **ptrs) == code
+@pytest.mark.parametrize("entry", ENTRIES)
+def test_scan_rejects_bad_arguments(L, kw, chunk, ptrs, code, entry):
+    assert scan(L, dims(**kw), chunk, entry=entry, **ptrs) == code
     assert L.ssd_last_error().decode()
 
 
-def test_scan_null_dims(L):
-    assert scan(L, None) == 1
+@pytest.mark.parametrize("entry", ENTRIES)
+def test_scan_null_dims(L, entry):
+    assert scan(L, None, entry=entry) == 1
+
+
+@pytest.mark.parametrize("entry", ENTRIES)
+def test_empty_scan_without_states_is_a_host_side_no_op(L, entry):
+    # no tokens and no final_state to fill: nothing reaches a device
+    assert scan(L, dims(seqlen=0), entry=entry, x=None, dt=None, B=None, C=None, y=None) == 0
+    assert scan(L, dims(batch=0), entry=entry) == 0
 
 
 def update(L, d, **ptrs):
@@ -114,11 +126,12 @@ def test_state_update_rejects_bad_arguments(L):
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a CUDA device")
-def test_valid_call_without_device_reports_cuda_error(L):
-    # All arguments valid: the first CUDA call (workspace allocation) fails
-    # cleanly because this host has no GPU.
-    assert scan(L, dims()) == 6
-    assert "cuda" in L.ssd_last_error().decode().lower() or L.ssd_last_error()
+@pytest.mark.parametrize("entry", ENTRIES)
+def test_valid_call_without_device_reports_cuda_error(L, entry):
+    # All arguments valid: the first CUDA call (workspace allocation, or the
+    # scratch array's address) fails cleanly because this host has no GPU.
+    assert scan(L, dims(), entry=entry) == 6
+    assert L.ssd_last_error().decode()
 
 
 def test_python_wrapper_fails_loudly_without_library(monkeypatch, tmp_path):
