@@ -353,7 +353,11 @@ class Machine:
 # tokens; `partial` = the last tile is shorter (its y leaves by row stores,
 # not through the staging tile).
 
-def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -> Machine:
+def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), zero_b: str = "") -> Machine:
+    """`zero_b` models ways of zeroing the B rows past the sequence end in a partial last tile
+    (not done by the kernel today): "p" has the P warps do it right after C B^T has read B
+    (cb_full), with W17 waiting for c_scaled before B^T (w o x) on that tile; "e" has the E
+    warps do it before x_ready, unordered with W18's C B^T read."""
     m = Machine()
     for i in range(4):
         m.barrier(f"scan_done{i}", 1)
@@ -417,6 +421,9 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -
             st, ph = t & 1, t >> 1
             if not (yield ("wait", f"x_ready{st}", ph)) or not (yield ("wait", f"full{st}", ph)):
                 break
+            if zero_b == "p" and not full_tile(t):
+                if not (yield ("wait", f"c_scaled{st}", ph)):
+                    break
             yield ("mma", (f"b{st}", "wx"), ("tSt",))
             yield ("commit", f"s_done{st}")
             if not (yield ("wait", f"hs_ready{st}", ph)) or not (yield ("wait", f"c_scaled{st}", ph)):
@@ -442,6 +449,8 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -
                 break
             yield ("read", f"ring{sl}", f"tC{st}")
             yield ("write", f"tC{st}")
+            if zero_b == "p" and not full_tile(t):
+                yield ("write", f"b{st}")
             yield ("arrive", f"c_scaled{st}", 8)
             yield ("read", "tCB", f"ring{sl}")
             yield ("arrive", f"cb_free{st}", 8)
@@ -495,6 +504,8 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset()) -
                 yield ("arrive", f"scan_free{k & 3}", 8)
                 yield ("read", f"x{k & 1}")
                 yield ("write", f"x{k & 1}", "wx")
+                if zero_b == "e" and not full_tile(k):
+                    yield ("write", f"b{k & 1}")
                 yield ("arrive", f"x_ready{k & 1}", 8)
 
     for name, gen in (("W19", w19()), ("W16", w16()), ("W18", w18()), ("W17", w17()), ("P", p_role()),

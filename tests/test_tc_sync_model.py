@@ -202,3 +202,17 @@ def test_scan1_timeout_path_needs_its_mma_drains(n):
     exit; without that, a timeout can leave MMAs writing TMEM after it is freed."""
     assert _faults(build_scan1, n=n) is None
     assert "in flight" in (_faults(build_scan1, n=n, fin=False) or "")
+
+
+def test_planned_zeroing_of_b_rows_past_a_sequence_end():
+    """k_tc_scan3 does not yet zero the B rows past a sequence's end in its partial last tile
+    (they feed B^T (w o x) against exact zeros, so only a non-finite B of the next sequence
+    matters).  Of two ways to add it, zeroing in the P warps after C B^T has read B, with W17
+    waiting for c_scaled before B^T (w o x) on that tile, is race-free, also on the timeout path;
+    zeroing in the E warps before x_ready races with W18's C B^T read."""
+    for nt in (1, 2, 3, 5, 8):
+        check(build_scan3, 40, seed=400 + nt, nt=nt, partial=True, zero_b="p")
+        check(build_scan3, 20, seed=500 + nt, nt=nt, partial=True, zero_b="p", faults=True)
+    with pytest.raises(ProtocolError, match="race on b"):
+        for nt in (1, 2, 3, 5, 8):
+            check(build_scan3, 40, seed=600 + nt, nt=nt, partial=True, zero_b="e")
