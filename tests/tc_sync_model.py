@@ -353,20 +353,27 @@ class Machine:
 # tokens; `partial` = the last tile is shorter (its y leaves by row stores,
 # not through the staging tile).
 
-def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), zero_b: str = "") -> Machine:
+def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), zero_b: str = "",
+                conv: str = "E") -> Machine:
     """`zero_b` models ways of zeroing the B rows past the sequence end in a partial last tile
     (not done by the kernel today): "p" has the P warps do it right after C B^T has read B
     (cb_full), with W17 waiting for c_scaled before B^T (w o x) on that tile; "e" has the E
-    warps do it before x_ready, unordered with W18's C B^T read."""
+    warps do it before x_ready, unordered with W18's C B^T read.
+
+    `conv` names the role that turns x into the fp16 operands x and w o x: "E" (the kernel
+    today: the E warps, between the state update of tile t - 1 and x_ready of tile t) or "Y"
+    (a candidate: the four epilogue warps convert x of tile t + 1 as soon as B^T (w o x) of
+    tile t has completed, and the E warps do only the state update, which then leaves the loop
+    between consecutive B^T (w o x) MMAs)."""
     m = Machine()
     for i in range(4):
         m.barrier(f"scan_done{i}", 1)
-        m.barrier(f"scan_free{i}", 16)
+        m.barrier(f"scan_free{i}", 16 if conv == "E" else 20)
     for i in range(2):
         for name, count in (("full", 1), ("cb_full", 1), ("cb_free", 8), ("c_scaled", 8), ("s_ready", 8),
                             ("x_ready", 8), ("hs_ready", 8), ("e_done", 4), ("stg_free", 1), ("s_done", 1),
-                            ("y_full", 1), ("fin", 1)):
-            m.barrier(f"{name}{i}", count)
+                            ("y_full", 1), ("fin", 1), ("st_free", 8)):
+            m.barrier(f"{name}{i}", count if not (name == "x_ready" and conv == "Y") else 4)
     full_tile = lambda u: not (partial and u == nt - 1)
 
     def w19():      # decay scan into the four-slot ring
@@ -421,6 +428,10 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
             st, ph = t & 1, t >> 1
             if not (yield ("wait", f"x_ready{st}", ph)) or not (yield ("wait", f"full{st}", ph)):
                 break
+            if conv == "Y" and t >= 1 and "w17_st_free" not in drop:
+                # the single s buffer: E has loaded s of tile t - 1
+                if not (yield ("wait", f"st_free{st ^ 1}", (t - 1) >> 1)):
+                    break
             if zero_b == "p" and not full_tile(t):
                 if not (yield ("wait", f"c_scaled{st}", ph)):
                     break
@@ -461,10 +472,28 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
             yield ("write", "tS")
             yield ("arrive", f"s_ready{st}", 8)
 
+    def convert(k, weight):   # x of tile k -> fp16 x and w o x
+        if not (yield ("wait", f"scan_done{k & 3}", k >> 2)) or not (yield ("wait", f"full{k & 1}", k >> 1)):
+            return False
+        yield ("read", f"ring{k & 3}")
+        yield ("arrive", f"scan_free{k & 3}", weight)
+        yield ("read", f"x{k & 1}")
+        yield ("write", f"x{k & 1}", "wx")
+        if zero_b == "e" and not full_tile(k):
+            yield ("write", f"b{k & 1}")
+        yield ("arrive", f"x_ready{k & 1}", weight)
+        return True
+
     def y_role():   # epilogue and TMA store of y
         stored = False
+        if conv == "Y" and nt > 0 and not (yield from convert(0, 4)):
+            return
         for u in range(nt):
             st = u & 1
+            if conv == "Y" and u + 1 < nt:
+                # w o x is free once B^T (w o x) of tile u has completed
+                if not (yield ("wait", f"s_done{st}", u >> 1)) or not (yield from convert(u + 1, 4)):
+                    break
             if not (yield ("wait", f"y_full{st}", u >> 1)):
                 break
             yield ("read", f"tY{st}")
@@ -493,20 +522,20 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
                 if 2 <= k < nt and "e_stg_free" not in drop:
                     if not (yield ("wait", f"stg_free{k & 1}", (k - 2) >> 1)):
                         break
+                if conv == "Y":
+                    # 2^cs_last of tile u from the ring (ordered after the decay scan through
+                    # x_ready -> s_done); the slot is released here
+                    yield ("read", f"ring{u & 3}")
+                    yield ("arrive", f"scan_free{u & 3}", 8)
                 yield ("read", "tSt")
+                if conv == "Y":
+                    yield ("arrive", f"st_free{u & 1}", 8)
                 if k < nt:
                     yield ("write", f"hs{k & 1}")
                     yield ("arrive", f"hs_ready{k & 1}", 8)
-            if k < nt:
-                if not (yield ("wait", f"scan_done{k & 3}", k >> 2)) or not (yield ("wait", f"full{k & 1}", k >> 1)):
+            if k < nt and conv == "E":
+                if not (yield from convert(k, 8)):
                     break
-                yield ("read", f"ring{k & 3}")
-                yield ("arrive", f"scan_free{k & 3}", 8)
-                yield ("read", f"x{k & 1}")
-                yield ("write", f"x{k & 1}", "wx")
-                if zero_b == "e" and not full_tile(k):
-                    yield ("write", f"b{k & 1}")
-                yield ("arrive", f"x_ready{k & 1}", 8)
 
     for name, gen in (("W19", w19()), ("W16", w16()), ("W18", w18()), ("W17", w17()), ("P", p_role()),
                       ("Y", y_role()), ("E", e_role())):

@@ -216,3 +216,19 @@ def test_planned_zeroing_of_b_rows_past_a_sequence_end():
     with pytest.raises(ProtocolError, match="race on b"):
         for nt in (1, 2, 3, 5, 8):
             check(build_scan3, 40, seed=600 + nt, nt=nt, partial=True, zero_b="e")
+
+
+def test_candidate_conversion_in_the_epilogue_warps():
+    """A candidate restructuring of k_tc_scan3 (not built yet): the epilogue warps convert x of
+    tile t + 1 as soon as B^T (w o x) of tile t has completed, and the E warps only update the
+    state.  The single TMEM buffer of the tile's own state term then needs its own release: E
+    arrives at st_free right after loading s, and W17 waits for it before the next B^T (w o x).
+    With that the protocol is clean, also on the timeout path; without it the next MMA can
+    overwrite s while E is still reading it."""
+    for nt in (0, 1, 2, 3, 5, 9):
+        for partial in (False, True):
+            check(build_scan3, 30, seed=700 + nt, nt=nt, partial=partial, conv="Y")
+            check(build_scan3, 15, seed=800 + nt, nt=nt, partial=partial, conv="Y", faults=True)
+    with pytest.raises(ProtocolError, match="race on tSt"):
+        for nt in (2, 3, 5, 9):
+            check(build_scan3, 40, seed=900 + nt, nt=nt, conv="Y", drop=frozenset(["w17_st_free"]))
