@@ -273,6 +273,41 @@ MUTANTS = {
                     "memset(state, 0, sizeof(double) * N * P);"),
     "no_softplus": ("const double d = oracle_softplus(j->dt[tok * H + h] + bias);",
                     "const double d = j->dt[tok * H + h] + bias;"),
+    "dt_bias_sign": ("const double d = oracle_softplus(j->dt[tok * H + h] + bias);",
+                     "const double d = oracle_softplus(j->dt[tok * H + h] - bias);"),
+    "B_without_d": ("const double dB = d * Bt[n];", "const double dB = Bt[n];"),
+    "A_per_group": ("const double Ah = j->A[h];", "const double Ah = j->A[g];"),
+    "D_per_group": ("const double Dh = j->D ? j->D[h] : 0.0;", "const double Dh = j->D ? j->D[g] : 0.0;"),
+    # y read from h_{t-1}: the output loop runs before the state update
+    "output_before_update": (
+        """        /* h_t = exp(d A) h_{t-1} + d B_t x_t^T */
+        for (int64_t n = 0; n < N; ++n) {
+            const double dB = d * Bt[n];
+            double *hn = state + n * P;
+            for (int64_t p = 0; p < P; ++p) hn[p] = decay * hn[p] + dB * xt[p];
+        }
+        /* y_t = C_t^T h_t + D x_t */
+        for (int64_t p = 0; p < P; ++p) yt[p] = Dh * xt[p];
+        for (int64_t n = 0; n < N; ++n) {
+            const double c = Ct[n];
+            const double *hn = state + n * P;
+            for (int64_t p = 0; p < P; ++p) yt[p] += c * hn[p];
+        }
+""",
+        """        for (int64_t p = 0; p < P; ++p) yt[p] = Dh * xt[p];
+        for (int64_t n = 0; n < N; ++n) {
+            const double c = Ct[n];
+            const double *hn = state + n * P;
+            for (int64_t p = 0; p < P; ++p) yt[p] += c * hn[p];
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            const double dB = d * Bt[n];
+            double *hn = state + n * P;
+            for (int64_t p = 0; p < P; ++p) hn[p] = decay * hn[p] + dB * xt[p];
+        }
+"""),
+    "decode_B_without_d": ("st[n * P + p] = decay * st[n * P + p] + d * Bt[n] * xt[p];",
+                           "st[n * P + p] = decay * st[n * P + p] + Bt[n] * xt[p];"),
 }
 
 
@@ -304,7 +339,7 @@ def test_planted_mistake_is_caught(tmp_path, monkeypatch, name):
     pins = [test_single_token_closed_form, test_constant_input_geometric_series,
             test_matches_bruteforce_semiseparable_matrix, test_no_decay_is_cumulative_sum,
             lambda: test_matches_block_decomposition(16), test_state_cache_split_continuation,
-            test_groups_map_to_contiguous_head_blocks]
+            test_groups_map_to_contiguous_head_blocks, test_decode_step_equals_one_token_scan]
     pins += [lambda c=c: test_golden_worked_examples(c) for c in json.load(open(GOLDEN))["cases"]]
     failures = 0
     for pin in pins:
