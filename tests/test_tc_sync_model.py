@@ -232,3 +232,7 @@ def test_candidate_conversion_in_the_epilogue_warps():
     with pytest.raises(ProtocolError, match="race on tSt"):
         for nt in (2, 3, 5, 9):
             check(build_scan3, 40, seed=900 + nt, nt=nt, conv="Y", drop=frozenset(["w17_st_free"]))
+    # together with the zeroing of B rows past a sequence end
+    for nt in (1, 2, 5):
+        check(build_scan3, 30, seed=950 + nt, nt=nt, partial=True, conv="Y", zero_b="p")
+        check(build_scan3, 15, seed=960 + nt, nt=nt, partial=True, conv="Y", zero_b="p", faults=True)
