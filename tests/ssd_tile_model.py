@@ -142,3 +142,40 @@ def segment_split_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, se
                 total = np.exp2(np.sum(d * np.asarray(A, np.float64)[h] * LOG2E))
                 h_in[bb, h] = fk[bb, h] + (0.0 if k == 0 else total * h_in[bb, h])
     return y, h_in
+
+
+def segment_rerun_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, segments=3, seg_len=None):
+    """The long-sequence split that reruns the scan instead of correcting y, in fp64.
+
+    Segments of `seg_len` tokens (default ceil(L / segments)); the last one takes the rest.
+    Pass 1 scans segments 0 .. K-2 independently: segment 0 from the real initial state (its y
+    is final), the others from zero (only their final states are used).  The chain gives the
+    state entering segment k >= 1: h_in(1) = final(0), h_in(k) = exp(sum of d A over segment
+    k - 1) h_in(k - 1) + final(k - 1).  Pass 2 rescans segments 1 .. K-1 from h_in(k), giving
+    their y and, from the last one, the final state."""
+    x, dt, B, C = (np.asarray(v, dtype=np.float64) for v in (x, dt, B, C))
+    A = np.asarray(A, dtype=np.float64)
+    b, L, H, P = x.shape
+    N = B.shape[3]
+    bias = np.zeros(H) if dt_bias is None else np.asarray(dt_bias, dtype=np.float64)
+    Ls = seg_len or -(-L // segments)
+    bounds = [min(k * Ls, L) for k in range(segments)] + [L]
+    assert all(bounds[k] < bounds[k + 1] for k in range(segments)), "every segment needs tokens"
+    seg = lambda v, k: v[:, bounds[k]:bounds[k + 1]]
+    y = np.zeros((b, L, H, P))
+    finals = []
+    for k in range(segments - 1):                                                      # pass 1
+        h0 = init_state if k == 0 else None
+        yk, fk = tile_form(seg(x, k), seg(dt, k), A, seg(B, k), seg(C, k), dt_bias, D, h0)
+        if k == 0:
+            y[:, bounds[0]:bounds[1]] = yk
+        finals.append(fk)
+    h_in = [None, finals[0]]                                                           # chain
+    for k in range(2, segments):
+        total = np.exp(np.sum(_softplus(seg(dt, k - 1) + bias) * A, axis=1))           # (b, H)
+        h_in.append(total[:, :, None, None] * h_in[k - 1] + finals[k - 1])
+    fs = None
+    for k in range(1, segments):                                                       # pass 2
+        yk, fs = tile_form(seg(x, k), seg(dt, k), A, seg(B, k), seg(C, k), dt_bias, D, h_in[k])
+        y[:, bounds[k]:bounds[k + 1]] = yk
+    return y, fs

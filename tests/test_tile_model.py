@@ -77,3 +77,16 @@ def test_kernel_roundings_hold_at_dstate_256():
     assert _rel(y16, yr) < 1e-2 and _rel(f16, fr) < 1e-2
     yb, _ = tile_form(**args, rounding="bf16_operands")
     assert _rel(yb, yr) > 2e-2
+
+
+def test_rerun_split_is_exact():
+    """The two-pass split for long sequences with few heads (pass 1 over segments 0 .. K-2,
+    the chain of segment states, pass 2 rescanning segments 1 .. K-1 from their entering
+    states) reproduces the recurrence, for tile-aligned and ragged segment lengths, batch > 1
+    and an initial state."""
+    from tests.ssd_tile_model import segment_rerun_form
+    args, yr, fr = _case("long_context", batch=2, seqlen=700, nheads=2, ngroups=1)
+    for segments, seg_len in ((3, 256), (3, None), (4, 128), (5, None)):
+        y, fs = segment_rerun_form(**args, segments=segments, seg_len=seg_len)
+        assert _rel(y, yr) < 1e-9, (segments, seg_len)
+        assert _rel(fs, fr) < 1e-9, (segments, seg_len)
