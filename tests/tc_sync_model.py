@@ -711,3 +711,61 @@ def check(build, schedules: int, seed: int, faults: bool = False, **kw) -> None:
     for _ in range(schedules):
         m = build(**kw)
         m.run(rng, fault_at=rng.randrange(0, 40 * (kw.get("nt", 1) + 1)) if faults else None)
+
+
+# ---------------------------------------------------------------------------
+# Leader waits inside a role.  A role of several warps waits as one: the leader
+# polls the mbarrier, writes the result to a flag in shared memory, all warps
+# meet at a named barrier (bar.sync, no timeout) and each reads the flag.  With
+# one flag the leader's next write can land before a slow warp has read the
+# previous result; warps of one role then disagree, and a warp that leaves
+# while the others go on to the next bar.sync leaves them waiting forever.
+# Alternating between two flags closes this: the leader writes a slot again
+# only after the next bar.sync, which every warp passes after its read.
+
+def role_leader_waits(nwarps: int, results, slots: int, rng: random.Random) -> str | None:
+    """Runs one random schedule of `nwarps` warps through consecutive leader waits whose
+    outcomes are `results` (False = the leader's wait gave up); returns None, or a description
+    of a warp that read another wait's result or of a hang at a named barrier."""
+    flag = [None] * slots
+    arrived, gen = 0, 0
+    pc = [("write" if w == 0 else "sync", 0) for w in range(nwarps)]   # (next action, call index)
+    waiting_gen = [None] * nwarps
+    done = [False] * nwarps
+    weight = [10 ** rng.uniform(-3, 0) for _ in range(nwarps)]
+    ncalls = len(results)
+    while not all(done):
+        runnable = []
+        for w in range(nwarps):
+            if done[w]:
+                continue
+            act, i = pc[w]
+            if act == "blocked" and gen == waiting_gen[w]:
+                continue                                   # still parked at the named barrier
+            runnable.append(w)
+        if not runnable:
+            return "hang: warps parked at a named barrier that a departed warp never reaches"
+        w = rng.choices(runnable, [weight[v] for v in runnable])[0]
+        act, i = pc[w]
+        if act == "write":                                 # leader: the wait's result
+            flag[i % slots] = (i, results[i])
+            pc[w] = ("sync", i)
+        elif act == "sync":
+            arrived += 1
+            if arrived == nwarps:                          # last arrival releases the barrier
+                arrived, gen = 0, gen + 1
+                pc[w] = ("read", i)
+            else:
+                waiting_gen[w] = gen
+                pc[w] = ("blocked", i)
+        elif act == "blocked":                             # released
+            pc[w] = ("read", i)
+        elif act == "read":
+            call, value = flag[i % slots]
+            if call != i:
+                return f"warp {w} read the result of wait {call} for wait {i}"
+            if not value or i + 1 == ncalls:
+                done[w] = True                             # leaves the role's loop
+            else:
+                pc[w] = ("write" if w == 0 else "sync", i + 1)
+    return None

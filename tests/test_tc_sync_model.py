@@ -236,3 +236,17 @@ def test_candidate_conversion_in_the_epilogue_warps():
     for nt in (1, 2, 5):
         check(build_scan3, 30, seed=950 + nt, nt=nt, partial=True, conv="Y", zero_b="p")
         check(build_scan3, 15, seed=960 + nt, nt=nt, partial=True, conv="Y", zero_b="p", faults=True)
+
+
+def test_role_leader_flag_needs_two_slots():
+    """One flag per role lets a slow warp read the leader's next result (and, when that wait
+    gave up, leave while the others park at the next named barrier); two alternating flags
+    never do, whatever the schedule."""
+    from tests.tc_sync_model import role_leader_waits
+    rng = random.Random(5)
+    results = [True] * 5 + [False]
+    one = [role_leader_waits(8, results, 1, rng) for _ in range(400)]
+    assert any(r is not None for r in one)
+    for _ in range(400):
+        assert role_leader_waits(8, results, 2, rng) is None
+        assert role_leader_waits(4, [True] * 7, 2, rng) is None
