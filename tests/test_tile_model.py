@@ -90,3 +90,25 @@ def test_rerun_split_is_exact():
         y, fs = segment_rerun_form(**args, segments=segments, seg_len=seg_len)
         assert _rel(y, yr) < 1e-9, (segments, seg_len)
         assert _rel(fs, fr) < 1e-9, (segments, seg_len)
+
+
+def test_state_rows_are_separable():
+    """The recurrence never mixes state rows: scanning the first and the second half of B and C
+    (d_state 256 split into 128 + 128) separately, with the D skip in one of them, gives y as
+    the sum of the two and the final state as their stack (the basis of running a d_state 256
+    scan as two d_state 128 halves on a CTA pair)."""
+    w = inputs.scaled(inputs.WORKLOADS["packed_varlen"], nheads=4, ngroups=2)
+    d = inputs.make_inputs(w, "cpu", lengths=[300])
+    yr, fr = oracle.ssd_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
+                             init_state=d["init_state"], dt_bias=d["dt_bias"])
+    half = d["B"].shape[-1] // 2
+    parts = []
+    for k, Dk in ((0, d["D"]), (1, None)):
+        sl = slice(k * half, (k + 1) * half)
+        parts.append(oracle.ssd_scan(d["x"], d["dt"], d["A"], d["B"][..., sl].contiguous(),
+                                     d["C"][..., sl].contiguous(), D=Dk, dt_bias=d["dt_bias"],
+                                     init_state=d["init_state"][:, :, sl].contiguous()))
+    y = parts[0][0] + parts[1][0]
+    fs = np.concatenate([parts[0][1], parts[1][1]], axis=2)
+    assert _rel(y, np.asarray(yr)) < 1e-12
+    assert _rel(fs, np.asarray(fr)) < 1e-12
