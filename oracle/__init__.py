@@ -6,8 +6,9 @@ reference arm may import this package.  The product path
 nothing from the product path: the two share no code.
 
 The arithmetic lives in ``ssd_oracle.c`` (a literal token-by-token loop in
-double precision, see the header there for the definition and its sources).
-This module only marshals numpy arrays to it.
+double precision, see the header there for the definition and its sources) and
+``ssd_oracle_bwd.c`` (the gradient of that loop: the adjoint reverse sweep).
+This module only marshals numpy arrays to them.
 
 Every input is taken as the exact values the GPU sees: bf16 / fp32 tensors are
 widened to float64 without rounding before the call.
@@ -22,6 +23,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ssd_oracle.c")
+_SRC_BWD = os.path.join(_HERE, "ssd_oracle_bwd.c")
 _LIB = os.path.join(_HERE, "libssd_oracle.so")
 _lib = None
 
@@ -31,11 +33,13 @@ _i64 = ctypes.c_int64
 
 
 def build(force: bool = False) -> str:
-    """Compiles ssd_oracle.c into libssd_oracle.so (plain gcc, no fast-math,
-    no FMA contraction, so the loop is evaluated exactly as written)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    """Compiles ssd_oracle.c and ssd_oracle_bwd.c into libssd_oracle.so (plain
+    gcc, no fast-math, no FMA contraction, so the loops are evaluated exactly as
+    written)."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_BWD))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
-               "-fno-fast-math", "-pthread", _SRC, "-o", _LIB + ".tmp", "-lm"]
+               "-fno-fast-math", "-pthread", _SRC, _SRC_BWD, "-o", _LIB + ".tmp", "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(_LIB + ".tmp", _LIB)
     return _LIB
@@ -51,6 +55,8 @@ def _load():
         lib.oracle_ssd_scan.argtypes = [_i64] * 7 + [_D] * 8 + [_I32, _D, _D, ctypes.c_int]
         lib.oracle_state_update.restype = ctypes.c_int
         lib.oracle_state_update.argtypes = [_i64] * 5 + [_D] * 9
+        lib.oracle_ssd_scan_bwd.restype = ctypes.c_int
+        lib.oracle_ssd_scan_bwd.argtypes = [_i64] * 7 + [_D] * 8 + [_I32] + [_D] * 10
         _lib = lib
     return _lib
 
@@ -135,3 +141,40 @@ def state_update(state, x, dt, A, B, C, dt_bias=None, D=None):
     if rc != 0:
         raise ValueError(f"oracle_state_update rejected its arguments (rc={rc})")
     return st, y
+
+
+def ssd_scan_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, seq_idx=None,
+                 nseqs=None, dfinal=None):
+    """Gradient of J = sum(dy * y) + sum(dfinal * final_state) through the scan.
+
+    Same inputs and shapes as ``ssd_scan``; dy (b, L, H, P); dfinal (S, H, N, P)
+    or None.  Returns a dict of float64 arrays: x, dt, dt_bias, A, B, C, D,
+    init_state (the last is the gradient for the initial state, zero or not).
+    """
+    x, dt, A, B, C, dy = (_f64(v) for v in (x, dt, A, B, C, dy))
+    dt_bias, D, init_state, dfinal = _f64(dt_bias), _f64(D), _f64(init_state), _f64(dfinal)
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    si = None
+    if seq_idx is not None:
+        if hasattr(seq_idx, "detach"):
+            seq_idx = seq_idx.detach().to("cpu").numpy()
+        si = np.ascontiguousarray(np.asarray(seq_idx, dtype=np.int32).reshape(-1))
+        assert b == 1 and si.shape == (L,)
+        if nseqs is None:
+            nseqs = int(si[-1]) + 1 if L > 0 else 0
+        S = nseqs
+    else:
+        nseqs = b
+        S = b
+    assert dy.shape == x.shape
+    out = {"x": np.zeros_like(x), "dt": np.zeros((b, L, H)), "dt_bias": np.zeros(H), "A": np.zeros(H),
+           "B": np.zeros((b, L, G, N)), "C": np.zeros((b, L, G, N)), "D": np.zeros(H),
+           "init_state": np.zeros((S, H, N, P))}
+    rc = _load().oracle_ssd_scan_bwd(
+        b, L, H, P, N, G, nseqs, _ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+        _ptr(init_state), _ptr(si, _I32), _ptr(dy), _ptr(dfinal),
+        *(_ptr(out[k]) for k in ("x", "dt", "dt_bias", "A", "B", "C", "D", "init_state")))
+    if rc != 0:
+        raise ValueError(f"oracle_ssd_scan_bwd rejected its arguments (rc={rc})")
+    return out
