@@ -38,6 +38,22 @@ def _round(a, kind):
     return t.to(dt).to(torch.float64).numpy()
 
 
+_FP8 = {"e4m3": (torch.float8_e4m3fn, 448.0), "e5m2": (torch.float8_e5m2, 57344.0)}
+
+
+def _round_op(a, kind, axis):
+    """Rounds one GEMM operand.  fp8 kinds carry one scale per slice along `axis` (the
+    contracted dimension: a row of A, a column of B), as a scaled fp8 MMA would: the scales
+    multiply back in its epilogue."""
+    if kind not in _FP8:
+        return _round(a, kind)
+    dt, top = _FP8[kind]
+    amax = np.max(np.abs(a), axis=axis, keepdims=True)
+    scale = np.where(amax > 0, top / np.where(amax > 0, amax, 1.0), 1.0)
+    t = torch.from_numpy(np.ascontiguousarray(a * scale, dtype=np.float32))
+    return t.to(dt).to(torch.float64).numpy() / scale
+
+
 def _softplus(z):
     return np.where(z > 0, z + np.log1p(np.exp(-np.abs(z))), np.log1p(np.exp(np.minimum(z, 0))))
 
@@ -61,10 +77,15 @@ def _mask(CB, cs, d, Dh, q):
     return S
 
 
-def tile_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, rounding=None):
+def tile_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, rounding=None, operands=None):
     """x (b,L,H,P), dt (b,L,H), B/C (b,L,G,N), A/dt_bias/D (H,), init_state (b,H,N,P).
 
+    `operands` (with rounding="kernel") overrides the operand type of single GEMMs: keys "cb"
+    (C B^T), "state" (B^T (w o x)), "out" (C' h_prev), "diag" (S x); values "f16", "bf16",
+    "e4m3", "e5m2" (fp8 with one scale per row of A and per column of B).
+
     Returns (y, final_state) as fp64 arrays."""
+    ops = dict(operands or {})
     x, dt, B, C = (np.asarray(v, dtype=np.float64) for v in (x, dt, B, C))
     A = np.asarray(A, dtype=np.float64)
     b, L, H, P = x.shape
@@ -93,14 +114,27 @@ def tile_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, rounding=No
                 Bt[:q] = B[bb, t0:t0 + q, g]
                 Ct = np.zeros((T, N))
                 Ct[:q] = C[bb, t0:t0 + q, g]
+                Braw, Craw, xraw = Bt, Ct, xt
                 Bt, Ct, x16 = _round(Bt, kop), _round(Ct, kop), _round(xt, kop)
-                CB = _round(Ct @ Bt.T, k32)
-                S = _round(_mask(CB, cs, d, Dv[h], q), k16)
+                if "cb" in ops:
+                    CB = _round(_round_op(Craw, ops["cb"], 1) @ _round_op(Braw, ops["cb"], 1).T, k32)
+                else:
+                    CB = _round(Ct @ Bt.T, k32)
+                S = _mask(CB, cs, d, Dv[h], q)
                 w = d * np.exp2(cs[q - 1] - cs)
-                wx = _round(w[:, None] * x16, k16)
-                s_tile = _round(Bt.T @ wx, k32)
-                Cp = _round(np.exp2(cs)[:, None] * Ct, kop)
-                Y = S @ x16 + Cp @ _round(hst, k16)
+                if "state" in ops:
+                    s_tile = _round(_round_op(Braw, ops["state"], 0).T @ _round_op(w[:, None] * xraw, ops["state"], 0), k32)
+                else:
+                    s_tile = _round(Bt.T @ _round(w[:, None] * x16, k16), k32)
+                if "out" in ops:
+                    Yo = _round_op(np.exp2(cs)[:, None] * Craw, ops["out"], 1) @ _round_op(hst, ops["out"], 0)
+                else:
+                    Yo = _round(np.exp2(cs)[:, None] * Ct, kop) @ _round(hst, k16)
+                if "diag" in ops:
+                    Yd = _round_op(S, ops["diag"], 1) @ _round_op(xraw, ops["diag"], 0)
+                else:
+                    Yd = _round(S, k16) @ x16
+                Y = Yd + Yo
                 yt = _round(Y, "bf16") if rounding else Y
                 y[bb, t0:t0 + q, h] = yt[:q]
                 hst = _round(np.exp2(cs[q - 1]) * hst + s_tile, k32)

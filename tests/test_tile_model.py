@@ -112,3 +112,20 @@ def test_state_rows_are_separable():
     fs = np.concatenate([parts[0][1], parts[1][1]], axis=2)
     assert _rel(y, np.asarray(yr)) < 1e-12
     assert _rel(fs, np.asarray(fr)) < 1e-12
+
+
+def test_fp8_operands_miss_the_bound_on_every_gemm():
+    """The tolerance study behind fp8 tensor-core operands: rounding the two operands of any one
+    of the tile's GEMMs to fp8 (e4m3 or e5m2, one scale per row of A and per column of B, the
+    other GEMMs as the kernel has them) takes y far over the 1e-2 (1 + |ref|) bound on the bench
+    workload's distributions (seeded: 0.13 - 1.8), so fp8 is out for this path at that
+    tolerance.  Per GEMM, bf16 operands pass for C B^T (exact: B and C are bf16 inputs),
+    B^T (w o x) and C' h_prev, and fail only for S x."""
+    args, yr, _ = _case("mamba2_2.7b_layer", batch=1, seqlen=640, nheads=6)
+    for gemm in ("cb", "state", "out", "diag"):
+        for kind in ("e4m3", "e5m2"):
+            y, _ = tile_form(**args, rounding="kernel", operands={gemm: kind})
+            assert _rel(y, yr) > 0.1, (gemm, kind)
+    for gemm, passes in (("cb", True), ("state", True), ("out", True), ("diag", False)):
+        y, _ = tile_form(**args, rounding="kernel", operands={gemm: "bf16"})
+        assert (_rel(y, yr) < 1e-2) == passes, gemm
