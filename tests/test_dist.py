@@ -32,7 +32,7 @@ def _worker(rank, world, port, out):
 
 def test_timing_is_max_over_ranks_and_throughput_counts_all_replicas():
     world = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
