@@ -364,7 +364,9 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
     today: the E warps, between the state update of tile t - 1 and x_ready of tile t) or "Y"
     (a candidate: the four epilogue warps convert x of tile t + 1 as soon as B^T (w o x) of
     tile t has completed, and the E warps do only the state update, which then leaves the loop
-    between consecutive B^T (w o x) MMAs)."""
+    between consecutive B^T (w o x) MMAs), or "Y2" (the same, in two phases: x of tile t + 1 is
+    converted in place as soon as it has landed, kept in registers, and only w o x is written
+    after B^T (w o x) of tile t)."""
     m = Machine()
     for i in range(4):
         m.barrier(f"scan_done{i}", 1)
@@ -373,7 +375,7 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
         for name, count in (("full", 1), ("cb_full", 1), ("cb_free", 8), ("c_scaled", 8), ("s_ready", 8),
                             ("x_ready", 8), ("hs_ready", 8), ("e_done", 4), ("stg_free", 1), ("s_done", 1),
                             ("y_full", 1), ("fin", 1), ("st_free", 8)):
-            m.barrier(f"{name}{i}", count if not (name == "x_ready" and conv == "Y") else 4)
+            m.barrier(f"{name}{i}", count if not (name == "x_ready" and conv != "E") else 4)
     full_tile = lambda u: not (partial and u == nt - 1)
 
     def w19():      # decay scan into the four-slot ring
@@ -428,7 +430,7 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
             st, ph = t & 1, t >> 1
             if not (yield ("wait", f"x_ready{st}", ph)) or not (yield ("wait", f"full{st}", ph)):
                 break
-            if conv == "Y" and t >= 1 and "w17_st_free" not in drop:
+            if conv != "E" and t >= 1 and "w17_st_free" not in drop:
                 # the single s buffer: E has loaded s of tile t - 1
                 if not (yield ("wait", f"st_free{st ^ 1}", (t - 1) >> 1)):
                     break
@@ -484,16 +486,39 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
         yield ("arrive", f"x_ready{k & 1}", weight)
         return True
 
+    def convert_in_place(k):   # phase 1 of "Y2": x of tile k -> fp16 in place (kept in registers)
+        if not (yield ("wait", f"scan_done{k & 3}", k >> 2)) or not (yield ("wait", f"full{k & 1}", k >> 1)):
+            return False
+        yield ("read", f"ring{k & 3}")
+        yield ("arrive", f"scan_free{k & 3}", 4)
+        yield ("read", f"x{k & 1}")
+        yield ("write", f"x{k & 1}")
+        return True
+
+    def write_wx(k):           # phase 2 of "Y2": w o x from the registers
+        yield ("write", "wx")
+        yield ("arrive", f"x_ready{k & 1}", 4)
+
     def y_role():   # epilogue and TMA store of y
         stored = False
         if conv == "Y" and nt > 0 and not (yield from convert(0, 4)):
             return
+        if conv == "Y2" and nt > 0:
+            if not (yield from convert_in_place(0)):
+                return
+            yield from write_wx(0)
         for u in range(nt):
             st = u & 1
             if conv == "Y" and u + 1 < nt:
                 # w o x is free once B^T (w o x) of tile u has completed
                 if not (yield ("wait", f"s_done{st}", u >> 1)) or not (yield from convert(u + 1, 4)):
                     break
+            if conv == "Y2" and u + 1 < nt:
+                if not (yield from convert_in_place(u + 1)):
+                    break
+                if not (yield ("wait", f"s_done{st}", u >> 1)):
+                    break
+                yield from write_wx(u + 1)
             if not (yield ("wait", f"y_full{st}", u >> 1)):
                 break
             yield ("read", f"tY{st}")
@@ -522,13 +547,13 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
                 if 2 <= k < nt and "e_stg_free" not in drop:
                     if not (yield ("wait", f"stg_free{k & 1}", (k - 2) >> 1)):
                         break
-                if conv == "Y":
+                if conv != "E":
                     # 2^cs_last of tile u from the ring (ordered after the decay scan through
                     # x_ready -> s_done); the slot is released here
                     yield ("read", f"ring{u & 3}")
                     yield ("arrive", f"scan_free{u & 3}", 8)
                 yield ("read", "tSt")
-                if conv == "Y":
+                if conv != "E":
                     yield ("arrive", f"st_free{u & 1}", 8)
                 if k < nt:
                     yield ("write", f"hs{k & 1}")

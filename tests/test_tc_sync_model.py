@@ -232,10 +232,14 @@ def test_candidate_conversion_in_the_epilogue_warps():
     with pytest.raises(ProtocolError, match="race on tSt"):
         for nt in (2, 3, 5, 9):
             check(build_scan3, 40, seed=900 + nt, nt=nt, conv="Y", drop=frozenset(["w17_st_free"]))
-    # together with the zeroing of B rows past a sequence end
-    for nt in (1, 2, 5):
-        check(build_scan3, 30, seed=950 + nt, nt=nt, partial=True, conv="Y", zero_b="p")
-        check(build_scan3, 15, seed=960 + nt, nt=nt, partial=True, conv="Y", zero_b="p", faults=True)
+    # together with the zeroing of B rows past a sequence end, and in the two-phase form (x
+    # converted in place as soon as it lands, w o x written after B^T (w o x) of the tile before)
+    for conv in ("Y", "Y2"):
+        for nt in (1, 2, 5):
+            check(build_scan3, 30, seed=950 + nt, nt=nt, partial=True, conv=conv, zero_b="p")
+            check(build_scan3, 15, seed=960 + nt, nt=nt, partial=True, conv=conv, zero_b="p", faults=True)
+    for nt in (0, 3, 9):
+        check(build_scan3, 30, seed=970 + nt, nt=nt, conv="Y2")
 
 
 def test_role_leader_flag_needs_two_slots():
