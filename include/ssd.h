@@ -188,6 +188,19 @@ typedef struct {
 /* on != 0 turns event timing on, 0 off.  Returns the previous setting. */
 SSD_API int ssd_profile_enable(int on);
 
+/*
+ * Self-test of the bounded device waits.  Every mbarrier wait in the library's
+ * kernels gives up after a bounded number of SM clock cycles, records the
+ * timeout in a device status word and lets the kernel return.  This call runs
+ * that same wait, on `stream`, in one thread waiting on an mbarrier that
+ * nothing ever arrives at, with a limit of `limit_cycles` (1000 .. 4e9; about
+ * 2e6 is a millisecond).  It then synchronises `stream` and reads the status
+ * word.  Returns SSD_ERR_TIMEOUT when the path works (the wait ran out and was
+ * reported), SSD_ERR_SHAPE for a limit out of range, SSD_ERR_CUDA on a CUDA
+ * failure.  No fault, trap or hang is involved.
+ */
+SSD_API int ssd_selftest_bounded_wait(int64_t limit_cycles, void* stream);
+
 /* Waits for the recorded events, folds them into the per-kernel totals and
  * copies up to max_entries entries (kernels launched at least once) into
  * out.  reset != 0 clears all counters afterwards.  Returns the number of

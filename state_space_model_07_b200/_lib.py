@@ -15,7 +15,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE"
           5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA", 7: "SSD_ERR_TIMEOUT", 8: "SSD_ERR_SEQIDX"}
 # Every function include/ssd.h declares.
 EXPORTS = ("ssd_chunk_scan_fwd", "ssd_state_update", "ssd_status_string", "ssd_last_error",
-           "ssd_profile_enable", "ssd_profile_read", "ssd_chunk_scan_fwd_noalloc")
+           "ssd_profile_enable", "ssd_profile_read", "ssd_chunk_scan_fwd_noalloc", "ssd_selftest_bounded_wait")
 
 
 class SsdDims(ctypes.Structure):
@@ -63,6 +63,8 @@ def lib():
         L.ssd_profile_enable.argtypes = [ctypes.c_int]
         L.ssd_profile_read.restype = ctypes.c_int
         L.ssd_profile_read.argtypes = [ctypes.POINTER(SsdKernelStat), ctypes.c_int, ctypes.c_int]
+        L.ssd_selftest_bounded_wait.restype = ctypes.c_int
+        L.ssd_selftest_bounded_wait.argtypes = [ctypes.c_int64, _VP]
         _lib = L
     return _lib
 

@@ -313,6 +313,33 @@ int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const vo
 
 }  // extern "C"
 
+// ---- Self-test of the bounded device waits -------------------------------------------
+
+extern "C" int ssd_selftest_bounded_wait(int64_t limit_cycles, void* stream) {
+    g_last_error[0] = 0;
+    if (limit_cycles < 1000 || limit_cycles > 4000000000LL)
+        return fail(SSD_ERR_SHAPE, "limit_cycles %lld outside [1000, 4e9]", (long long)limit_cycles);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    cudaMemPool_t pool = workspace_pool();
+    if (!pool) return fail(SSD_ERR_CUDA, "could not create the workspace memory pool");
+    int32_t* status = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync((void**)&status, 256, pool, st);
+    if (e != cudaSuccess) return cuda_fail("cudaMallocFromPoolAsync(status)", e);
+    int rc = SSD_OK;
+    e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) rc = cuda_fail("status reset", e);
+    if (rc == SSD_OK) {
+        ssd::launch_selftest_wait((long long)limit_cycles, status, st);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) rc = cuda_fail("kernel launch", e);
+    }
+    if (rc == SSD_OK) rc = debug_sync(st, status);   // waits for the kernel, reads the status word
+    cudaError_t ef = cudaFreeAsync(status, st);
+    if (rc == SSD_OK && ef != cudaSuccess) rc = cuda_fail("cudaFreeAsync(status)", ef);
+    return rc;
+}
+
 // ---- Scan without any device allocation ---------------------------------------------
 //
 // Some callers cannot let a library allocate device memory: a serving engine

@@ -41,4 +41,8 @@ struct UpdateArgs {
 };
 void launch_state_update(const UpdateArgs& a, cudaStream_t st);
 
+// One thread waits, with the kernels' bounded wait and `limit_cycles`, on an
+// mbarrier nothing arrives at, and writes the outcome to *status.
+void launch_selftest_wait(long long limit_cycles, int32_t* status, cudaStream_t st);
+
 }  // namespace ssd

@@ -14,6 +14,7 @@ enum KernelId : int {
     K_STATE_UPDATE,
     K_TC_PREP,
     K_TC_SCAN,
+    K_SELFTEST_WAIT,
     K_COUNT
 };
 

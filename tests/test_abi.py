@@ -168,3 +168,14 @@ def test_python_wrapper_rejects_host_and_mistyped_tensors_before_any_call():
     st = torch.zeros(1, 2, 16, 16)
     with pytest.raises(ValueError, match="CUDA tensor"):
         ssd.state_update(st, x[:, 0], dt[:, 0], A, B[:, 0], B[:, 0])
+
+
+def test_selftest_wait_checks_its_limit_on_the_host(L):
+    assert L.ssd_selftest_bounded_wait(10, None) == 2
+    assert L.ssd_selftest_bounded_wait(5_000_000_000, None) == 2
+    assert "limit_cycles" in L.ssd_last_error().decode()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a CUDA device")
+def test_selftest_wait_without_device_reports_cuda_error(L):
+    assert L.ssd_selftest_bounded_wait(2_000_000, None) == 6
