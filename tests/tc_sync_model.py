@@ -349,12 +349,40 @@ class Machine:
 # catches each of them.
 
 
+def _prefixed(gen, pre: str, peer: str):
+    """Runs a role script inside one CTA of a cluster: every barrier and buffer name gets the
+    CTA's prefix, names written "peer:..." get the other CTA's (distributed shared memory)."""
+    nm = lambda x: peer + x[5:] if x.startswith("peer:") else pre + x
+
+    def conv(op):
+        k = op[0]
+        if k in ("wait", "bwait", "arrive", "arrive_tx", "commit"):
+            return (k, nm(op[1])) + tuple(op[2:])
+        if k in ("read", "write"):
+            return (k,) + tuple(nm(b) for b in op[1:])
+        if k == "tma_load":
+            return (k, nm(op[1]), nm(op[2]))
+        if k == "mma":
+            return (k, tuple(nm(b) for b in op[1]), tuple(nm(b) for b in op[2]))
+        if k == "store":
+            return (k, tuple(nm(b) for b in op[1]))
+        return op
+
+    try:
+        op = gen.send(None)
+        while True:
+            val = yield conv(op)
+            op = gen.send(val)
+    except StopIteration:
+        return
+
+
 # The decoupled-state kernel (k_tc_scan3, d_state 128).  `nt` tiles of 128
 # tokens; `partial` = the last tile is shorter (its y leaves by row stores,
 # not through the staging tile).
 
 def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), zero_b: str = "",
-                conv: str = "E") -> Machine:
+                conv: str = "E", m: Machine | None = None, rank: int | None = None) -> Machine:
     """`zero_b` models ways of zeroing the B rows past the sequence end in a partial last tile
     (not done by the kernel today): "p" has the P warps do it right after C B^T has read B
     (cb_full), with W17 waiting for c_scaled before B^T (w o x) on that tile; "e" has the E
@@ -366,16 +394,24 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
     tile t has completed, and the E warps do only the state update, which then leaves the loop
     between consecutive B^T (w o x) MMAs), or "Y2" (the same, in two phases: x of tile t + 1 is
     converted in place as soon as it has landed, kept in registers, and only w o x is written
-    after B^T (w o x) of tile t)."""
-    m = Machine()
+    after B^T (w o x) of tile t).
+
+    `rank` (0 or 1, with a shared `m`) builds one CTA of the d_state 256 pair candidate (see
+    build_scan3_pair): C gets one shared-memory stage on its own barrier, and the epilogues
+    exchange Y through distributed shared memory."""
+    pre, peer = ("", "") if rank is None else (("a.", "b.") if rank == 0 else ("b.", "a."))
+    m = m or Machine()
+    reg = lambda name, count: m.barrier(pre + name, count)
     for i in range(4):
-        m.barrier(f"scan_done{i}", 1)
-        m.barrier(f"scan_free{i}", 16 if conv == "E" else 20)
+        reg(f"scan_done{i}", 1)
+        reg(f"scan_free{i}", 16 if conv == "E" else 20)
     for i in range(2):
         for name, count in (("full", 1), ("cb_full", 1), ("cb_free", 8), ("c_scaled", 8), ("s_ready", 8),
                             ("x_ready", 8), ("hs_ready", 8), ("e_done", 4), ("stg_free", 1), ("s_done", 1),
-                            ("y_full", 1), ("fin", 1), ("st_free", 8)):
-            m.barrier(f"{name}{i}", count if not (name == "x_ready" and conv != "E") else 4)
+                            ("y_full", 1), ("fin", 1), ("st_free", 8), ("rcv_full", 1), ("rcv_free", 1)):
+            reg(f"{name}{i}", count if not (name == "x_ready" and conv != "E") else 4)
+    reg("cfull", 1)
+    pair = rank is not None
     full_tile = lambda u: not (partial and u == nt - 1)
 
     def w19():      # decay scan into the four-slot ring
@@ -394,14 +430,23 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
             if u >= 2 and "w16_y_full" not in drop:
                 if not (yield ("wait", f"y_full{st}", (u - 2) >> 1)):
                     break
-            yield ("arrive_tx", f"full{st}", 3)
-            for buf in ("x", "b", "c"):
+            yield ("arrive_tx", f"full{st}", 2 if pair else 3)
+            for buf in (("x", "b") if pair else ("x", "b", "c")):
                 yield ("tma_load", f"full{st}", f"{buf}{st}")
             issued += 1
+            if pair:
+                # one C stage: free once the copy of C(u - 1) to TMEM has completed
+                if u >= 1 and "pair_c_stage" not in drop:
+                    if not (yield ("wait", f"cb_full{st ^ 1}", (u - 1) >> 1)):
+                        break
+                yield ("arrive_tx", "cfull", 1)
+                yield ("tma_load", "cfull", "c0")
         if m.abort and "w16_drain" not in drop:
             # let the copies in flight land before the CTA exits
             for u in range(issued):
                 yield ("bwait", f"full{u & 1}", u >> 1)
+                if pair:
+                    yield ("bwait", "cfull", u)
 
     def w18():      # C -> TMEM copy and C B^T
         if nt == 0:
@@ -413,7 +458,9 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
             if t >= 2 and "w18_y_full" not in drop:
                 if not (yield ("wait", f"y_full{st}", (t - 2) >> 1)):
                     break
-            yield ("mma", (f"c{st}",), (f"tC{st}",))                       # tcgen05.cp
+            if pair and not (yield ("wait", "cfull", t)):
+                break
+            yield ("mma", ("c0" if pair else f"c{st}",), (f"tC{st}",))     # tcgen05.cp
             if t >= 1 and "w18_cb_free" not in drop:
                 if not (yield ("wait", f"cb_free{st ^ 1}", (t - 1) >> 1)):
                     break
@@ -522,6 +569,22 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
             if not (yield ("wait", f"y_full{st}", u >> 1)):
                 break
             yield ("read", f"tY{st}")
+            if rank == 1:
+                # the second CTA hands its fp32 Y partial to the first one's shared memory
+                yield ("arrive", f"e_done{st}", 4)
+                if u >= 2 and "pair_rcv_free" not in drop:
+                    if not (yield ("wait", f"rcv_free{st}", (u - 2) >> 1)):
+                        break
+                yield ("write", f"peer:rcv{st}")
+                yield ("arrive", f"peer:rcv_full{st}")
+                yield ("arrive", f"stg_free{st}")
+                continue
+            if rank == 0:
+                if "pair_rcv_full" not in drop:
+                    if not (yield ("wait", f"rcv_full{st}", u >> 1)):
+                        break
+                yield ("read", f"rcv{st}")
+                yield ("arrive", f"peer:rcv_free{st}")
             if full_tile(u):
                 yield ("write", f"hs{st}")
             yield ("arrive", f"e_done{st}", 4)
@@ -564,7 +627,20 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
 
     for name, gen in (("W19", w19()), ("W16", w16()), ("W18", w18()), ("W17", w17()), ("P", p_role()),
                       ("Y", y_role()), ("E", e_role())):
-        m.role(name, gen)
+        m.role(pre + name, _prefixed(gen, pre, peer) if pair else gen)
+    return m
+
+
+def build_scan3_pair(nt: int, partial: bool = False, drop: frozenset = frozenset(), zero_b: str = "",
+                     conv: str = "E") -> Machine:
+    """The d_state 256 candidate: a cluster of two CTAs, each running the k_tc_scan3 roles on
+    one half of the state rows (B and C halves), with one shared-memory stage for C.  The
+    second CTA's epilogue writes its fp32 Y partial into the first CTA's receive buffer
+    (two, by tile parity) and arrives on its rcv_full; the first CTA's epilogue adds it, stores
+    y and arrives on the second CTA's rcv_free.  Both CTAs leave together (a cluster barrier)."""
+    m = Machine()
+    build_scan3(nt, partial, drop, zero_b, conv, m=m, rank=0)
+    build_scan3(nt, partial, drop, zero_b, conv, m=m, rank=1)
     return m
 
 
