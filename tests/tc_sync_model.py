@@ -572,19 +572,20 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
             if rank == 1:
                 # the second CTA hands its fp32 Y partial to the first one's shared memory
                 yield ("arrive", f"e_done{st}", 4)
-                if u >= 2 and "pair_rcv_free" not in drop:
-                    if not (yield ("wait", f"rcv_free{st}", (u - 2) >> 1)):
+                # one receive buffer (32 KB): free once the first CTA has read tile u - 1's
+                if u >= 1 and "pair_rcv_free" not in drop:
+                    if not (yield ("wait", "rcv_free0", u - 1)):
                         break
-                yield ("write", f"peer:rcv{st}")
-                yield ("arrive", f"peer:rcv_full{st}")
+                yield ("write", "peer:rcv0")
+                yield ("arrive", "peer:rcv_full0")
                 yield ("arrive", f"stg_free{st}")
                 continue
             if rank == 0:
                 if "pair_rcv_full" not in drop:
-                    if not (yield ("wait", f"rcv_full{st}", u >> 1)):
+                    if not (yield ("wait", "rcv_full0", u)):
                         break
-                yield ("read", f"rcv{st}")
-                yield ("arrive", f"peer:rcv_free{st}")
+                yield ("read", "rcv0")
+                yield ("arrive", "peer:rcv_free0")
             if full_tile(u):
                 yield ("write", f"hs{st}")
             yield ("arrive", f"e_done{st}", 4)
@@ -635,9 +636,10 @@ def build_scan3_pair(nt: int, partial: bool = False, drop: frozenset = frozenset
                      conv: str = "E") -> Machine:
     """The d_state 256 candidate: a cluster of two CTAs, each running the k_tc_scan3 roles on
     one half of the state rows (B and C halves), with one shared-memory stage for C.  The
-    second CTA's epilogue writes its fp32 Y partial into the first CTA's receive buffer
-    (two, by tile parity) and arrives on its rcv_full; the first CTA's epilogue adds it, stores
-    y and arrives on the second CTA's rcv_free.  Both CTAs leave together (a cluster barrier)."""
+    second CTA's epilogue writes its fp32 Y partial into the first CTA's receive buffer (one,
+    32 KB: what the single C stage frees) and arrives on its rcv_full; the first CTA's epilogue
+    adds it, stores y and arrives on the second CTA's rcv_free.  Both CTAs leave together (a
+    cluster barrier)."""
     m = Machine()
     build_scan3(nt, partial, drop, zero_b, conv, m=m, rank=0)
     build_scan3(nt, partial, drop, zero_b, conv, m=m, rank=1)

@@ -260,7 +260,7 @@ def test_dstate_256_pair_candidate():
     """The d_state 256 candidate: two CTAs of a cluster run the k_tc_scan3 roles on the two
     halves of the state rows, C has one shared-memory stage (reloaded once its copy to TMEM has
     completed), and the second CTA's fp32 Y partial travels to the first CTA through distributed
-    shared memory (rcv_full / rcv_free by tile parity).  Clean, also on the timeout path and
+    shared memory (one receive buffer, rcv_full / rcv_free).  Clean, also on the timeout path and
     with the conversion and tail-zeroing candidates; each of its three new waits is needed."""
     from tests.tc_sync_model import build_scan3_pair
     for nt in (0, 1, 2, 3, 5, 9):
@@ -269,7 +269,7 @@ def test_dstate_256_pair_candidate():
             check(build_scan3_pair, 8, seed=1100 + nt, nt=nt, partial=partial, faults=True)
     for nt in (2, 5):
         check(build_scan3_pair, 15, seed=1200 + nt, nt=nt, partial=True, conv="Y2", zero_b="p")
-    for drop, what in (("pair_rcv_full", r"a\.rcv"), ("pair_rcv_free", r"a\.rcv"),
+    for drop, what in (("pair_rcv_full", r"a\.rcv"), ("pair_rcv_free", r"rcv"),
                        ("pair_c_stage", r"cfull|c0")):
         with pytest.raises(ProtocolError, match=what):
             for nt in (3, 5, 8):
