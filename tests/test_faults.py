@@ -48,3 +48,72 @@ def test_context_stays_usable_after_a_timeout():
     yr, fr = oracle_scan(to_cpu(d))
     assert_close(y, yr, TOL[torch.bfloat16], "y after a timeout")
     assert_close(fs, fr, TOL[torch.bfloat16], "final_state after a timeout")
+
+
+# --- every output element is written -------------------------------------------------------
+
+CANARY_CASES = [
+    ("tensor-core, ragged", dict(name="mamba2_2.7b_layer", batch=2, seqlen=333, nheads=4), None),
+    ("tensor-core, packed", dict(name="packed_varlen", nheads=4, dstate=128), [300, 17, 129, 128, 1]),
+    ("tensor-core, d_state 256, packed", dict(name="packed_varlen", nheads=4), [200, 1, 130]),
+    ("CUDA cores, fp32", dict(name="tiny_fp32", seqlen=77), None),
+]
+
+
+@pytest.mark.parametrize("what,kw,lens", CANARY_CASES, ids=[c[0] for c in CANARY_CASES])
+def test_every_output_element_is_written(what, kw, lens):
+    """y and final_state start as NaN: after the call none may be left (inputs are finite)."""
+    kw = dict(kw)
+    w = inputs.scaled(inputs.WORKLOADS[kw.pop("name")], **kw)
+    d = inputs.make_inputs(w, "cuda", lengths=lens)
+    y = torch.full_like(d["x"], float("nan"))
+    S = d["nseqs"]
+    fs = torch.full((S, w.nheads, w.dstate, w.headdim), float("nan"), device="cuda")
+    ssd.chunk_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_bias=d["dt_bias"], D=d["D"],
+                       init_state=d["init_state"], seq_idx=d["seq_idx"], nseqs=S, chunk=w.chunk, y=y,
+                       final_state=fs)
+    torch.cuda.synchronize()
+    assert not torch.isnan(y).any(), what
+    assert not torch.isnan(fs).any(), what
+
+
+# --- a broken seq_idx is reported in debug mode -------------------------------------------------
+
+_BROKEN_SEQ_IDX = r"""
+import sys, torch
+sys.path.insert(0, {root!r})
+import state_space_model_07_b200 as ssd
+from state_space_model_07_b200 import inputs
+w = inputs.scaled(inputs.WORKLOADS["packed_varlen"], nheads=4, dstate=128)
+d = inputs.make_inputs(w, "cuda", lengths=[100, 50, 30])
+si = d["seq_idx"].clone()
+si[0, 100:] += 1          # 0 -> 2 at token 100 (a step of +2), and it ends at 3 > nseqs - 1
+try:
+    ssd.chunk_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_bias=d["dt_bias"], D=d["D"],
+                       init_state=d["init_state"], seq_idx=si, nseqs=3, chunk=w.chunk)
+    torch.cuda.synchronize()
+    print("status 0")
+except ssd.SsdError as e:
+    print("status", e.code)
+# the context is still usable: a valid call right after
+y, fs = ssd.chunk_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_bias=d["dt_bias"], D=d["D"],
+                           init_state=d["init_state"], seq_idx=d["seq_idx"], nseqs=3, chunk=w.chunk)
+torch.cuda.synchronize()
+print("after ok", bool(torch.isfinite(y).all()))
+"""
+
+
+def test_broken_seq_idx_is_reported_in_debug_mode():
+    """With SSD_DEBUG_CHECK=1 every call synchronises and reads the device status word: a
+    seq_idx that breaks its contract comes back as SSD_ERR_SEQIDX (8), never as an
+    out-of-bounds access, and the next valid call works."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SSD_DEBUG_CHECK="1")
+    out = subprocess.run([sys.executable, "-c", _BROKEN_SEQ_IDX.format(root=root)], env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert "status 8" in out.stdout, out.stdout
+    assert "after ok True" in out.stdout, out.stdout
