@@ -77,12 +77,15 @@ def _mask(CB, cs, d, Dh, q):
     return S
 
 
-def tile_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, rounding=None, operands=None):
+def tile_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, rounding=None, operands=None, stats=None):
     """x (b,L,H,P), dt (b,L,H), B/C (b,L,G,N), A/dt_bias/D (H,), init_state (b,H,N,P).
 
     `operands` (with rounding="kernel") overrides the operand type of single GEMMs: keys "cb"
     (C B^T), "state" (B^T (w o x)), "out" (C' h_prev), "diag" (S x); values "f16", "bf16",
     "e4m3", "e5m2" (fp8 with one scale per row of A and per column of B).
+
+    `stats` (a dict) collects the largest magnitude of each thread-made tensor-core operand
+    ("S", "h_prev", "wx", "Cp"), to check their fp16 range.
 
     Returns (y, final_state) as fp64 arrays."""
     ops = dict(operands or {})
@@ -122,6 +125,10 @@ def tile_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, rounding=No
                     CB = _round(Ct @ Bt.T, k32)
                 S = _mask(CB, cs, d, Dv[h], q)
                 w = d * np.exp2(cs[q - 1] - cs)
+                if stats is not None:
+                    for k, v in (("S", S), ("h_prev", hst), ("wx", w[:, None] * xraw),
+                                 ("Cp", np.exp2(cs)[:, None] * Craw)):
+                        stats[k] = max(stats.get(k, 0.0), float(np.max(np.abs(v))))
                 if "state" in ops:
                     s_tile = _round(_round_op(Braw, ops["state"], 0).T @ _round_op(w[:, None] * xraw, ops["state"], 0), k32)
                 else:
