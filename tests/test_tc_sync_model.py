@@ -240,6 +240,12 @@ def test_candidate_conversion_in_the_epilogue_warps():
             check(build_scan3, 15, seed=960 + nt, nt=nt, partial=True, conv=conv, zero_b="p", faults=True)
     for nt in (0, 3, 9):
         check(build_scan3, 30, seed=970 + nt, nt=nt, conv="Y2")
+    # the lean form of the draft: without the two waits that other waits imply (W18's y_full,
+    # W17's e_done, hence no e_done barrier at all)
+    lean = frozenset(["w17_e_done", "w18_y_full"])
+    for nt in (1, 2, 5, 9):
+        check(build_scan3, 30, seed=980 + nt, nt=nt, partial=True, conv="Y2", zero_b="p", drop=lean)
+        check(build_scan3, 15, seed=990 + nt, nt=nt, partial=True, conv="Y2", zero_b="p", drop=lean, faults=True)
 
 
 def test_role_leader_flag_needs_two_slots():
