@@ -31,9 +31,22 @@ def _sigmoid(z):
     return np.where(z >= 0, 1.0 / (1.0 + np.exp(-np.abs(z))), np.exp(-np.abs(z)) / (1.0 + np.exp(-np.abs(z))))
 
 
-def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfinal=None, Q=16):
+def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfinal=None, Q=16, operands=None):
     """x, dy (b,L,H,P); dt (b,L,H); B, C (b,L,G,N); A, dt_bias, D (H,); init_state, dfinal
-    (b,H,N,P) or None.  Returns the same dict of gradients as the oracle."""
+    (b,H,N,P) or None.  Returns the same dict of gradients as the oracle.
+
+    `operands` ("f16" or "bf16") rounds both operands of every matrix product (the work a
+    tensor-core kernel would do) to that type, with products and sums kept in fp32; the
+    decay arithmetic stays in fp64.  None: everything fp64."""
+    if operands is None:
+        rd = lambda a: a
+        mm = lambda a, b: a @ b
+    else:
+        import torch
+        dt_ = {"f16": torch.float16, "bf16": torch.bfloat16}[operands]
+        rd = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dt_).double().numpy()
+        f32 = lambda a: np.asarray(a, dtype=np.float32).astype(np.float64)
+        mm = lambda a, b: f32(rd(a) @ rd(b))
     x, dt, B, C, dy = (np.asarray(v, dtype=np.float64) for v in (x, dt, B, C, dy))
     A = np.asarray(A, dtype=np.float64)
     b, L, H, P = x.shape
@@ -56,7 +69,7 @@ def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfina
                 t1 = min(t0 + Q, L)
                 cs = np.cumsum(d[t0:t1] * A[h])
                 u = np.exp(cs[-1] - cs) * d[t0:t1]
-                h_prev.append(np.exp(cs[-1]) * h_prev[-1] + (B[bb, t0:t1, g] * u[:, None]).T @ x[bb, t0:t1, h])
+                h_prev.append(np.exp(cs[-1]) * h_prev[-1] + mm((B[bb, t0:t1, g] * u[:, None]).T, x[bb, t0:t1, h]))
             # backward over chunks, last first
             dh_end = dfin[bb, h].copy()
             for c in reversed(range(len(starts))):
@@ -71,14 +84,14 @@ def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfina
                 q = t1 - t0
                 mask = np.tril(np.ones((q, q), dtype=bool))
                 Lm = np.where(mask, np.exp(np.where(mask, cs[:, None] - cs[None, :], 0.0)), 0.0)  # [j, i]
-                CB = Cc @ Bc.T                                   # [j, i]
+                CB = mm(Cc, Bc.T)                                # [j, i]
                 W = CB * Lm * dc[None, :]
-                dyx = dyc @ xc.T                                 # [j, i] = dy_j . x_i
+                dyx = mm(dyc, xc.T)                              # [j, i] = dy_j . x_i
                 # x, B, C, D
-                dx = Dv[h] * dyc + W.T @ dyc + u[:, None] * (Bc @ dh_end)
+                dx = Dv[h] * dyc + mm(W.T, dyc) + u[:, None] * mm(Bc, dh_end)
                 K = Lm * dyx * dc[None, :]                       # [j, i]
-                dB = K.T @ Cc + u[:, None] * (xc @ dh_end.T)
-                dC = K @ Bc + e[:, None] * (dyc @ hp.T)
+                dB = mm(K.T, Cc) + u[:, None] * mm(xc, dh_end.T)
+                dC = mm(K, Bc) + e[:, None] * mm(dyc, hp.T)
                 out["x"][bb, t0:t1, h] += dx
                 out["B"][bb, t0:t1, g] += dB
                 out["C"][bb, t0:t1, g] += dC
@@ -99,6 +112,6 @@ def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfina
                 out["dt"][bb, t0:t1, h] += dz
                 out["dt_bias"][h] += np.sum(dz)
                 # reverse state passing
-                dh_end = E * dh_end + (Cc * e[:, None]).T @ dyc
+                dh_end = E * dh_end + mm((Cc * e[:, None]).T, dyc)
             out["init_state"][bb, h] = dh_end
     return out
