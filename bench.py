@@ -107,7 +107,7 @@ REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_c
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML while the timed region runs."""
 
-    def __init__(self, torch_device, period_s=0.002):
+    def __init__(self, torch_device, period_s=0.0005):
         self.period = period_s
         self.samples = []
         self.max_mhz = None
@@ -368,13 +368,15 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    for k in range(args.warmup):
-        step(k)
-    barrier()
-    _lib.profile_read(reset=True)
-    _lib.profile_enable(True)
+    # clocks are sampled through the warm-up steps and the timed region (both keep the GPU busy),
+    # so that a short timed region still has several samples under load
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev) as clk:
+        for k in range(args.warmup):
+            step(k)
+        barrier()
+        _lib.profile_read(reset=True)
+        _lib.profile_enable(True)
         barrier()
         e0.record(stream)
         for k in range(args.steps):

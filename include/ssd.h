@@ -61,7 +61,9 @@ typedef enum {
     SSD_ERR_UNSUPPORTED = 5, /* valid request this build does not implement         */
     SSD_ERR_CUDA = 6,        /* a CUDA call failed; see ssd_last_error()            */
     SSD_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up (debug check)     */
-    SSD_ERR_SEQIDX = 8       /* seq_idx breaks its contract (debug check only)       */
+    SSD_ERR_SEQIDX = 8,      /* seq_idx breaks its contract (debug check only)       */
+    SSD_ERR_RANGE = 9        /* values outside the tensor-core path's fp16 operand
+                                range (debug check only; see ssd_chunk_scan_fwd)    */
 } ssd_status;
 
 /* Problem sizes.  b = batch, L = seqlen, H = nheads, P = headdim, N = dstate,
@@ -100,6 +102,20 @@ typedef struct {
  *
  * Supported sizes: P and N multiples of 16 with 16 <= P, N <= 256; H % G == 0;
  * b, L >= 0 (empty inputs are a no-op apart from final_state = init_state).
+ *
+ * Value range.  bf16 calls with P = 64, N in {128, 256} and chunk in {128, 256}
+ * run on the tensor cores, whose operands are fp16 (11-bit significand, largest
+ * finite value 65504) with fp32 accumulation; every other call runs on CUDA
+ * cores in fp32.  On the tensor-core path:
+ *   - every x, B, C and init_state value must be finite with magnitude at most
+ *     65504 (a larger bf16 value cannot be represented and becomes inf);
+ *   - the masked score matrix (C_j . B_i) exp(sum of d A from i+1 to j) d_i and
+ *     the state carried between 128-token tiles must also stay within 65504
+ *     in magnitude (for N(0,1) inputs of the sizes above they stay below ~20,
+ *     so B and C may grow ~58x, x and the state ~2e4x, before this binds).
+ * Outside these limits the result holds inf or NaN where the recurrence is
+ * finite.  With SSD_DEBUG_CHECK=1 such calls return SSD_ERR_RANGE: an input
+ * beyond 65504, or a non-finite y / final_state from finite inputs.
  * Returns an ssd_status.
  */
 SSD_API int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
@@ -123,6 +139,7 @@ SSD_API int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* 
  *           arguments keep the order of the problem statement; it must be the
  *           same bias the prefill scan used for the continuation to be exact.
  * Uses dims->batch, nheads, headdim, dstate, ngroups, dtype (seqlen, nseqs ignored).
+ * state, x and y must be 16-byte aligned (SSD_ERR_SHAPE otherwise).
  */
 SSD_API int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const void* dt,
                      const float* A, const void* B, const void* C, const float* D, void* y,

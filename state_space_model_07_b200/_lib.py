@@ -12,7 +12,8 @@ PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
 
 SSD_F32, SSD_BF16 = 0, 1
 STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE", 4: "SSD_ERR_CHUNK",
-          5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA", 7: "SSD_ERR_TIMEOUT", 8: "SSD_ERR_SEQIDX"}
+          5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA", 7: "SSD_ERR_TIMEOUT", 8: "SSD_ERR_SEQIDX",
+          9: "SSD_ERR_RANGE"}
 # Every function include/ssd.h declares.
 EXPORTS = ("ssd_chunk_scan_fwd", "ssd_state_update", "ssd_status_string", "ssd_last_error",
            "ssd_profile_enable", "ssd_profile_read", "ssd_chunk_scan_fwd_noalloc", "ssd_selftest_bounded_wait")

@@ -109,8 +109,9 @@ cudaMemPool_t workspace_pool() {
     return pools[dev];
 }
 
-// Waits for the stream and reports device-side status (debug mode only).
-int debug_sync(cudaStream_t st, const int32_t* status_dev) {
+// Waits for the stream and reports device-side status (debug mode only):
+// the status word and, after a tensor-core scan, the value-check counters.
+int debug_sync(cudaStream_t st, const int32_t* status_dev, const uint32_t* counters_dev = nullptr) {
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail("kernel execution", e);
     if (status_dev) {
@@ -119,6 +120,19 @@ int debug_sync(cudaStream_t st, const int32_t* status_dev) {
         if (e != cudaSuccess) return cuda_fail("status read", e);
         if (s == ssd::kStatusSeqIdx) return fail(SSD_ERR_SEQIDX, "seq_idx breaks its contract");
         if (s == ssd::kStatusTimeout) return fail(SSD_ERR_TIMEOUT, "a bounded device wait gave up");
+    }
+    if (counters_dev) {
+        uint32_t c[3] = {0, 0, 0};
+        e = cudaMemcpy(c, counters_dev, sizeof(c), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail("value-check read", e);
+        if (c[1])
+            return fail(SSD_ERR_RANGE,
+                        "%u finite x, B, C or init_state values exceed 65504, the fp16 operand range of the "
+                        "tensor-core path", c[1]);
+        if (c[2] && !c[0])
+            return fail(SSD_ERR_RANGE,
+                        "finite inputs gave %u non-finite outputs: an intermediate (score matrix or carried "
+                        "state) left the fp16 operand range of the tensor-core path", c[2]);
     }
     return SSD_OK;
 }
@@ -200,11 +214,15 @@ size_t scan_table_bytes(const ssd::ScanArgs& a) {
 }
 
 // Carves the status word and the sequence table out of `cv` (after the path's
-// workspace), fills the sequence description and, for packed input, launches
-// the kernels that build the table.
-ssd::SeqInfo scan_tables(const ssd::ScanArgs& a, Carve& cv, bool dbg, int32_t** status, cudaStream_t st) {
+// workspace), fills the sequence description *out and, for packed input,
+// launches the kernels that build the table.  Returns an ssd_status.
+int scan_tables(const ssd::ScanArgs& a, Carve& cv, bool dbg, int32_t** status, ssd::SeqInfo* out,
+                cudaStream_t st) {
     *status = (int32_t*)cv.take(sizeof(int32_t));
-    if (dbg) cudaMemsetAsync(*status, 0, sizeof(int32_t), st);
+    if (dbg) {
+        cudaError_t e = cudaMemsetAsync(*status, 0, sizeof(int32_t), st);
+        if (e != cudaSuccess) return cuda_fail("status word reset", e);
+    }
     ssd::SeqInfo si;
     si.L = a.L; si.S = (int32_t)a.S; si.Q = a.Q; si.packed = a.seq_idx ? 1 : 0;
     si.nc_row = (int32_t)((a.L + a.Q - 1) / a.Q);
@@ -216,7 +234,8 @@ ssd::SeqInfo scan_tables(const ssd::ScanArgs& a, Carve& cv, bool dbg, int32_t** 
         ssd::launch_seq_table(a.seq_idx, a.L, (int32_t)a.S, a.Q, start, end, off, dbg ? *status : nullptr, st);
         si.start = start; si.end = end; si.chunk_off = off;
     }
-    return si;
+    *out = si;
+    return SSD_OK;
 }
 
 }  // namespace
@@ -234,6 +253,7 @@ const char* ssd_status_string(int s) {
         case SSD_ERR_CUDA: return "CUDA error";
         case SSD_ERR_TIMEOUT: return "bounded device wait timed out";
         case SSD_ERR_SEQIDX: return "seq_idx breaks its contract";
+        case SSD_ERR_RANGE: return "values outside the fp16 operand range of the tensor-core path";
         default: return "unknown status";
     }
 }
@@ -259,7 +279,8 @@ int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, cons
     const size_t ws_path = use_tc ? ssd::tc_workspace_bytes(a, max_chunks)
                                   : ssd::simt_workspace_bytes(a, max_chunks);
     const bool dbg = debug_check();
-    const size_t ws_bytes = Carve::round(ws_path) + scan_table_bytes(a);
+    const bool value_check = dbg && use_tc;
+    const size_t ws_bytes = Carve::round(ws_path) + scan_table_bytes(a) + (value_check ? Carve::round(16) : 0);
 
     Carve cv;
     cudaMemPool_t pool = workspace_pool();
@@ -268,14 +289,29 @@ int ssd_chunk_scan_fwd(const ssd_dims* dims, const void* x, const void* dt, cons
     if (e != cudaSuccess) return cuda_fail("cudaMallocFromPoolAsync(workspace)", e);
     void* ws_main = cv.take(ws_path);
     int32_t* status = nullptr;
-    const ssd::SeqInfo si = scan_tables(a, cv, dbg, &status, st);
-    if (use_tc)
-        rc = ssd::launch_tc_scan(a, si, max_chunks, ws_main, dbg ? status : nullptr, st);
-    else
-        ssd::launch_simt_scan(a, si, max_chunks, ws_main, st);
+    ssd::SeqInfo si;
+    rc = scan_tables(a, cv, dbg, &status, &si, st);
+    if (rc) {
+        cudaFreeAsync(cv.base, st);
+        return rc;
+    }
+    uint32_t* counters = nullptr;
+    if (value_check) {
+        counters = (uint32_t*)cv.take(16);
+        e = cudaMemsetAsync(counters, 0, 16, st);
+        if (e != cudaSuccess) rc = cuda_fail("value-check reset", e);
+        else ssd::launch_range_check_inputs(a, counters, st);
+    }
+    if (rc == SSD_OK) {
+        if (use_tc)
+            rc = ssd::launch_tc_scan(a, si, max_chunks, ws_main, dbg ? status : nullptr, st);
+        else
+            ssd::launch_simt_scan(a, si, max_chunks, ws_main, st);
+    }
+    if (rc == SSD_OK && value_check) ssd::launch_range_check_outputs(a, counters, st);
     e = cudaGetLastError();
     if (rc == SSD_OK && e != cudaSuccess) rc = cuda_fail("kernel launch", e);
-    if (rc == SSD_OK && dbg) rc = debug_sync(st, status);
+    if (rc == SSD_OK && dbg) rc = debug_sync(st, status, counters);
     cudaError_t ef = cudaFreeAsync(cv.base, st);
     if (rc == SSD_OK && ef != cudaSuccess) rc = cuda_fail("cudaFreeAsync(workspace)", ef);
     return rc;
@@ -292,12 +328,13 @@ int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const vo
     if (b == 0) return SSD_OK;
     if (!state || !x || !dt || !A || !B || !C || !y)
         return fail(SSD_ERR_NULL, "state, x, dt, A, B, C and y are required");
-    if (!aligned16(state)) return fail(SSD_ERR_SHAPE, "state must be 16-byte aligned");
+    if (!aligned16(state) || !aligned16(x) || !aligned16(y))
+        return fail(SSD_ERR_SHAPE, "state, x and y must be 16-byte aligned");
     const size_t es = dims->dtype == SSD_BF16 ? 2 : 4;
     if (overlaps(y, (size_t)b * H * P * es, state, (size_t)b * H * N * P * 4) ||
         overlaps(y, (size_t)b * H * P * es, x, (size_t)b * H * P * es))
         return fail(SSD_ERR_SHAPE, "y overlaps state or x");
-    if (b * H > 0x7fffffffLL) return fail(SSD_ERR_SHAPE, "batch * nheads too large");
+    if (b * H > 0x7fffffffLL / 8) return fail(SSD_ERR_SHAPE, "batch * nheads too large");
     cudaStream_t st = (cudaStream_t)stream;
     cudaGetLastError();
     ssd::UpdateArgs a;
@@ -417,7 +454,9 @@ extern "C" int ssd_chunk_scan_fwd_noalloc(const ssd_dims* dims, const void* x, c
     void* ws_main = cv.take(ws_path);
     const bool dbg = debug_check();
     int32_t* status = nullptr;
-    const ssd::SeqInfo si = scan_tables(a, cv, dbg, &status, st);
+    ssd::SeqInfo si;
+    rc = scan_tables(a, cv, dbg, &status, &si, st);
+    if (rc) return rc;
     ssd::launch_simt_scan(a, si, max_chunks, ws_main, st);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("kernel launch", e);

@@ -41,6 +41,12 @@ struct UpdateArgs {
 };
 void launch_state_update(const UpdateArgs& a, cudaStream_t st);
 
+// Debug-mode value checks around a tensor-core scan (ssd_check.cu): counters[0]
+// += non-finite inputs, counters[1] += finite x / B / C / init_state values
+// beyond the fp16 range, counters[2] += non-finite outputs.
+void launch_range_check_inputs(const ScanArgs& a, uint32_t* counters, cudaStream_t st);
+void launch_range_check_outputs(const ScanArgs& a, uint32_t* counters, cudaStream_t st);
+
 // One thread waits, with the kernels' bounded wait and `limit_cycles`, on an
 // mbarrier nothing arrives at, and writes the outcome to *status.
 void launch_selftest_wait(long long limit_cycles, int32_t* status, cudaStream_t st);

@@ -38,9 +38,11 @@
 // All waits are bounded: on a timeout the kernel records SSD_ERR_TIMEOUT in the
 // status word and returns after freeing its TMEM.
 #include <cuda.h>
+#include <algorithm>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <stdio.h>
+#include <stdlib.h>
 
 #include "ssd_common.cuh"
 #include "ssd_prof.h"
@@ -82,7 +84,7 @@ struct Cfg {
 
 struct TcCtl {
     int abort;
-    int p_flag, e_flag, y_flag;    // leader-wait results handed to the rest of a role
+    int p_flag, e_flag;            // leader-wait results handed to the rest of a role (k_tc_scan<N>)
 };
 
 template <int N>
@@ -441,8 +443,10 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 uint32_t sv[8];
 #pragma unroll
                 for (int k = 0; k < 16; k += 2) {
-                    float v0 = __uint_as_float(r[k]) * f[k];
-                    float v1 = __uint_as_float(r[k + 1]) * f[k + 1];
+                    // a select, not a multiply by zero: C B^T above the diagonal may hold B rows
+                    // of the next packed sequence (past this one's end), and inf * 0 is NaN
+                    float v0 = i0 + k <= j ? __uint_as_float(r[k]) * f[k] : 0.f;
+                    float v1 = i0 + k + 1 <= j ? __uint_as_float(r[k + 1]) * f[k + 1] : 0.f;
                     if (i0 + k == j) v0 += Dh;
                     if (i0 + k + 1 == j) v1 += Dh;
                     sv[k / 2] = pack_f16x2(v0, v1);
@@ -661,8 +665,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 // tile t, so no waiter can see a barrier two phases ahead.
 namespace v3 {
 
-constexpr int kThreads3 = 768;
-constexpr int kYWarps = 4;          // epilogue warps, one per TMEM lane quarter
+constexpr int kThreads3 = 800;
 
 // Per-tile event timestamps of CTA 0, compiled in only with -DSSD_TC_TRACE
 // (performance analysis builds); a no-op otherwise.
@@ -725,11 +728,10 @@ struct __align__(1024) Smem {
     uint64_t s_ready[2];              // P (S in TMEM) -> W17
     uint64_t x_ready[2];              // E (x, w o x written) -> W17
     uint64_t hs_ready[2];             // E -> W17
-    uint64_t e_done[2];               // Y (Y read from TMEM) -> W17
     uint64_t stg_free[2];             // Y (y staged in hs[t & 1] has been stored) -> E
     uint64_t s_done[2];               // W17 commit -> E
     uint64_t y_full[2];               // W17 commit -> E, P, W16, W18
-    uint64_t fin[2];                  // W17, W18: own tcgen05 work drained before exit
+    uint64_t fin[3];                  // W18, W17, W24: own tcgen05 work drained before exit
     uint32_t tmem_base;
     TcCtl ctl;
 };
@@ -767,12 +769,12 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             mbar_init(&s.s_ready[i], kRoleWarps);
             mbar_init(&s.x_ready[i], kRoleWarps);
             mbar_init(&s.hs_ready[i], kRoleWarps);
-            mbar_init(&s.e_done[i], kYWarps);
             mbar_init(&s.stg_free[i], 1);
             mbar_init(&s.s_done[i], 1);
             mbar_init(&s.y_full[i], 1);
             mbar_init(&s.fin[i], 1);
         }
+        mbar_init(&s.fin[2], 1);
         ctl.abort = 0;
         fence_mbar_init();
     }
@@ -782,6 +784,12 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = s.tmem_base;
     const float kLog2e = 1.4426950408889634f;
+    // Every warp of a role polls the mbarrier itself (no rendezvous inside the role: a warp that
+    // lags its siblings does not hold the others back); the result is uniform per warp.
+    auto wait_w = [&](uint64_t* bar, uint32_t par) { return wait_bar_w(ctl, bar, par, p.status); };
+    auto wait_w2 = [&](uint64_t* b1, uint32_t p1, uint64_t* b2, uint32_t p2) {
+        return wait_bar_w(ctl, b1, p1, p.status) && (!b2 || wait_bar_w(ctl, b2, p2, p.status));
+    };
 #ifdef SSD_TC_TRACE
     if (tid == 0 && blockIdx.x < 8192) {
         uint32_t smid;
@@ -862,10 +870,16 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             tma_prefetch_desc(&tm_b);
             tma_prefetch_desc(&tm_c);
             int issued = 0;
+            // x comes from HBM with a latency of a few thousand cycles, more than the two stages
+            // hide: each tile's x is pulled into L2 four tiles before its load
+            for (int u = 0; u < 4 && u < nt; ++u) tma_prefetch_l2_3d(&tm_x, 0, h, (int)(tok0 + (int64_t)u * kT));
             for (int u = 0; u < nt; ++u) {
                 const int st = u & 1;
-                // stage st is free once every MMA of tile u - 2 has completed
+                if (u + 4 < nt) tma_prefetch_l2_3d(&tm_x, 0, h, (int)(tok0 + (int64_t)(u + 4) * kT));
+                // stage st is free once every MMA of tile u - 2 has completed: W24's output chain
+                // (y_full) and W17's B^T (w o x) (s_done), issued by different threads
                 if (u >= 2 && !wait_bar(ctl, &s.y_full[st], ((u - 2) >> 1) & 1, p.status)) break;
+                if (u >= 2 && !wait_bar(ctl, &s.s_done[st], ((u - 2) >> 1) & 1, p.status)) break;
                 const int tok = (int)(tok0 + (int64_t)u * kT);
                 mbar_expect_tx(&s.full[st], kTileBytesX + 4 * kBoxBytes);
                 tma_load_3d(s.x[st], &tm_x, &s.full[st], 0, h, tok);
@@ -888,8 +902,8 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             for (int t = 0; t < nt; ++t) {
                 const int st = t & 1;
                 if (!wait_bar(ctl, &s.full[st], (t >> 1) & 1, p.status)) break;
-                // TMEM C buffer st is free once C' h_prev of tile t - 2 has completed
-                if (t >= 2 && !wait_bar(ctl, &s.y_full[st], ((t - 2) >> 1) & 1, p.status)) break;
+                // (TMEM C buffer st is free again: full(t) follows W16's wait for y_full(t - 2), which
+                // follows C' h_prev of tile t - 2)
                 tc_fence_after();
                 // descriptors differ per K step only in the start address (low bits, in 16-byte units)
                 const uint64_t dc = sdesc_sw128(smem_u32(s.c[st][0]), 16, 1024);
@@ -913,20 +927,20 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             mbar_wait(&s.fin[0], 0, 400000000ll);
         }
     } else if (warp == 17) {
-        // ------------------------------------------ W17: s, C' h_prev, S x
+        // -------------------------------------------------- W17: s = B^T (w o x)
         if (lane == 0 && nt > 0) {
             const uint32_t id_st = idesc_f16(128, 64, 1, 1);   // MN-major A (B^T) and B (w o x)
-            const uint32_t id_y = idesc_f16(128, 64, 0, 1);    // A from TMEM, MN-major B
             for (int t = 0; t < nt; ++t) {
                 const int st = t & 1;
                 const uint32_t par = (t >> 1) & 1;
                 const uint64_t db = sdesc_sw128(smem_u32(s.b[st][0]), kBoxBytes, 1024);
                 const uint64_t dwx = sdesc_sw128(smem_u32(s.wx), kBoxBytes, 1024);
-                const uint64_t dx = sdesc_sw128(smem_u32(s.x[st]), kBoxBytes, 1024);
-                const uint64_t dhs = sdesc_sw128(smem_u32(s.hs[st]), kBoxBytes, 1024);
-                // s = B^T (w o x)  (state rows 0..127 = TMEM lanes)
+                // (the single s buffer is free again: E loads s of tile t - 1 before it writes the
+                // w o x of tile t that x_ready announces)
                 if (!wait_bar(ctl, &s.x_ready[st], par, p.status)) break;
                 if (!wait_bar(ctl, &s.full[st], par, p.status)) break;
+                // a partial tile's B rows past the sequence end are zeroed by P before c_scaled
+                if (tile_len(t) < kT && !wait_bar(ctl, &s.c_scaled[st], par, p.status)) break;
                 TC_TRACE(3, t);
                 tc_fence_after();
 #pragma unroll 1
@@ -934,18 +948,36 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     mma_ss(tmem + kColSt, db + (uint64_t)(k * 128), dwx + (uint64_t)(k * 128), id_st, k > 0);
                 mma_commit(&s.s_done[st]);
                 TC_TRACE(4, t);
-                // Y = C' h_prev: needs the state entering tile t, C' and a free Y buffer
+            }
+            mma_commit(&s.fin[1]);
+            mbar_wait(&s.fin[1], 0, 400000000ll);
+        }
+    } else if (warp == 24) {
+        // --------------------------------------------- W24: Y = C' h_prev + S x
+        // A second MMA-issuing thread: an issuing thread is held for each tcgen05.mma it issues,
+        // and a chain accumulating into one TMEM buffer waits for its previous step, so the
+        // tile's two independent chains (s on W17, Y here) run side by side.
+        if (lane == 0 && nt > 0) {
+            const uint32_t id_y = idesc_f16(128, 64, 0, 1);    // A from TMEM, MN-major B
+            for (int t = 0; t < nt; ++t) {
+                const int st = t & 1;
+                const uint32_t par = (t >> 1) & 1;
+                const uint64_t dx = sdesc_sw128(smem_u32(s.x[st]), kBoxBytes, 1024);
+                const uint64_t dhs = sdesc_sw128(smem_u32(s.hs[st]), kBoxBytes, 1024);
+                // Y = C' h_prev: needs the state entering tile t and C'.  (The Y buffer is free
+                // again: hs_ready(t) follows E's wait for stg_free(t - 2), which the epilogue
+                // arrives at after reading Y of tile t - 2.)
                 if (!wait_bar(ctl, &s.hs_ready[st], par, p.status)) break;
                 if (!wait_bar(ctl, &s.c_scaled[st], par, p.status)) break;
-                if (t >= 2 && !wait_bar(ctl, &s.e_done[st], ((t - 2) >> 1) & 1, p.status)) break;
                 TC_TRACE(5, t);
                 tc_fence_after();
 #pragma unroll 1
                 for (int k = 0; k < N / 16; ++k)
                     mma_ts(tmem + kColY + 64 * st, tmem + kColC + 64 * st + 8 * k, dhs + (uint64_t)(k * 128), id_y, k > 0);
                 TC_TRACE(6, t);
-                // Y += S x
+                // Y += S x: needs S and the converted x of tile t
                 if (!wait_bar(ctl, &s.s_ready[st], par, p.status)) break;
+                if (!wait_bar(ctl, &s.x_ready[st], par, p.status)) break;
                 TC_TRACE(7, t);
                 tc_fence_after();
 #pragma unroll 1
@@ -954,15 +986,14 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 mma_commit(&s.y_full[st]);
                 TC_TRACE(8, t);
             }
-            mma_commit(&s.fin[1]);
-            mbar_wait(&s.fin[1], 0, 400000000ll);
+            mma_commit(&s.fin[2]);
+            mbar_wait(&s.fin[2], 0, 400000000ll);
         }
     } else if (warp < 8) {
         // -------------------------------------- P: C', decay mask, decay scan
         const int quarter = warp & 3, half = warp >> 2;
         const int j = 32 * quarter + lane;
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-        const bool leader = warp == 4;
         const float Dh = p.D ? p.D[h] : 0.f;
         // S blocks right of this quarter's diagonal stay zero: write them once.
         {
@@ -974,7 +1005,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             const int st = t & 1;
             const uint32_t par = (t >> 1) & 1;
             const int sl = t & 3;
-            if (!wait_role2<1>(ctl, &s.scan_done[sl], (t >> 2) & 1, &s.cb_full[st], par, p.status, leader, &ctl.p_flag))
+            if (!wait_w2(&s.scan_done[sl], (t >> 2) & 1, &s.cb_full[st], par))
                 break;
             if (tid == 128) TC_TRACE(9, t);
             tc_fence_after();
@@ -995,6 +1026,14 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 tmem_st16(ct, r0);
                 tmem_st16(ct + 16, r1);
                 tmem_st_wait();
+                if (tile_len(t) < kT && j >= tile_len(t)) {
+                    // C B^T has read B: zero this row past the sequence end so that B^T (w o x)
+                    // meets exact zeros there even for non-finite values of the next sequence
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(s.b[st][half] + sw128_off(j, c)) = z;
+                    fence_proxy_async_smem();
+                }
                 tc_fence_before();
                 warp_arrive(&s.c_scaled[st]);
                 if (tid == 128) TC_TRACE(10, t);
@@ -1060,7 +1099,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (tid == 128) TC_TRACE(11, t);
             if (tid == 96) TC_TRACE(15, t);
             // the S buffer is free once S x of tile t - 1 has completed
-            if (t > 0 && !wait_role<1>(ctl, &s.y_full[st ^ 1], ((t - 1) >> 1) & 1, p.status, leader, &ctl.p_flag))
+            if (t > 0 && !wait_w(&s.y_full[st ^ 1], ((t - 1) >> 1) & 1))
                 break;
             if (tid == 128) TC_TRACE(12, t);
             tc_fence_after();
@@ -1076,7 +1115,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
 
             if (tid == 128) TC_TRACE(14, t);
         }
-    } else if (warp >= 20) {
+    } else if (warp >= 20 && warp < 24) {
         // ---------------------------------------------- Y: epilogue, y = Y
         // A full tile is staged (bf16, 128-byte swizzled rows) in hs[u & 1], free once C' h_prev
         // of tile u has completed and until E writes the state entering tile u + 2 there, and
@@ -1090,13 +1129,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         if (issuer) tma_prefetch_desc(&tm_y);
         for (int u = 0; u < nt; ++u) {
             const int q = tile_len(u);
-            // one warp polls, the four decide together (they meet at named barrier 3 below)
-            if (warp == 20) {
-                const bool okw = wait_bar_w(ctl, &s.y_full[u & 1], (u >> 1) & 1, p.status);
-                if (lane == 0) *(volatile int*)&ctl.y_flag = okw ? 1 : 0;
-            }
-            asm volatile("bar.sync 3, 128;" ::: "memory");
-            if (!*(volatile int*)&ctl.y_flag) break;
+            if (!wait_w(&s.y_full[u & 1], (u >> 1) & 1)) break;
             tc_fence_after();
             const uint32_t ya = tmem + lane_base + kColY + 64 * (u & 1);
             uint8_t* stg = s.hs[u & 1];
@@ -1107,12 +1140,6 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 tmem_ld16(ya + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(r));
                 tmem_ld16(ya + 32 * hh + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
                 tmem_ld_wait();
-                if (hh == 1) {
-                    // Y is in registers: release the buffer before storing
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s.e_done[u & 1]);
-                }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const uint4 val = make_uint4(
@@ -1127,6 +1154,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 }
             }
             if (q == kT) fence_proxy_async_smem();
+            tc_fence_before();      // the Y reads precede stg_free, hence the next MMA into this buffer
             asm volatile("bar.sync 3, 128;" ::: "memory");
             if (issuer) {
                 if (q == kT) {
@@ -1146,7 +1174,6 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         const int j = 32 * quarter + lane;     // token row (x, y) and state row (s, h)
         const int col0 = 32 * half;
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-        const bool leader = warp == 8;
         float hreg[32];
         {
             const float* src = p.init_state ? p.init_state + (((int64_t)seq * H + h) * N + j) * kP + col0 : nullptr;
@@ -1171,78 +1198,98 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             fence_proxy_async_smem();
             warp_arrive(&s.hs_ready[u & 1]);
         };
-        if (nt > 0) put_state(0);
-        float e_state = 1.f;   // 2^cs_last of the tile whose s is pending
-        bool ok = true;
-        for (int k = 0; ok && k <= nt; ++k) {
-            if (k >= 1) {
-                // h <- 2^cs_last h + s for tile k - 1
-                const int u = k - 1;
-                // (and hs[k & 1] free again: it held y of tile k - 2 on its way out)
-                if (!(ok = wait_role2<2>(ctl, &s.s_done[u & 1], (u >> 1) & 1,
-                                         (k >= 2 && k < nt) ? &s.stg_free[k & 1] : nullptr, ((k - 2) >> 1) & 1,
-                                         p.status, leader, &ctl.e_flag)))
-                    break;
-                if (tid == 256) TC_TRACE(17, u);
-                tc_fence_after();
-                {
-                    uint32_t r0[16], r1[16];
-                    tmem_ld16(tmem + lane_base + kColSt + col0, r0);
-                    tmem_ld16(tmem + lane_base + kColSt + col0 + 16, r1);
-                    tmem_ld_wait();
-                    const uint64_t e2 = f2pack(e_state, e_state);
+        // x of tile k -> fp16 in place (zero past the sequence end); returns the tile's total
+        // decay 2^cs_last and this row's weight w_j = d_j 2^(cs_last - cs_j).
+        auto convert_x = [&](int k, float& e_tot, __half2& w2) {
+            const int q = tile_len(k);
+            const float cs_last = s.cs[k & 3][q - 1];
+            e_tot = ex2(cs_last);
+            w2 = __float2half2_rn(s.d[k & 3][j] * ex2(cs_last - s.cs[k & 3][j]));
+            warp_arrive(&s.scan_free[k & 3]);
+            uint8_t* xt = s.x[k & 1];
 #pragma unroll
-                    for (int i = 0; i < 16; i += 2) {
-                        float lo, hi;
-                        f2unpack(f2fma(e2, f2pack(hreg[i], hreg[i + 1]),
-                                       f2pack(__uint_as_float(r0[i]), __uint_as_float(r0[i + 1]))), lo, hi);
-                        hreg[i] = lo; hreg[i + 1] = hi;
-                        f2unpack(f2fma(e2, f2pack(hreg[16 + i], hreg[17 + i]),
-                                       f2pack(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1]))), lo, hi);
-                        hreg[16 + i] = lo; hreg[17 + i] = hi;
-                    }
-                }
-                if (tid == 256) TC_TRACE(38, u);
-                tc_fence_before();
-                if (k < nt) put_state(k);
-                if (tid == 256) TC_TRACE(18, u);
+            for (int m = 0; m < 4; ++m) {
+                const uint32_t off = sw128_off(j, col0 / 8 + m);
+                const uint4 xv = *reinterpret_cast<const uint4*>(xt + off);
+                uint4 o;
+                o.x = pack_f16x2(bf16lo(xv.x), bf16hi(xv.x));
+                o.y = pack_f16x2(bf16lo(xv.y), bf16hi(xv.y));
+                o.z = pack_f16x2(bf16lo(xv.z), bf16hi(xv.z));
+                o.w = pack_f16x2(bf16lo(xv.w), bf16hi(xv.w));
+                if (j >= q) o = make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(xt + off) = o;
             }
-            if (k < nt) {
-                // x of tile k to the fp16 operands x and w o x (zero past the sequence end)
-                if (!(ok = wait_role2<2>(ctl, &s.scan_done[k & 3], (k >> 2) & 1, &s.full[k & 1], (k >> 1) & 1, p.status,
-                                         leader, &ctl.e_flag)))
-                    break;
+        };
+        // w o x of tile k from its converted x, then x_ready
+        auto write_wx = [&](int k, __half2 w2) {
+            const uint8_t* xt = s.x[k & 1];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const uint32_t off = sw128_off(j, col0 / 8 + m);
+                const uint4 o = *reinterpret_cast<const uint4*>(xt + off);
+                uint4 w;
+                w.x = h2u(__hmul2(u2h(o.x), w2));
+                w.y = h2u(__hmul2(u2h(o.y), w2));
+                w.z = h2u(__hmul2(u2h(o.z), w2));
+                w.w = h2u(__hmul2(u2h(o.w), w2));
+                *reinterpret_cast<uint4*>(s.wx + off) = w;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            warp_arrive(&s.x_ready[k & 1]);
+        };
+        bool ok = true;
+        float e_cur = 1.f, e_next = 1.f;   // 2^cs_last of tiles t and t + 1
+        __half2 w_next = __float2half2_rn(0.f);
+        if (nt > 0) {
+            put_state(0);
+            if ((ok = wait_w2(&s.scan_done[0], 0, &s.full[0], 0))) {
+                convert_x(0, e_cur, w_next);
+                write_wx(0, w_next);
+            }
+        }
+        // Tile t: x of tile t + 1 is converted while B^T (w o x) of tile t runs; once it has
+        // completed, s(t) is taken into the state, and w o x of tile t + 1 (the single w o x
+        // buffer is free again) and the state entering tile t + 1 are written.
+        for (int t = 0; ok && t < nt; ++t) {
+            if (t + 1 < nt) {
+                const int k = t + 1;
+                if (!(ok = wait_w2(&s.scan_done[k & 3], (k >> 2) & 1, &s.full[k & 1], (k >> 1) & 1))) break;
                 if (tid == 256) TC_TRACE(19, k);
-                const int q = tile_len(k);
-                const float cs_last = s.cs[k & 3][q - 1];
-                e_state = ex2(cs_last);
-                const __half2 w2 = __float2half2_rn(s.d[k & 3][j] * ex2(cs_last - s.cs[k & 3][j]));
-                warp_arrive(&s.scan_free[k & 3]);
-                if (tid == 256) TC_TRACE(39, k);
-                uint8_t* xt = s.x[k & 1];
-#pragma unroll 1
-                for (int m = 0; m < 4; ++m) {
-                    const uint4 xv = *reinterpret_cast<const uint4*>(xt + sw128_off(j, col0 / 8 + m));
-                    uint4 o, w;
-                    o.x = pack_f16x2(bf16lo(xv.x), bf16hi(xv.x));
-                    o.y = pack_f16x2(bf16lo(xv.y), bf16hi(xv.y));
-                    o.z = pack_f16x2(bf16lo(xv.z), bf16hi(xv.z));
-                    o.w = pack_f16x2(bf16lo(xv.w), bf16hi(xv.w));
-                    if (j >= q) o = make_uint4(0u, 0u, 0u, 0u);
-                    w.x = h2u(__hmul2(u2h(o.x), w2));
-                    w.y = h2u(__hmul2(u2h(o.y), w2));
-                    w.z = h2u(__hmul2(u2h(o.z), w2));
-                    w.w = h2u(__hmul2(u2h(o.w), w2));
-                    const uint32_t off = sw128_off(j, col0 / 8 + m);
-                    *reinterpret_cast<uint4*>(xt + off) = o;
-                    *reinterpret_cast<uint4*>(s.wx + off) = w;
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                warp_arrive(&s.x_ready[k & 1]);
-                if (tid == 256) TC_TRACE(20, k);
-                if (tid == 480) TC_TRACE(23, k);
+                convert_x(k, e_next, w_next);
+                if (tid == 256) TC_TRACE(21, k);
             }
+            // s(t) is complete (and hs[(t + 1) & 1] free again: it held y of tile t - 1 on its way out)
+            if (!(ok = wait_w2(&s.s_done[t & 1], (t >> 1) & 1,
+                                     (t >= 1 && t + 1 < nt) ? &s.stg_free[(t + 1) & 1] : nullptr,
+                                     ((t - 1) >> 1) & 1)))
+                break;
+            if (tid == 256) TC_TRACE(17, t);
+            tc_fence_after();
+            {
+                uint32_t r0[16], r1[16];
+                tmem_ld16(tmem + lane_base + kColSt + col0, r0);
+                tmem_ld16(tmem + lane_base + kColSt + col0 + 16, r1);
+                tmem_ld_wait();
+                const uint64_t e2 = f2pack(e_cur, e_cur);
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                    float lo, hi;
+                    f2unpack(f2fma(e2, f2pack(hreg[i], hreg[i + 1]),
+                                   f2pack(__uint_as_float(r0[i]), __uint_as_float(r0[i + 1]))), lo, hi);
+                    hreg[i] = lo; hreg[i + 1] = hi;
+                    f2unpack(f2fma(e2, f2pack(hreg[16 + i], hreg[17 + i]),
+                                   f2pack(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1]))), lo, hi);
+                    hreg[16 + i] = lo; hreg[17 + i] = hi;
+                }
+            }
+            if (t + 1 < nt) {
+                write_wx(t + 1, w_next);
+                if (tid == 256) TC_TRACE(20, t + 1);
+                put_state(t + 1);
+                if (tid == 256) TC_TRACE(18, t + 1);
+            }
+            e_cur = e_next;
         }
         if (p.final_state && (ok || nt == 0)) {
             float* dst = p.final_state + (((int64_t)seq * H + h) * N + j) * kP + col0;
@@ -1278,6 +1325,138 @@ __global__ void k_tc_prep(const uint4* __restrict__ b, const uint4* __restrict__
         b16[i] = ob;
         c16[i] = oc;
     }
+}
+
+// ---- Long sequences with few (sequence, head) pairs: the two-pass split ----------------
+//
+// With b H CTAs well below the SM count, each sequence is cut into K segments of Ls tokens
+// (tile-aligned; the last takes the rest).  Pass 1 scans segments 0 .. K-2 of every row as
+// independent spans (segment 0 from the real initial state, so its y is final; the others from
+// zero, for their final states); the chain forms the state entering each segment k >= 1,
+//   h_in(1) = F(0),  h_in(k) = exp(sum over segment k - 1 of d A) h_in(k - 1) + F(k - 1);
+// pass 2 rescans segments 1 .. K-1 from h_in (overwriting their y) and the last one's final
+// state is the row's.  Both passes are the unchanged scan kernel over span tables.
+
+struct SplitPlan {
+    int K = 0;
+    int64_t Ls = 0;
+};
+
+// Spans of segments first .. first + nseg - 1 of every row, on the flat (b L) token axis.
+__global__ void k_split_spans(int64_t L, int64_t Ls, int K, int first, int nseg, int64_t b, int32_t* start,
+                              int32_t* end) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < b * nseg; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / nseg, k = first + i % nseg;
+        const int64_t t0 = k * Ls, t1 = (k == K - 1 || (k + 1) * Ls > L) ? L : (k + 1) * Ls;   // the last runs to L
+        start[i] = (int32_t)(r * L + t0);
+        end[i] = (int32_t)(r * L + t1);
+    }
+}
+
+// Initial states of pass 1: the row's own for segment 0, zero for the others.
+__global__ void k_split_init(const float* __restrict__ init, float* __restrict__ I1, int64_t b, int nseg,
+                             int64_t HNP) {
+    const int64_t n = b * nseg * HNP;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t span = e / HNP, r = span / nseg;
+        I1[e] = (span % nseg == 0 && init) ? init[r * HNP + e % HNP] : 0.f;
+    }
+}
+
+// Sum of d A over segment k = 1 .. K-2 of every row and head (natural log of its total decay).
+// One block per (row, segment, head).
+__global__ void k_split_decay(const __nv_bfloat16* __restrict__ dt, const float* __restrict__ dt_bias,
+                              const float* __restrict__ A, int64_t L, int64_t Ls, int K, int H,
+                              float* __restrict__ dsum) {
+    const int h = blockIdx.x % H;
+    const int k = 1 + (int)((blockIdx.x / H) % (K - 2));
+    const int64_t r = blockIdx.x / ((int64_t)H * (K - 2));
+    const float bias = dt_bias ? dt_bias[h] : 0.f;
+    float acc = 0.f;
+    for (int64_t t = k * Ls + threadIdx.x; t < (k + 1) * Ls && t < L; t += blockDim.x)
+        acc += softplus_f(__bfloat162float(dt[(r * L + t) * H + h]) + bias);
+    __shared__ float red[32];
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        acc = threadIdx.x < blockDim.x / 32 ? red[threadIdx.x] : 0.f;
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (threadIdx.x == 0) dsum[blockIdx.x] = acc * A[h];
+    }
+}
+
+// h_in of segments 1 .. K-1 (pass 2's initial states) from pass 1's final states F1.
+__global__ void k_split_chain(const float* __restrict__ F1, const float* __restrict__ dsum,
+                              float* __restrict__ I2, int64_t b, int K, int H, int64_t NP) {
+    const int64_t n = b * H * NP;
+    const int64_t HNP = (int64_t)H * NP;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = e / HNP, he = e % HNP, h = he / NP;
+        float hin = F1[(r * (K - 1)) * HNP + he];
+        I2[(r * (K - 1)) * HNP + he] = hin;
+        for (int k = 2; k < K; ++k) {
+            const float dec = expf(dsum[(r * (K - 2) + (k - 1 - 1)) * H + h]);
+            hin = dec * hin + F1[(r * (K - 1) + (k - 1)) * HNP + he];
+            I2[(r * (K - 1) + (k - 1)) * HNP + he] = hin;
+        }
+    }
+}
+
+// SMs of the current device (queried once per device), and SSD_TC_SPLIT=K, read once: forces
+// K segments whenever the sequence has at least K tiles (for tests and tuning; 0 or unset: the
+// plan below).
+int sm_count() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        cache[dev] = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+int forced_split() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("SSD_TC_SPLIT");
+        v = e ? atoi(e) : 0;
+        if (v < 0 || v > 64) v = 0;
+    }
+    return v;
+}
+
+// K and Ls for a call, or K = 0 when the split does not pay: packed input (spans per sequence,
+// not handled), at least half the SMs already busy, or fewer than 8 tiles per segment.
+SplitPlan plan_split(const ScanArgs& a) {
+    SplitPlan pl;
+    const int64_t ctas = a.b * a.H;
+    const int64_t tiles = (a.L + kT - 1) / kT;
+    if (a.seq_idx || ctas <= 0) return pl;
+    int K;
+    if (forced_split() >= 2) {
+        K = forced_split();
+        if (tiles < K) return pl;
+    } else {
+        const int sms = sm_count();
+        if (ctas * 2 > sms) return pl;
+        K = (int)(1 + sms / ctas);
+        if (K > 8) K = 8;
+        if (K < 3 || tiles < 8 * (int64_t)K) return pl;
+    }
+    const int64_t Ls = ((tiles + K - 1) / K) * kT;
+    if ((K - 1) * Ls >= a.L) return pl;
+    pl.K = K;
+    pl.Ls = Ls;
+    return pl;
+}
+
+size_t split_workspace_bytes(const ScanArgs& a, const SplitPlan& pl) {
+    if (!pl.K) return 0;
+    const size_t states = (size_t)a.b * (pl.K - 1) * a.H * a.N * a.P * sizeof(float);
+    const size_t spans = (size_t)a.b * (pl.K - 1) * sizeof(int32_t);
+    return 3 * ((states + 255) & ~(size_t)255) + 4 * ((spans + 255) & ~(size_t)255) +
+           (((size_t)a.b * pl.K * a.H * sizeof(float) + 255) & ~(size_t)255);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -1327,7 +1506,8 @@ bool tc_supported(const ScanArgs& a) {
 }
 
 size_t tc_workspace_bytes(const ScanArgs& a, int64_t) {
-    return 2 * (size_t)a.b * a.L * a.G * a.N * sizeof(__half) + 256;
+    const size_t bc = (2 * (size_t)a.b * a.L * a.G * a.N * sizeof(__half) + 255) & ~(size_t)255;
+    return bc + 256 + split_workspace_bytes(a, plan_split(a));
 }
 
 int launch_tc_scan(const ScanArgs& a, const SeqInfo& si, int64_t, void* ws, int32_t* status, cudaStream_t st) {
@@ -1362,6 +1542,63 @@ int launch_tc_scan(const ScanArgs& a, const SeqInfo& si, int64_t, void* ws, int3
     p.status = status;
     p.H = (int)a.H;
     p.G = (int)a.G;
+    const SplitPlan pl = a.N == 128 ? plan_split(a) : SplitPlan();
+    if (pl.K) {
+        const size_t smem = sizeof(v3::Smem) + 1024;
+        cudaFuncSetAttribute(v3::k_tc_scan3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const int K = pl.K, nseg = K - 1;
+        const int64_t HNP = a.H * a.N * a.P, S2 = a.b * nseg;
+        const size_t states = ((size_t)S2 * HNP * sizeof(float) + 255) & ~(size_t)255;
+        const size_t spans = ((size_t)S2 * sizeof(int32_t) + 255) & ~(size_t)255;
+        char* w = reinterpret_cast<char*>(ws) + ((2 * (size_t)ntok * a.G * a.N * sizeof(__half) + 255) & ~(size_t)255) + 256;
+        float* I1 = reinterpret_cast<float*>(w); w += states;       // pass 1 initial states, then pass 2's final
+        float* F1 = reinterpret_cast<float*>(w); w += states;       // pass 1 final states
+        float* I2 = reinterpret_cast<float*>(w); w += states;       // pass 2 initial states (the chain)
+        int32_t* st1 = reinterpret_cast<int32_t*>(w); w += spans;
+        int32_t* en1 = reinterpret_cast<int32_t*>(w); w += spans;
+        int32_t* st2 = reinterpret_cast<int32_t*>(w); w += spans;
+        int32_t* en2 = reinterpret_cast<int32_t*>(w); w += spans;
+        float* dsum = reinterpret_cast<float*>(w);
+        const unsigned gs = (unsigned)((S2 + 255) / 256);
+        const int64_t ne = S2 * HNP;
+        const unsigned ge = (unsigned)std::min<int64_t>((ne + 255) / 256, 148 * 16);
+        {
+            ProfScope pt(K_TC_PREP, st);
+            k_split_spans<<<gs, 256, 0, st>>>(a.L, pl.Ls, K, 0, nseg, a.b, st1, en1);
+            k_split_spans<<<gs, 256, 0, st>>>(a.L, pl.Ls, K, 1, nseg, a.b, st2, en2);
+            k_split_init<<<ge, 256, 0, st>>>(a.init_state, I1, a.b, nseg, HNP);
+            if (K > 2)
+                k_split_decay<<<(unsigned)(a.b * (K - 2) * a.H), 256, 0, st>>>(
+                    (const __nv_bfloat16*)a.dt, a.dt_bias, a.A, a.L, pl.Ls, K, (int)a.H, dsum);
+        }
+        SeqInfo s1 = si;
+        s1.packed = 1; s1.S = (int32_t)S2; s1.L = ntok; s1.start = st1; s1.end = en1; s1.chunk_off = nullptr;
+        TcParams p1 = p;
+        p1.si = s1; p1.init_state = I1; p1.final_state = F1;
+        {
+            ProfScope ps(K_TC_SCAN, st);
+            v3::k_tc_scan3<<<(unsigned)(S2 * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, tm_y, p1);
+        }
+        {
+            ProfScope pt(K_TC_PREP, st);
+            const unsigned gc = (unsigned)std::min<int64_t>((a.b * HNP + 255) / 256, 148 * 16);
+            k_split_chain<<<gc, 256, 0, st>>>(F1, dsum, I2, a.b, K, (int)a.H, a.N * a.P);
+        }
+        SeqInfo s2 = s1;
+        s2.start = st2; s2.end = en2;
+        TcParams p2 = p;
+        p2.si = s2; p2.init_state = I2; p2.final_state = I1;       // pass 1's initial states are spent
+        {
+            ProfScope ps(K_TC_SCAN, st);
+            v3::k_tc_scan3<<<(unsigned)(S2 * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, tm_y, p2);
+        }
+        if (a.final_state &&
+            cudaMemcpy2DAsync(a.final_state, HNP * sizeof(float), I1 + (size_t)(nseg - 1) * HNP,
+                              (size_t)nseg * HNP * sizeof(float), HNP * sizeof(float), (size_t)a.b,
+                              cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return 6;
+        return 0;
+    }
     ProfScope ps(K_TC_SCAN, st);
     if (a.N == 128) {
         const size_t smem = sizeof(v3::Smem) + 1024;

@@ -145,6 +145,13 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
         : "memory");
 }
 
+// Brings a 3-D tile into L2 ahead of its load (no shared memory, no completion
+// signal); coordinates as for tma_load_3d.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
+
 // Shared -> global tile store through the tensor map (coordinates must be
 // non-negative; rows past the tensor's outer extent are not written).
 // Completion is tracked per thread with the bulk async-group.

@@ -382,7 +382,8 @@ def _prefixed(gen, pre: str, peer: str):
 # not through the staging tile).
 
 def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), zero_b: str = "",
-                conv: str = "E", m: Machine | None = None, rank: int | None = None) -> Machine:
+                conv: str = "E", m: Machine | None = None, rank: int | None = None,
+                y_issuer: bool = False) -> Machine:
     """`zero_b` models ways of zeroing the B rows past the sequence end in a partial last tile
     (not done by the kernel today): "p" has the P warps do it right after C B^T has read B
     (cb_full), with W17 waiting for c_scaled before B^T (w o x) on that tile; "e" has the E
@@ -394,7 +395,14 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
     tile t has completed, and the E warps do only the state update, which then leaves the loop
     between consecutive B^T (w o x) MMAs), or "Y2" (the same, in two phases: x of tile t + 1 is
     converted in place as soon as it has landed, kept in registers, and only w o x is written
-    after B^T (w o x) of tile t).
+    after B^T (w o x) of tile t), or "E2" (the kernel's form: the E warps convert x of tile
+    t + 1 in place while B^T (w o x) of tile t runs, and once it has completed they load s,
+    release the s buffer, write w o x of tile t + 1 from the converted x and then the state
+    entering tile t + 1).
+
+    `y_issuer` moves the output chain (C' h_prev, then S x into one accumulator) from W17 to a
+    warp of its own (W24), as the kernel has it: W17 then issues only B^T (w o x); W24 also waits
+    for x_ready, since S x reads the converted x.
 
     `rank` (0 or 1, with a shared `m`) builds one CTA of the d_state 256 pair candidate (see
     build_scan3_pair): C gets one shared-memory stage on its own barrier, and the epilogues
@@ -404,13 +412,14 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
     reg = lambda name, count: m.barrier(pre + name, count)
     for i in range(4):
         reg(f"scan_done{i}", 1)
-        reg(f"scan_free{i}", 16 if conv == "E" else 20)
+        reg(f"scan_free{i}", 16 if conv in ("E", "E2") else 20)
     for i in range(2):
         for name, count in (("full", 1), ("cb_full", 1), ("cb_free", 8), ("c_scaled", 8), ("s_ready", 8),
                             ("x_ready", 8), ("hs_ready", 8), ("e_done", 4), ("stg_free", 1), ("s_done", 1),
                             ("y_full", 1), ("fin", 1), ("st_free", 8), ("rcv_full", 1), ("rcv_free", 1)):
-            reg(f"{name}{i}", count if not (name == "x_ready" and conv != "E") else 4)
+            reg(f"{name}{i}", count if not (name == "x_ready" and conv in ("Y", "Y2")) else 4)
     reg("cfull", 1)
+    reg("fin2", 1)
     pair = rank is not None
     full_tile = lambda u: not (partial and u == nt - 1)
 
@@ -429,6 +438,10 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
             st = u & 1
             if u >= 2 and "w16_y_full" not in drop:
                 if not (yield ("wait", f"y_full{st}", (u - 2) >> 1)):
+                    break
+            if u >= 2 and y_issuer and "w16_s_done" not in drop:
+                # B^T (w o x) of tile u - 2 is W17's, not covered by W24's y_full commit
+                if not (yield ("wait", f"s_done{st}", (u - 2) >> 1)):
                     break
             yield ("arrive_tx", f"full{st}", 2 if pair else 3)
             for buf in (("x", "b") if pair else ("x", "b", "c")):
@@ -486,6 +499,8 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
                     break
             yield ("mma", (f"b{st}", "wx"), ("tSt",))
             yield ("commit", f"s_done{st}")
+            if y_issuer:
+                continue
             if not (yield ("wait", f"hs_ready{st}", ph)) or not (yield ("wait", f"c_scaled{st}", ph)):
                 break
             if t >= 2 and "w17_e_done" not in drop:
@@ -500,6 +515,29 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
         if "w17_fin" not in drop:
             yield ("commit", "fin1")
             yield ("bwait", "fin1", 0)
+
+    def w24():      # the output chain on its own warp: C' h_prev, then S x
+        if nt == 0:
+            return
+        for t in range(nt):
+            st, ph = t & 1, t >> 1
+            if not (yield ("wait", f"hs_ready{st}", ph)) or not (yield ("wait", f"c_scaled{st}", ph)):
+                break
+            if t >= 2 and "w17_e_done" not in drop:
+                if not (yield ("wait", f"e_done{st}", (t - 2) >> 1)):
+                    break
+            yield ("mma", (f"tC{st}", f"hs{st}"), (f"tY{st}",))
+            if "w17_s_ready" not in drop:
+                if not (yield ("wait", f"s_ready{st}", ph)):
+                    break
+            if "w24_x_ready" not in drop:
+                if not (yield ("wait", f"x_ready{st}", ph)):
+                    break
+            yield ("mma", ("tS", f"x{st}", f"tY{st}"), (f"tY{st}",))
+            yield ("commit", f"y_full{st}")
+        if "w24_fin" not in drop:
+            yield ("commit", "fin2")
+            yield ("bwait", "fin2", 0)
 
     def p_role():   # C' scaling and the decay mask S
         yield ("write", "tS")                       # blocks right of the diagonal, zeroed once
@@ -599,6 +637,44 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
         if stored:
             yield ("store_wait",)
 
+    def e2_role():  # "E2": two-phase conversion in the E warps, then the fp32 state
+        if nt == 0:
+            return
+        yield ("write", "hs0")
+        yield ("arrive", "hs_ready0", 8)
+
+        def convert_x(k):
+            if not (yield ("wait", f"scan_done{k & 3}", k >> 2)) or not (yield ("wait", f"full{k & 1}", k >> 1)):
+                return False
+            yield ("read", f"ring{k & 3}")
+            yield ("arrive", f"scan_free{k & 3}", 8)
+            yield ("read", f"x{k & 1}")
+            yield ("write", f"x{k & 1}")
+            return True
+
+        def write_wx(k):
+            yield ("read", f"x{k & 1}")
+            yield ("write", "wx")
+            yield ("arrive", f"x_ready{k & 1}", 8)
+
+        if not (yield from convert_x(0)):
+            return
+        yield from write_wx(0)
+        for t in range(nt):
+            if t + 1 < nt and not (yield from convert_x(t + 1)):
+                break
+            if not (yield ("wait", f"s_done{t & 1}", t >> 1)):
+                break
+            if t >= 1 and t + 1 < nt and "e_stg_free" not in drop:
+                if not (yield ("wait", f"stg_free{(t + 1) & 1}", (t - 1) >> 1)):
+                    break
+            yield ("read", "tSt")
+            yield ("arrive", f"st_free{t & 1}", 8)
+            if t + 1 < nt:
+                yield from write_wx(t + 1)
+                yield ("write", f"hs{(t + 1) & 1}")
+                yield ("arrive", f"hs_ready{(t + 1) & 1}", 8)
+
     def e_role():   # x operands and the fp32 state
         if nt > 0:
             yield ("write", "hs0")
@@ -626,8 +702,11 @@ def build_scan3(nt: int, partial: bool = False, drop: frozenset = frozenset(), z
                 if not (yield from convert(k, 8)):
                     break
 
-    for name, gen in (("W19", w19()), ("W16", w16()), ("W18", w18()), ("W17", w17()), ("P", p_role()),
-                      ("Y", y_role()), ("E", e_role())):
+    roles = [("W19", w19()), ("W16", w16()), ("W18", w18()), ("W17", w17()), ("P", p_role()),
+             ("Y", y_role()), ("E", e2_role() if conv == "E2" else e_role())]
+    if y_issuer:
+        roles.append(("W24", w24()))
+    for name, gen in roles:
         m.role(pre + name, _prefixed(gen, pre, peer) if pair else gen)
     return m
 

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in range(9):
+    for code in range(10):
         s = L.ssd_status_string(code).decode()
         assert s and s != "unknown status"
     assert L.ssd_status_string(99).decode() == "unknown status"

@@ -5,23 +5,29 @@ import bench
 
 
 def test_roofline_traffic_is_attached_to_the_measured_code_only(tmp_path, monkeypatch):
-    # the committed DRAM capture is reported for the kernel as it stands ...
-    rec = json.load(open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")))["tc_scan"]
-    assert rec["source_sha"] == bench.kernel_source_sha("tc_scan")
-    assert bench.traffic_for("tc_scan", rec["units"]) == rec["dram_bytes"]
-    # ... scales with the units a launch processes ...
-    assert bench.traffic_for("tc_scan", 2 * rec["units"]) == 2 * rec["dram_bytes"]
-    # ... and is dropped once the recorded hash no longer matches the code
-    bad = dict(rec, source_sha="0" * 16)
-    p = tmp_path / "profiles"
-    p.mkdir()
-    (p / "traffic.json").write_text(json.dumps({"tc_scan": bad}))
+    src = open(bench.os.path.join(bench.ROOT, "state_space_model_07_b200", "csrc", "ssd_tc.cu")).read()
     csrc = tmp_path / "state_space_model_07_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "ssd_tc.cu").write_text(open(bench.os.path.join(bench.ROOT, "state_space_model_07_b200", "csrc",
-                                                            "ssd_tc.cu")).read())
+    (csrc / "ssd_tc.cu").write_text(src)
+    p = tmp_path / "profiles"
+    p.mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.traffic_for("tc_scan", rec["units"]) is None
+    rec = {"source_sha": bench.kernel_source_sha("tc_scan"), "dram_bytes": 1000, "units": 10}
+    (p / "traffic.json").write_text(json.dumps({"tc_scan": rec}))
+    # a DRAM capture is reported for the kernel as it stands ...
+    assert bench.traffic_for("tc_scan", 10) == 1000
+    # ... scales with the units a launch processes ...
+    assert bench.traffic_for("tc_scan", 20) == 2000
+    # ... and is dropped once the recorded hash no longer matches the code
+    (p / "traffic.json").write_text(json.dumps({"tc_scan": dict(rec, source_sha="0" * 16)}))
+    assert bench.traffic_for("tc_scan", 10) is None
+
+
+def test_committed_traffic_record_names_its_kernel_and_summary():
+    rec = json.load(open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for name, r in rec.items():
+        assert {"kernel", "workload", "source_sha", "dram_bytes", "units", "summary"} <= set(r), name
+        assert bench.os.path.exists(bench.os.path.join(bench.ROOT, "profiles", r["summary"])), name
 
 
 def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):

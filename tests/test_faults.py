@@ -117,3 +117,57 @@ def test_broken_seq_idx_is_reported_in_debug_mode():
     assert out.returncode == 0, out.stderr[-2000:]
     assert "status 8" in out.stdout, out.stdout
     assert "after ok True" in out.stdout, out.stdout
+
+
+# --- the tensor-core path's fp16 operand range -----------------------------------------------
+
+_RANGE = r"""
+import sys, torch
+sys.path.insert(0, {root!r})
+import state_space_model_07_b200 as ssd
+from state_space_model_07_b200 import inputs
+w = inputs.scaled(inputs.WORKLOADS["mamba2_2.7b_layer"], batch=1, seqlen=300, nheads=4)
+d = inputs.make_inputs(w, "cuda")
+def run(dd):
+    try:
+        y, fs = ssd.chunk_scan_fwd(dd["x"], dd["dt"], dd["A"], dd["B"], dd["C"], dt_bias=dd["dt_bias"],
+                                   D=dd["D"], chunk=w.chunk)
+        torch.cuda.synchronize()
+        return "0 finite" if bool(torch.isfinite(y).all() and torch.isfinite(fs).all()) else "0 nonfinite"
+    except ssd.SsdError as e:
+        return str(e.code)
+over = dict(d, x=d["x"].clone())
+over["x"][0, 5, 1, 3] = 1e5                      # finite in bf16, beyond fp16
+big = dict(d, B=d["B"] * 1000, C=d["C"] * 1000)  # every input in range; the score matrix is not
+nan = dict(d, x=d["x"].clone())
+nan["x"][0, 5, 1, 3] = float("nan")
+print("plain", run(d))
+print("x over", run(over))
+print("scores over", run(big))
+print("nan input", run(nan))
+"""
+
+
+@pytest.mark.parametrize("debug", [True, False])
+def test_fp16_operand_range_of_the_tensor_core_path(debug):
+    """The tensor-core path's operands are fp16.  With SSD_DEBUG_CHECK=1 an input beyond 65504
+    and a non-finite result from finite inputs (B and C 1000x larger than N(0, 1): the score
+    matrix passes 65504) come back as SSD_ERR_RANGE (9); a NaN input is the caller's and is not
+    a range error.  Without the debug check the same calls return non-finite values, as the
+    header states."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SSD_DEBUG_CHECK="1" if debug else "0")
+    out = subprocess.run([sys.executable, "-c", _RANGE.format(root=root)], env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = out.stdout.splitlines()
+    assert "plain 0 finite" in lines, out.stdout
+    if debug:
+        assert "x over 9" in lines and "scores over 9" in lines, out.stdout
+        assert "nan input 0 nonfinite" in lines, out.stdout
+    else:
+        assert "x over 0 nonfinite" in lines and "scores over 0 nonfinite" in lines, out.stdout
+        assert "nan input 0 nonfinite" in lines, out.stdout

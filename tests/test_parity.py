@@ -151,9 +151,16 @@ def test_causality_bitwise():
     assert not torch.equal(y1[:, t:], y2[:, t:])
 
 
+@pytest.mark.parametrize("poison", ["finite", "x", "B", "C", "dt"])
 @pytest.mark.parametrize("dstate", [128, 256])
-def test_packed_isolation_bitwise(dstate):
-    """Changing one sequence's inputs leaves every other sequence unchanged, bit for bit."""
+def test_packed_isolation_bitwise(dstate, poison):
+    """Changing one sequence's inputs leaves every other sequence unchanged, bit
+    for bit, even when the changed values are not finite.
+
+    Sequence 3 starts inside the last, partial 128-token tile of sequence 2
+    (lengths 300 + 17 + 129 = 446), so the tensor-core kernels load its first
+    rows of x, dt, B and C as part of sequence 2's tile and must mask all of
+    them; `poison` names the input that gets inf / NaN there."""
     w = inputs.scaled(W["packed_varlen"], nheads=8, dstate=dstate)
     lens = [300, 17, 129, 128, 600, 1]
     d = inputs.make_inputs(w, "cuda", lengths=lens)
@@ -164,9 +171,17 @@ def test_packed_isolation_bitwise(dstate):
               init_state=d["init_state"].clone())
     d2["x"][:, t0:t1] = torch.randn_like(d2["x"][:, t0:t1]) * 7
     d2["B"][:, t0:t1] = torch.randn_like(d2["B"][:, t0:t1])
-    d2["C"][:, t0:t1] = float("inf")          # even non-finite values must not leak
+    d2["C"][:, t0:t1] = torch.randn_like(d2["C"][:, t0:t1])
     d2["dt"][:, t0:t1] = 30.0
     d2["init_state"][k] = 5.0
+    if poison == "x":
+        d2["x"][:, t0:t1] = float("nan")
+    elif poison == "B":
+        d2["B"][:, t0:t1] = float("inf")
+    elif poison == "C":
+        d2["C"][:, t0:t1] = float("inf")
+    elif poison == "dt":
+        d2["dt"][:, t0:t1] = float("inf")
     y2, f2 = gpu_scan(d2)
     torch.cuda.synchronize()
     assert torch.equal(y1[:, :t0], y2[:, :t0]) and torch.equal(y1[:, t1:], y2[:, t1:])
@@ -189,7 +204,8 @@ def test_final_state_is_taken_at_each_sequence_end():
 
 # --- decode state update --------------------------------------------------------------------
 
-@pytest.mark.parametrize("dtype,b,H,P,N,G", [("bf16", 64, 64, 64, 128, 1), ("f32", 3, 4, 16, 16, 2),
+@pytest.mark.parametrize("dtype,b,H,P,N,G", [("bf16", 64, 64, 64, 128, 1), ("bf16", 8, 80, 64, 128, 1),
+                                              ("f32", 3, 4, 16, 16, 2),
                                               ("bf16", 2, 8, 128, 256, 4), ("f32", 5, 6, 256, 64, 3),
                                               ("bf16", 1, 3, 48, 80, 1)])
 def test_state_update_matches_oracle(dtype, b, H, P, N, G):

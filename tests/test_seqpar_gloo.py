@@ -1,4 +1,4 @@
-"""Sequence parallelism across ranks (the survey's NEXT-1), checked at the algorithm level on CPU.
+"""Sequence parallelism across ranks, checked at the algorithm level on CPU.
 
 "5.3 Tensor Parallelism support and large-cluster training", section 4.2, splits a long
 sequence across GPUs and hands the N x P state from one GPU to the next by point-to-point

@@ -280,3 +280,47 @@ def test_dstate_256_pair_candidate():
         with pytest.raises(ProtocolError, match=what):
             for nt in (3, 5, 8):
                 check(build_scan3_pair, 30, seed=1300 + nt, nt=nt, drop=frozenset([drop]))
+
+
+def test_two_phase_conversion_in_the_e_warps():
+    """The E warps convert x of tile t + 1 in place while B^T (w o x) of tile t runs; after it
+    completes they load s, write w o x of tile t + 1 and the state entering it.  With the B rows
+    past a sequence end zeroed by P and without the waits other waits imply, the protocol is
+    clean, also on the timeout path.  Implied waits: W18's y_full and W17's e_done (as in the
+    epilogue-warp forms), and here also W17's st_free: E loads s(t) before it writes w o x of
+    tile t + 1, so x_ready(t + 1) already orders the next B^T (w o x) after that load.  The
+    stg_free wait before the state copy (hs doubles as the y staging buffer) is needed."""
+    lean = frozenset(["w17_e_done", "w18_y_full", "w17_st_free"])
+    for nt in (0, 1, 2, 3, 5, 9):
+        for partial in (False, True):
+            check(build_scan3, 30, seed=1300 + nt, nt=nt, partial=partial, conv="E2", zero_b="p", drop=lean)
+            check(build_scan3, 15, seed=1400 + nt, nt=nt, partial=partial, conv="E2", zero_b="p", drop=lean,
+                  faults=True)
+    with pytest.raises(ProtocolError):
+        for nt in (3, 5, 9):
+            check(build_scan3, 40, seed=1600 + nt, nt=nt, conv="E2", zero_b="p", drop=lean | {"e_stg_free"})
+
+
+def test_kernel_form_with_a_separate_output_chain_issuer():
+    """k_tc_scan3 as built: the two-phase conversion in the E warps, the B rows past a sequence
+    end zeroed by P, and the output chain (C' h_prev, S x) on its own issuing warp (W24) beside
+    W17's B^T (w o x), without the waits other waits imply.  Clean, also on the timeout path;
+    W24's own waits for x_ready (S x reads the converted x), s_ready and its drain are each
+    needed, and so is W16's wait for s_done before it reloads a stage: W24's y_full commit does
+    not cover W17's B^T (w o x), which reads the stage's B."""
+    lean = frozenset(["w17_e_done", "w18_y_full", "w17_st_free"])
+    kw = dict(conv="E2", zero_b="p", y_issuer=True)
+    for nt in (0, 1, 2, 3, 5, 9):
+        for partial in (False, True):
+            check(build_scan3, 30, seed=1700 + nt, nt=nt, partial=partial, drop=lean, **kw)
+            check(build_scan3, 15, seed=1800 + nt, nt=nt, partial=partial, drop=lean, faults=True, **kw)
+    with pytest.raises(ProtocolError, match="race on x"):
+        for nt in (1, 2, 3):
+            check(build_scan3, 40, seed=1900 + nt, nt=nt, drop=lean | {"w24_x_ready"}, **kw)
+    with pytest.raises(ProtocolError, match="race on tS"):
+        for nt in (2, 3, 5):
+            check(build_scan3, 40, seed=2000 + nt, nt=nt, drop=lean | {"w17_s_ready"}, **kw)
+    assert "in flight" in (_faults(build_scan3, drop=lean | {"w24_fin"}, **kw) or "")
+    with pytest.raises(ProtocolError, match="race on b"):
+        for nt in (3, 5, 9):
+            check(build_scan3, 60, seed=2100 + nt, nt=nt, drop=lean | {"w16_s_done"}, **kw)

@@ -4,10 +4,11 @@ It exists for callers that cannot let the library allocate device memory (a
 serving engine whose pool already owns almost all of HBM, or code that must
 not allocate after start-up).  It keeps its scratch in a fixed 32 MiB device
 array inside the library, so these tests check that (1) through the C ABI it
-gives the same results as the allocating ssd_chunk_scan_fwd, within the
-parity tolerance, on two different calls in a row (the second call must not
-be disturbed by what the first left in the shared scratch), and (2) a call
-whose scratch would not fit is refused before anything runs.
+matches the fp64 oracle element by element within the parity tolerance, and
+agrees with the allocating ssd_chunk_scan_fwd within the same tolerance, on two
+different calls in a row (the second call must not be disturbed by what the
+first left in the shared scratch), and (2) a call whose scratch would not fit
+is refused before anything runs.
 
 The file name makes pytest collect it last.
 """
@@ -18,7 +19,7 @@ import torch
 
 import state_space_model_07_b200 as ssd
 from state_space_model_07_b200 import _lib, inputs
-from tests.helpers import TOL, assert_close
+from tests.helpers import TOL, assert_close, oracle_scan, to_cpu
 
 pytestmark = pytest.mark.gpu
 
@@ -61,10 +62,13 @@ def test_noalloc_matches_allocating_scan_on_two_calls_in_a_row():
         assert rc == 0, _lib.lib().ssd_last_error().decode()
         outs.append((y, fs))
     torch.cuda.synchronize()
-    for (y, fs), (yr, fr), d in zip(outs, refs, (d1, d2)):
+    for (y, fs), (ya, fa), d in zip(outs, refs, (d1, d2)):
         tol = TOL[d["x"].dtype]
-        assert_close(y, yr.double().cpu().numpy(), tol, "no-alloc y")
-        assert_close(fs, fr.double().cpu().numpy(), tol, "no-alloc final_state")
+        yo, fo = oracle_scan(to_cpu(d))
+        assert_close(y, yo, tol, "no-alloc y vs oracle")
+        assert_close(fs, fo, tol, "no-alloc final_state vs oracle")
+        assert_close(y, ya.double().cpu().numpy(), tol, "no-alloc y vs allocating scan")
+        assert_close(fs, fa.double().cpu().numpy(), tol, "no-alloc final_state vs allocating scan")
 
 
 def test_noalloc_refuses_calls_beyond_its_scratch():
