@@ -146,6 +146,35 @@ SSD_API int ssd_state_update(const ssd_dims* dims, float* state, const void* x, 
                      void* stream, const float* dt_bias);
 
 /*
+ * ssd_chunk_scan_bwd -- gradient of the scan (the backward of the training step
+ * the pages describe: "5.3 Tensor Parallelism support and large-cluster
+ * training", section 6.3 and Table 5.3.1; the pages print no gradient
+ * formulas, these are the chain rule applied to the recurrence above).
+ *
+ * For the objective J = sum_t <dy_t, y_t> + <dfinal, final_state> it writes
+ *   dx, ddt   dJ/dx (b, L, H, P) and dJ/d(raw dt) (b, L, H), dtype of x
+ *   dB, dC    (b, L, G, N), dtype of x, summed over the heads of each group
+ *   ddt_bias, dA, dD  (H) float32, summed over tokens and sequences
+ *   dinit     (S, H, N, P) float32, dJ/d init_state (NULL = not written)
+ * Inputs are those of ssd_chunk_scan_fwd with the same meaning, plus
+ *   dy        (b, L, H, P)  dtype of x, required
+ *   dfinal    (S, H, N, P)  float32, NULL = zero
+ * chunk is validated as in the forward; the result does not depend on it.
+ * Every output is overwritten (none is read).  Gradient buffers must not
+ * overlap the inputs or each other.  Computed on CUDA cores in fp32 with
+ * checkpoints of the state every 64 tokens; workspace (stream-ordered, from
+ * the library's pool) is 4 N P H (blocks + 64 S) + 8 b L G N bytes, blocks =
+ * the number of 64-token blocks over all sequences.  Supported: headdim
+ * dividing 256 and headdim * dstate in {256, 512, ..., 8192}; other shapes
+ * return SSD_ERR_UNSUPPORTED.
+ */
+SSD_API int ssd_chunk_scan_bwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
+                               const float* A, const void* B, const void* C, const float* D,
+                               const float* init_state, const int32_t* seq_idx, int chunk, const void* dy,
+                               const float* dfinal, void* dx, void* ddt, float* ddt_bias, float* dA,
+                               void* dB, void* dC, float* dD, float* dinit, void* stream);
+
+/*
  * ssd_chunk_scan_fwd_noalloc -- the same scan, for callers that cannot let the
  * library allocate device memory (for example a serving engine that has
  * already given nearly all of HBM to its own pool, or a caller that forbids

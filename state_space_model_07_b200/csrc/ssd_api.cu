@@ -350,6 +350,86 @@ int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const vo
 
 }  // extern "C"
 
+// ---- Backward of the scan -------------------------------------------------------------
+
+extern "C" int ssd_chunk_scan_bwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
+                                  const float* A, const void* B, const void* C, const float* D,
+                                  const float* init_state, const int32_t* seq_idx, int chunk, const void* dy,
+                                  const float* dfinal, void* dx, void* ddt, float* ddt_bias, float* dA,
+                                  void* dB, void* dC, float* dD, float* dinit, void* stream) {
+    g_last_error[0] = 0;
+    ssd::ScanArgs a;
+    int64_t max_chunks = 0;
+    size_t nstate = 0;
+    // the forward's validation, with dx in the place of y and dinit in that of final_state
+    int rc = prepare_scan(dims, x, dt, dt_bias, A, B, C, D, init_state, seq_idx, chunk, dx, dinit, a,
+                          max_chunks, nstate);
+    if (rc) return rc;
+    if (!ddt_bias || !dA || !dD) return fail(SSD_ERR_NULL, "ddt_bias, dA and dD are required");
+    const int64_t ntok = a.b * a.L;
+    const size_t es = a.dtype == SSD_BF16 ? 2 : 4;
+    if (ntok > 0) {
+        if (!dy || !ddt || !dB || !dC) return fail(SSD_ERR_NULL, "dy, ddt, dB and dC are required");
+        const size_t nx = (size_t)ntok * a.H * a.P * es, nbc = (size_t)ntok * a.G * a.N * es;
+        const size_t ndt = (size_t)ntok * a.H * es;
+        const void* outs[4] = {dx, ddt, dB, dC};
+        const size_t nout[4] = {nx, ndt, nbc, nbc};
+        const void* ins[5] = {x, dt, B, C, dy};
+        const size_t nin[5] = {nx, ndt, nbc, nbc, nx};
+        for (int i = 0; i < 4; ++i) {
+            for (int k = 0; k < 5; ++k)
+                if (overlaps(outs[i], nout[i], ins[k], nin[k])) return fail(SSD_ERR_SHAPE, "a gradient overlaps an input");
+            for (int k = i + 1; k < 4; ++k)
+                if (overlaps(outs[i], nout[i], outs[k], nout[k])) return fail(SSD_ERR_SHAPE, "two gradients overlap");
+        }
+    }
+    if (dfinal && !aligned16(dfinal)) return fail(SSD_ERR_SHAPE, "dfinal must be 16-byte aligned");
+    if (!ssd::bwd_supported(a))
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "the backward handles headdim dividing 256 and headdim * dstate a power-of-two multiple of "
+                    "256 up to 8192 (got headdim %lld, dstate %lld)", (long long)a.P, (long long)a.N);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    if (ntok == 0 || a.S == 0) {
+        cudaError_t e = cudaMemsetAsync(ddt_bias, 0, sizeof(float) * a.H, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dA, 0, sizeof(float) * a.H, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dD, 0, sizeof(float) * a.H, st);
+        if (e == cudaSuccess && dinit && a.S > 0)
+            e = dfinal ? cudaMemcpyAsync(dinit, dfinal, nstate, cudaMemcpyDeviceToDevice, st)
+                       : cudaMemsetAsync(dinit, 0, nstate, st);
+        if (e != cudaSuccess) return cuda_fail("empty-input gradients", e);
+        return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
+    }
+    // sequence tables with 64-token blocks (the backward's checkpoint spacing)
+    ssd::ScanArgs a64 = a;
+    a64.Q = 64;
+    const bool dbg = debug_check();
+    const size_t ws_path = ssd::bwd_workspace_bytes(a);
+    const size_t ws_bytes = Carve::round(ws_path) + scan_table_bytes(a64);
+    Carve cv;
+    cudaMemPool_t pool = workspace_pool();
+    if (!pool) return fail(SSD_ERR_CUDA, "could not create the workspace memory pool");
+    cudaError_t e = cudaMallocFromPoolAsync((void**)&cv.base, ws_bytes, pool, st);
+    if (e != cudaSuccess) return cuda_fail("cudaMallocFromPoolAsync(workspace)", e);
+    void* ws_main = cv.take(ws_path);
+    int32_t* status = nullptr;
+    ssd::SeqInfo si;
+    rc = scan_tables(a64, cv, dbg, &status, &si, st);
+    if (rc == SSD_OK) {
+        ssd::BwdArgs g;
+        g.dy = dy; g.dfinal = dfinal; g.dx = dx; g.ddt = ddt; g.dB = dB; g.dC = dC;
+        g.ddt_bias = ddt_bias; g.dA = dA; g.dD = dD; g.dinit = dinit;
+        rc = ssd::launch_scan_bwd(a, g, si, ws_main, st);
+        if (rc) rc = fail(SSD_ERR_CUDA, "could not clear the gradient accumulators");
+    }
+    e = cudaGetLastError();
+    if (rc == SSD_OK && e != cudaSuccess) rc = cuda_fail("kernel launch", e);
+    if (rc == SSD_OK && dbg) rc = debug_sync(st, status);
+    cudaError_t ef = cudaFreeAsync(cv.base, st);
+    if (rc == SSD_OK && ef != cudaSuccess) rc = cuda_fail("cudaFreeAsync(workspace)", ef);
+    return rc;
+}
+
 // ---- Self-test of the bounded device waits -------------------------------------------
 
 extern "C" int ssd_selftest_bounded_wait(int64_t limit_cycles, void* stream) {

@@ -41,6 +41,22 @@ struct UpdateArgs {
 };
 void launch_state_update(const UpdateArgs& a, cudaStream_t st);
 
+// Backward of the scan (ssd_bwd.cu): the gradients' buffers of one
+// ssd_chunk_scan_bwd call.
+struct BwdArgs {
+    const void* dy;            // (b, L, H, P), dtype of x
+    const float* dfinal;       // (S, H, N, P) or null
+    void *dx, *ddt, *dB, *dC;  // dtype of x
+    float *ddt_bias, *dA, *dD; // (H)
+    float* dinit;              // (S, H, N, P) or null
+};
+// Shapes the CUDA-core backward handles: P divides 256, N P a power-of-two
+// multiple of 256 up to 8192.
+bool bwd_supported(const ScanArgs& a);
+size_t bwd_workspace_bytes(const ScanArgs& a);
+// `si64` describes the sequences with 64-token blocks (chunk_off counts them).
+int launch_scan_bwd(const ScanArgs& a, const BwdArgs& g, const SeqInfo& si64, void* ws, cudaStream_t st);
+
 // Debug-mode value checks around a tensor-core scan (ssd_check.cu): counters[0]
 // += non-finite inputs, counters[1] += finite x / B / C / init_state values
 // beyond the fp16 range, counters[2] += non-finite outputs.

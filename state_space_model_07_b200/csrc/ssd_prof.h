@@ -15,6 +15,8 @@ enum KernelId : int {
     K_TC_PREP,
     K_TC_SCAN,
     K_SELFTEST_WAIT,
+    K_SCAN_BWD,
+    K_BWD_CAST,
     K_COUNT
 };
 
