@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--workload", default="mamba2_2.7b_layer")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqpar", action="store_true",
+                    help="split each sequence of the workload over the ranks (state passed along a ring); "
+                         "default: every rank runs its own replica")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (small cases for profiling; not a bench line)")
     return ap.parse_args()
@@ -493,10 +496,97 @@ def run_ours(args):
     return 0
 
 
+def run_seqpar(args):
+    """One scan of the workload split along the sequence over the ranks: rank r holds tokens
+    [r L/N, (r + 1) L/N) of every batch row, scans them, receives the state entering its slice
+    from rank r - 1 (NCCL point-to-point), passes the state leaving it on and rescans from the
+    state it received (state_space_model_07_b200.seqpar).  Total work is fixed as N grows."""
+    import torch
+    import torch.distributed as dist
+    from state_space_model_07_b200 import _lib, inputs, seqpar
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    w = workload_of(args)
+    if w.packed_nseqs:
+        raise SystemExit("--seqpar splits batch rows; packed workloads are not supported")
+    d = inputs.make_inputs(w, dev)
+    b, L, H, P = d["x"].shape
+    lo, hi = rank * L // world, (rank + 1) * L // world
+    part = {k: d[k][:, lo:hi].contiguous() for k in ("x", "dt", "B", "C")}
+    del d["x"], d["B"], d["C"]
+    comm = seqpar.TorchDistComm() if world > 1 else seqpar.LocalRing(1)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return seqpar.chunk_scan_fwd_seqpar(part["x"], part["dt"], d["A"], part["B"], part["C"], comm=comm,
+                                            dt_bias=d["dt_bias"], D=d["D"], init_state=d["init_state"],
+                                            chunk=w.chunk)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        for _ in range(args.warmup):
+            step()
+        barrier()
+        _lib.profile_read(reset=True)
+        _lib.profile_enable(True)
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        barrier()
+    _lib.profile_enable(False)
+    stats = _lib.profile_read(reset=True)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    tokens = b * L
+    value = tokens * args.steps / (ms * 1e-3)
+    pk, pk_src = peaks()
+    nl, nt, tot = stats.get("tc_scan", stats.get("simt_chunk_out", (0, 0, 0.0)))
+    avg_ms = tot / max(nt, 1)
+    runs = 1 if world == 1 or rank == 0 else 2     # ranks >= 1 scan their slice twice
+    alg = workload_bytes(inputs.scaled(w, seqlen=hi - lo), b, b * (hi - lo), part["x"].element_size())
+    roof = {"kernel": "tc_scan", "bound": "hbm", "achieved": alg / (avg_ms * 1e-3) / 1e9 if avg_ms else None,
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_source": pk_src, "avg_launch_ms": avg_ms,
+            "launches": nl, "algorithmic_bytes_per_launch": alg, "traffic": None,
+            "scans_per_step_on_this_rank": runs}
+    roof["frac"] = roof["achieved"] / roof["peak"] if roof["achieved"] else None
+    launches = sum(v[0] for v in stats.values())
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    cfg = config_of(w)
+    cfg.update(parallelism=f"seqpar{world}", step="one ssd_chunk_scan_fwd of the workload split along the "
+               "sequence over the ranks: local scan, state ring (NCCL send / recv), rescan on ranks >= 1",
+               tokens_per_rank=hi - lo)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16" if part["x"].element_size() == 2 else "f32", "data": "synthetic",
+            "config": cfg, "roofline": roof, "cpu_baseline": None,
+            "e2e": None, "e2e_note": "sequence-parallel mode times device-resident slices only",
+            "gpu_launches": launches, "kernels": {k: {"launches": v[0], "avg_ms": v[2] / max(v[1], 1)}
+                                                  for k, v in stats.items()},
+            "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.seqpar:
+        return run_seqpar(args)
     return run_ours(args)
 
 

@@ -146,6 +146,26 @@ SSD_API int ssd_state_update(const ssd_dims* dims, float* state, const void* x, 
                      void* stream, const float* dt_bias);
 
 /*
+ * Sequence-parallel state passing ("5.3 Tensor Parallelism ...", section 4.2:
+ * a long sequence split over devices, the N x P state handed from each device
+ * to the next).  A slice scanned from a zero state (final state F) leaves the
+ * state h_out = exp(D) h_in + F for a state h_in entering it, with D its total
+ * log-decay; these two calls compute D and that step, on the device.
+ *
+ * ssd_segment_logdecay -- D[b, h] = sum_t softplus(dt[b, t, h] + dt_bias_h) A_h
+ *   dt (b, L, H) dtype of dims; dt_bias (H) float32, NULL = 0; A (H) float32;
+ *   out (b, H) float32.  Uses dims->batch, seqlen, nheads, dtype.
+ * ssd_state_chain -- h_out = exp(logdecay) h_in + F per (batch, head)
+ *   h_in, F, h_out (b, H, N, P) float32, 16-byte aligned; logdecay (b, H)
+ *   float32.  h_out may alias h_in or F exactly.  Uses dims->batch, nheads,
+ *   headdim, dstate.
+ */
+SSD_API int ssd_segment_logdecay(const ssd_dims* dims, const void* dt, const float* dt_bias, const float* A,
+                                 float* out, void* stream);
+SSD_API int ssd_state_chain(const ssd_dims* dims, const float* h_in, const float* logdecay, const float* F,
+                            float* h_out, void* stream);
+
+/*
  * ssd_chunk_scan_bwd -- gradient of the scan (the backward of the training step
  * the pages describe: "5.3 Tensor Parallelism support and large-cluster
  * training", section 6.3 and Table 5.3.1; the pages print no gradient

@@ -350,6 +350,50 @@ int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const vo
 
 }  // extern "C"
 
+// ---- Sequence-parallel state passing ---------------------------------------------------
+
+extern "C" int ssd_segment_logdecay(const ssd_dims* dims, const void* dt, const float* dt_bias, const float* A,
+                                    float* out, void* stream) {
+    g_last_error[0] = 0;
+    if (!dims) return fail(SSD_ERR_NULL, "dims is NULL");
+    int rc = check_sizes(dims);
+    if (rc) return rc;
+    const int64_t b = dims->batch, L = dims->seqlen, H = dims->nheads;
+    if (L < 0) return fail(SSD_ERR_SHAPE, "seqlen %lld < 0", (long long)L);
+    if (b == 0) return SSD_OK;
+    if (!A || !out || (L > 0 && !dt)) return fail(SSD_ERR_NULL, "dt, A and out are required");
+    if (b * H > 0x7fffffffLL) return fail(SSD_ERR_SHAPE, "batch * nheads too large");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    ssd::launch_segment_logdecay(b, L, H, dims->dtype, dt, dt_bias, A, out, st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("kernel launch", e);
+    return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
+}
+
+extern "C" int ssd_state_chain(const ssd_dims* dims, const float* h_in, const float* logdecay, const float* F,
+                               float* h_out, void* stream) {
+    g_last_error[0] = 0;
+    if (!dims) return fail(SSD_ERR_NULL, "dims is NULL");
+    int rc = check_sizes(dims);
+    if (rc) return rc;
+    const int64_t b = dims->batch, H = dims->nheads, NP = dims->dstate * dims->headdim;
+    if (b == 0) return SSD_OK;
+    if (!h_in || !logdecay || !F || !h_out) return fail(SSD_ERR_NULL, "h_in, logdecay, F and h_out are required");
+    if (!aligned16(h_in) || !aligned16(F) || !aligned16(h_out))
+        return fail(SSD_ERR_SHAPE, "h_in, F and h_out must be 16-byte aligned");
+    const size_t ns = (size_t)b * H * NP * sizeof(float);
+    if ((h_out != h_in && overlaps(h_out, ns, h_in, ns)) || (h_out != F && overlaps(h_out, ns, F, ns)) ||
+        overlaps(h_out, ns, logdecay, (size_t)b * H * sizeof(float)))
+        return fail(SSD_ERR_SHAPE, "h_out partially overlaps an input");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    ssd::launch_state_chain(b * H, NP, h_in, logdecay, F, h_out, st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("kernel launch", e);
+    return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
+}
+
 // ---- Backward of the scan -------------------------------------------------------------
 
 extern "C" int ssd_chunk_scan_bwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,

@@ -57,6 +57,14 @@ size_t bwd_workspace_bytes(const ScanArgs& a);
 // `si64` describes the sequences with 64-token blocks (chunk_off counts them).
 int launch_scan_bwd(const ScanArgs& a, const BwdArgs& g, const SeqInfo& si64, void* ws, cudaStream_t st);
 
+// Sequence-parallel state passing (ssd_seqpar.cu): the total log-decay of
+// each batch row's slice, out (b, H); and h_out = exp(logdecay) h_in + F over
+// bh (batch, head) pairs of N P floats.
+void launch_segment_logdecay(int64_t b, int64_t L, int64_t H, int dtype, const void* dt, const float* dt_bias,
+                             const float* A, float* out, cudaStream_t st);
+void launch_state_chain(int64_t bh, int64_t NP, const float* h_in, const float* logdecay, const float* F,
+                        float* h_out, cudaStream_t st);
+
 // Debug-mode value checks around a tensor-core scan (ssd_check.cu): counters[0]
 // += non-finite inputs, counters[1] += finite x / B / C / init_state values
 // beyond the fp16 range, counters[2] += non-finite outputs.

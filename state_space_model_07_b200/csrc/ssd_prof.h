@@ -17,6 +17,8 @@ enum KernelId : int {
     K_SELFTEST_WAIT,
     K_SCAN_BWD,
     K_BWD_CAST,
+    K_SEG_DECAY,
+    K_STATE_CHAIN,
     K_COUNT
 };
 

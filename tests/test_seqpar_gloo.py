@@ -10,8 +10,11 @@ and exchange real tensors:
      but the last sends h_out = exp(D_r) h_in + F_r (rank 0: h_out = F_0) to rank r + 1;
   3. every rank r >= 1 rescans its slice from h_in (the rerun form pinned in
      tests/test_tile_model.py), and the last rank's final state is the sequence's.
-The stitched y and final state equal one oracle scan of the whole sequence.  The per-slice scans
-are the fp64 oracle: this checks the distributed algorithm and its message order, not GPU code.
+The ranks run the library's own ring code (state_space_model_07_b200.seqpar: its send / receive
+order over torch.distributed and its use of the scan, decay and chain steps) with those steps
+supplied in fp64 on the CPU (the scan by the oracle), so the stitched y and final state must
+equal one oracle scan of the whole sequence to rounding.  The GPU kernels of the steps are
+checked in tests/test_seqpar_gpu.py.
 """
 import os
 import socket
@@ -40,36 +43,45 @@ def _softplus(z):
     return np.where(z > 0, z + np.log1p(np.exp(-np.abs(z))), np.log1p(np.exp(np.minimum(z, 0))))
 
 
+def _oracle_ops():
+    """The compute steps in fp64 on the CPU (the scan by the oracle), so that the library's ring
+    code (chunk_scan_fwd_seqpar, TorchDistComm) runs unchanged on gloo ranks without a GPU."""
+    import torch
+    import oracle
+    from state_space_model_07_b200.seqpar import SeqParOps
+
+    class OracleOps(SeqParOps):
+        def scan(self, x, dt, A, B, C, *, dt_bias, D, init_state, chunk, y=None):
+            h0 = None if init_state is None else init_state.numpy()
+            yy, F = oracle.ssd_scan(x.numpy(), dt.numpy(), A.numpy(), B.numpy(), C.numpy(), dt_bias=dt_bias.numpy(),
+                                    D=D.numpy(), init_state=h0, nthreads=1)
+            return torch.from_numpy(yy), torch.from_numpy(np.ascontiguousarray(F))
+
+        def logdecay(self, dt, A, *, dt_bias):
+            return torch.from_numpy(np.sum(_softplus(dt.numpy() + dt_bias.numpy()) * A.numpy(), axis=1))
+
+        def chain(self, h_in, logdecay, F):
+            return torch.exp(logdecay)[:, :, None, None] * h_in + F
+
+    return OracleOps()
+
+
 def _worker(rank, world, port, out):
     import torch
     import torch.distributed as dist
-    import oracle
+    from state_space_model_07_b200.seqpar import TorchDistComm, chunk_scan_fwd_seqpar
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        a = _inputs()
+        a = {k: (None if v is None else torch.from_numpy(v)) for k, v in _inputs().items()}
         L = a["x"].shape[1]
         bounds = np.linspace(0, L, world + 1).astype(int)
         sl = slice(bounds[rank], bounds[rank + 1])
-        part = {k: a[k][:, sl] for k in ("x", "dt", "B", "C")}
-        scan = lambda h0: oracle.ssd_scan(part["x"], part["dt"], a["A"], part["B"], part["C"],
-                                          dt_bias=a["dt_bias"], D=a["D"], init_state=h0, nthreads=1)
-        # 1. local scan (rank 0 from the real initial state) and the slice's log-decay
-        y, F = scan(a["init_state"] if rank == 0 else None)
-        D = np.sum(_softplus(part["dt"] + a["dt_bias"]) * a["A"], axis=1)          # (b, H)
-        # 2. the ring of entering states
-        h_in = None
-        if rank > 0:
-            buf = torch.empty(F.shape, dtype=torch.float64)
-            dist.recv(buf, src=rank - 1)
-            h_in = buf.numpy()
-        if rank < world - 1:
-            h_out = F if rank == 0 else np.exp(D)[:, :, None, None] * h_in + F
-            dist.send(torch.from_numpy(np.ascontiguousarray(h_out)), dst=rank + 1)
-        # 3. rescan from the entering state
-        if rank > 0:
-            y, F = scan(h_in)
-        out[rank] = (y, F)
+        part = {k: a[k][:, sl].contiguous() for k in ("x", "dt", "B", "C")}
+        y, F = chunk_scan_fwd_seqpar(part["x"], part["dt"], a["A"], part["B"], part["C"], comm=TorchDistComm(),
+                                     dt_bias=a["dt_bias"], D=a["D"], init_state=a["init_state"], chunk=64,
+                                     ops_=_oracle_ops())
+        out[rank] = (y.numpy(), F.numpy())
         dist.barrier()
     finally:
         dist.destroy_process_group()
