@@ -2,7 +2,9 @@
  * Calling libssd.so from plain C (no Python, no torch): one fp32 scan over two
  * short sequences, then one decode step that continues from the scan's final
  * state.  Built by tests/test_c_api.py against include/ssd.h and the in-tree
- * library; run it on a machine with a GPU to see the status codes come back 0.
+ * library.  Run with a file name, it writes every input and output there
+ * (float32, in the order of dump() below) so that a test can check them
+ * against an independent implementation.
  */
 #include <cuda_runtime.h>
 #include <stdio.h>
@@ -29,7 +31,15 @@ static float* dev_fill(size_t n, float scale) {
     return d;
 }
 
-int main(void) {
+static int dump(FILE* f, const float* d, size_t n) {
+    float* h = (float*)malloc(n * sizeof(float));
+    if (!h || cudaMemcpy(h, d, n * sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess) return 1;
+    const int bad = fwrite(h, sizeof(float), n, f) != n;
+    free(h);
+    return bad;
+}
+
+int main(int argc, char** argv) {
     const int64_t b = 2, L = 100, H = 4, P = 16, N = 16, G = 2;
     ssd_dims dims = {b, L, H, P, N, G, 0, SSD_F32};
     float *x = dev_fill(b * L * H * P, 1.f), *dt = dev_fill(b * L * H, 1.f);
@@ -58,6 +68,18 @@ int main(void) {
         return 3;
     }
     CHECK_CUDA(cudaDeviceSynchronize());
+    if (argc > 1) {
+        FILE* f = fopen(argv[1], "wb");
+        if (!f) return 4;
+        int bad = 0;
+        bad |= dump(f, x, b * L * H * P) | dump(f, dt, b * L * H) | dump(f, Bm, b * L * G * N);
+        bad |= dump(f, Cm, b * L * G * N) | dump(f, A, H) | dump(f, D, H) | dump(f, bias, H);
+        bad |= dump(f, y, b * L * H * P) | dump(f, x1, b * H * P) | dump(f, dt1, b * H);
+        bad |= dump(f, B1, b * G * N) | dump(f, C1, b * G * N) | dump(f, y1, b * H * P);
+        bad |= dump(f, state, b * H * N * P);
+        fclose(f);
+        if (bad) return 5;
+    }
     printf("ok\n");
     return 0;
 }
