@@ -84,7 +84,6 @@ struct Cfg {
 
 struct TcCtl {
     int abort;
-    int p_flag, e_flag;            // leader-wait results handed to the rest of a role (k_tc_scan<N>)
 };
 
 template <int N>
@@ -145,37 +144,10 @@ __device__ __forceinline__ bool wait_bar(TcCtl& c, uint64_t* bar, uint32_t parit
 
 // Bounded wait of a whole warp; the result is the same in every lane, so the
 // warp-collective TMEM instructions that follow stay uniform even on the
-// error path.
+// error path.  Every warp of a role polls its waits itself: a rendezvous of the
+// role's warps at each wait would let one lagging warp hold the whole role back.
 __device__ __forceinline__ bool wait_bar_w(TcCtl& c, uint64_t* bar, uint32_t parity, int32_t* status) {
     return __all_sync(0xffffffffu, wait_bar(c, bar, parity, status));
-}
-
-// Bounded wait of a whole 8-warp role: only the role's first warp polls the
-// mbarrier; the other seven sleep in a hardware named barrier, so waiting
-// warps take no issue slots from the warps doing work.  `flag` carries the
-// leader's result (false once the CTA has given up) to the others.
-template <int kBarId>
-__device__ __forceinline__ bool wait_role(TcCtl& c, uint64_t* bar, uint32_t parity, int32_t* status,
-                                          bool leader, int* flag) {
-    if (leader) {
-        const bool ok = wait_bar_w(c, bar, parity, status);
-        if ((threadIdx.x & 31) == 0) *(volatile int*)flag = ok ? 1 : 0;
-    }
-    asm volatile("bar.sync %0, 256;" ::"n"(kBarId) : "memory");
-    return *(volatile int*)flag != 0;
-}
-
-// The same for two barriers at once (one named-barrier round for both);
-// `bar2` may be null.
-template <int kBarId>
-__device__ __forceinline__ bool wait_role2(TcCtl& c, uint64_t* bar1, uint32_t par1, uint64_t* bar2, uint32_t par2,
-                                           int32_t* status, bool leader, int* flag) {
-    if (leader) {
-        const bool ok = wait_bar_w(c, bar1, par1, status) && (!bar2 || wait_bar_w(c, bar2, par2, status));
-        if ((threadIdx.x & 31) == 0) *(volatile int*)flag = ok ? 1 : 0;
-    }
-    asm volatile("bar.sync %0, 256;" ::"n"(kBarId) : "memory");
-    return *(volatile int*)flag != 0;
 }
 
 template <int N>
@@ -364,7 +336,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             const int buf = t & 1, bst = t % C::kBCStages;
             const int q = (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT);
             // E is done with tile t - 2, whose decay arrays share this parity
-            if (t >= 2 && !wait_role<1>(ctl, &s.e_done[buf], ((t - 2) >> 1) & 1, p.status, warp == 0, &ctl.p_flag))
+            if (t >= 2 && !wait_bar_w(ctl, &s.e_done[buf], ((t - 2) >> 1) & 1, p.status))
                 break;
             // both warps of a quarter compute the scan; the first one publishes it
             float dj = 0.f, a = 0.f;
@@ -393,7 +365,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             }
             mbar_arrive(&s.scan_done[buf]);
             p_bar();
-            if (!wait_role<1>(ctl, &s.cb_done, t & 1, p.status, warp == 0, &ctl.p_flag)) break;
+            if (!wait_bar_w(ctl, &s.cb_done, t & 1, p.status)) break;
             if (j >= q) {
                 // C B^T has read this tile's B: zero the rows past the sequence end
                 // so that B^T (w o x) sees exact zeros there (even for non-finite data)
@@ -405,7 +377,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             }
             // S of the previous tile has been consumed by its S x
             if (t > 0 &&
-                !wait_role<1>(ctl, &s.yd_par[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status, warp == 0, &ctl.p_flag))
+                !wait_bar_w(ctl, &s.yd_par[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status))
                 break;
             tc_fence_after();
             // S = C B^T o 2^(cs_j - cs_i) d_i for i <= j, plus D on the diagonal.  This warp
@@ -471,7 +443,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
         auto prepare = [&](int u, bool first) -> bool {
             const int st = u & 1;
             const int qu = (int)(len - (int64_t)u * kT < kT ? len - (int64_t)u * kT : kT);
-            if (!wait_role<2>(ctl, &s.scan_done[st], (u >> 1) & 1, p.status, warp == 8, &ctl.e_flag)) return false;
+            if (!wait_bar_w(ctl, &s.scan_done[st], (u >> 1) & 1, p.status)) return false;
             const float cs2j = s.cs[st][j], dj = s.d[st][j], cs2_last = s.cs[st][qu - 1];
             const float e = ex2(cs2_last);
 #pragma unroll 1
@@ -515,7 +487,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 }
             }
             tmem_st_wait();
-            if (!wait_role<2>(ctl, &s.xfull[st], (u >> 1) & 1, p.status, warp == 8, &ctl.e_flag)) return false;
+            if (!wait_bar_w(ctl, &s.xfull[st], (u >> 1) & 1, p.status)) return false;
             const __half2 w2 = __float2half2_rn(dj * ex2(cs2_last - cs2j));
             uint8_t* xt = s.x[st];
             uint4 v[4];
@@ -552,7 +524,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 // the state entering tile k is complete once B^T (w o x) of tile k - 1 has been
                 // added; that also frees hs and (w o x) for tile k
                 if (k > 0) {
-                    if (!(ok = wait_role<2>(ctl, &s.sc_done, (k - 1) & 1, p.status, warp == 8, &ctl.e_flag))) break;
+                    if (!(ok = wait_bar_w(ctl, &s.sc_done, (k - 1) & 1, p.status))) break;
                     tc_fence_after();
                 }
                 if (!(ok = prepare(k, k == 0))) break;
@@ -561,7 +533,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             const int t = k - 1, st = t & 1;
             const int q = (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT);
             // epilogue of tile t: y = Yd + 2^cs_j Yo   (D x is inside Yd)
-            if (!(ok = wait_role<2>(ctl, &s.yd_par[st], (t >> 1) & 1, p.status, warp == 8, &ctl.e_flag))) break;
+            if (!(ok = wait_bar_w(ctl, &s.yd_par[st], (t >> 1) & 1, p.status))) break;
             tc_fence_after();
             {
                 const float ej = ex2(s.cs[st][j]);
