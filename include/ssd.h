@@ -211,8 +211,10 @@ SSD_API int ssd_chunk_scan_bwd(const ssd_dims* dims, const void* x, const void* 
  *     ceil(L / chunk) + nseqs when packed.  Larger calls are rejected with
  *     SSD_ERR_UNSUPPORTED before anything is launched (ssd_last_error() says
  *     how much was needed);
- *   - the array is held by every GPU that uses this call, from its first use
- *     until the process exits;
+ *   - the array is part of the library's device code: every GPU on which that
+ *     code is loaded holds it until the process exits (loaded at first use
+ *     under CUDA's default lazy module loading, at context creation with
+ *     CUDA_MODULE_LOADING=EAGER);
  *   - the first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
  *     stream capture;

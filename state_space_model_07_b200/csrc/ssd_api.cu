@@ -334,7 +334,8 @@ int ssd_state_update(const ssd_dims* dims, float* state, const void* x, const vo
     if (overlaps(y, (size_t)b * H * P * es, state, (size_t)b * H * N * P * 4) ||
         overlaps(y, (size_t)b * H * P * es, x, (size_t)b * H * P * es))
         return fail(SSD_ERR_SHAPE, "y overlaps state or x");
-    if (b * H > 0x7fffffffLL / 8) return fail(SSD_ERR_SHAPE, "batch * nheads too large");
+    // the decode grid has up to b H P / 16 blocks
+    if (b * H > 0x7fffffffLL / 16) return fail(SSD_ERR_SHAPE, "batch * nheads too large");
     cudaStream_t st = (cudaStream_t)stream;
     cudaGetLastError();
     ssd::UpdateArgs a;
