@@ -150,7 +150,9 @@ SSD_API int ssd_state_update(const ssd_dims* dims, float* state, const void* x, 
  * a long sequence split over devices, the N x P state handed from each device
  * to the next).  A slice scanned from a zero state (final state F) leaves the
  * state h_out = exp(D) h_in + F for a state h_in entering it, with D its total
- * log-decay; these two calls compute D and that step, on the device.
+ * log-decay; these two calls compute D and that step, on the device.  The
+ * slice's own output then misses only the part that comes from h_in, which
+ * ssd_state_to_output adds.
  *
  * ssd_segment_logdecay -- D[b, h] = sum_t softplus(dt[b, t, h] + dt_bias_h) A_h
  *   dt (b, L, H) dtype of dims; dt_bias (H) float32, NULL = 0; A (H) float32;
@@ -164,6 +166,27 @@ SSD_API int ssd_segment_logdecay(const ssd_dims* dims, const void* dt, const flo
                                  float* out, void* stream);
 SSD_API int ssd_state_chain(const ssd_dims* dims, const float* h_in, const float* logdecay, const float* F,
                             float* h_out, void* stream);
+
+/*
+ * ssd_state_to_output -- the output of a state entering each row at its start
+ * (the state-to-output term of "5.3 Tensor Parallelism ...", section 3.2,
+ * measured from the row's first token):
+ *   y[b, t, h, :] += exp(sum_{i <= t} softplus(dt[b, i, h] + dt_bias_h) A_h)
+ *                    * sum_n C[b, t, g, n] h_in[b, h, n, :],   g = h / (H / G)
+ * so that a scan of the row from a zero state plus this call equals the scan
+ * from h_in (up to rounding: y is read as bf16 and written back as bf16).
+ *   dt (b, L, H), C (b, L, G, N), y (b, L, H, P): bfloat16; y is read and
+ *   written in place.  h_in (b, H, N, P), A (H) float32; dt_bias (H) float32,
+ *   NULL = 0.  C, h_in and y 16-byte aligned; y must not overlap the inputs.
+ * Runs on the tensor cores (C and h_in rounded to fp16 operands, fp32
+ * accumulation; the value range of ssd_chunk_scan_fwd applies): dtype
+ * SSD_BF16, headdim 64 and dstate 128 only, SSD_ERR_UNSUPPORTED otherwise, and
+ * for nseqs > 0.  Workspace (stream-ordered, from the library's pool):
+ * 2 b L G N + 520 b H ceil(L / 128) bytes.  Uses dims->batch, seqlen, nheads,
+ * headdim, dstate, ngroups, dtype.
+ */
+SSD_API int ssd_state_to_output(const ssd_dims* dims, const void* dt, const float* dt_bias, const float* A,
+                                const void* C, const float* h_in, void* y, void* stream);
 
 /*
  * ssd_chunk_scan_bwd -- gradient of the scan (the backward of the training step

@@ -17,7 +17,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE"
 # Every function include/ssd.h declares.
 EXPORTS = ("ssd_chunk_scan_fwd", "ssd_state_update", "ssd_status_string", "ssd_last_error",
            "ssd_profile_enable", "ssd_profile_read", "ssd_chunk_scan_fwd_noalloc", "ssd_selftest_bounded_wait",
-           "ssd_chunk_scan_bwd", "ssd_segment_logdecay", "ssd_state_chain")
+           "ssd_chunk_scan_bwd", "ssd_segment_logdecay", "ssd_state_chain", "ssd_state_to_output")
 
 
 class SsdDims(ctypes.Structure):
@@ -61,6 +61,8 @@ def lib():
         L.ssd_segment_logdecay.argtypes = [dims] + [_VP] * 5
         L.ssd_state_chain.restype = ctypes.c_int
         L.ssd_state_chain.argtypes = [dims] + [_VP] * 5
+        L.ssd_state_to_output.restype = ctypes.c_int
+        L.ssd_state_to_output.argtypes = [dims] + [_VP] * 7
         L.ssd_state_update.restype = ctypes.c_int
         L.ssd_state_update.argtypes = [dims] + [_VP] * 10
         L.ssd_status_string.restype = ctypes.c_char_p

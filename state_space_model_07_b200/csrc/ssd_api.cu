@@ -397,6 +397,53 @@ extern "C" int ssd_state_chain(const ssd_dims* dims, const float* h_in, const fl
 
 // ---- Backward of the scan -------------------------------------------------------------
 
+extern "C" int ssd_state_to_output(const ssd_dims* dims, const void* dt, const float* dt_bias, const float* A,
+                                   const void* C, const float* h_in, void* y, void* stream) {
+    g_last_error[0] = 0;
+    if (!dims) return fail(SSD_ERR_NULL, "dims is NULL");
+    int rc = check_sizes(dims);
+    if (rc) return rc;
+    if (dims->nseqs) return fail(SSD_ERR_UNSUPPORTED, "packed sequences (nseqs > 0) are not taken by this call");
+    const int64_t b = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim, N = dims->dstate,
+                  G = dims->ngroups;
+    if (L < 0) return fail(SSD_ERR_SHAPE, "seqlen %lld < 0", (long long)L);
+    if (b * L == 0) return SSD_OK;
+    if (!dt || !A || !C || !h_in || !y) return fail(SSD_ERR_NULL, "dt, A, C, h_in and y are required");
+    ssd::ScanArgs a{};
+    a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G; a.S = b; a.dtype = dims->dtype; a.Q = 128;
+    a.dt = dt; a.C = C; a.dt_bias = dt_bias; a.A = A; a.y = y;
+    if (!ssd::state_out_supported(a))
+        return fail(SSD_ERR_UNSUPPORTED, "needs bfloat16 inputs, headdim 64 and dstate 128 (tensor-core path)");
+    if (!aligned16(C) || !aligned16(h_in) || !aligned16(y))
+        return fail(SSD_ERR_SHAPE, "C, h_in and y must be 16-byte aligned");
+    const size_t ny = (size_t)b * L * H * P * 2;
+    if (overlaps(y, ny, dt, (size_t)b * L * H * 2) || overlaps(y, ny, C, (size_t)b * L * G * N * 2) ||
+        overlaps(y, ny, h_in, (size_t)b * H * N * P * 4))
+        return fail(SSD_ERR_SHAPE, "y overlaps dt, C or h_in");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    const bool dbg = debug_check();
+    const size_t ws_path = ssd::state_out_workspace_bytes(a);
+    Carve cv;
+    cudaMemPool_t pool = workspace_pool();
+    if (!pool) return fail(SSD_ERR_CUDA, "could not create the workspace memory pool");
+    cudaError_t e = cudaMallocFromPoolAsync((void**)&cv.base, Carve::round(ws_path) + Carve::round(16), pool, st);
+    if (e != cudaSuccess) return cuda_fail("cudaMallocFromPoolAsync(workspace)", e);
+    void* ws = cv.take(ws_path);
+    int32_t* status = (int32_t*)cv.take(16);
+    if (dbg) {
+        e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
+        if (e != cudaSuccess) rc = cuda_fail("status reset", e);
+    }
+    if (rc == SSD_OK) rc = ssd::launch_state_to_output(a, h_in, ws, dbg ? status : nullptr, st);
+    e = cudaGetLastError();
+    if (rc == SSD_OK && e != cudaSuccess) rc = cuda_fail("kernel launch", e);
+    if (rc == SSD_OK && dbg) rc = debug_sync(st, status);
+    cudaError_t ef = cudaFreeAsync(cv.base, st);
+    if (rc == SSD_OK && ef != cudaSuccess) rc = cuda_fail("cudaFreeAsync(workspace)", ef);
+    return rc;
+}
+
 extern "C" int ssd_chunk_scan_bwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
                                   const float* A, const void* B, const void* C, const float* D,
                                   const float* init_state, const int32_t* seq_idx, int chunk, const void* dy,

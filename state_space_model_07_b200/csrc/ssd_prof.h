@@ -19,6 +19,8 @@ enum KernelId : int {
     K_BWD_CAST,
     K_SEG_DECAY,
     K_STATE_CHAIN,
+    K_STATE_OUT,
+    K_TILE_DECAY,
     K_COUNT
 };
 

@@ -113,6 +113,19 @@ struct __align__(1024) TcSmem {
     TcCtl ctl;
 };
 
+// Rows split into segments (k_tc_scan3 only).  Span index s >= first is segment
+// (s - first) % K of batch row row0 + (s - first) / K: tokens [k Ls, (k + 1) Ls) of the
+// row, the last segment running to the row's end.  Segment 0 starts from the row's
+// initial state and the others from zero; every segment's final state goes to fin
+// and the running base-2 log-decay from the segment start through each of its tokens
+// to cs (128 `tiles` floats per (segment, head)).  first = INT32_MAX: no split.
+struct SplitSpec {
+    int32_t first = 0x7fffffff, K = 0, row0 = 0, tiles = 0;
+    int64_t Ls = 0;
+    float* fin = nullptr;
+    float* cs = nullptr;
+};
+
 struct TcParams {
     SeqInfo si;
     const __nv_bfloat16* dt;
@@ -124,6 +137,7 @@ struct TcParams {
     __nv_bfloat16* y;
     int32_t* status;
     int H, G;
+    SplitSpec split;
 };
 
 __device__ __forceinline__ void p_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -708,6 +722,9 @@ struct __align__(1024) Smem {
     TcCtl ctl;
 };
 
+// kSplit: the launch holds split segments (SplitSpec); the plain instantiation carries none
+// of their bookkeeping.
+template <bool kSplit>
 __global__ void __launch_bounds__(kThreads3, 1)
 k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
            const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const TcParams p) {
@@ -722,7 +739,24 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     const int g = h / (H / G);
 
     int64_t row, t0, t1;
-    seq_span(p.si, seq, row, t0, t1);
+    const float* init_src = nullptr;   // state entering the span (null: zero)
+    float* final_dst = nullptr;        // state leaving it (null: not wanted)
+    float* tok_cs = nullptr;           // running log-decay per token (split segments only)
+    bool y_f16 = false;                // y written as fp16 (a segment after the first of its row)
+    if (kSplit && seq >= p.split.first) {
+        const int sp = seq - p.split.first, k = sp % p.split.K;
+        row = p.split.row0 + sp / p.split.K;
+        t0 = (int64_t)k * p.split.Ls;
+        t1 = k == p.split.K - 1 || t0 + p.split.Ls > p.si.L ? p.si.L : t0 + p.split.Ls;
+        if (k == 0 && p.init_state) init_src = p.init_state + (row * H + h) * N * kP;
+        final_dst = p.split.fin + ((int64_t)sp * H + h) * N * kP;
+        tok_cs = p.split.cs + ((int64_t)sp * H + h) * p.split.tiles * kT;
+        y_f16 = k > 0;
+    } else {
+        seq_span(p.si, seq, row, t0, t1);
+        if (p.init_state) init_src = p.init_state + ((int64_t)seq * H + h) * N * kP;
+        if (p.final_state) final_dst = p.final_state + ((int64_t)seq * H + h) * N * kP;
+    }
     const int64_t len = t1 > t0 ? t1 - t0 : 0;
     const int nt = (int)((len + kT - 1) / kT);
     const int64_t tok0 = row * p.si.L + t0;
@@ -803,6 +837,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
         };
         if (nt > 0) load_dt(0);
+        float run = 0.f;   // log-decay from the span start through the tile before u
         for (int u = 0; u < nt; ++u) {
             const int sl = u & 3, qu = tile_len(u);
             // P and E have read slot sl for tile u - 4
@@ -828,11 +863,18 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 cs[i] += excl;
                 cf[i] = ex2(pivot - cs[i]) * dd[i];
             }
+
             *reinterpret_cast<float4*>(&s.cs[sl][4 * lane]) = make_float4(cs[0], cs[1], cs[2], cs[3]);
             *reinterpret_cast<float4*>(&s.d[sl][4 * lane]) = make_float4(dd[0], dd[1], dd[2], dd[3]);
             *reinterpret_cast<float4*>(&s.colfac[sl][4 * lane]) = make_float4(cf[0], cf[1], cf[2], cf[3]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.scan_done[sl]);
+            if (kSplit) {
+                if (tok_cs)
+                    *reinterpret_cast<float4*>(tok_cs + (int64_t)u * kT + 4 * lane) =
+                        make_float4(run + cs[0], run + cs[1], run + cs[2], run + cs[3]);
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
             if (u + 1 < nt) load_dt(u + 1);
         }
     } else if (warp == 16) {
@@ -1114,11 +1156,14 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 tmem_ld_wait();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const uint4 val = make_uint4(
-                        pack_bf16x2(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
-                        pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
-                        pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
-                        pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+                    // a split segment's partial y waits in fp16 for the state-to-output pass
+                    // (11 significant bits: its later rounding to bf16 stays the only one that
+                    // counts even where that pass cancels most of it)
+                    auto pk = [&](int e) {
+                        const float lo = __uint_as_float(r[8 * c + e]), hi = __uint_as_float(r[8 * c + e + 1]);
+                        return kSplit && y_f16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+                    };
+                    const uint4 val = make_uint4(pk(0), pk(2), pk(4), pk(6));
                     if (q == kT)
                         *reinterpret_cast<uint4*>(stg + sw128_off(j, 4 * hh + c)) = val;
                     else if (j < q)
@@ -1148,7 +1193,7 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         float hreg[32];
         {
-            const float* src = p.init_state ? p.init_state + (((int64_t)seq * H + h) * N + j) * kP + col0 : nullptr;
+            const float* src = init_src ? init_src + (int64_t)j * kP + col0 : nullptr;
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
                 const float4 v = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1263,8 +1308,8 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
             e_cur = e_next;
         }
-        if (p.final_state && (ok || nt == 0)) {
-            float* dst = p.final_state + (((int64_t)seq * H + h) * N + j) * kP + col0;
+        if (final_dst && (ok || nt == 0)) {
+            float* dst = final_dst + (int64_t)j * kP + col0;
 #pragma unroll
             for (int c = 0; c < 32; c += 4)
                 *reinterpret_cast<float4*>(dst + c) = make_float4(hreg[c], hreg[c + 1], hreg[c + 2], hreg[c + 3]);
@@ -1281,103 +1326,412 @@ k_tc_scan3(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
 
 }  // namespace v3
 
+// ---- Contribution of an entering state to the output -------------------------------------
+//
+// For a span of tokens entered by the state h_in (N x P) and scanned from zero, the full
+// output adds, at every token j of the span,
+//   y_j += 2^(cs_j) C_j^T h_in,   cs_j = sum over the span's tokens i <= j of d_i A log2(e)
+// (the state term of section 3.2 of "5.3 Tensor Parallelism support and large-cluster
+// training", taken from the span start instead of the chunk start).  Per 128-token tile that
+// is one 128 x 64 x 128 product C h_in on the tensor core (fp16 operands, as the scan's own
+// C' h_prev), scaled by 2^cs_j per row in the epilogue and added to y in place.
+//
+// A CTA takes `tpp` consecutive tiles of one (span, head); its entering state is either given
+// (h_in) or chained from the spans before it in the row: h_in(k) = 2^D(k-1) h_in(k-1) + F(k-1),
+// with F the spans' own final states and D their total log-decay (the last entry of the
+// running log-decay table cs).  The CTA holding the first tiles of a row's last span writes
+// the row's final state 2^D h_in + F.
+//
+// Roles (384 threads, one CTA per SM):
+//   warps 0-7:  prologue (the fp16 copy of h_in), then the epilogue: TMEM -> registers,
+//               y tile (shared memory) += 2^cs_j (C h_in)_j.  Two warps per TMEM lane
+//               quarter split the 64 columns; each warp hands its part on by itself.
+//   warp 8:     TMA loads of the C and y tiles and a bulk copy of the tile's running
+//               log-decays cs_j (a table the scan wrote), kStagesSO deep: no epilogue thread
+//               waits on a global load.
+//   warps 9, 10: the MMAs of the even and of the odd tiles (an issuing thread is held for
+//               each tcgen05.mma it issues, so two of them keep up with the memory rate);
+//               warp 9 also owns the TMEM allocation.
+//   warp 11:    the TMA store of each finished y tile, which hands the stage back as soon as
+//               the store has read it.
+namespace so {
+
+constexpr int kEpiWarps = 8;
+constexpr int kThreadsSO = 32 * (kEpiWarps + 4);
+constexpr int kStagesSO = 4;
+constexpr uint32_t kTmemColsSO = 64 * kStagesSO;
+
+struct __align__(1024) SmemSO {
+    uint8_t c[kStagesSO][2][kBoxBytes];   // C (fp16), two 64-column boxes per stage
+    uint8_t y[kStagesSO][kTileBytesX];    // y (bf16), updated in place and stored from here
+    uint8_t hs[kTileBytesX];              // h_in (fp16), state rows, 128-byte swizzled
+    float cs[kStagesSO][kT];              // running log-decay cs_j of the tile's tokens
+    uint64_t full[kStagesSO];             // TMA (C, y) -> MMA, epilogue
+    uint64_t acc_full[kStagesSO];         // MMA commit -> epilogue
+    uint64_t acc_free[kStagesSO];         // epilogue (accumulator read) -> MMA
+    uint64_t y_ready[kStagesSO];          // epilogue warps (y tile updated) -> store warp
+    uint64_t stage_free[kStagesSO];       // store warp (y stored or written) -> TMA
+    uint64_t hs_ready;                    // epilogue warps (h_in in shared memory) -> MMA
+    uint64_t fin[2];                      // MMA warps: own MMAs drained before exit
+    uint32_t tmem_base;
+    TcCtl ctl;
+};
+
+struct SOParams {
+    const __nv_bfloat16* dt;
+    const float* dt_bias;
+    const float* A;
+    const float* h_in;     // (rows, H, N, P) given entering states, or null: chain from fin
+    const float* fin;      // chained mode: final state of every span, (rows K, H, N, P)
+    const float* cs;       // running log-decay from the span start through each token, 128 tiles
+                           // floats per (span, head)
+    float* final_state;    // chained mode: the rows' final states (batch rows, H, N, P) or null
+    __nv_bfloat16* y;      // (batch rows, L, H, P), updated in place
+    int y_f16;             // y holds fp16 partial outputs (chained mode), written back as bf16
+    int32_t* status;
+    int64_t L;             // tokens per batch row
+    int64_t Ls;            // tokens per span (the last span of a row runs to its end)
+    int H, G;
+    int K;                 // spans per row
+    int k0;                // first span corrected (chained mode 1: span 0 has its own state)
+    int row0;              // batch row of the first row taken
+    int tiles;             // tiles of the longest span
+    int nparts, tpp;       // parts per span, tiles per part
+};
+
+__global__ void __launch_bounds__(kThreadsSO, 1)
+k_state_out(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const SOParams p) {
+    constexpr int N = 128;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    SmemSO& s = *reinterpret_cast<SmemSO*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    TcCtl& ctl = s.ctl;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.H;
+    const int h = blockIdx.x % H;
+    int64_t rest = blockIdx.x / H;
+    const int part = (int)(rest % p.nparts);
+    rest /= p.nparts;
+    const int nk = p.K - p.k0;
+    const int k = p.k0 + (int)(rest % nk);
+    const int rr = (int)(rest / nk);               // row taken, relative to row0
+    const int64_t row = p.row0 + rr;
+    const int g = h / (H / p.G);
+    const int64_t NP = (int64_t)N * kP;
+
+    const int64_t s0 = (int64_t)k * p.Ls;
+    const int64_t s1 = k == p.K - 1 || s0 + p.Ls > p.L ? p.L : s0 + p.Ls;
+    const int nts = (int)((s1 - s0 + kT - 1) / kT);           // tiles of the span
+    const int ft = part * p.tpp;                              // first tile of this part
+    const int nt = ft < nts ? min(p.tpp, nts - ft) : 0;       // tiles of this part
+    const int64_t span = (int64_t)rr * p.K + k;
+    const float* cs_span = p.cs + (span * H + h) * p.tiles * kT;   // running log-decay per token
+    const int64_t tok_base = row * p.L + s0 + (int64_t)ft * kT;   // flat token of the first tile
+
+    if (tid == 0) {
+        for (int i = 0; i < kStagesSO; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.acc_full[i], 1);
+            mbar_init(&s.acc_free[i], kEpiWarps);
+            mbar_init(&s.y_ready[i], kEpiWarps);
+            mbar_init(&s.stage_free[i], 1);
+        }
+        mbar_init(&s.hs_ready, kEpiWarps);
+        mbar_init(&s.fin[0], 1);
+        mbar_init(&s.fin[1], 1);
+        ctl.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) tmem_alloc(&s.tmem_base, kTmemColsSO);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+
+    if (warp < kEpiWarps) {
+        // ---- prologue (while the first tiles load): the entering state, and the row's final
+        // state; thread = (column half, state row)
+        const int n = 32 * (warp & 3) + lane, c0 = 32 * (warp >> 2);
+        float hv[32];
+        if (p.h_in) {
+            const float* src = p.h_in + (row * H + h) * NP + (int64_t)n * kP + c0;
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(src + c);
+                hv[c] = v.x; hv[c + 1] = v.y; hv[c + 2] = v.z; hv[c + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) hv[c] = 0.f;
+            for (int j = 0; j < k; ++j) {
+                const int64_t sj = (int64_t)rr * p.K + j;
+                // spans before the last hold Ls tokens; the decay of span j enters from j + 1 on
+                const float e = j ? ex2(p.cs[(sj * H + h) * p.tiles * kT + p.Ls - 1]) : 0.f;
+                const float* f = p.fin + (sj * H + h) * NP + (int64_t)n * kP + c0;
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(f + c);
+                    hv[c] = e * hv[c] + v.x; hv[c + 1] = e * hv[c + 1] + v.y;
+                    hv[c + 2] = e * hv[c + 2] + v.z; hv[c + 3] = e * hv[c + 3] + v.w;
+                }
+            }
+            if (p.final_state && k == p.K - 1 && part == 0) {
+                const float e = ex2(cs_span[s1 - s0 - 1]);
+                const float* f = p.fin + (span * H + h) * NP + (int64_t)n * kP + c0;
+                float* dst = p.final_state + (row * H + h) * NP + (int64_t)n * kP + c0;
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(f + c);
+                    *reinterpret_cast<float4*>(dst + c) = make_float4(e * hv[c] + v.x, e * hv[c + 1] + v.y,
+                                                                      e * hv[c + 2] + v.z, e * hv[c + 3] + v.w);
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+            uint4 v;
+            v.x = pack_f16x2(hv[c], hv[c + 1]);
+            v.y = pack_f16x2(hv[c + 2], hv[c + 3]);
+            v.z = pack_f16x2(hv[c + 4], hv[c + 5]);
+            v.w = pack_f16x2(hv[c + 6], hv[c + 7]);
+            *reinterpret_cast<uint4*>(s.hs + sw128_off(n, (c0 + c) / 8)) = v;
+        }
+        fence_proxy_async_smem();
+        v3::warp_arrive(&s.hs_ready);
+    }
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA: C and y tiles
+        if (lane == 0 && nt > 0) {
+            tma_prefetch_desc(&tm_c);
+            tma_prefetch_desc(&tm_y);
+            int issued = 0;
+            for (int i = 0; i < nt; ++i) {
+                const int st = i % kStagesSO;
+                if (i >= kStagesSO && !wait_bar(ctl, &s.stage_free[st], ((i / kStagesSO) - 1) & 1, p.status)) break;
+                const int tok = (int)(tok_base + (int64_t)i * kT);
+                mbar_expect_tx(&s.full[st], 2 * kBoxBytes + kTileBytesX + kT * sizeof(float));
+                tma_load_3d(s.c[st][0], &tm_c, &s.full[st], 0, g, tok);
+                tma_load_3d(s.c[st][1], &tm_c, &s.full[st], 64, g, tok);
+                tma_load_3d(s.y[st], &tm_y, &s.full[st], 0, h, tok);
+                bulk_load(s.cs[st], cs_span + (int64_t)(ft + i) * kT, kT * sizeof(float), &s.full[st]);
+                ++issued;
+            }
+            if (*(volatile int*)&ctl.abort)
+                for (int i = 0; i < issued; ++i) mbar_wait(&s.full[i % kStagesSO], (i / kStagesSO) & 1, 400000000ll);
+        }
+    } else if (warp == 9 || warp == 10) {
+        // ----------------------------------------------- MMA: C h_in, even / odd tiles
+        const int par0 = warp == 9 ? 0 : 1;
+        if (lane == 0 && nt > par0) {
+            const uint32_t id = idesc_f16(128, 64, 0, 1);   // K-major A (C rows), MN-major B (state rows)
+            const uint32_t hsb = smem_u32(s.hs);
+            bool go = wait_bar(ctl, &s.hs_ready, 0, p.status);
+            for (int i = par0; go && i < nt; i += 2) {
+                const int st = i % kStagesSO;
+                if (!wait_bar(ctl, &s.full[st], (i / kStagesSO) & 1, p.status)) break;
+                if (i >= kStagesSO && !wait_bar(ctl, &s.acc_free[st], ((i / kStagesSO) - 1) & 1, p.status)) break;
+                tc_fence_after();
+                const uint32_t cb = smem_u32(s.c[st][0]);
+                for (int kk = 0; kk < N / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                    mma_ss(tmem + 64 * st, sdesc_sw128(cb + off, 16, 1024), sdesc_sw128(hsb + kk * 2048, kBoxBytes, 1024),
+                           id, kk > 0);
+                }
+                mma_commit(&s.acc_full[st]);
+            }
+            mma_commit(&s.fin[par0]);
+            mbar_wait(&s.fin[par0], 0, 400000000ll);
+        }
+    } else if (warp == 11) {
+        // ------------------------------------------------------------ TMA stores of y tiles
+        if (lane == 0 && nt > 0) {
+            bool stored = false;
+            for (int i = 0; i < nt; ++i) {
+                const int st = i % kStagesSO;
+                if (!wait_bar(ctl, &s.y_ready[st], (i / kStagesSO) & 1, p.status)) break;
+                const int64_t left = s1 - (s0 + (int64_t)(ft + i) * kT);
+                if (left >= kT) {
+                    tma_store_3d(&tm_y, s.y[st], 0, h, (int)(tok_base + (int64_t)i * kT));
+                    bulk_commit();
+                    bulk_wait_read0();
+                    stored = true;
+                }
+                mbar_arrive(&s.stage_free[st]);
+            }
+            if (stored) bulk_wait0();
+        }
+    }
+    if (warp < kEpiWarps) {
+        // ---------------------------------------------------------------------- epilogue
+        const int quarter = warp & 3, half = warp >> 2;
+        const int j = 32 * quarter + lane;                      // token row of the tile = TMEM lane
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        for (int i = 0; i < nt; ++i) {
+            const int st = i % kStagesSO;
+            const int64_t tok = tok_base + (int64_t)i * kT;
+            const int64_t left = s1 - (s0 + (int64_t)(ft + i) * kT);
+            const int q = left < kT ? (int)left : kT;
+            const bool ok = wait_bar_w(ctl, &s.acc_full[st], (i / kStagesSO) & 1, p.status) &&
+                            wait_bar_w(ctl, &s.full[st], (i / kStagesSO) & 1, p.status);
+            const float f = j < q ? ex2(s.cs[st][j]) : 0.f;
+            if (ok) {
+                tc_fence_after();
+                uint32_t r[32];
+                uint32_t (&r0)[16] = *reinterpret_cast<uint32_t (*)[16]>(&r[0]);
+                uint32_t (&r1)[16] = *reinterpret_cast<uint32_t (*)[16]>(&r[16]);
+                tmem_ld16(tmem + lane_base + 64 * st + 32 * half, r0);
+                tmem_ld16(tmem + lane_base + 64 * st + 32 * half + 16, r1);
+                tmem_ld_wait();
+                tc_fence_before();
+                v3::warp_arrive(&s.acc_free[st]);
+                // a full tile goes back through shared memory and one TMA store; the rows of a
+                // partial tile (a span's end) are written one by one, since the rows past its end
+                // belong to the next batch row
+                if (j < q) {
+                    uint8_t* yrow = s.y[st];
+                    __nv_bfloat16* yg = p.y + (tok + j) * H * kP + (int64_t)h * kP + 32 * half;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4* pv = reinterpret_cast<uint4*>(yrow + sw128_off(j, 4 * half + c));
+                        uint4 v = *pv;
+                        uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float lo, hi;
+                            if (p.y_f16) {
+                                const float2 v2 = __half22float2(u2h(w[e]));
+                                lo = v2.x;
+                                hi = v2.y;
+                            } else {
+                                lo = bf16lo(w[e]);
+                                hi = bf16hi(w[e]);
+                            }
+                            w[e] = pack_bf16x2(lo + f * __uint_as_float(r[8 * c + 2 * e]),
+                                               hi + f * __uint_as_float(r[8 * c + 2 * e + 1]));
+                        }
+                        if (q == kT)
+                            *pv = v;
+                        else
+                            *reinterpret_cast<uint4*>(yg + 8 * c) = v;
+                    }
+                }
+                fence_proxy_async_smem();
+            }
+            if (!ok) break;
+            v3::warp_arrive(&s.y_ready[st]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, kTmemColsSO);
+}
+
+}  // namespace so
+
 // bf16 -> fp16 copies of B and C (8 elements per thread step).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+    return make_uint4(pack_f16x2(bf16lo(v.x), bf16hi(v.x)), pack_f16x2(bf16lo(v.y), bf16hi(v.y)),
+                      pack_f16x2(bf16lo(v.z), bf16hi(v.z)), pack_f16x2(bf16lo(v.w), bf16hi(v.w)));
+}
+
 __global__ void k_tc_prep(const uint4* __restrict__ b, const uint4* __restrict__ c, uint4* __restrict__ b16,
                           uint4* __restrict__ c16, int64_t n8) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-        uint4 vb = b[i], vc = c[i], ob, oc;
-        ob.x = pack_f16x2(bf16lo(vb.x), bf16hi(vb.x));
-        ob.y = pack_f16x2(bf16lo(vb.y), bf16hi(vb.y));
-        ob.z = pack_f16x2(bf16lo(vb.z), bf16hi(vb.z));
-        ob.w = pack_f16x2(bf16lo(vb.w), bf16hi(vb.w));
-        oc.x = pack_f16x2(bf16lo(vc.x), bf16hi(vc.x));
-        oc.y = pack_f16x2(bf16lo(vc.y), bf16hi(vc.y));
-        oc.z = pack_f16x2(bf16lo(vc.z), bf16hi(vc.z));
-        oc.w = pack_f16x2(bf16lo(vc.w), bf16hi(vc.w));
-        b16[i] = ob;
-        c16[i] = oc;
+        b16[i] = bf16x8_to_f16x8(b[i]);
+        c16[i] = bf16x8_to_f16x8(c[i]);
     }
 }
 
-// ---- Long sequences with few (sequence, head) pairs: the two-pass split ----------------
+// ---- The output of a given entering state (ssd_state_to_output) --------------------------
+
+// bf16 -> fp16 copy of one array (as k_tc_prep).
+__global__ void k_to_f16(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n8) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = bf16x8_to_f16x8(src[i]);
+}
+
+// Sum of d A log2(e) over each 128-token tile of every row and head: one block per (row, tile),
+// one thread per head (consecutive heads are consecutive in dt).
+__global__ void k_tile_sums(const __nv_bfloat16* __restrict__ dt, const float* __restrict__ dt_bias,
+                            const float* __restrict__ A, int64_t L, int H, int nt, float* __restrict__ tsum) {
+    const int64_t row = blockIdx.x / nt;
+    const int tile = (int)(blockIdx.x % nt);
+    const int64_t t0 = (int64_t)tile * kT;
+    const int q = L - t0 < kT ? (int)(L - t0) : kT;
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+        const float bias = dt_bias ? dt_bias[h] : 0.f;
+        const __nv_bfloat16* d = dt + (row * L + t0) * H + h;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < q; ++j) acc += v3::softplus_fast(__bfloat162float(d[(int64_t)j * H]) + bias);
+        tsum[(int64_t)blockIdx.x * H + h] = acc * A[h] * 1.4426950408889634f;
+    }
+}
+
+// Running sums of the tile sums along each row: run[(row H + h) nt + t] = log-decay from the
+// row's start through tile t.  One thread per (row, head).
+__global__ void k_tile_running(const float* __restrict__ tsum, int64_t bh, int H, int nt, float* __restrict__ run) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= bh) return;
+    const int64_t row = i / H;
+    const int h = (int)(i % H);
+    float r = 0.f;
+    for (int t = 0; t < nt; ++t) {
+        r += tsum[(row * nt + t) * H + h];
+        run[i * nt + t] = r;
+    }
+}
+
+// Per token: cs[((row H + h) nt + t) 128 + j] = log-decay from the row's start through token
+// j of tile t.  One block of 128 threads (one per token) per (row, tile), heads in turn.
+__global__ void __launch_bounds__(kT)
+k_token_running(const __nv_bfloat16* __restrict__ dt, const float* __restrict__ dt_bias, const float* __restrict__ A,
+                const float* __restrict__ run, int64_t L, int H, int nt, float* __restrict__ cs) {
+    __shared__ float wsum[kT / 32];
+    const int64_t row = blockIdx.x / nt;
+    const int tile = (int)(blockIdx.x % nt);
+    const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
+    const int64_t t0 = (int64_t)tile * kT;
+    const int q = L - t0 < kT ? (int)(L - t0) : kT;
+    for (int h = 0; h < H; ++h) {
+        float a = j < q ? v3::softplus_fast(__bfloat162float(dt[(row * L + t0 + j) * H + h]) + (dt_bias ? dt_bias[h] : 0.f)) *
+                              A[h] * 1.4426950408889634f
+                        : 0.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v = __shfl_up_sync(0xffffffffu, a, o);
+            if (lane >= o) a += v;
+        }
+        if (lane == 31) wsum[warp] = a;
+        __syncthreads();
+        float before = tile > 0 ? run[(row * H + h) * nt + tile - 1] : 0.f;
+        for (int w = 0; w < warp; ++w) before += wsum[w];
+        cs[((row * H + h) * nt + tile) * kT + j] = before + a;
+        __syncthreads();
+    }
+}
+
+// ---- Few long rows: the segment split ------------------------------------------------------
 //
-// With b H CTAs well below the SM count, each sequence is cut into K segments of Ls tokens
-// (tile-aligned; the last takes the rest).  Pass 1 scans segments 0 .. K-2 of every row as
-// independent spans (segment 0 from the real initial state, so its y is final; the others from
-// zero, for their final states); the chain forms the state entering each segment k >= 1,
-//   h_in(1) = F(0),  h_in(k) = exp(sum over segment k - 1 of d A) h_in(k - 1) + F(k - 1);
-// pass 2 rescans segments 1 .. K-1 from h_in (overwriting their y) and the last one's final
-// state is the row's.  Both passes are the unchanged scan kernel over span tables.
+// One CTA scans one (row, head) from start to end, so when b H is small (few long rows) most
+// SMs sit idle.  The rows from W on (all rows, unless forced otherwise) are then cut into K
+// segments of Ls tokens (tile-aligned; the last runs to the row's end).  One launch of the
+// scan takes the whole rows and every segment (segment 0 from the row's initial state, the
+// others from zero; see SplitSpec), and k_state_out adds to every later segment the output
+// of the state entering it, chained from the segments' final states and total decays
+// (section 4.2 of "5.3 Tensor Parallelism support and large-cluster training", state
+// passing at segment granularity), and writes the row's final state.
 
 struct SplitPlan {
-    int K = 0;
-    int64_t Ls = 0;
+    int K = 0;                 // segments per split row; 0: no split
+    int64_t W = 0;             // whole rows 0 .. W - 1; rows W .. b - 1 are split
+    int64_t Ls = 0;            // tokens per segment
+    int tiles = 0;             // Ls / 128
+    int nparts = 1, tpp = 0;   // k_state_out: parts per segment and tiles per part
 };
 
-// Spans of segments first .. first + nseg - 1 of every row, on the flat (b L) token axis.
-__global__ void k_split_spans(int64_t L, int64_t Ls, int K, int first, int nseg, int64_t b, int32_t* start,
-                              int32_t* end) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < b * nseg; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / nseg, k = first + i % nseg;
-        const int64_t t0 = k * Ls, t1 = (k == K - 1 || (k + 1) * Ls > L) ? L : (k + 1) * Ls;   // the last runs to L
-        start[i] = (int32_t)(r * L + t0);
-        end[i] = (int32_t)(r * L + t1);
-    }
-}
-
-// Initial states of pass 1: the row's own for segment 0, zero for the others.
-__global__ void k_split_init(const float* __restrict__ init, float* __restrict__ I1, int64_t b, int nseg,
-                             int64_t HNP) {
-    const int64_t n = b * nseg * HNP;
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t span = e / HNP, r = span / nseg;
-        I1[e] = (span % nseg == 0 && init) ? init[r * HNP + e % HNP] : 0.f;
-    }
-}
-
-// Sum of d A over segment k = 1 .. K-2 of every row and head (natural log of its total decay).
-// One block per (row, segment, head).
-__global__ void k_split_decay(const __nv_bfloat16* __restrict__ dt, const float* __restrict__ dt_bias,
-                              const float* __restrict__ A, int64_t L, int64_t Ls, int K, int H,
-                              float* __restrict__ dsum) {
-    const int h = blockIdx.x % H;
-    const int k = 1 + (int)((blockIdx.x / H) % (K - 2));
-    const int64_t r = blockIdx.x / ((int64_t)H * (K - 2));
-    const float bias = dt_bias ? dt_bias[h] : 0.f;
-    float acc = 0.f;
-    for (int64_t t = k * Ls + threadIdx.x; t < (k + 1) * Ls && t < L; t += blockDim.x)
-        acc += softplus_f(__bfloat162float(dt[(r * L + t) * H + h]) + bias);
-    __shared__ float red[32];
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        acc = threadIdx.x < blockDim.x / 32 ? red[threadIdx.x] : 0.f;
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (threadIdx.x == 0) dsum[blockIdx.x] = acc * A[h];
-    }
-}
-
-// h_in of segments 1 .. K-1 (pass 2's initial states) from pass 1's final states F1.
-__global__ void k_split_chain(const float* __restrict__ F1, const float* __restrict__ dsum,
-                              float* __restrict__ I2, int64_t b, int K, int H, int64_t NP) {
-    const int64_t n = b * H * NP;
-    const int64_t HNP = (int64_t)H * NP;
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = e / HNP, he = e % HNP, h = he / NP;
-        float hin = F1[(r * (K - 1)) * HNP + he];
-        I2[(r * (K - 1)) * HNP + he] = hin;
-        for (int k = 2; k < K; ++k) {
-            const float dec = expf(dsum[(r * (K - 2) + (k - 1 - 1)) * H + h]);
-            hin = dec * hin + F1[(r * (K - 1) + (k - 1)) * HNP + he];
-            I2[(r * (K - 1) + (k - 1)) * HNP + he] = hin;
-        }
-    }
-}
-
-// SMs of the current device (queried once per device), and SSD_TC_SPLIT=K, read once: forces
-// K segments whenever the sequence has at least K tiles (for tests and tuning; 0 or unset: the
-// plan below).
+// SMs of the current device (queried once per device).
 int sm_count() {
     static int cache[64] = {};
     int dev = 0;
@@ -1388,47 +1742,82 @@ int sm_count() {
     }
     return cache[dev];
 }
-int forced_split() {
-    static int v = -1;
-    if (v < 0) {
+
+// SSD_TC_SPLIT="K" or "K,R", read once: split the last R rows (default: all) into K segments
+// whenever a row has at least K tiles; "1": never split (for tests and tuning); "0" or unset:
+// the plan below.
+struct ForcedSplit {
+    int K = 0, R = 0;
+};
+ForcedSplit forced_split() {
+    static ForcedSplit v;
+    static bool read = false;
+    if (!read) {
         const char* e = getenv("SSD_TC_SPLIT");
-        v = e ? atoi(e) : 0;
-        if (v < 0 || v > 64) v = 0;
+        int k = 0, r = 0;
+        if (e && sscanf(e, "%d,%d", &k, &r) >= 1 && k >= 1 && k <= 64) v = {k, r > 0 ? r : 0};
+        read = true;
     }
     return v;
 }
 
-// K and Ls for a call, or K = 0 when the split does not pay: packed input (spans per sequence,
-// not handled), at least half the SMs already busy, or fewer than 8 tiles per segment.
+// Parts per segment for k_state_out: the count whose CTAs best fill whole waves, with at
+// least four tiles per part.
+void plan_parts(SplitPlan& pl, int64_t items, int S) {
+    double best = -1.0;
+    pl.nparts = 1;
+    pl.tpp = pl.tiles;
+    for (int np = 1; np <= 32 && pl.tiles / np >= 4; ++np) {
+        const int tpp = (pl.tiles + np - 1) / np;
+        const int used = (pl.tiles + tpp - 1) / tpp;
+        const double x = (double)(items * used) / S;
+        const double eff = x / std::ceil(x);
+        if (eff > best + 0.02) {
+            best = eff;
+            pl.nparts = used;
+            pl.tpp = tpp;
+        }
+    }
+}
+
+// The plan: split only rows that leave at least half the SMs idle (b H <= S / 2), every row
+// into the most segments that still run in one wave (b H K <= S), with at least 8 tiles per
+// segment.  Measured on B200 (b1 L131072 H64): K = 2 beats the single pass by 30 % and K = 3
+// (two waves) by a further 40 %.  Filling only the last, partial wave of a long batch does
+// not pay: a CTA's tiles run faster when fewer CTAs share the GPU (about 1.8 us per tile
+// with 48 CTAs against 2.9 us with 148 on b8 L4096 H80), so the time won in the scan (~25 us)
+// goes to the state-to-output pass.
 SplitPlan plan_split(const ScanArgs& a) {
     SplitPlan pl;
-    const int64_t ctas = a.b * a.H;
-    const int64_t tiles = (a.L + kT - 1) / kT;
-    if (a.seq_idx || ctas <= 0) return pl;
+    const int64_t nt = (a.L + kT - 1) / kT;
+    if (a.seq_idx || a.b * a.H <= 0 || a.N != 128) return pl;
+    const int S = sm_count();
+    const ForcedSplit f = forced_split();
     int K;
-    if (forced_split() >= 2) {
-        K = forced_split();
-        if (tiles < K) return pl;
+    int64_t R = a.b;   // rows split (the last R)
+    if (f.K) {
+        if (f.K == 1 || nt < f.K) return pl;
+        K = f.K;
+        if (f.R && f.R < a.b) R = f.R;
     } else {
-        const int sms = sm_count();
-        if (ctas * 2 > sms) return pl;
-        K = (int)(1 + sms / ctas);
-        if (K > 8) K = 8;
-        if (K < 3 || tiles < 8 * (int64_t)K) return pl;
+        if (a.b * a.H * 2 > S) return pl;
+        K = (int)std::min<int64_t>(8, S / (a.b * a.H));
+        if (K < 2 || nt < 8 * (int64_t)K) return pl;
     }
-    const int64_t Ls = ((tiles + K - 1) / K) * kT;
-    if ((K - 1) * Ls >= a.L) return pl;
+    pl.tiles = (int)((nt + K - 1) / K);
+    pl.Ls = (int64_t)pl.tiles * kT;
+    if ((K - 1) * pl.Ls >= a.L) return SplitPlan();
     pl.K = K;
-    pl.Ls = Ls;
+    pl.W = a.b - R;
+    plan_parts(pl, R * (K - 1) * a.H, S);
     return pl;
 }
 
 size_t split_workspace_bytes(const ScanArgs& a, const SplitPlan& pl) {
     if (!pl.K) return 0;
-    const size_t states = (size_t)a.b * (pl.K - 1) * a.H * a.N * a.P * sizeof(float);
-    const size_t spans = (size_t)a.b * (pl.K - 1) * sizeof(int32_t);
-    return 3 * ((states + 255) & ~(size_t)255) + 4 * ((spans + 255) & ~(size_t)255) +
-           (((size_t)a.b * pl.K * a.H * sizeof(float) + 255) & ~(size_t)255);
+    const size_t spans = (size_t)(a.b - pl.W) * pl.K * a.H;
+    return ((spans * a.N * a.P * sizeof(float) + 255) & ~(size_t)255) +
+           ((spans * pl.tiles * kT * sizeof(float) + 255) & ~(size_t)255);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -1516,71 +1905,130 @@ int launch_tc_scan(const ScanArgs& a, const SeqInfo& si, int64_t, void* ws, int3
     p.G = (int)a.G;
     const SplitPlan pl = a.N == 128 ? plan_split(a) : SplitPlan();
     if (pl.K) {
-        const size_t smem = sizeof(v3::Smem) + 1024;
-        cudaFuncSetAttribute(v3::k_tc_scan3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        const int K = pl.K, nseg = K - 1;
-        const int64_t HNP = a.H * a.N * a.P, S2 = a.b * nseg;
-        const size_t states = ((size_t)S2 * HNP * sizeof(float) + 255) & ~(size_t)255;
-        const size_t spans = ((size_t)S2 * sizeof(int32_t) + 255) & ~(size_t)255;
+        const int64_t R = a.b - pl.W, spans = R * pl.K;
+        const size_t states = ((size_t)spans * a.H * a.N * a.P * sizeof(float) + 255) & ~(size_t)255;
         char* w = reinterpret_cast<char*>(ws) + ((2 * (size_t)ntok * a.G * a.N * sizeof(__half) + 255) & ~(size_t)255) + 256;
-        float* I1 = reinterpret_cast<float*>(w); w += states;       // pass 1 initial states, then pass 2's final
-        float* F1 = reinterpret_cast<float*>(w); w += states;       // pass 1 final states
-        float* I2 = reinterpret_cast<float*>(w); w += states;       // pass 2 initial states (the chain)
-        int32_t* st1 = reinterpret_cast<int32_t*>(w); w += spans;
-        int32_t* en1 = reinterpret_cast<int32_t*>(w); w += spans;
-        int32_t* st2 = reinterpret_cast<int32_t*>(w); w += spans;
-        int32_t* en2 = reinterpret_cast<int32_t*>(w); w += spans;
-        float* dsum = reinterpret_cast<float*>(w);
-        const unsigned gs = (unsigned)((S2 + 255) / 256);
-        const int64_t ne = S2 * HNP;
-        const unsigned ge = (unsigned)std::min<int64_t>((ne + 255) / 256, 148 * 16);
+        p.split.first = (int32_t)pl.W;
+        p.split.K = pl.K;
+        p.split.row0 = (int32_t)pl.W;
+        p.split.tiles = pl.tiles;
+        p.split.Ls = pl.Ls;
+        p.split.fin = reinterpret_cast<float*>(w);
+        p.split.cs = reinterpret_cast<float*>(w + states);
         {
-            ProfScope pt(K_TC_PREP, st);
-            k_split_spans<<<gs, 256, 0, st>>>(a.L, pl.Ls, K, 0, nseg, a.b, st1, en1);
-            k_split_spans<<<gs, 256, 0, st>>>(a.L, pl.Ls, K, 1, nseg, a.b, st2, en2);
-            k_split_init<<<ge, 256, 0, st>>>(a.init_state, I1, a.b, nseg, HNP);
-            if (K > 2)
-                k_split_decay<<<(unsigned)(a.b * (K - 2) * a.H), 256, 0, st>>>(
-                    (const __nv_bfloat16*)a.dt, a.dt_bias, a.A, a.L, pl.Ls, K, (int)a.H, dsum);
-        }
-        SeqInfo s1 = si;
-        s1.packed = 1; s1.S = (int32_t)S2; s1.L = ntok; s1.start = st1; s1.end = en1; s1.chunk_off = nullptr;
-        TcParams p1 = p;
-        p1.si = s1; p1.init_state = I1; p1.final_state = F1;
-        {
+            const size_t smem = sizeof(v3::Smem) + 1024;
+            cudaFuncSetAttribute(v3::k_tc_scan3<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             ProfScope ps(K_TC_SCAN, st);
-            v3::k_tc_scan3<<<(unsigned)(S2 * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, tm_y, p1);
+            v3::k_tc_scan3<true><<<(unsigned)((pl.W + spans) * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, tm_y, p);
         }
-        {
-            ProfScope pt(K_TC_PREP, st);
-            const unsigned gc = (unsigned)std::min<int64_t>((a.b * HNP + 255) / 256, 148 * 16);
-            k_split_chain<<<gc, 256, 0, st>>>(F1, dsum, I2, a.b, K, (int)a.H, a.N * a.P);
-        }
-        SeqInfo s2 = s1;
-        s2.start = st2; s2.end = en2;
-        TcParams p2 = p;
-        p2.si = s2; p2.init_state = I2; p2.final_state = I1;       // pass 1's initial states are spent
-        {
-            ProfScope ps(K_TC_SCAN, st);
-            v3::k_tc_scan3<<<(unsigned)(S2 * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, tm_y, p2);
-        }
-        if (a.final_state &&
-            cudaMemcpy2DAsync(a.final_state, HNP * sizeof(float), I1 + (size_t)(nseg - 1) * HNP,
-                              (size_t)nseg * HNP * sizeof(float), HNP * sizeof(float), (size_t)a.b,
-                              cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-            return 6;
+        so::SOParams q;
+        q.dt = p.dt;
+        q.dt_bias = a.dt_bias;
+        q.A = a.A;
+        q.h_in = nullptr;
+        q.fin = p.split.fin;
+        q.cs = p.split.cs;
+        q.final_state = a.final_state;
+        q.y = p.y;
+        q.y_f16 = 1;
+        q.status = status;
+        q.L = a.L;
+        q.Ls = pl.Ls;
+        q.H = (int)a.H;
+        q.G = (int)a.G;
+        q.K = pl.K;
+        q.k0 = 1;
+        q.row0 = (int)pl.W;
+        q.tiles = pl.tiles;
+        q.nparts = pl.nparts;
+        q.tpp = pl.tpp;
+        const size_t smem = sizeof(so::SmemSO) + 1024;
+        cudaFuncSetAttribute(so::k_state_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        ProfScope ps(K_STATE_OUT, st);
+        so::k_state_out<<<(unsigned)(R * (pl.K - 1) * pl.nparts * a.H), so::kThreadsSO, smem, st>>>(tm_c, tm_y, q);
         return 0;
     }
     ProfScope ps(K_TC_SCAN, st);
     if (a.N == 128) {
         const size_t smem = sizeof(v3::Smem) + 1024;
-        cudaFuncSetAttribute(v3::k_tc_scan3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        v3::k_tc_scan3<<<(unsigned)(a.S * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, tm_y, p);
+        cudaFuncSetAttribute(v3::k_tc_scan3<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        v3::k_tc_scan3<false><<<(unsigned)(a.S * a.H), v3::kThreads3, smem, st>>>(tm_x, tm_b, tm_c, tm_y, p);
     } else {
         const size_t smem = sizeof(TcSmem<256>) + 1024;
         cudaFuncSetAttribute(k_tc_scan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k_tc_scan<256><<<(unsigned)(a.S * a.H), kThreads, smem, st>>>(tm_x, tm_b, tm_c, p);
     }
+    return 0;
+}
+
+bool state_out_supported(const ScanArgs& a) {
+    return a.dtype == 1 && a.P == kP && a.N == 128 && a.b * a.L < ((int64_t)1 << 31) && get_encode() != nullptr;
+}
+
+size_t state_out_workspace_bytes(const ScanArgs& a) {
+    const int64_t nt = (a.L + kT - 1) / kT;
+    const size_t c16 = ((size_t)a.b * a.L * a.G * a.N * sizeof(__half) + 255) & ~(size_t)255;
+    const size_t tab = ((size_t)a.b * nt * a.H * sizeof(float) + 255) & ~(size_t)255;
+    const size_t tok = ((size_t)a.b * nt * kT * a.H * sizeof(float) + 255) & ~(size_t)255;
+    return c16 + 2 * tab + tok;
+}
+
+int launch_state_to_output(const ScanArgs& a, const float* h_in, void* ws, int32_t* status, cudaStream_t st) {
+    const int64_t ntok = a.b * a.L, nt = (a.L + kT - 1) / kT;
+    char* w = reinterpret_cast<char*>(ws);
+    __half* c16 = reinterpret_cast<__half*>(w);
+    w += ((size_t)ntok * a.G * a.N * sizeof(__half) + 255) & ~(size_t)255;
+    const size_t tab = ((size_t)a.b * nt * a.H * sizeof(float) + 255) & ~(size_t)255;
+    float* tsum = reinterpret_cast<float*>(w);
+    float* run = reinterpret_cast<float*>(w + tab);
+    float* cs = reinterpret_cast<float*>(w + 2 * tab);
+    {
+        const int64_t n8 = ntok * a.G * a.N / 8;
+        const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, 148 * 16);
+        ProfScope ps(K_TC_PREP, st);
+        k_to_f16<<<(unsigned)blocks, 256, 0, st>>>((const uint4*)a.C, (uint4*)c16, n8);
+    }
+    {
+        ProfScope ps(K_TILE_DECAY, st);
+        const int threads = a.H < 256 ? (int)((a.H + 31) / 32 * 32) : 256;
+        k_tile_sums<<<(unsigned)(a.b * nt), threads, 0, st>>>((const __nv_bfloat16*)a.dt, a.dt_bias, a.A, a.L,
+                                                              (int)a.H, (int)nt, tsum);
+        k_tile_running<<<(unsigned)((a.b * a.H + 127) / 128), 128, 0, st>>>(tsum, a.b * a.H, (int)a.H, (int)nt, run);
+        k_token_running<<<(unsigned)(a.b * nt), kT, 0, st>>>((const __nv_bfloat16*)a.dt, a.dt_bias, a.A, run, a.L,
+                                                            (int)a.H, (int)nt, cs);
+    }
+    CUtensorMap tm_c, tm_y;
+    if (!make_map(&tm_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c16, (uint64_t)a.N, (uint64_t)a.G, (uint64_t)ntok) ||
+        !make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, (uint64_t)a.P, (uint64_t)a.H, (uint64_t)ntok))
+        return 6;  // SSD_ERR_CUDA
+    SplitPlan pl;
+    pl.tiles = (int)nt;
+    plan_parts(pl, a.b * a.H, sm_count());
+    so::SOParams q;
+    q.dt = (const __nv_bfloat16*)a.dt;
+    q.dt_bias = a.dt_bias;
+    q.A = a.A;
+    q.h_in = h_in;
+    q.fin = nullptr;
+    q.cs = cs;
+    q.final_state = nullptr;
+    q.y = (__nv_bfloat16*)a.y;
+    q.y_f16 = 0;
+    q.status = status;
+    q.L = a.L;
+    q.Ls = a.L;
+    q.H = (int)a.H;
+    q.G = (int)a.G;
+    q.K = 1;
+    q.k0 = 0;
+    q.row0 = 0;
+    q.tiles = (int)nt;
+    q.nparts = pl.nparts;
+    q.tpp = pl.tpp;
+    const size_t smem = sizeof(so::SmemSO) + 1024;
+    cudaFuncSetAttribute(so::k_state_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ProfScope ps(K_STATE_OUT, st);
+    so::k_state_out<<<(unsigned)(a.b * pl.nparts * a.H), so::kThreadsSO, smem, st>>>(tm_c, tm_y, q);
     return 0;
 }
 

@@ -10,8 +10,10 @@ by point-to-point send / receive.  Rank r holds tokens [r Ls, (r + 1) Ls) of eve
 3. the ring: rank r >= 1 receives the state entering its slice h_in from rank r - 1, and every
    rank but the last sends h_out = exp(D_r) h_in + F_r (rank 0: h_out = F_0) to rank r + 1
    (the chain step is a library kernel too);
-4. every rank r >= 1 scans its slice again from h_in, which gives its final y; the last rank's
-   final state is the sequence's.
+4. every rank r >= 1 adds to its y the part that comes from h_in (the state-to-output term
+   exp(cs_t) C_t^T h_in, one library call), or, where that call does not take the inputs'
+   dtype and shape, scans its slice again from h_in; the last rank's h_out is the
+   sequence's final state.
 
 Only the entering states cross between ranks (b H N P float32 per boundary).  The compute
 steps go through the library (``SeqParOps``); the exchange goes through a communicator with
@@ -69,6 +71,34 @@ def state_chain(h_in, logdecay, F, *, out=None, stream=None):
     return out
 
 
+def state_to_output(dt, A, C, h_in, y, *, dt_bias=None, stream=None):
+    """Adds to y (b, L, H, P), in place, the output of the state h_in (b, H, N, P) entering each
+    row at its start: y_t += exp(sum_{i <= t} softplus(dt_i + dt_bias) A) C_t^T h_in.  bf16 dt, C
+    and y, P = 64, N = 128 (the library's tensor-core path).  Returns y."""
+    ops._need(dt, "dt", torch.bfloat16, 3)
+    dev = dt.device
+    ops._need(C, "C", torch.bfloat16, 4, dev)
+    ops._need(y, "y", torch.bfloat16, 4, dev)
+    ops._need(h_in, "h_in", torch.float32, 4, dev)
+    ops._need(A, "A", torch.float32, 1, dev)
+    ops._need(dt_bias, "dt_bias", torch.float32, 1, dev)
+    b, L, H, P = y.shape
+    G, N = C.shape[2], C.shape[3]
+    if dt.shape != (b, L, H) or C.shape[:2] != (b, L) or h_in.shape != (b, H, N, P):
+        raise ValueError("shapes of dt, C, h_in and y disagree")
+    dims = ops.SsdDims(b, L, H, P, N, G, 0, _lib.SSD_BF16)
+    with torch.cuda.device(dev):
+        rc = _lib.lib().ssd_state_to_output(ctypes.byref(dims), ops._p(dt), ops._p(dt_bias), ops._p(A),
+                                            ops._p(C), ops._p(h_in), ops._p(y), ops._stream(stream, dev))
+    _lib.check(rc)
+    return y
+
+
+def state_to_output_supported(x, B) -> bool:
+    """True when state_to_output takes inputs of this dtype and shape."""
+    return x.dtype == torch.bfloat16 and x.shape[-1] == 64 and B.shape[-1] == 128
+
+
 class SeqParOps:
     """The compute steps of one rank: the library's kernels."""
 
@@ -83,6 +113,14 @@ class SeqParOps:
 
     def empty_state(self, like_F):
         return torch.empty_like(like_F)
+
+    def add_state(self, x, dt, A, B, C, *, dt_bias, h_in, y):
+        """y += the output of h_in entering the slice; False when the library has no such call
+        for these inputs (the ring then scans the slice again from h_in)."""
+        if not state_to_output_supported(x, B):
+            return False
+        state_to_output(dt, A, C, h_in, y, dt_bias=dt_bias)
+        return True
 
 
 class TorchDistComm:
@@ -128,7 +166,7 @@ def chunk_scan_fwd_seqpar(x, dt, A, B, C, *, comm, dt_bias=None, D=None, init_st
         h_out = F
     if rank < world - 1:
         comm.send_next(h_out)
-    if rank > 0:
+    if rank > 0 and not o.add_state(x, dt, A, B, C, dt_bias=dt_bias, h_in=h_in, y=y):
         y, h_out = o.scan(x, dt, A, B, C, dt_bias=dt_bias, D=D, init_state=h_in, chunk=chunk, y=y)
     return y, h_out
 

@@ -8,8 +8,9 @@ and exchange real tensors:
      giving its local final state F_r, and sums its slice's log-decay D_r;
   2. a ring: rank r >= 1 receives the state entering its slice from rank r - 1, and every rank
      but the last sends h_out = exp(D_r) h_in + F_r (rank 0: h_out = F_0) to rank r + 1;
-  3. every rank r >= 1 rescans its slice from h_in (the rerun form pinned in
-     tests/test_tile_model.py), and the last rank's final state is the sequence's.
+  3. every rank r >= 1 adds to its y the output of h_in entering its slice (here the oracle scan
+     of a zero input from h_in, which by linearity is that term), and the last rank's h_out is
+     the sequence's final state.
 The ranks run the library's own ring code (state_space_model_07_b200.seqpar: its send / receive
 order over torch.distributed and its use of the scan, decay and chain steps) with those steps
 supplied in fp64 on the CPU (the scan by the oracle), so the stitched y and final state must
@@ -62,6 +63,13 @@ def _oracle_ops():
 
         def chain(self, h_in, logdecay, F):
             return torch.exp(logdecay)[:, :, None, None] * h_in + F
+
+        def add_state(self, x, dt, A, B, C, *, dt_bias, h_in, y):
+            # the output of h_in alone: the scan of a zero input entered by h_in (D x = 0)
+            yy, _ = oracle.ssd_scan(np.zeros_like(x.numpy()), dt.numpy(), A.numpy(), B.numpy(), C.numpy(),
+                                    dt_bias=dt_bias.numpy(), D=None, init_state=h_in.numpy(), nthreads=1)
+            y.add_(torch.from_numpy(yy))
+            return True
 
     return OracleOps()
 

@@ -4,6 +4,7 @@
 over devices, the state handed from each device to the next.  Checked here:
 * ssd_segment_logdecay against the fp64 sum of softplus(dt + dt_bias) A written out in numpy;
 * ssd_state_chain against exp(D) h_in + F in fp64;
+* ssd_state_to_output: a scan from zero plus the output of h_in equals the oracle's scan from h_in;
 * chunk_scan_fwd_seqpar with 1 to 4 ranks emulated in order on one GPU (LocalRing), slices
   tile-aligned or ragged, batch 2, with an initial state: the stitched y and the last rank's
   final state equal one oracle scan of the whole sequence within 1e-2 (1 + |ref|).
@@ -12,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import state_space_model_07_b200 as ssd
 from state_space_model_07_b200 import inputs, seqpar
 from tests.helpers import TOL, assert_close, oracle_scan, to_cpu
 
@@ -67,3 +69,18 @@ def test_ring_over_ranks_reproduces_the_whole_scan(world, bounds):
     tol = TOL[torch.bfloat16]
     assert_close(y, yr, tol, "stitched y")
     assert_close(res[-1][1], fr, tol, "final state")
+
+
+@pytest.mark.parametrize("b,L,H,G", [(2, 1000, 8, 2), (1, 129, 4, 1), (3, 300, 8, 8), (1, 5000, 16, 2)])
+def test_state_to_output_adds_the_entering_state(b, L, H, G):
+    """A scan from a zero state plus ssd_state_to_output(h_in) equals the scan from h_in (the
+    oracle's); rows whose length is not a multiple of 128 exercise the partial last tile."""
+    w = inputs.scaled(inputs.WORKLOADS["long_context"], batch=b, seqlen=L, nheads=H, ngroups=G)
+    d = inputs.make_inputs(w, "cuda")
+    y, _ = ssd.chunk_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_bias=d["dt_bias"], D=d["D"],
+                              chunk=w.chunk)
+    out = seqpar.state_to_output(d["dt"], d["A"], d["C"], d["init_state"], y, dt_bias=d["dt_bias"])
+    torch.cuda.synchronize()
+    assert out is y
+    yr, _ = oracle_scan(to_cpu(d))
+    assert_close(y, yr, TOL[torch.bfloat16], "y")
