@@ -52,6 +52,11 @@ def parse():
     ap.add_argument("--seqpar", action="store_true",
                     help="split each sequence of the workload over the ranks (state passed along a ring); "
                          "default: every rank runs its own replica")
+    ap.add_argument("--mixer", default=None, metavar="CONFIG",
+                    help="time the head-sharded mixer layer (tensor parallel over the ranks, quantised "
+                         "all-reduce) on this configuration, e.g. mixer_2.7b, instead of the scan")
+    ap.add_argument("--exact-allreduce", action="store_true",
+                    help="with --mixer: an fp32 all-reduce instead of the quantised one")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (small cases for profiling; not a bench line)")
     return ap.parse_args()
@@ -503,8 +508,8 @@ def run_ours(args):
 def run_seqpar(args):
     """One scan of the workload split along the sequence over the ranks: rank r holds tokens
     [r L/N, (r + 1) L/N) of every batch row, scans them, receives the state entering its slice
-    from rank r - 1 (NCCL point-to-point), passes the state leaving it on and rescans from the
-    state it received (state_space_model_07_b200.seqpar).  Total work is fixed as N grows."""
+    from rank r - 1 (NCCL point-to-point), passes the state leaving it on and adds the output of
+    the state it received (state_space_model_07_b200.seqpar).  Total work is fixed as N grows."""
     import torch
     import torch.distributed as dist
     from state_space_model_07_b200 import _lib, inputs, seqpar
@@ -556,7 +561,7 @@ def run_seqpar(args):
     value = tokens * args.steps / (ms * 1e-3)
     pk, pk_src = peaks()
     nl, nt, tot = stats.get("tc_scan", stats.get("simt_chunk_out", (0, 0, 0.0)))
-    per_step = max(1, round(nl / args.steps))      # ranks >= 1 scan their slice twice; long slices split
+    per_step = max(1, round(nl / args.steps))
     step_ms = tot / max(nt, 1) * per_step
     alg = workload_bytes(inputs.scaled(w, seqlen=hi - lo), b, b * (hi - lo), part["x"].element_size())
     roof = {"kernel": "tc_scan", "bound": "hbm", "achieved": alg / (step_ms * 1e-3) / 1e9 if step_ms else None,
@@ -571,7 +576,8 @@ def run_seqpar(args):
         return 0
     cfg = config_of(w)
     cfg.update(parallelism=f"seqpar{world}", step="one ssd_chunk_scan_fwd of the workload split along the "
-               "sequence over the ranks: local scan, state ring (NCCL send / recv), rescan on ranks >= 1",
+               "sequence over the ranks: local scan, state ring (NCCL send / recv), the entering state's "
+               "output added on ranks >= 1",
                tokens_per_rank=hi - lo)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
@@ -585,12 +591,98 @@ def run_seqpar(args):
     return 0
 
 
+def run_mixer(args):
+    """The head-sharded mixer layer ("5.3 Tensor Parallelism support and large-cluster training",
+    section 4.1) on the ranks: each holds H / N heads, computes its projections (cuBLAS), scan and
+    group norm (library kernels) and its partial output projection, and the partials are summed by
+    the quantised all-reduce (library quantisation kernels; all-to-all and all-gather over NCCL).
+    Every rank holds the whole input; total work is fixed as N grows."""
+    import torch
+    import torch.distributed as dist
+    from state_space_model_07_b200 import _lib, inputs, tp
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    cfg = inputs.MIXERS[args.mixer]
+    if args.batch:
+        cfg = inputs.dataclasses.replace(cfg, batch=args.batch)
+    u, w = inputs.make_mixer(cfg, dev)
+    sh = tp.shard(w, rank, world)
+    del w
+    comm = tp.TorchDistTPComm() if world > 1 else tp.SingleRankComm()
+    quantized = not args.exact_allreduce
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return tp.mixer_fwd(u, sh, comm, ngroups=cfg.ngroups, dstate=cfg.dstate, headdim=cfg.headdim,
+                            chunk=cfg.chunk, quantized=quantized)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        for _ in range(args.warmup):
+            step()
+        barrier()
+        _lib.profile_read(reset=True)
+        _lib.profile_enable(True)
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        barrier()
+    _lib.profile_enable(False)
+    stats = _lib.profile_read(reset=True)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    T = cfg.batch * cfg.seqlen
+    value = T * args.steps / (ms * 1e-3)
+    launches = sum(v[0] for v in stats.values())
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    Hr = cfg.nheads // world
+    gemm_flops = 2 * T * cfg.d_model * (Hr * cfg.headdim * 2 + 2 * cfg.ngroups // world * cfg.dstate + Hr)
+    code_bytes = 2 * (world - 1) / world * T * cfg.d_model * (1 + 4 / 64)
+    pk, pk_src = peaks()
+    line = {"metric": "head-sharded SSD mixer layer tokens/s (tensor parallel over the GPUs)", "value": value,
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen, "d_model": cfg.d_model,
+                       "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
+                       "ngroups": cfg.ngroups, "chunk": cfg.chunk, "parallelism": f"tp{world}",
+                       "allreduce": "int8 codes, one fp32 scale per 64 columns" if quantized else "fp32",
+                       "step": "input projections (cuBLAS), scan and group norm of the rank's heads, partial "
+                               "output projection, all-reduce of the partials"},
+            "per_rank": {"heads": Hr, "gemm_flops": gemm_flops,
+                         "allreduce_bytes_sent": code_bytes if quantized else 2 * (world - 1) / world * T *
+                         cfg.d_model * 4},
+            "roofline": None, "cpu_baseline": None, "e2e": None,
+            "note": "the layer around the scan: GEMMs by cuBLAS; the scan's own roofline is the scan line's",
+            "gpu_launches": launches, "kernels": {k: {"launches": v[0], "avg_ms": v[2] / max(v[1], 1)}
+                                                  for k, v in stats.items()},
+            "peaks": {"source": pk_src}, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.seqpar:
         return run_seqpar(args)
+    if args.mixer:
+        return run_mixer(args)
     return run_ours(args)
 
 

@@ -189,6 +189,44 @@ SSD_API int ssd_state_to_output(const ssd_dims* dims, const void* dt, const floa
                                 const void* C, const float* h_in, void* y, void* stream);
 
 /*
+ * Head-sharded (tensor-parallel) mixer ("5.3 Tensor Parallelism ...", section 4.1;
+ * "Scaling State-Space Models on Multiple GPUs with Tensor Parallelism", abstract):
+ * each of `ranks` devices holds H / ranks heads; the layer's output is the sum of
+ * the devices' partial output projections, formed by a quantised all-reduce.
+ *
+ * ssd_group_norm -- out[r, c] = (x[r, c] - mean_g) / sqrt(var_g + eps) * gamma[c]
+ *   + beta[c], mean_g and var_g (biased) over the channels of c's group in row r
+ *   (ngroups groups of channels / ngroups consecutive channels, at most 2048).
+ *   x, out (rows, channels) of dtype (SSD_F32 or SSD_BF16; out may be x);
+ *   gamma, beta (channels) float32.  Statistics in fp32.
+ *
+ * The quantised all-reduce of (T, D) float32 partials over `ranks` devices, with
+ * int8 codes and one float32 scale per block of 64 consecutive columns of a row
+ * (scale = amax / 127 in fp32; code = rint(x * (127 / amax)) with round-half-even,
+ * in [-127, 127]; 0 for an all-zero block).  Column chunk j = columns
+ * [j D / ranks, (j + 1) D / ranks), Dc = D / ranks a multiple of 64:
+ * ssd_quant_chunks -- x (T, D) float32 -> q (ranks, T, Dc) int8,
+ *   scale (ranks, T, Dc / 64): chunk-major, so chunk j is contiguous (it goes to
+ *   rank j in an all-to-all).
+ * ssd_dequant_sum_quant -- the chunks from every rank, q_in (ranks, T, Dc) and
+ *   scale_in (ranks, T, Dc / 64) -> their dequantised sum in float32 (added in
+ *   rank order, each product and sum rounded separately) -> q_out (T, Dc),
+ *   scale_out (T, Dc / 64).
+ * ssd_dequant_chunks -- gathered chunks q (ranks, T, Dc), scale -> out (T, D) of
+ *   dtype, out[t, j Dc + c] = scale * code (rounded once to dtype).
+ * Every buffer 16-byte aligned; sizes and alignment checked on the host
+ * (SSD_ERR_SHAPE).
+ */
+SSD_API int ssd_group_norm(int64_t rows, int64_t channels, int64_t ngroups, int dtype, const void* x,
+                           const float* gamma, const float* beta, float eps, void* out, void* stream);
+SSD_API int ssd_quant_chunks(int64_t T, int64_t D, int64_t ranks, const float* x, int8_t* q, float* scale,
+                             void* stream);
+SSD_API int ssd_dequant_sum_quant(int64_t T, int64_t Dc, int64_t ranks, const int8_t* q_in, const float* scale_in,
+                                  int8_t* q_out, float* scale_out, void* stream);
+SSD_API int ssd_dequant_chunks(int64_t T, int64_t D, int64_t ranks, int dtype, const int8_t* q, const float* scale,
+                               void* out, void* stream);
+
+/*
  * ssd_chunk_scan_bwd -- gradient of the scan (the backward of the training step
  * the pages describe: "5.3 Tensor Parallelism support and large-cluster
  * training", section 6.3 and Table 5.3.1; the pages print no gradient

@@ -17,7 +17,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE"
 # Every function include/ssd.h declares.
 EXPORTS = ("ssd_chunk_scan_fwd", "ssd_state_update", "ssd_status_string", "ssd_last_error",
            "ssd_profile_enable", "ssd_profile_read", "ssd_chunk_scan_fwd_noalloc", "ssd_selftest_bounded_wait",
-           "ssd_chunk_scan_bwd", "ssd_segment_logdecay", "ssd_state_chain", "ssd_state_to_output")
+           "ssd_chunk_scan_bwd", "ssd_segment_logdecay", "ssd_state_chain", "ssd_state_to_output",
+           "ssd_group_norm", "ssd_quant_chunks", "ssd_dequant_sum_quant", "ssd_dequant_chunks")
 
 
 class SsdDims(ctypes.Structure):
@@ -63,6 +64,15 @@ def lib():
         L.ssd_state_chain.argtypes = [dims] + [_VP] * 5
         L.ssd_state_to_output.restype = ctypes.c_int
         L.ssd_state_to_output.argtypes = [dims] + [_VP] * 7
+        i64 = ctypes.c_int64
+        L.ssd_group_norm.restype = ctypes.c_int
+        L.ssd_group_norm.argtypes = [i64, i64, i64, ctypes.c_int, _VP, _VP, _VP, ctypes.c_float, _VP, _VP]
+        L.ssd_quant_chunks.restype = ctypes.c_int
+        L.ssd_quant_chunks.argtypes = [i64, i64, i64, _VP, _VP, _VP, _VP]
+        L.ssd_dequant_sum_quant.restype = ctypes.c_int
+        L.ssd_dequant_sum_quant.argtypes = [i64, i64, i64, _VP, _VP, _VP, _VP, _VP]
+        L.ssd_dequant_chunks.restype = ctypes.c_int
+        L.ssd_dequant_chunks.argtypes = [i64, i64, i64, ctypes.c_int, _VP, _VP, _VP, _VP]
         L.ssd_state_update.restype = ctypes.c_int
         L.ssd_state_update.argtypes = [dims] + [_VP] * 10
         L.ssd_status_string.restype = ctypes.c_char_p

@@ -397,6 +397,83 @@ extern "C" int ssd_state_chain(const ssd_dims* dims, const float* h_in, const fl
 
 // ---- Backward of the scan -------------------------------------------------------------
 
+extern "C" int ssd_group_norm(int64_t rows, int64_t channels, int64_t ngroups, int dtype, const void* x,
+                              const float* gamma, const float* beta, float eps, void* out, void* stream) {
+    g_last_error[0] = 0;
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return fail(SSD_ERR_DTYPE, "dtype %d is not SSD_F32 or SSD_BF16", dtype);
+    if (rows < 0 || channels < 1) return fail(SSD_ERR_SHAPE, "rows must be >= 0 and channels >= 1");
+    if (!ssd::group_norm_supported(channels, ngroups))
+        return fail(SSD_ERR_SHAPE, "ngroups must divide channels, with at most 2048 channels per group");
+    if (rows == 0) return SSD_OK;
+    if (!x || !gamma || !beta || !out) return fail(SSD_ERR_NULL, "x, gamma, beta and out are required");
+    if (!(eps >= 0.f)) return fail(SSD_ERR_SHAPE, "eps must be >= 0");
+    if (rows * ngroups > 0x7fffffffLL / 32) return fail(SSD_ERR_SHAPE, "rows * ngroups too large");
+    const size_t es = dtype == SSD_BF16 ? 2 : 4, n = (size_t)rows * channels * es;
+    if (overlaps(out, n, x, n) && out != x) return fail(SSD_ERR_SHAPE, "out overlaps x without being x");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    ssd::launch_group_norm(dtype, x, gamma, beta, eps, rows, channels, ngroups, out, st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("kernel launch", e);
+    return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
+}
+
+namespace {
+int quant_shape(int64_t T, int64_t D, int64_t Tp) {
+    if (T < 0 || D < 1 || Tp < 1 || Tp > 64) return fail(SSD_ERR_SHAPE, "need T >= 0, D >= 1, 1 <= ranks <= 64");
+    if (D % (64 * Tp)) return fail(SSD_ERR_SHAPE, "D (%lld) must be a multiple of 64 * ranks", (long long)D);
+    if (T * (D / 64) > 0x7fffffffLL / 32) return fail(SSD_ERR_SHAPE, "T * D too large");
+    return SSD_OK;
+}
+int launched(cudaStream_t st) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("kernel launch", e);
+    return debug_check() ? debug_sync(st, nullptr) : SSD_OK;
+}
+}  // namespace
+
+extern "C" int ssd_quant_chunks(int64_t T, int64_t D, int64_t ranks, const float* x, int8_t* q, float* scale,
+                                void* stream) {
+    g_last_error[0] = 0;
+    int rc = quant_shape(T, D, ranks);
+    if (rc || T == 0) return rc;
+    if (!x || !q || !scale) return fail(SSD_ERR_NULL, "x, q and scale are required");
+    if (!aligned16(x) || !aligned16(q) || !aligned16(scale)) return fail(SSD_ERR_SHAPE, "x, q and scale must be 16-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    ssd::launch_quant_chunks(x, T, D, ranks, q, scale, st);
+    return launched(st);
+}
+
+extern "C" int ssd_dequant_sum_quant(int64_t T, int64_t Dc, int64_t ranks, const int8_t* q_in, const float* scale_in,
+                                     int8_t* q_out, float* scale_out, void* stream) {
+    g_last_error[0] = 0;
+    int rc = quant_shape(T, Dc, 1);
+    if (rc || T == 0) return rc;
+    if (ranks < 1 || ranks > 64) return fail(SSD_ERR_SHAPE, "1 <= ranks <= 64");
+    if (!q_in || !scale_in || !q_out || !scale_out) return fail(SSD_ERR_NULL, "all buffers are required");
+    if (!aligned16(q_in) || !aligned16(q_out) || !aligned16(scale_in) || !aligned16(scale_out))
+        return fail(SSD_ERR_SHAPE, "codes and scales must be 16-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    ssd::launch_dequant_sum_quant(q_in, scale_in, ranks, T, Dc, q_out, scale_out, st);
+    return launched(st);
+}
+
+extern "C" int ssd_dequant_chunks(int64_t T, int64_t D, int64_t ranks, int dtype, const int8_t* q, const float* scale,
+                                  void* out, void* stream) {
+    g_last_error[0] = 0;
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return fail(SSD_ERR_DTYPE, "dtype %d is not SSD_F32 or SSD_BF16", dtype);
+    int rc = quant_shape(T, D, ranks);
+    if (rc || T == 0) return rc;
+    if (!q || !scale || !out) return fail(SSD_ERR_NULL, "q, scale and out are required");
+    if (!aligned16(q) || !aligned16(scale) || !aligned16(out)) return fail(SSD_ERR_SHAPE, "q, scale and out must be 16-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    ssd::launch_dequant_chunks(dtype, q, scale, ranks, T, D / ranks, out, st);
+    return launched(st);
+}
+
 extern "C" int ssd_state_to_output(const ssd_dims* dims, const void* dt, const float* dt_bias, const float* A,
                                    const void* C, const float* h_in, void* y, void* stream) {
     g_last_error[0] = 0;

@@ -65,6 +65,17 @@ void launch_segment_logdecay(int64_t b, int64_t L, int64_t H, int dtype, const v
 void launch_state_chain(int64_t bh, int64_t NP, const float* h_in, const float* logdecay, const float* F,
                         float* h_out, cudaStream_t st);
 
+// Head-sharded mixer (ssd_tp.cu): group norm of (rows, C) with C / ngroups channels per group,
+// and the steps of the quantised all-reduce (int8 codes, one fp32 scale per 64 columns).
+bool group_norm_supported(int64_t C, int64_t ngroups);
+void launch_group_norm(int dtype, const void* x, const float* gamma, const float* beta, float eps, int64_t rows,
+                       int64_t C, int64_t ngroups, void* out, cudaStream_t st);
+void launch_quant_chunks(const float* x, int64_t T, int64_t D, int64_t Tp, int8_t* q, float* scale, cudaStream_t st);
+void launch_dequant_sum_quant(const int8_t* qin, const float* sin, int64_t Tp, int64_t T, int64_t Dc, int8_t* qout,
+                              float* sout, cudaStream_t st);
+void launch_dequant_chunks(int dtype, const int8_t* q, const float* s, int64_t Tp, int64_t T, int64_t Dc, void* out,
+                           cudaStream_t st);
+
 // Debug-mode value checks around a tensor-core scan (ssd_check.cu): counters[0]
 // += non-finite inputs, counters[1] += finite x / B / C / init_state values
 // beyond the fp16 range, counters[2] += non-finite outputs.

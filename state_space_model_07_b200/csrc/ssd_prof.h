@@ -21,6 +21,8 @@ enum KernelId : int {
     K_STATE_CHAIN,
     K_STATE_OUT,
     K_TILE_DECAY,
+    K_GROUP_NORM,
+    K_QUANT,
     K_COUNT
 };
 

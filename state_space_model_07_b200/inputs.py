@@ -144,3 +144,58 @@ def make_decode_inputs(w: Workload, step: int, batch: int, device="cpu"):
         "B": _bf16_or_f32(B, dt_).to(device),
         "C": _bf16_or_f32(C, dt_).to(device),
     }
+
+
+# ---- Head-sharded mixer (tensor parallelism): synthetic layer weights and input -------------
+#
+# Shapes of a Mamba-2-2.7B-like layer with the SSM groups raised to 8 so that they divide among
+# up to 8 devices: d_model 2560, 80 heads of 64, d_state 128.  Recipe (one default_rng(seed)
+# stream, float32 draws, bf16 RNE for the matrices and the input):
+#   u              ~ N(0, 1)                              (b, L, d_model)
+#   W_x, W_B, W_C  ~ N(0, 1 / d_model)                    (d_model, H P), (d_model, G N) x 2
+#   W_dt           ~ N(0, 1 / d_model)                    (d_model, H)
+#   dt_bias, A, D  as for the scan (per head, float32)
+#   gamma ~ 1 + N(0, 0.1^2), beta ~ N(0, 0.1^2)           (H P) float32
+#   W_out          ~ N(0, 1 / (H P))                      (H P, d_model)
+
+@dataclasses.dataclass(frozen=True)
+class MixerConfig:
+    name: str
+    batch: int
+    seqlen: int
+    d_model: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int          # SSM groups (B, C) and also the group-norm groups
+    chunk: int
+    seed: int
+
+
+MIXERS = {
+    "mixer_2.7b": MixerConfig("mixer_2.7b", 8, 4096, 2560, 80, 64, 128, 8, 256, 5),
+    "mixer_small": MixerConfig("mixer_small", 2, 300, 256, 8, 64, 128, 4, 128, 6),
+}
+
+
+def make_mixer(cfg: MixerConfig, device="cpu"):
+    """Returns (u, weights dict) for one layer; matrices and u in bf16, vectors float32."""
+    rng = np.random.default_rng(cfg.seed)
+    Dm, H, P, N, G = cfg.d_model, cfg.nheads, cfg.headdim, cfg.dstate, cfg.ngroups
+    bf = lambda a: torch.from_numpy(a).to(torch.bfloat16).to(device)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    u = rng.standard_normal((cfg.batch, cfg.seqlen, Dm), dtype=np.float32)
+    sd = np.float32(1.0 / math.sqrt(Dm))
+    w = {
+        "W_x": bf(rng.standard_normal((Dm, H * P), dtype=np.float32) * sd),
+        "W_B": bf(rng.standard_normal((Dm, G * N), dtype=np.float32) * sd),
+        "W_C": bf(rng.standard_normal((Dm, G * N), dtype=np.float32) * sd),
+        "W_dt": bf(rng.standard_normal((Dm, H), dtype=np.float32) * sd),
+        "dt_bias": f32(rng.uniform(math.log(1e-3), math.log(1e-1), H)),
+        "A": f32(-np.exp(rng.uniform(0.0, math.log(16.0), H))),
+        "D": f32(rng.standard_normal(H, dtype=np.float32)),
+        "gamma": f32(1.0 + 0.1 * rng.standard_normal(H * P, dtype=np.float32)),
+        "beta": f32(0.1 * rng.standard_normal(H * P, dtype=np.float32)),
+        "W_out": bf(rng.standard_normal((H * P, Dm), dtype=np.float32) * np.float32(1.0 / math.sqrt(H * P))),
+    }
+    return bf(u), w
