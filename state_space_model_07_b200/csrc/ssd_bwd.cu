@@ -26,6 +26,7 @@
 // it recomputes the block's per-token states into a per-(sequence, head)
 // scratch area and then runs the adjoint sweep over the block's tokens, last
 // to first.  Every quantity is fp32; inputs are read in their own dtype.
+#include <cuda_fp16.h>
 #include <stdio.h>
 
 #include "ssd_common.cuh"
@@ -252,6 +253,636 @@ k_scan_bwd(const BwdParams p) {
     }
 }
 
+// ---- Chunked backward (P = 64, N = 64 or 128) ---------------------------------------------
+//
+// The same gradients in the block-decomposed form of section 3.2, a chunk of Qb = 64 tokens at a
+// time.  Inside a chunk, with a_i = d_i A (natural log-decay), chunk-local cs_j = sum_{k<=j} a_k,
+// e_j = exp(cs_j), E = exp(cs_last), u_i = exp(cs_last - cs_i) d_i, the forward is
+//   y_j   = sum_{i<=j} (C_j . B_i) exp(cs_j - cs_i) d_i x_i + e_j C_j^T h_prev + D x_j,
+//   h_end = E h_prev + sum_i u_i B_i x_i^T,
+// and with dh_end the adjoint of the state leaving the chunk:
+//   dh_prev = E dh_end + sum_j e_j C_j dy_j^T                       (reverse state passing)
+//   dx = D dy + W^T dy + u o (B dh_end),      W[j,i] = (C_j.B_i) L[j,i] d_i
+//   dB = K^T C + u o (x dh_end^T),            K[j,i] = L[j,i] (dy_j.x_i) d_i
+//   dC = K B + e o (dy h_prev^T)
+// with L[j,i] = exp(cs_j - cs_i) for i <= j, else 0; and for the decays, with
+// R[j,i] = (C_j.B_i)(dy_j.x_i) L[j,i], Z_i = B_i^T dh_end x_i, Y_j = C_j^T h_prev dy_j:
+//   dJ/dd_i (direct) = sum_j R[j,i] + exp(cs_last - cs_i) Z_i
+//   dJ/dcs_k = sum_i R[k,i] d_i - sum_j R[j,k] d_k + e_k Y_k - u_k Z_k
+//              (+ E <dh_end, h_prev> + sum_i u_i Z_i at k = last)
+//   dJ/da_m = sum_{k>=m} dJ/dcs_k,  dd = direct + A dJ/da,  dA += d dJ/da,  dz = dd sigmoid(z).
+// Three kernels: k_bwd_terms (per chunk and head: the chunk's own state term S = sum_i u_i B_i
+// x_i^T and adjoint term T = sum_j e_j C_j dy_j^T, and E), k_bwd_pass (per state element: the
+// state entering every chunk, forwards, and the adjoint leaving every chunk, backwards), and
+// k_bwd_grads (per chunk and group: every gradient of the chunk's tokens; C B^T is shared by the
+// group's heads, and dB, dC are summed over them in registers, so no atomics touch them).
+
+constexpr int kQb = 64;   // tokens per chunk of the chunked backward
+constexpr int kPb = 64;   // headdim of the chunked backward
+
+bool bwd_chunked(const ScanArgs& a) { return a.P == kPb && (a.N == 64 || a.N == 128); }
+
+// Chunk-local decay quantities of tokens 2 lane, 2 lane + 1 of a chunk (one warp): d, z, cs and
+// the chunk's last cs; tokens past q get d = 0.
+template <typename T>
+__device__ __forceinline__ void chunk_decay(const T* dt, int64_t tok0, int H, int h, int q, float bias, float Ah,
+                                            float* sd, float* sz, float* scs, float* slast) {
+    const int lane = threadIdx.x & 31;
+    float dd[2], zz[2], cc[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int j = 2 * lane + k;
+        zz[k] = j < q ? to_f<T>(dt[(tok0 + j) * H + h]) + bias : 0.f;
+        dd[k] = j < q ? softplus_f(zz[k]) : 0.f;
+    }
+    cc[0] = dd[0] * Ah;
+    cc[1] = cc[0] + dd[1] * Ah;
+    float incl = cc[1];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    const float excl = incl - cc[1];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        sd[2 * lane + k] = dd[k];
+        sz[2 * lane + k] = zz[k];
+        scs[2 * lane + k] = excl + cc[k];
+    }
+    if (lane == 31) *slast = incl;   // tokens past q add 0, so this is cs of token q - 1
+}
+
+// acc[i][j] += sum_k A(r0 + i, k) Bm(k, c0 + j), A(r, k) = A[r ar + k ak], Bm(k, c) = Bm[k bk + c bc],
+// four k at a time with 16-byte shared-memory reads: AI (ar == 1) reads A along i, else along k
+// (ak == 1); BJ (bc == 1) reads Bm along j, else along k (bk == 1).  r0, c0, TM, TN, K, the
+// non-unit strides and every row start are multiples of 4 floats.
+template <int TM, int TN, bool AI, bool BJ>
+__device__ __forceinline__ void mm_acc(float (&acc)[TM][TN], const float* A, int ar, int ak, const float* Bm, int bk,
+                                       int bc, int r0, int c0, int K) {
+#pragma unroll 1
+    for (int k = 0; k < K; k += 4) {
+        float av[4][TM], bv[4][TN];
+        if (AI) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int i = 0; i < TM; i += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(A + r0 + i + (k + kk) * ak);
+                    av[kk][i] = v.x; av[kk][i + 1] = v.y; av[kk][i + 2] = v.z; av[kk][i + 3] = v.w;
+                }
+        } else {
+#pragma unroll
+            for (int i = 0; i < TM; ++i) {
+                const float4 v = *reinterpret_cast<const float4*>(A + (r0 + i) * ar + k);
+                av[0][i] = v.x; av[1][i] = v.y; av[2][i] = v.z; av[3][i] = v.w;
+            }
+        }
+        if (BJ) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int j = 0; j < TN; j += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(Bm + (k + kk) * bk + c0 + j);
+                    bv[kk][j] = v.x; bv[kk][j + 1] = v.y; bv[kk][j + 2] = v.z; bv[kk][j + 3] = v.w;
+                }
+        } else {
+#pragma unroll
+            for (int j = 0; j < TN; ++j) {
+                const float4 v = *reinterpret_cast<const float4*>(Bm + (c0 + j) * bc + k);
+                bv[0][j] = v.x; bv[1][j] = v.y; bv[2][j] = v.z; bv[3][j] = v.w;
+            }
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[kk][i], bv[kk][j], acc[i][j]);
+    }
+}
+
+// Warp products on the tensor cores: mma.sync m16n8k16, fp16 operands (rounded from the fp32
+// shared-memory values), fp32 accumulators.  A warp computes an (16 MT) x (8 NT) tile at rows
+// r0.., columns c0.. of sum_k A(r, k) Bm(k, c), A(r, k) = A[r ar + k ak], Bm(k, c) = Bm[k bk + c bc];
+// AK1 / BK1: ak == 1 / bk == 1 (the fragment's pairs of consecutive k are adjacent: one 8-byte
+// read).  Fragment layout (PTX ISA, m16n8k16 with .row A and .col B), g = lane / 4, t = lane % 4:
+// A regs {(g, 2t..2t+1), (g+8, 2t..), (g, 2t+8..), (g+8, 2t+8..)}; B regs {(2t..2t+1, g),
+// (2t+8..2t+9, g)}; accumulator {(g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1)}.
+__device__ __forceinline__ uint32_t h2pack(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <bool K1>
+__device__ __forceinline__ uint32_t pair_k(const float* M, int64_t at, int kstride) {
+    if (K1) {
+        const float2 v = *reinterpret_cast<const float2*>(M + at);
+        return h2pack(v.x, v.y);
+    }
+    return h2pack(M[at], M[at + kstride]);
+}
+
+template <int MT, int NT, bool AK1, bool BK1>
+__device__ __forceinline__ void mma_tile(float (&acc)[MT][NT][4], const float* A, int ar, int ak, const float* Bm,
+                                         int bk, int bc, int r0, int c0, int K) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll 1
+    for (int k = 0; k < K; k += 16) {
+        uint32_t af[MT][4], bf[NT][2];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int ra = r0 + 16 * mt + g;
+            af[mt][0] = pair_k<AK1>(A, (int64_t)ra * ar + (k + 2 * t) * ak, ak);
+            af[mt][1] = pair_k<AK1>(A, (int64_t)(ra + 8) * ar + (k + 2 * t) * ak, ak);
+            af[mt][2] = pair_k<AK1>(A, (int64_t)ra * ar + (k + 2 * t + 8) * ak, ak);
+            af[mt][3] = pair_k<AK1>(A, (int64_t)(ra + 8) * ar + (k + 2 * t + 8) * ak, ak);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int n = c0 + 8 * nt + g;
+            bf[nt][0] = pair_k<BK1>(Bm, (int64_t)(k + 2 * t) * bk + n * bc, bk);
+            bf[nt][1] = pair_k<BK1>(Bm, (int64_t)(k + 2 * t + 8) * bk + n * bc, bk);
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                asm volatile(
+                    "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                    "{%8, %9}, {%0, %1, %2, %3};"
+                    : "+f"(acc[mt][nt][0]), "+f"(acc[mt][nt][1]), "+f"(acc[mt][nt][2]), "+f"(acc[mt][nt][3])
+                    : "r"(af[mt][0]), "r"(af[mt][1]), "r"(af[mt][2]), "r"(af[mt][3]), "r"(bf[nt][0]),
+                      "r"(bf[nt][1]));
+    }
+}
+
+// The same tile in fp32 on the CUDA cores, each thread computing the elements an m16n8k16
+// accumulator would hold (fp32 inputs: their accuracy bound leaves no room for fp16 operands).
+template <int MT, int NT>
+__device__ __forceinline__ void fma_tile(float (&acc)[MT][NT][4], const float* A, int ar, int ak, const float* Bm,
+                                         int bk, int bc, int r0, int c0, int K) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll 2
+    for (int k = 0; k < K; ++k) {
+        float av[MT][2], bv[NT][2];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            av[mt][0] = A[(int64_t)(r0 + 16 * mt + g) * ar + k * ak];
+            av[mt][1] = A[(int64_t)(r0 + 16 * mt + g + 8) * ar + k * ak];
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            bv[nt][0] = Bm[(int64_t)k * bk + (c0 + 8 * nt + 2 * t) * bc];
+            bv[nt][1] = Bm[(int64_t)k * bk + (c0 + 8 * nt + 2 * t + 1) * bc];
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[mt][nt][e] = fmaf(av[mt][e >> 1], bv[nt][e & 1], acc[mt][nt][e]);
+    }
+}
+
+// Tensor cores for bf16 inputs, fp32 CUDA cores for fp32 inputs.
+template <typename T, int MT, int NT, bool AK1, bool BK1>
+__device__ __forceinline__ void prod(float (&acc)[MT][NT][4], const float* A, int ar, int ak, const float* Bm, int bk,
+                                     int bc, int r0, int c0, int K) {
+    if constexpr (sizeof(T) == 2)
+        mma_tile<MT, NT, AK1, BK1>(acc, A, ar, ak, Bm, bk, bc, r0, c0, K);
+    else
+        fma_tile<MT, NT>(acc, A, ar, ak, Bm, bk, bc, r0, c0, K);
+}
+
+// Row and column of accumulator element e of tile (mt, nt) of a warp tile at (r0, c0).
+__device__ __forceinline__ int frag_row(int r0, int mt, int e) { return r0 + 16 * mt + ((threadIdx.x & 31) >> 2) + 8 * (e >> 1); }
+__device__ __forceinline__ int frag_col(int c0, int nt, int e) { return c0 + 8 * nt + 2 * (threadIdx.x & 3) + (e & 1); }
+
+template <int MT, int NT>
+__device__ __forceinline__ void zero_frag(float (&acc)[MT][NT][4]) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+}
+
+template <int TM, int TN>
+__device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+}
+
+struct ChunkedBwd {
+    SeqInfo si;                        // 64-token chunks
+    const void *x, *dt, *B, *C, *dy;
+    const float *dt_bias, *A, *D, *init_state, *dfinal;
+    void *dx, *ddt, *dB, *dC;
+    float *ddt_bias, *dA, *dD, *dinit;
+    float *S, *T, *E;                  // (chunks, H, N P), (chunks, H, N P), (chunks, H)
+    int H, N, G;
+};
+
+// Loads rows [0, q) of a (tokens, stride) slab of T into shared fp32 (rows, cols) with row
+// stride ld, zero past q.
+template <typename T>
+__device__ __forceinline__ void load_rows(float* dst, const T* src, int64_t stride, int q, int rows, int cols,
+                                          int ld) {
+    for (int e = threadIdx.x; e < rows * cols; e += blockDim.x) {
+        const int r = e / cols, c = e % cols;
+        dst[r * ld + c] = r < q ? to_f<T>(src[(int64_t)r * stride + c]) : 0.f;
+    }
+}
+
+// ---- k_bwd_terms: S = sum_i u_i B_i x_i^T, T = sum_j e_j C_j dy_j^T (N x 64 each), E = exp(cs_last)
+template <typename T, int N>
+__global__ void __launch_bounds__(256) k_bwd_terms(const ChunkedBwd p) {
+    constexpr int P = kPb;
+    extern __shared__ float smf[];
+    float* sB = smf;                    // kQb x N
+    float* sX = sB + kQb * N;           // kQb x P
+    __shared__ float sd[kQb], sz[kQb], scs[kQb], slast;
+    const int H = p.H, G = p.G;
+    const int64_t f = blockIdx.x / H;
+    const int h = (int)(blockIdx.x % H), g = h / (H / G);
+    ChunkRef r;
+    if (!chunk_ref(p.si, f, r)) return;
+    const int q = (int)(r.t1 - r.t0);
+    const int64_t tok0 = r.row * p.si.L + r.t0;
+    const float bias = p.dt_bias ? p.dt_bias[h] : 0.f, Ah = p.A[h];
+    if (threadIdx.x < 32) chunk_decay<T>((const T*)p.dt, tok0, H, h, q, bias, Ah, sd, sz, scs, &slast);
+    __syncthreads();
+    // warp tiles of the N x 64 result: (16 MT) x 32
+    constexpr int MT = N / 64;
+    const int warp = threadIdx.x >> 5;
+    const int n0 = 16 * MT * (warp >> 1), c0 = 32 * (warp & 1);
+    for (int pass = 0; pass < 2; ++pass) {
+        // pass 0: B with u and x -> S; pass 1: C with e and dy -> T
+        const T* mat = (const T*)(pass == 0 ? p.B : p.C) + (tok0 * G + g) * N;
+        const T* vec = (const T*)(pass == 0 ? p.x : p.dy) + (tok0 * H + h) * P;
+        load_rows<T>(sB, mat, (int64_t)G * N, q, kQb, N, N);
+        for (int e = threadIdx.x; e < kQb * P; e += blockDim.x) {
+            const int j = e / P, c = e % P;
+            float w = 0.f;
+            if (j < q) w = pass == 0 ? expf(slast - scs[j]) * sd[j] : expf(scs[j]);
+            sX[e] = j < q ? w * to_f<T>(vec[(int64_t)j * H * P + c]) : 0.f;
+        }
+        __syncthreads();
+        float acc[MT][4][4];
+        zero_frag(acc);
+        prod<T, MT, 4, false, false>(acc, sB, 1, N, sX, P, 1, n0, c0, kQb);
+        float* out = (pass == 0 ? p.S : p.T) + ((int64_t)f * H + h) * N * P;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; e += 2)
+                    *reinterpret_cast<float2*>(out + (int64_t)frag_row(n0, mt, e) * P + frag_col(c0, nt, e)) =
+                        make_float2(acc[mt][nt][e], acc[mt][nt][e + 1]);
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) p.E[f * H + h] = expf(slast);
+}
+
+// ---- k_bwd_pass: per state element of a (sequence, head), the state entering every chunk
+// (overwriting S) and the adjoint leaving every chunk (overwriting T); dinit.  The chain is
+// sequential over the chunks, so each thread keeps the terms and decays of the next kPre chunks
+// in flight while it advances.
+constexpr int kPre = 8;
+
+__device__ __forceinline__ float chain(float* __restrict__ M, const float* __restrict__ E, int64_t idx0, int64_t eidx0,
+                                       int64_t step, int64_t estep, int nc, float v) {
+    float mv[kPre], ev[kPre];
+#pragma unroll
+    for (int k = 0; k < kPre; ++k)
+        if (k < nc) {
+            mv[k] = M[idx0 + k * step];
+            ev[k] = E[eidx0 + k * estep];
+        }
+    for (int c0 = 0; c0 < nc; c0 += kPre) {
+#pragma unroll
+        for (int k = 0; k < kPre; ++k) {
+            const int c = c0 + k;
+            if (c < nc) {
+                const float mc = mv[k], ec = ev[k];
+                if (c + kPre < nc) {
+                    mv[k] = M[idx0 + (int64_t)(c + kPre) * step];
+                    ev[k] = E[eidx0 + (int64_t)(c + kPre) * estep];
+                }
+                M[idx0 + (int64_t)c * step] = v;
+                v = ec * v + mc;
+            }
+        }
+    }
+    return v;
+}
+
+__global__ void k_bwd_pass(float* __restrict__ S, float* __restrict__ Tm, const float* __restrict__ E,
+                           const float* __restrict__ init, const float* __restrict__ dfinal,
+                           float* __restrict__ dinit, SeqInfo si, int H, int64_t NP) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)si.S * H * NP) return;
+    const int64_t sh = i / NP, e = i % NP;
+    const int s = (int)(sh / H), h = (int)(sh % H);
+    const int nc = seq_nchunks(si, s);
+    const int64_t c0 = seq_chunk0(si, s);
+    const int64_t step = (int64_t)H * NP;
+    // forwards: the state entering chunk c replaces its own term
+    chain(S, E, (c0 * H + h) * NP + e, c0 * H + h, step, H, nc, init ? init[sh * NP + e] : 0.f);
+    // backwards: the adjoint leaving chunk c replaces its adjoint term
+    const float g = chain(Tm, E, ((c0 + nc - 1) * H + h) * NP + e, (c0 + nc - 1) * H + h, -step, -(int64_t)H, nc,
+                          dfinal ? dfinal[sh * NP + e] : 0.f);
+    if (dinit) dinit[sh * NP + e] = g;
+}
+
+// ---- k_bwd_grads: every gradient of one chunk's tokens for one group (its heads in turn)
+template <typename T, int N>
+__global__ void __launch_bounds__(256, 1) k_bwd_grads(const ChunkedBwd p) {
+    constexpr int P = kPb, Q = kQb;
+    // warp tiles: 64 x 64 products 16 x 32 per warp; 64 x N products (16 MTN) x 32
+    constexpr int WC = N / 32, MTN = WC / 2;
+    // rows of the matrices read along a row by the threads of different rows (B, C, x, dy and
+    // the two states) padded by 4 floats, so that those reads spread over the banks
+    constexpr int LN = N + 4, LP = P + 4, LQ = Q;
+    extern __shared__ float smf[];
+    float* sB = smf;                  // Q x N (row stride LN)
+    float* sC = sB + Q * LN;          // Q x N
+    float* sCB = sC + Q * LN;         // Q x Q, C_j . B_i at [j LQ + i]
+    float* sX = sCB + Q * LQ;         // Q x P (row stride LP)
+    float* sDY = sX + Q * LP;         // Q x P
+    float* sHP = sDY + Q * LP;        // N x P, state entering the chunk
+    float* sDH = sHP + N * LP;        // N x P, adjoint of the state leaving it
+    float* sW = sDH + N * LP;         // Q x Q
+    float* sK = sW + Q * LQ;          // Q x Q
+    float* sd = sK + Q * LQ;          // Q each below
+    float* sz = sd + Q;
+    float* scs = sz + Q;
+    float* se = scs + Q;
+    float* su = se + Q;
+    float* colR = su + Q;
+    float* rowRd = colR + Q;
+    float* rowZ = rowRd + Q;
+    float* rowY = rowZ + Q;
+    float* sred = rowY + Q;           // [0] <dh_end, h_prev>, [1] sum dy x, [2] last cs
+    const int H = p.H, G = p.G, HG = H / G;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int64_t f = blockIdx.x / G;
+    const int g = (int)(blockIdx.x % G);
+    ChunkRef r;
+    if (!chunk_ref(p.si, f, r)) return;
+    const int q = (int)(r.t1 - r.t0);
+    const int64_t tok0 = r.row * p.si.L + r.t0;
+    const T* dtg = (const T*)p.dt;
+    load_rows<T>(sB, (const T*)p.B + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N, LN);
+    load_rows<T>(sC, (const T*)p.C + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N, LN);
+    __syncthreads();
+    const int warp = tid >> 5;
+    const int r64 = 16 * (warp >> 1), c64 = 32 * (warp & 1);        // 64 x 64 warp tiles
+    const int rN = 16 * MTN * (warp / WC), cN = 32 * (warp % WC);   // 64 x N warp tiles
+    {
+        float acc[1][4][4];
+        zero_frag(acc);
+        prod<T, 1, 4, true, true>(acc, sC, LN, 1, sB, 1, LN, r64, c64, N);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sCB[frag_row(r64, 0, e) * LQ + frag_col(c64, nt, e)] = acc[0][nt][e];
+    }
+    float dBa[MTN][4][4], dCa[MTN][4][4];
+    zero_frag(dBa);
+    zero_frag(dCa);
+    for (int hh = 0; hh < HG; ++hh) {
+        const int h = g * HG + hh;
+        const float bias = p.dt_bias ? p.dt_bias[h] : 0.f, Ah = p.A[h], Dh = p.D ? p.D[h] : 0.f;
+        load_rows<T>(sX, (const T*)p.x + (tok0 * H + h) * P, (int64_t)H * P, q, Q, P, LP);
+        load_rows<T>(sDY, (const T*)p.dy + (tok0 * H + h) * P, (int64_t)H * P, q, Q, P, LP);
+        {
+            const float4* hp = reinterpret_cast<const float4*>(p.S + ((int64_t)f * H + h) * N * P);
+            const float4* dh = reinterpret_cast<const float4*>(p.T + ((int64_t)f * H + h) * N * P);
+            for (int e = tid; e < N * P / 4; e += blockDim.x) {
+                const int n = e / (P / 4), c = 4 * (e % (P / 4));
+                *reinterpret_cast<float4*>(sHP + n * LP + c) = hp[e];
+                *reinterpret_cast<float4*>(sDH + n * LP + c) = dh[e];
+            }
+        }
+        if (tid < Q) {
+            colR[tid] = 0.f; rowRd[tid] = 0.f; rowZ[tid] = 0.f; rowY[tid] = 0.f;
+        }
+        if (tid < 2) sred[tid] = 0.f;      // sred[2] is written by the decay scan below
+        if (tid < 32) {
+            chunk_decay<T>(dtg, tok0, H, h, q, bias, Ah, sd, sz, scs, &sred[2]);
+            __syncwarp();
+            const float last = sred[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int j = 2 * lane + k;
+                se[j] = j < q ? expf(scs[j]) : 0.f;
+                su[j] = j < q ? expf(last - scs[j]) * sd[j] : 0.f;
+            }
+        }
+        __syncthreads();
+        {
+            float a1 = 0.f, a2 = 0.f;
+            for (int e = tid; e < N * P; e += blockDim.x) a1 += sHP[(e / P) * LP + e % P] * sDH[(e / P) * LP + e % P];
+            for (int e = tid; e < Q * P; e += blockDim.x) a2 += sDY[(e / P) * LP + e % P] * sX[(e / P) * LP + e % P];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+                a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+            }
+            if (lane == 0) {
+                atomicAdd(&sred[0], a1);
+                atomicAdd(&sred[1], a2);
+            }
+        }
+        // (1) dy_j . x_i, the masked forms W, K and the sums of R
+        {
+            float acc[1][4][4];
+            zero_frag(acc);
+            prod<T, 1, 4, true, true>(acc, sDY, LP, 1, sX, 1, LP, r64, c64, P);
+            float rrow[2] = {0.f, 0.f}, rcol[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = frag_row(r64, 0, e), i = frag_col(c64, nt, e);
+                    const float L = (i <= j && j < q) ? expf(scs[j] - scs[i]) : 0.f;
+                    const float cb = sCB[j * LQ + i], di = sd[i], dyx = acc[0][nt][e];
+                    sW[j * LQ + i] = cb * L * di;
+                    sK[j * LQ + i] = L * dyx * di;
+                    const float R = cb * dyx * L;
+                    rrow[e >> 1] += R * di;
+                    rcol[nt][e & 1] += R;
+                }
+#pragma unroll
+            for (int a = 0; a < 2; ++a) atomicAdd(&rowRd[frag_row(r64, 0, 2 * a)], rrow[a]);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) atomicAdd(&colR[frag_col(c64, nt, b)], rcol[nt][b]);
+        }
+        __syncthreads();
+        // (2) dx = D dy + W^T dy + u o (B dh_end), and Z_i = B_i^T dh_end x_i
+        {
+            float bd[1][4][4], wd[1][4][4];
+            zero_frag(bd);
+            zero_frag(wd);
+            prod<T, 1, 4, true, false>(bd, sB, LN, 1, sDH, LP, 1, r64, c64, N);
+            prod<T, 1, 4, false, false>(wd, sW, 1, LQ, sDY, LP, 1, r64, c64, Q);
+            T* dxg = (T*)p.dx + (tok0 * H + h) * P;
+            float z[2] = {0.f, 0.f};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = frag_row(r64, 0, e), c = frag_col(c64, nt, e);
+                    z[e >> 1] += bd[0][nt][e] * sX[i * LP + c];
+                    if (i < q)
+                        dxg[(int64_t)i * H * P + c] = from_f<T>(Dh * sDY[i * LP + c] + wd[0][nt][e] + su[i] * bd[0][nt][e]);
+                }
+#pragma unroll
+            for (int a = 0; a < 2; ++a) atomicAdd(&rowZ[frag_row(r64, 0, 2 * a)], z[a]);
+        }
+        // (3) Y_j = C_j^T h_prev dy_j
+        {
+            float ch[1][4][4];
+            zero_frag(ch);
+            prod<T, 1, 4, true, false>(ch, sC, LN, 1, sHP, LP, 1, r64, c64, N);
+            float y[2] = {0.f, 0.f};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    y[e >> 1] += ch[0][nt][e] * sDY[frag_row(r64, 0, e) * LP + frag_col(c64, nt, e)];
+#pragma unroll
+            for (int a = 0; a < 2; ++a) atomicAdd(&rowY[frag_row(r64, 0, 2 * a)], y[a]);
+        }
+        // (4) dB += K^T C + u o (x dh_end^T),  dC += K B + e o (dy h_prev^T)
+        {
+            float t[MTN][4][4];
+            prod<T, MTN, 4, false, false>(dBa, sK, 1, LQ, sC, LN, 1, rN, cN, Q);
+            zero_frag(t);
+            prod<T, MTN, 4, true, true>(t, sX, LP, 1, sDH, 1, LP, rN, cN, P);
+#pragma unroll
+            for (int mt = 0; mt < MTN; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dBa[mt][nt][e] += su[frag_row(rN, mt, e)] * t[mt][nt][e];
+            prod<T, MTN, 4, true, false>(dCa, sK, LQ, 1, sB, LN, 1, rN, cN, Q);
+            zero_frag(t);
+            prod<T, MTN, 4, true, true>(t, sDY, LP, 1, sHP, 1, LP, rN, cN, P);
+#pragma unroll
+            for (int mt = 0; mt < MTN; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dCa[mt][nt][e] += se[frag_row(rN, mt, e)] * t[mt][nt][e];
+        }
+        __syncthreads();
+        // (5) the decays, on warp 0: tokens 2 lane, 2 lane + 1
+        if (tid < 32) {
+            const float last = sred[2], E = expf(last);
+            float ddir[2], dcs[2], uz = 0.f;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int j = 2 * lane + k;
+                const bool in = j < q;
+                const float Z = rowZ[j];
+                ddir[k] = in ? colR[j] + expf(last - scs[j]) * Z : 0.f;
+                dcs[k] = in ? rowRd[j] - sd[j] * colR[j] + se[j] * rowY[j] - su[j] * Z : 0.f;
+                uz += in ? su[j] * Z : 0.f;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) uz += __shfl_xor_sync(0xffffffffu, uz, o);
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+                if (2 * lane + k == q - 1) dcs[k] += E * sred[0] + uz;
+            // dJ/da_m = sum_{k >= m} dJ/dcs_k: suffix sums over the lanes
+            const float pair = dcs[0] + dcs[1];
+            float suf = pair;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float t = __shfl_down_sync(0xffffffffu, suf, o);
+                if (lane + o < 32) suf += t;
+            }
+            const float above = suf - pair;
+            const float da[2] = {above + pair, above + dcs[1]};
+            float sdA = 0.f, sbias = 0.f;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int j = 2 * lane + k;
+                if (j < q) {
+                    const float dd = ddir[k] + Ah * da[k];
+                    const float z = sz[j];
+                    const float sg = z >= 0.f ? 1.f / (1.f + expf(-z)) : expf(z) / (1.f + expf(z));
+                    const float dz = dd * sg;
+                    ((T*)p.ddt)[(tok0 + j) * H + h] = from_f<T>(dz);
+                    sdA += sd[j] * da[k];
+                    sbias += dz;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                sdA += __shfl_xor_sync(0xffffffffu, sdA, o);
+                sbias += __shfl_xor_sync(0xffffffffu, sbias, o);
+            }
+            if (lane == 0) {
+                atomicAdd(&p.dA[h], sdA);
+                atomicAdd(&p.ddt_bias[h], sbias);
+                atomicAdd(&p.dD[h], sred[1]);
+            }
+        }
+        __syncthreads();
+    }
+    T* dBg = (T*)p.dB + (tok0 * G + g) * N;
+    T* dCg = (T*)p.dC + (tok0 * G + g) * N;
+#pragma unroll
+    for (int mt = 0; mt < MTN; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = frag_row(rN, mt, e), n = frag_col(cN, nt, e);
+                if (i < q) {
+                    dBg[(int64_t)i * G * N + n] = from_f<T>(dBa[mt][nt][e]);
+                    dCg[(int64_t)i * G * N + n] = from_f<T>(dCa[mt][nt][e]);
+                }
+            }
+}
+
+template <int N>
+constexpr size_t grads_smem() {
+    return sizeof(float) * (2 * kQb * (N + 4) + 3 * kQb * kQb + 2 * kQb * (kPb + 4) + 2 * N * (kPb + 4) +
+                            10 * kQb + 4);
+}
+
+template <typename T, int N>
+void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
+    const size_t sm_terms = sizeof(float) * (kQb * N + kQb * kPb);
+    cudaFuncSetAttribute(k_bwd_terms<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_terms);
+    cudaFuncSetAttribute(k_bwd_grads<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grads_smem<N>());
+    {
+        ProfScope ps(K_SCAN_BWD, st);
+        k_bwd_terms<T, N><<<(unsigned)(chunks * p.H), 256, sm_terms, st>>>(p);
+    }
+    {
+        ProfScope ps(K_BWD_PASS, st);
+        const int64_t n = (int64_t)p.si.S * p.H * N * kPb;
+        k_bwd_pass<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p.S, p.T, p.E, p.init_state, p.dfinal, p.dinit, p.si,
+                                                                p.H, (int64_t)N * kPb);
+    }
+    {
+        ProfScope ps(K_BWD_GRADS, st);
+        k_bwd_grads<T, N><<<(unsigned)(chunks * p.G), 256, grads_smem<N>(), st>>>(p);
+    }
+}
+
 template <typename T>
 __global__ void k_bwd_cast(const float* __restrict__ src, T* __restrict__ dst, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
@@ -290,6 +921,7 @@ size_t bwd_workspace_bytes(const ScanArgs& a) {
                                      : a.b * ((a.L + kBwdBlock - 1) / kBwdBlock);
     const size_t NP = (size_t)a.N * a.P;
     auto r = [](size_t v) { return (v + 255) & ~(size_t)255; };
+    if (bwd_chunked(a)) return 2 * r(sizeof(float) * blocks * a.H * NP) + r(sizeof(float) * blocks * a.H);
     return r(sizeof(float) * blocks * a.H * NP) + r(sizeof(float) * a.S * a.H * kBwdBlock * NP) +
            2 * r(sizeof(float) * a.b * a.L * a.G * a.N);
 }
@@ -300,6 +932,30 @@ int launch_scan_bwd(const ScanArgs& a, const BwdArgs& g, const SeqInfo& si64, vo
     const int64_t blocks = a.seq_idx ? (a.L + kBwdBlock - 1) / kBwdBlock + a.S
                                      : a.b * ((a.L + kBwdBlock - 1) / kBwdBlock);
     char* w = (char*)ws;
+    if (bwd_chunked(a)) {
+        ChunkedBwd c;
+        c.si = si64;
+        c.x = a.x; c.dt = a.dt; c.B = a.B; c.C = a.C; c.dy = g.dy;
+        c.dt_bias = a.dt_bias; c.A = a.A; c.D = a.D; c.init_state = a.init_state; c.dfinal = g.dfinal;
+        c.dx = g.dx; c.ddt = g.ddt; c.dB = g.dB; c.dC = g.dC;
+        c.ddt_bias = g.ddt_bias; c.dA = g.dA; c.dD = g.dD; c.dinit = g.dinit;
+        c.S = (float*)w; w += r(sizeof(float) * blocks * a.H * NP);
+        c.T = (float*)w; w += r(sizeof(float) * blocks * a.H * NP);
+        c.E = (float*)w;
+        c.H = (int)a.H; c.N = (int)a.N; c.G = (int)a.G;
+        cudaError_t e = cudaMemsetAsync(g.ddt_bias, 0, sizeof(float) * a.H, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(g.dA, 0, sizeof(float) * a.H, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(g.dD, 0, sizeof(float) * a.H, st);
+        if (e != cudaSuccess) return 6;
+        if (a.dtype == 0) {
+            if (a.N == 128) launch_chunked_t<float, 128>(c, blocks, st);
+            else launch_chunked_t<float, 64>(c, blocks, st);
+        } else {
+            if (a.N == 128) launch_chunked_t<__nv_bfloat16, 128>(c, blocks, st);
+            else launch_chunked_t<__nv_bfloat16, 64>(c, blocks, st);
+        }
+        return 0;
+    }
     BwdParams p;
     p.si = si64;
     p.ck_per_row = (a.L + kBwdBlock - 1) / kBwdBlock;

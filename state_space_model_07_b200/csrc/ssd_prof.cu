@@ -13,7 +13,7 @@ namespace {
 const char* const kNames[K_COUNT] = {
     "seq_bounds", "seq_table", "simt_chunk_state", "simt_state_pass", "simt_chunk_out",
     "state_update", "tc_prep", "tc_scan", "selftest_wait", "scan_bwd", "bwd_cast",
-    "segment_logdecay", "state_chain", "state_out", "tile_logdecay", "group_norm", "quant_allreduce",
+    "segment_logdecay", "state_chain", "state_out", "tile_logdecay", "group_norm", "quant_allreduce", "bwd_pass", "bwd_grads",
 };
 
 struct Pending {

@@ -23,6 +23,8 @@ enum KernelId : int {
     K_TILE_DECAY,
     K_GROUP_NORM,
     K_QUANT,
+    K_BWD_PASS,
+    K_BWD_GRADS,
     K_COUNT
 };
 

@@ -13,13 +13,7 @@
 #include "ssd_internal.h"
 #include "ssd_prof.h"
 
-// tc_ptx.cuh defines the out-of-line polling loop of the bounded wait with
-// external linkage for the tensor-core kernels' translation unit.  This file
-// compiles the same code under another name, so that both units link into one
-// library and the kernels' own build stays exactly as it is.
-#define mbar_wait_slow selftest_mbar_wait_slow
 #include "tc_ptx.cuh"
-#undef mbar_wait_slow
 
 namespace ssd {
 namespace {

@@ -18,4 +18,11 @@ bool state_out_supported(const ScanArgs& a);
 size_t state_out_workspace_bytes(const ScanArgs& a);
 int launch_state_to_output(const ScanArgs& a, const float* h_in, void* ws, int32_t* status, cudaStream_t st);
 
+// The state-to-output pass of the segment split (ssd_state_out.cu): rows W .. b - 1 of `a` are
+// split into K segments of Ls tokens (`tiles` tiles); fin holds every segment's final state and
+// cs the running log-decay of its tokens, c16 the fp16 copy of C; adds each later segment's
+// entering-state output to y and writes those rows' final states.
+int launch_state_out_split(const ScanArgs& a, const void* c16, const float* fin, const float* cs, int64_t W, int K,
+                           int64_t Ls, int tiles, int32_t* status, cudaStream_t st);
+
 }  // namespace ssd

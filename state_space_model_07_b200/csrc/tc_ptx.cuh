@@ -84,7 +84,8 @@ __device__ __forceinline__ bool mbar_try_wait_ns(uint64_t* bar, uint32_t parity,
 __device__ unsigned long long g_poll_iters[32];
 __device__ unsigned long long g_poll_calls[32];
 #endif
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long long limit_cycles) {
+// (internal linkage: every translation unit that includes this header has its own copy)
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long long limit_cycles) {
     const long long t0 = clock64();
 #ifdef SSD_TC_TRACE
     unsigned long long iters = 0;
