@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--mixer", default=None, metavar="CONFIG",
                     help="time the head-sharded mixer layer (tensor parallel over the ranks, quantised "
                          "all-reduce) on this configuration, e.g. mixer_2.7b, instead of the scan")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward of the scan (ssd_chunk_scan_bwd) on the workload instead")
     ap.add_argument("--exact-allreduce", action="store_true",
                     help="with --mixer: an fp32 all-reduce instead of the quantised one")
     ap.add_argument("--batch", type=int, default=None,
@@ -591,6 +593,94 @@ def run_seqpar(args):
     return 0
 
 
+def bwd_flops(w, tokens):
+    """Multiply-adds of the chunked backward (64-token chunks, as evaluated) x 2: per token and
+    head the chunk's state and adjoint terms (2 N P), dy x^T and W^T dy (2 Q P), B dh_end and
+    C h_prev (2 N P), K^T C, K B (2 Q N) and x dh_end^T, dy h_prev^T (2 P N); per token and group
+    C B^T (Q N)."""
+    Q, P, N, H, G = 64, w.headdim, w.dstate, w.nheads, w.ngroups
+    per_head = 2 * N * P + 2 * Q * P + 2 * N * P + 2 * Q * N + 2 * P * N
+    return 2.0 * tokens * (H * per_head + G * Q * N)
+
+
+def run_bwd(args):
+    """The backward of the scan on the workload (one GPU; replicas under torchrun): dx, ddt, dB,
+    dC, ddt_bias, dA, dD and the initial state's gradient from a seeded upstream gradient dy (and
+    dfinal where the workload has an initial state)."""
+    import torch
+    import torch.distributed as dist
+    import state_space_model_07_b200 as ssd
+    from state_space_model_07_b200 import _lib, inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    w = workload_of(args)
+    d = inputs.make_inputs(w, dev)
+    gen = torch.Generator(device="cpu").manual_seed(7)
+    dy = torch.randn(d["x"].shape, generator=gen).to(d["x"].dtype).to(dev)
+    dfinal = None
+    if d["init_state"] is not None:
+        dfinal = torch.randn(d["init_state"].shape, generator=gen).to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return ssd.chunk_scan_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], dy, dt_bias=d["dt_bias"], D=d["D"],
+                                  init_state=d["init_state"], seq_idx=d["seq_idx"], nseqs=d["nseqs"], chunk=w.chunk,
+                                  dfinal=dfinal)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        for _ in range(args.warmup):
+            step()
+        barrier()
+        _lib.profile_read(reset=True)
+        _lib.profile_enable(True)
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        barrier()
+    _lib.profile_enable(False)
+    stats = _lib.profile_read(reset=True)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    tokens = int(d["x"].shape[0] * d["x"].shape[1])
+    value = tokens * world * args.steps / (ms * 1e-3)
+    pk, pk_src = peaks()
+    step_ms = ms / args.steps
+    flops = bwd_flops(w, tokens)
+    es = d["x"].element_size()
+    bytes_ = es * tokens * (w.nheads * (3 * w.headdim + 2) + 4 * w.ngroups * w.dstate)   # x, dy, dx; dt, ddt; B, C, dB, dC
+    line = {"metric": "SSD scan backward tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if es == 2 else "f32", "data": "synthetic",
+            "config": dict(config_of(w), step="ssd_chunk_scan_bwd over the workload (dy seeded)",
+                           parallelism=f"replicas{world}"),
+            "roofline": {"bound": "tensor", "algorithmic_flops": flops, "achieved": flops / (step_ms * 1e-3) / 1e12,
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "peak_source": pk_src,
+                         "frac": flops / (step_ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                         "hbm_min_bytes": bytes_, "hbm_frac": bytes_ / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
+            "cpu_baseline": None, "e2e": None,
+            "gpu_launches": sum(v[0] for v in stats.values()),
+            "kernels": {k: {"launches": v[0], "avg_ms": v[2] / max(v[1], 1)} for k, v in stats.items()},
+            "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_mixer(args):
     """The head-sharded mixer layer ("5.3 Tensor Parallelism support and large-cluster training",
     section 4.1) on the ranks: each holds H / N heads, computes its projections (cuBLAS), scan and
@@ -683,6 +773,8 @@ def main():
         return run_seqpar(args)
     if args.mixer:
         return run_mixer(args)
+    if args.bwd:
+        return run_bwd(args)
     return run_ours(args)
 
 
