@@ -856,6 +856,353 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads(const ChunkedBwd p) {
             }
 }
 
+
+// 8 packed bf16 -> 8 packed fp16 (exact for values in fp16's normal range).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8_bwd(uint4 v) {
+    auto cv = [](uint32_t w) { return h2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
+    return make_uint4(cv(v.x), cv(v.y), cv(v.z), cv(v.w));
+}
+
+// ---- k_bwd_grads_h: k_bwd_grads for bf16 inputs with fp16 operand tiles in shared memory ----
+//
+// The tensor-core operands are fp16 either way; holding them as fp16 halves the shared memory and
+// lets the MMA fragments be read as packed pairs.  Every tile is row-major [rows][W] fp16 with its
+// 4-byte words XOR-swizzled by row (word w of row r at w ^ 4 (r mod 8)): the eight rows and four
+// word offsets a fragment read touches then fall in 32 different banks, for reads along a row
+// (a pair of consecutive k in one word) and across rows (a pair in two rows) alike.
+__device__ __forceinline__ int hsw(int r, int c, int W) {
+    return r * W + ((((c >> 1) ^ ((r & 7) << 2))) << 1) + (c & 1);
+}
+
+// 16 bytes (8 fp16) for columns 8 c8 .. 8 c8 + 7 of row r.
+__device__ __forceinline__ __half* hsw8(__half* M, int r, int c8, int W) { return M + r * W + 8 * (c8 ^ (r & 7)); }
+
+// The pair (k, k + 1) at index `o` (the row of A / the column of B): ROWK = the tile holds k
+// along its rows (one word), else along its columns (two rows).
+template <bool ROWK>
+__device__ __forceinline__ uint32_t hpair(const __half* M, int W, int o, int k) {
+    if (ROWK) return *reinterpret_cast<const uint32_t*>(M + hsw(o, k, W));
+    const __half2 v = __halves2half2(M[hsw(k, o, W)], M[hsw(k + 1, o, W)]);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// mma_tile for fp16 tiles: A(r, k) = A[r][k] (AROWK) or A[k][r]; Bm(k, n) = Bm[n][k] (BROWK) or Bm[k][n].
+template <int MT, int NT, bool AROWK, bool BROWK>
+__device__ __forceinline__ void mma_tile_h(float (&acc)[MT][NT][4], const __half* A, int WA, const __half* Bm, int WB,
+                                           int r0, int c0, int K) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll 1
+    for (int k = 0; k < K; k += 16) {
+        uint32_t af[MT][4], bf[NT][2];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int ra = r0 + 16 * mt + g;
+            af[mt][0] = hpair<AROWK>(A, WA, ra, k + 2 * t);
+            af[mt][1] = hpair<AROWK>(A, WA, ra + 8, k + 2 * t);
+            af[mt][2] = hpair<AROWK>(A, WA, ra, k + 2 * t + 8);
+            af[mt][3] = hpair<AROWK>(A, WA, ra + 8, k + 2 * t + 8);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int n = c0 + 8 * nt + g;
+            bf[nt][0] = hpair<BROWK>(Bm, WB, n, k + 2 * t);
+            bf[nt][1] = hpair<BROWK>(Bm, WB, n, k + 2 * t + 8);
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                asm volatile(
+                    "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                    "{%8, %9}, {%0, %1, %2, %3};"
+                    : "+f"(acc[mt][nt][0]), "+f"(acc[mt][nt][1]), "+f"(acc[mt][nt][2]), "+f"(acc[mt][nt][3])
+                    : "r"(af[mt][0]), "r"(af[mt][1]), "r"(af[mt][2]), "r"(af[mt][3]), "r"(bf[nt][0]),
+                      "r"(bf[nt][1]));
+    }
+}
+
+// Rows [0, q) of a bf16 (tokens, stride) slab -> fp16 tile [rows][W] (swizzled), zero past q.
+__device__ __forceinline__ void load_rows_h(__half* dst, const __nv_bfloat16* src, int64_t stride, int q, int rows,
+                                            int W) {
+    const int c8n = W / 8;
+    for (int e = threadIdx.x; e < rows * c8n; e += blockDim.x) {
+        const int r = e / c8n, c8 = e % c8n;
+        uint4 o = make_uint4(0u, 0u, 0u, 0u);
+        if (r < q) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src + (int64_t)r * stride + 8 * c8);
+            o = bf16x8_to_f16x8_bwd(v);
+        }
+        *reinterpret_cast<uint4*>(hsw8(dst, r, c8, W)) = o;
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(256, 1) k_bwd_grads_h(const ChunkedBwd p) {
+    using T = __nv_bfloat16;
+    constexpr int P = kPb, Q = kQb;
+    constexpr int WC = N / 32, MTN = WC / 2;
+    extern __shared__ __align__(16) uint8_t smraw[];
+    __half* sB = reinterpret_cast<__half*>(smraw);   // [Q][N]
+    __half* sC = sB + Q * N;                         // [Q][N]
+    __half* sX = sC + Q * N;                         // [Q][P]
+    __half* sDY = sX + Q * P;                        // [Q][P]
+    __half* sHP = sDY + Q * P;                       // [N][P] state entering the chunk
+    __half* sDH = sHP + N * P;                       // [N][P] adjoint of the state leaving it
+    __half* sW = sDH + N * P;                        // [Q][Q]
+    __half* sK = sW + Q * Q;                         // [Q][Q]
+    float* sCB = reinterpret_cast<float*>(sK + Q * Q);   // [Q][Q] C_j . B_i in fp32 (it enters the decays)
+    float* sd = sCB + Q * Q;
+    float* sz = sd + Q;
+    float* scs = sz + Q;
+    float* se = scs + Q;
+    float* su = se + Q;
+    float* colR = su + Q;
+    float* rowRd = colR + Q;
+    float* rowZ = rowRd + Q;
+    float* rowY = rowZ + Q;
+    float* sred = rowY + Q;           // [0] <dh_end, h_prev>, [1] sum dy x, [2] last cs
+    const int H = p.H, G = p.G, HG = H / G;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int64_t f = blockIdx.x / G;
+    const int g = (int)(blockIdx.x % G);
+    ChunkRef r;
+    if (!chunk_ref(p.si, f, r)) return;
+    const int q = (int)(r.t1 - r.t0);
+    const int64_t tok0 = r.row * p.si.L + r.t0;
+    const T* dtg = (const T*)p.dt;
+    load_rows_h(sB, (const T*)p.B + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
+    load_rows_h(sC, (const T*)p.C + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
+    __syncthreads();
+    const int warp = tid >> 5;
+    const int r64 = 16 * (warp >> 1), c64 = 32 * (warp & 1);
+    const int rN = 16 * MTN * (warp / WC), cN = 32 * (warp % WC);
+    {
+        float acc[1][4][4];
+        zero_frag(acc);
+        mma_tile_h<1, 4, true, true>(acc, sC, N, sB, N, r64, c64, N);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                sCB[frag_row(r64, 0, e) * Q + frag_col(c64, nt, e)] = acc[0][nt][e];
+    }
+    float dBa[MTN][4][4], dCa[MTN][4][4];
+    zero_frag(dBa);
+    zero_frag(dCa);
+    for (int hh = 0; hh < HG; ++hh) {
+        const int h = g * HG + hh;
+        const float bias = p.dt_bias ? p.dt_bias[h] : 0.f, Ah = p.A[h], Dh = p.D ? p.D[h] : 0.f;
+        load_rows_h(sX, (const T*)p.x + (tok0 * H + h) * P, (int64_t)H * P, q, Q, P);
+        load_rows_h(sDY, (const T*)p.dy + (tok0 * H + h) * P, (int64_t)H * P, q, Q, P);
+        float hpdh = 0.f;   // <h_prev, dh_end> in fp32 from the fp32 states
+        {
+            const float* hp = p.S + ((int64_t)f * H + h) * N * P;
+            const float* dh = p.T + ((int64_t)f * H + h) * N * P;
+            for (int e = tid; e < N * P / 8; e += blockDim.x) {
+                const int n = e / (P / 8), c8 = e % (P / 8);
+                const float4 a0 = *reinterpret_cast<const float4*>(hp + (int64_t)n * P + 8 * c8);
+                const float4 a1 = *reinterpret_cast<const float4*>(hp + (int64_t)n * P + 8 * c8 + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(dh + (int64_t)n * P + 8 * c8);
+                const float4 b1 = *reinterpret_cast<const float4*>(dh + (int64_t)n * P + 8 * c8 + 4);
+                *reinterpret_cast<uint4*>(hsw8(sHP, n, c8, P)) =
+                    make_uint4(h2pack(a0.x, a0.y), h2pack(a0.z, a0.w), h2pack(a1.x, a1.y), h2pack(a1.z, a1.w));
+                *reinterpret_cast<uint4*>(hsw8(sDH, n, c8, P)) =
+                    make_uint4(h2pack(b0.x, b0.y), h2pack(b0.z, b0.w), h2pack(b1.x, b1.y), h2pack(b1.z, b1.w));
+                hpdh += a0.x * b0.x + a0.y * b0.y + a0.z * b0.z + a0.w * b0.w + a1.x * b1.x + a1.y * b1.y +
+                        a1.z * b1.z + a1.w * b1.w;
+            }
+        }
+        if (tid < Q) {
+            colR[tid] = 0.f; rowRd[tid] = 0.f; rowZ[tid] = 0.f; rowY[tid] = 0.f;
+        }
+        if (tid < 2) sred[tid] = 0.f;      // sred[2] is written by the decay scan below
+        if (tid < 32) {
+            chunk_decay<T>(dtg, tok0, H, h, q, bias, Ah, sd, sz, scs, &sred[2]);
+            __syncwarp();
+            const float last = sred[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int j = 2 * lane + k;
+                se[j] = j < q ? expf(scs[j]) : 0.f;
+                su[j] = j < q ? expf(last - scs[j]) * sd[j] : 0.f;
+            }
+        }
+        __syncthreads();
+        {
+            // x and dy share one swizzle, so element e is the same (row, column) in both
+            float a1 = hpdh, a2 = 0.f;
+            for (int e = tid; e < Q * P; e += blockDim.x) a2 += __half2float(sDY[e]) * __half2float(sX[e]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+                a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+            }
+            if (lane == 0) {
+                atomicAdd(&sred[0], a1);
+                atomicAdd(&sred[1], a2);
+            }
+        }
+        // (1) dy_j . x_i, the masked forms W, K and the sums of R
+        {
+            float acc[1][4][4];
+            zero_frag(acc);
+            mma_tile_h<1, 4, true, true>(acc, sDY, P, sX, P, r64, c64, P);
+            float rrow[2] = {0.f, 0.f}, rcol[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = frag_row(r64, 0, e), i = frag_col(c64, nt, e);
+                    const float L = (i <= j && j < q) ? expf(scs[j] - scs[i]) : 0.f;
+                    const float cb = sCB[j * Q + i], di = sd[i], dyx = acc[0][nt][e];
+                    sW[hsw(j, i, Q)] = __float2half_rn(cb * L * di);
+                    sK[hsw(j, i, Q)] = __float2half_rn(L * dyx * di);
+                    const float R = cb * dyx * L;
+                    rrow[e >> 1] += R * di;
+                    rcol[nt][e & 1] += R;
+                }
+#pragma unroll
+            for (int a = 0; a < 2; ++a) atomicAdd(&rowRd[frag_row(r64, 0, 2 * a)], rrow[a]);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) atomicAdd(&colR[frag_col(c64, nt, b)], rcol[nt][b]);
+        }
+        __syncthreads();
+        // (2) dx = D dy + W^T dy + u o (B dh_end), and Z_i = B_i^T dh_end x_i
+        {
+            float bd[1][4][4], wd[1][4][4];
+            zero_frag(bd);
+            zero_frag(wd);
+            mma_tile_h<1, 4, true, false>(bd, sB, N, sDH, P, r64, c64, N);
+            mma_tile_h<1, 4, false, false>(wd, sW, Q, sDY, P, r64, c64, Q);
+            T* dxg = (T*)p.dx + (tok0 * H + h) * P;
+            float z[2] = {0.f, 0.f};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = frag_row(r64, 0, e), c = frag_col(c64, nt, e);
+                    z[e >> 1] += bd[0][nt][e] * __half2float(sX[hsw(i, c, P)]);
+                    if (i < q)
+                        dxg[(int64_t)i * H * P + c] =
+                            from_f<T>(Dh * __half2float(sDY[hsw(i, c, P)]) + wd[0][nt][e] + su[i] * bd[0][nt][e]);
+                }
+#pragma unroll
+            for (int a = 0; a < 2; ++a) atomicAdd(&rowZ[frag_row(r64, 0, 2 * a)], z[a]);
+        }
+        // (3) Y_j = C_j^T h_prev dy_j
+        {
+            float ch[1][4][4];
+            zero_frag(ch);
+            mma_tile_h<1, 4, true, false>(ch, sC, N, sHP, P, r64, c64, N);
+            float y[2] = {0.f, 0.f};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    y[e >> 1] += ch[0][nt][e] * __half2float(sDY[hsw(frag_row(r64, 0, e), frag_col(c64, nt, e), P)]);
+#pragma unroll
+            for (int a = 0; a < 2; ++a) atomicAdd(&rowY[frag_row(r64, 0, 2 * a)], y[a]);
+        }
+        // (4) dB += K^T C + u o (x dh_end^T),  dC += K B + e o (dy h_prev^T)
+        {
+            float t[MTN][4][4];
+            mma_tile_h<MTN, 4, false, false>(dBa, sK, Q, sC, N, rN, cN, Q);
+            zero_frag(t);
+            mma_tile_h<MTN, 4, true, true>(t, sX, P, sDH, P, rN, cN, P);
+#pragma unroll
+            for (int mt = 0; mt < MTN; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dBa[mt][nt][e] += su[frag_row(rN, mt, e)] * t[mt][nt][e];
+            mma_tile_h<MTN, 4, true, false>(dCa, sK, Q, sB, N, rN, cN, Q);
+            zero_frag(t);
+            mma_tile_h<MTN, 4, true, true>(t, sDY, P, sHP, P, rN, cN, P);
+#pragma unroll
+            for (int mt = 0; mt < MTN; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dCa[mt][nt][e] += se[frag_row(rN, mt, e)] * t[mt][nt][e];
+        }
+        __syncthreads();
+        // (5) the decays, on warp 0: tokens 2 lane, 2 lane + 1
+        if (tid < 32) {
+            const float last = sred[2], E = expf(last);
+            float ddir[2], dcs[2], uz = 0.f;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int j = 2 * lane + k;
+                const bool in = j < q;
+                const float Z = rowZ[j];
+                ddir[k] = in ? colR[j] + expf(last - scs[j]) * Z : 0.f;
+                dcs[k] = in ? rowRd[j] - sd[j] * colR[j] + se[j] * rowY[j] - su[j] * Z : 0.f;
+                uz += in ? su[j] * Z : 0.f;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) uz += __shfl_xor_sync(0xffffffffu, uz, o);
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+                if (2 * lane + k == q - 1) dcs[k] += E * sred[0] + uz;
+            const float pair = dcs[0] + dcs[1];
+            float suf = pair;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float tt = __shfl_down_sync(0xffffffffu, suf, o);
+                if (lane + o < 32) suf += tt;
+            }
+            const float above = suf - pair;
+            const float da[2] = {above + pair, above + dcs[1]};
+            float sdA = 0.f, sbias = 0.f;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int j = 2 * lane + k;
+                if (j < q) {
+                    const float dd = ddir[k] + Ah * da[k];
+                    const float z = sz[j];
+                    const float sg = z >= 0.f ? 1.f / (1.f + expf(-z)) : expf(z) / (1.f + expf(z));
+                    const float dz = dd * sg;
+                    ((T*)p.ddt)[(tok0 + j) * H + h] = from_f<T>(dz);
+                    sdA += sd[j] * da[k];
+                    sbias += dz;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                sdA += __shfl_xor_sync(0xffffffffu, sdA, o);
+                sbias += __shfl_xor_sync(0xffffffffu, sbias, o);
+            }
+            if (lane == 0) {
+                atomicAdd(&p.dA[h], sdA);
+                atomicAdd(&p.ddt_bias[h], sbias);
+                atomicAdd(&p.dD[h], sred[1]);
+            }
+        }
+        __syncthreads();
+    }
+    T* dBg = (T*)p.dB + (tok0 * G + g) * N;
+    T* dCg = (T*)p.dC + (tok0 * G + g) * N;
+#pragma unroll
+    for (int mt = 0; mt < MTN; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = frag_row(rN, mt, e), n = frag_col(cN, nt, e);
+                if (i < q) {
+                    dBg[(int64_t)i * G * N + n] = from_f<T>(dBa[mt][nt][e]);
+                    dCg[(int64_t)i * G * N + n] = from_f<T>(dCa[mt][nt][e]);
+                }
+            }
+}
+
+template <int N>
+constexpr size_t grads_h_smem() {
+    return 2 * (2 * kQb * N + 2 * kQb * kPb + 2 * N * kPb + 2 * kQb * kQb) + sizeof(float) * (kQb * kQb + 9 * kQb + 4);
+}
+
 template <int N>
 constexpr size_t grads_smem() {
     return sizeof(float) * (2 * kQb * (N + 4) + 3 * kQb * kQb + 2 * kQb * (kPb + 4) + 2 * N * (kPb + 4) +
@@ -866,7 +1213,8 @@ template <typename T, int N>
 void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
     const size_t sm_terms = sizeof(float) * (kQb * N + kQb * kPb);
     cudaFuncSetAttribute(k_bwd_terms<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_terms);
-    cudaFuncSetAttribute(k_bwd_grads<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grads_smem<N>());
+    if constexpr (sizeof(T) == 4)
+        cudaFuncSetAttribute(k_bwd_grads<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grads_smem<N>());
     {
         ProfScope ps(K_SCAN_BWD, st);
         k_bwd_terms<T, N><<<(unsigned)(chunks * p.H), 256, sm_terms, st>>>(p);
@@ -879,7 +1227,12 @@ void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
     }
     {
         ProfScope ps(K_BWD_GRADS, st);
-        k_bwd_grads<T, N><<<(unsigned)(chunks * p.G), 256, grads_smem<N>(), st>>>(p);
+        if constexpr (sizeof(T) == 2) {
+            cudaFuncSetAttribute(k_bwd_grads_h<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grads_h_smem<N>());
+            k_bwd_grads_h<N><<<(unsigned)(chunks * p.G), 256, grads_h_smem<N>(), st>>>(p);
+        } else {
+            k_bwd_grads<T, N><<<(unsigned)(chunks * p.G), 256, grads_smem<N>(), st>>>(p);
+        }
     }
 }
 
