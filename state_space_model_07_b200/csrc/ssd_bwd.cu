@@ -936,11 +936,15 @@ __device__ __forceinline__ void load_rows_h(__half* dst, const __nv_bfloat16* sr
     }
 }
 
+// 512 threads (16 warps) per block: the 64 x 64 products in 16 x 16 warp tiles, the 64 x N
+// products in 16 x (N / 4) warp tiles.
+constexpr int kGradThreads = 512;
+
 template <int N>
-__global__ void __launch_bounds__(256, 1) k_bwd_grads_h(const ChunkedBwd p) {
+__global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBwd p) {
     using T = __nv_bfloat16;
     constexpr int P = kPb, Q = kQb;
-    constexpr int WC = N / 32, MTN = WC / 2;
+    constexpr int NTN = N / 32;   // 8-column MMA tiles per warp in the 64 x N products
     extern __shared__ __align__(16) uint8_t smraw[];
     __half* sB = reinterpret_cast<__half*>(smraw);   // [Q][N]
     __half* sC = sB + Q * N;                         // [Q][N]
@@ -974,19 +978,19 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads_h(const ChunkedBwd p) {
     load_rows_h(sC, (const T*)p.C + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
     __syncthreads();
     const int warp = tid >> 5;
-    const int r64 = 16 * (warp >> 1), c64 = 32 * (warp & 1);
-    const int rN = 16 * MTN * (warp / WC), cN = 32 * (warp % WC);
+    const int r64 = 16 * (warp >> 2), c64 = 16 * (warp & 3);
+    const int rN = 16 * (warp >> 2), cN = (N / 4) * (warp & 3);
     {
-        float acc[1][4][4];
+        float acc[1][2][4];
         zero_frag(acc);
-        mma_tile_h<1, 4, true, true>(acc, sC, N, sB, N, r64, c64, N);
+        mma_tile_h<1, 2, true, true>(acc, sC, N, sB, N, r64, c64, N);
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 sCB[frag_row(r64, 0, e) * Q + frag_col(c64, nt, e)] = acc[0][nt][e];
     }
-    float dBa[MTN][4][4], dCa[MTN][4][4];
+    float dBa[1][NTN][4], dCa[1][NTN][4];
     zero_frag(dBa);
     zero_frag(dCa);
     for (int hh = 0; hh < HG; ++hh) {
@@ -1044,12 +1048,12 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads_h(const ChunkedBwd p) {
         }
         // (1) dy_j . x_i, the masked forms W, K and the sums of R
         {
-            float acc[1][4][4];
+            float acc[1][2][4];
             zero_frag(acc);
-            mma_tile_h<1, 4, true, true>(acc, sDY, P, sX, P, r64, c64, P);
-            float rrow[2] = {0.f, 0.f}, rcol[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+            mma_tile_h<1, 2, true, true>(acc, sDY, P, sX, P, r64, c64, P);
+            float rrow[2] = {0.f, 0.f}, rcol[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = frag_row(r64, 0, e), i = frag_col(c64, nt, e);
@@ -1064,22 +1068,22 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads_h(const ChunkedBwd p) {
 #pragma unroll
             for (int a = 0; a < 2; ++a) atomicAdd(&rowRd[frag_row(r64, 0, 2 * a)], rrow[a]);
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int b = 0; b < 2; ++b) atomicAdd(&colR[frag_col(c64, nt, b)], rcol[nt][b]);
         }
         __syncthreads();
         // (2) dx = D dy + W^T dy + u o (B dh_end), and Z_i = B_i^T dh_end x_i
         {
-            float bd[1][4][4], wd[1][4][4];
+            float bd[1][2][4], wd[1][2][4];
             zero_frag(bd);
             zero_frag(wd);
-            mma_tile_h<1, 4, true, false>(bd, sB, N, sDH, P, r64, c64, N);
-            mma_tile_h<1, 4, false, false>(wd, sW, Q, sDY, P, r64, c64, Q);
+            mma_tile_h<1, 2, true, false>(bd, sB, N, sDH, P, r64, c64, N);
+            mma_tile_h<1, 2, false, false>(wd, sW, Q, sDY, P, r64, c64, Q);
             T* dxg = (T*)p.dx + (tok0 * H + h) * P;
             float z[2] = {0.f, 0.f};
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int i = frag_row(r64, 0, e), c = frag_col(c64, nt, e);
@@ -1093,12 +1097,12 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads_h(const ChunkedBwd p) {
         }
         // (3) Y_j = C_j^T h_prev dy_j
         {
-            float ch[1][4][4];
+            float ch[1][2][4];
             zero_frag(ch);
-            mma_tile_h<1, 4, true, false>(ch, sC, N, sHP, P, r64, c64, N);
+            mma_tile_h<1, 2, true, false>(ch, sC, N, sHP, P, r64, c64, N);
             float y[2] = {0.f, 0.f};
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     y[e >> 1] += ch[0][nt][e] * __half2float(sDY[hsw(frag_row(r64, 0, e), frag_col(c64, nt, e), P)]);
@@ -1107,25 +1111,21 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads_h(const ChunkedBwd p) {
         }
         // (4) dB += K^T C + u o (x dh_end^T),  dC += K B + e o (dy h_prev^T)
         {
-            float t[MTN][4][4];
-            mma_tile_h<MTN, 4, false, false>(dBa, sK, Q, sC, N, rN, cN, Q);
+            float t[1][NTN][4];
+            mma_tile_h<1, NTN, false, false>(dBa, sK, Q, sC, N, rN, cN, Q);
             zero_frag(t);
-            mma_tile_h<MTN, 4, true, true>(t, sX, P, sDH, P, rN, cN, P);
+            mma_tile_h<1, NTN, true, true>(t, sX, P, sDH, P, rN, cN, P);
 #pragma unroll
-            for (int mt = 0; mt < MTN; ++mt)
+            for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dBa[mt][nt][e] += su[frag_row(rN, mt, e)] * t[mt][nt][e];
-            mma_tile_h<MTN, 4, true, false>(dCa, sK, Q, sB, N, rN, cN, Q);
+                for (int e = 0; e < 4; ++e) dBa[0][nt][e] += su[frag_row(rN, 0, e)] * t[0][nt][e];
+            mma_tile_h<1, NTN, true, false>(dCa, sK, Q, sB, N, rN, cN, Q);
             zero_frag(t);
-            mma_tile_h<MTN, 4, true, true>(t, sDY, P, sHP, P, rN, cN, P);
+            mma_tile_h<1, NTN, true, true>(t, sDY, P, sHP, P, rN, cN, P);
 #pragma unroll
-            for (int mt = 0; mt < MTN; ++mt)
+            for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dCa[mt][nt][e] += se[frag_row(rN, mt, e)] * t[mt][nt][e];
+                for (int e = 0; e < 4; ++e) dCa[0][nt][e] += se[frag_row(rN, 0, e)] * t[0][nt][e];
         }
         __syncthreads();
         // (5) the decays, on warp 0: tokens 2 lane, 2 lane + 1
@@ -1185,17 +1185,70 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads_h(const ChunkedBwd p) {
     T* dBg = (T*)p.dB + (tok0 * G + g) * N;
     T* dCg = (T*)p.dC + (tok0 * G + g) * N;
 #pragma unroll
-    for (int mt = 0; mt < MTN; ++mt)
+    for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = frag_row(rN, mt, e), n = frag_col(cN, nt, e);
-                if (i < q) {
-                    dBg[(int64_t)i * G * N + n] = from_f<T>(dBa[mt][nt][e]);
-                    dCg[(int64_t)i * G * N + n] = from_f<T>(dCa[mt][nt][e]);
-                }
+        for (int e = 0; e < 4; ++e) {
+            const int i = frag_row(rN, 0, e), n = frag_col(cN, nt, e);
+            if (i < q) {
+                dBg[(int64_t)i * G * N + n] = from_f<T>(dBa[0][nt][e]);
+                dCg[(int64_t)i * G * N + n] = from_f<T>(dCa[0][nt][e]);
             }
+        }
+}
+
+// k_bwd_terms for bf16 inputs with fp16 operand tiles (swizzled as for k_bwd_grads_h).
+template <int N>
+__global__ void __launch_bounds__(256) k_bwd_terms_h(const ChunkedBwd p) {
+    using T = __nv_bfloat16;
+    constexpr int P = kPb, Q = kQb;
+    extern __shared__ __align__(16) uint8_t smraw[];
+    __half* sM = reinterpret_cast<__half*>(smraw);   // [Q][N]: B, then C
+    __half* sV = sM + Q * N;                         // [Q][P]: u_j x_j, then e_j dy_j
+    __shared__ float sd[kQb], sz[kQb], scs[kQb], slast;
+    const int H = p.H, G = p.G;
+    const int64_t f = blockIdx.x / H;
+    const int h = (int)(blockIdx.x % H), g = h / (H / G);
+    ChunkRef r;
+    if (!chunk_ref(p.si, f, r)) return;
+    const int q = (int)(r.t1 - r.t0);
+    const int64_t tok0 = r.row * p.si.L + r.t0;
+    if (threadIdx.x < 32)
+        chunk_decay<T>((const T*)p.dt, tok0, H, h, q, p.dt_bias ? p.dt_bias[h] : 0.f, p.A[h], sd, sz, scs, &slast);
+    __syncthreads();
+    constexpr int MT = N / 64;
+    const int warp = threadIdx.x >> 5;
+    const int n0 = 16 * MT * (warp >> 1), c0 = 32 * (warp & 1);
+    for (int pass = 0; pass < 2; ++pass) {
+        // pass 0: B with u and x -> S; pass 1: C with e and dy -> T
+        load_rows_h(sM, (const T*)(pass == 0 ? p.B : p.C) + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
+        const T* vec = (const T*)(pass == 0 ? p.x : p.dy) + (tok0 * H + h) * P;
+        for (int e = threadIdx.x; e < Q * (P / 8); e += blockDim.x) {
+            const int j = e / (P / 8), c8 = e % (P / 8);
+            uint4 o = make_uint4(0u, 0u, 0u, 0u);
+            if (j < q) {
+                const float w = pass == 0 ? expf(slast - scs[j]) * sd[j] : expf(scs[j]);
+                const uint4 v = *reinterpret_cast<const uint4*>(vec + (int64_t)j * H * P + 8 * c8);
+                auto cv = [&](uint32_t u) { return h2pack(w * __uint_as_float(u << 16), w * __uint_as_float(u & 0xffff0000u)); };
+                o = make_uint4(cv(v.x), cv(v.y), cv(v.z), cv(v.w));
+            }
+            *reinterpret_cast<uint4*>(hsw8(sV, j, c8, P)) = o;
+        }
+        __syncthreads();
+        float acc[MT][4][4];
+        zero_frag(acc);
+        mma_tile_h<MT, 4, false, false>(acc, sM, N, sV, P, n0, c0, Q);
+        float* out = (pass == 0 ? p.S : p.T) + ((int64_t)f * H + h) * N * P;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; e += 2)
+                    *reinterpret_cast<float2*>(out + (int64_t)frag_row(n0, mt, e) * P + frag_col(c0, nt, e)) =
+                        make_float2(acc[mt][nt][e], acc[mt][nt][e + 1]);
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) p.E[f * H + h] = expf(slast);
 }
 
 template <int N>
@@ -1217,7 +1270,13 @@ void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
         cudaFuncSetAttribute(k_bwd_grads<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grads_smem<N>());
     {
         ProfScope ps(K_SCAN_BWD, st);
-        k_bwd_terms<T, N><<<(unsigned)(chunks * p.H), 256, sm_terms, st>>>(p);
+        if constexpr (sizeof(T) == 2) {
+            const size_t sm_h = 2 * (kQb * N + kQb * kPb);
+            cudaFuncSetAttribute(k_bwd_terms_h<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_h);
+            k_bwd_terms_h<N><<<(unsigned)(chunks * p.H), 256, sm_h, st>>>(p);
+        } else {
+            k_bwd_terms<T, N><<<(unsigned)(chunks * p.H), 256, sm_terms, st>>>(p);
+        }
     }
     {
         ProfScope ps(K_BWD_PASS, st);
@@ -1229,7 +1288,7 @@ void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
         ProfScope ps(K_BWD_GRADS, st);
         if constexpr (sizeof(T) == 2) {
             cudaFuncSetAttribute(k_bwd_grads_h<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grads_h_smem<N>());
-            k_bwd_grads_h<N><<<(unsigned)(chunks * p.G), 256, grads_h_smem<N>(), st>>>(p);
+            k_bwd_grads_h<N><<<(unsigned)(chunks * p.G), kGradThreads, grads_h_smem<N>(), st>>>(p);
         } else {
             k_bwd_grads<T, N><<<(unsigned)(chunks * p.G), 256, grads_smem<N>(), st>>>(p);
         }
