@@ -549,55 +549,83 @@ __global__ void __launch_bounds__(256) k_bwd_terms(const ChunkedBwd p) {
     if (threadIdx.x == 0) p.E[f * H + h] = expf(slast);
 }
 
-// ---- k_bwd_pass: per state element of a (sequence, head), the state entering every chunk
-// (overwriting S) and the adjoint leaving every chunk (overwriting T); dinit.  The chain is
-// sequential over the chunks, so each thread keeps the terms and decays of the next kPre chunks
-// in flight while it advances.
-constexpr int kPre = 8;
+// ---- k_bwd_pass: per (sequence, head), the state entering every chunk (overwriting S) and the
+// adjoint of the state leaving every chunk (overwriting T), and dinit.  One 256-thread block per
+// (sequence, head) holds the N x 64 state in registers, kVec float4 per thread, and walks the
+// chunks with the next two chunks' terms in flight (every chunk is one contiguous N P slab).
+constexpr int kPassThreads = 256;
 
-__device__ __forceinline__ float chain(float* __restrict__ M, const float* __restrict__ E, int64_t idx0, int64_t eidx0,
-                                       int64_t step, int64_t estep, int nc, float v) {
-    float mv[kPre], ev[kPre];
+__device__ __forceinline__ float4 fma4(float e, float4 a, float4 b) {
+    return make_float4(fmaf(e, a.x, b.x), fmaf(e, a.y, b.y), fmaf(e, a.z, b.z), fmaf(e, a.w, b.w));
+}
+
+// h (in registers) runs through nc chunks whose slabs (N P floats, indexed chunk H + head, as E)
+// are first, first + dir, ...; every slab is replaced by the value entering its chunk, and h
+// becomes E h + (the slab's term).
+template <int kVec>
+__device__ __forceinline__ void chain_block(float4* M, const float* E, int64_t first, int64_t dir, int nc,
+                                            float4 (&hv)[kVec]) {
+    constexpr int64_t slab4 = (int64_t)kVec * kPassThreads;
+    const int tid = threadIdx.x;
+    auto at = [&](int c) { return M + (first + dir * c) * slab4 + tid; };
+    float4 m0[kVec], m1[kVec];
 #pragma unroll
-    for (int k = 0; k < kPre; ++k)
-        if (k < nc) {
-            mv[k] = M[idx0 + k * step];
-            ev[k] = E[eidx0 + k * estep];
+    for (int k = 0; k < kVec; ++k) {
+        if (nc > 0) m0[k] = at(0)[kPassThreads * k];
+        if (nc > 1) m1[k] = at(1)[kPassThreads * k];
+    }
+    for (int c = 0; c < nc; c += 2) {
+        {
+            const float e = E[first + dir * c];
+            float4* dst = at(c);
+#pragma unroll
+            for (int k = 0; k < kVec; ++k) {
+                const float4 mv = m0[k];
+                if (c + 2 < nc) m0[k] = at(c + 2)[kPassThreads * k];
+                dst[kPassThreads * k] = hv[k];
+                hv[k] = fma4(e, hv[k], mv);
+            }
         }
-    for (int c0 = 0; c0 < nc; c0 += kPre) {
+        if (c + 1 < nc) {
+            const float e = E[first + dir * (c + 1)];
+            float4* dst = at(c + 1);
 #pragma unroll
-        for (int k = 0; k < kPre; ++k) {
-            const int c = c0 + k;
-            if (c < nc) {
-                const float mc = mv[k], ec = ev[k];
-                if (c + kPre < nc) {
-                    mv[k] = M[idx0 + (int64_t)(c + kPre) * step];
-                    ev[k] = E[eidx0 + (int64_t)(c + kPre) * estep];
-                }
-                M[idx0 + (int64_t)c * step] = v;
-                v = ec * v + mc;
+            for (int k = 0; k < kVec; ++k) {
+                const float4 mv = m1[k];
+                if (c + 3 < nc) m1[k] = at(c + 3)[kPassThreads * k];
+                dst[kPassThreads * k] = hv[k];
+                hv[k] = fma4(e, hv[k], mv);
             }
         }
     }
-    return v;
 }
 
-__global__ void k_bwd_pass(float* __restrict__ S, float* __restrict__ Tm, const float* __restrict__ E,
-                           const float* __restrict__ init, const float* __restrict__ dfinal,
-                           float* __restrict__ dinit, SeqInfo si, int H, int64_t NP) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)si.S * H * NP) return;
-    const int64_t sh = i / NP, e = i % NP;
+template <int kVec>
+__global__ void __launch_bounds__(kPassThreads) k_bwd_pass(float* __restrict__ S, float* __restrict__ Tm,
+                                                             const float* __restrict__ E,
+                                                             const float* __restrict__ init,
+                                                             const float* __restrict__ dfinal,
+                                                             float* __restrict__ dinit, SeqInfo si, int H) {
+    constexpr int64_t slab4 = (int64_t)kVec * kPassThreads;   // N P / 4
+    const int64_t sh = blockIdx.x;
     const int s = (int)(sh / H), h = (int)(sh % H);
     const int nc = seq_nchunks(si, s);
     const int64_t c0 = seq_chunk0(si, s);
-    const int64_t step = (int64_t)H * NP;
-    // forwards: the state entering chunk c replaces its own term
-    chain(S, E, (c0 * H + h) * NP + e, c0 * H + h, step, H, nc, init ? init[sh * NP + e] : 0.f);
-    // backwards: the adjoint leaving chunk c replaces its adjoint term
-    const float g = chain(Tm, E, ((c0 + nc - 1) * H + h) * NP + e, (c0 + nc - 1) * H + h, -step, -(int64_t)H, nc,
-                          dfinal ? dfinal[sh * NP + e] : 0.f);
-    if (dinit) dinit[sh * NP + e] = g;
+    const int tid = threadIdx.x;
+    float4 hv[kVec];
+    const float4* i4 = init ? reinterpret_cast<const float4*>(init) + sh * slab4 + tid : nullptr;
+#pragma unroll
+    for (int k = 0; k < kVec; ++k) hv[k] = i4 ? i4[kPassThreads * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+    chain_block<kVec>(reinterpret_cast<float4*>(S), E, c0 * H + h, H, nc, hv);                    // forwards
+    const float4* d4 = dfinal ? reinterpret_cast<const float4*>(dfinal) + sh * slab4 + tid : nullptr;
+#pragma unroll
+    for (int k = 0; k < kVec; ++k) hv[k] = d4 ? d4[kPassThreads * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+    chain_block<kVec>(reinterpret_cast<float4*>(Tm), E, (c0 + nc - 1) * H + h, -(int64_t)H, nc, hv);  // backwards
+    if (dinit) {
+        float4* o4 = reinterpret_cast<float4*>(dinit) + sh * slab4 + tid;
+#pragma unroll
+        for (int k = 0; k < kVec; ++k) o4[kPassThreads * k] = hv[k];
+    }
 }
 
 // ---- k_bwd_grads: every gradient of one chunk's tokens for one group (its heads in turn)
@@ -1280,9 +1308,9 @@ void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
     }
     {
         ProfScope ps(K_BWD_PASS, st);
-        const int64_t n = (int64_t)p.si.S * p.H * N * kPb;
-        k_bwd_pass<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p.S, p.T, p.E, p.init_state, p.dfinal, p.dinit, p.si,
-                                                                p.H, (int64_t)N * kPb);
+        constexpr int kVec = N * kPb / 4 / kPassThreads;
+        k_bwd_pass<kVec><<<(unsigned)((int64_t)p.si.S * p.H), kPassThreads, 0, st>>>(p.S, p.T, p.E, p.init_state,
+                                                                                    p.dfinal, p.dinit, p.si, p.H);
     }
     {
         ProfScope ps(K_BWD_GRADS, st);
