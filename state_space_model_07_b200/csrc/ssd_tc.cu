@@ -1326,7 +1326,9 @@ ForcedSplit forced_split() {
 // The plan: split only rows that leave at least half the SMs idle (b H <= S / 2), every row
 // into the most segments that still run in one wave (b H K <= S), with at least 8 tiles per
 // segment.  Measured on B200 (b1 L131072 H64): K = 2 beats the single pass by 30 % and K = 3
-// (two waves) by a further 40 %.  Filling only the last, partial wave of a long batch does
+// (two waves) by a further 40 %; three unequal segments sized to fill all 148 SMs (443 + 443 + 138
+// tiles) take 1.42 ms against 1.26-1.32 ms for the two halves on 128 SMs, because a CTA's tiles
+// slow down as more CTAs run at once (below).  Filling only the last, partial wave of a long batch does
 // not pay: a CTA's tiles run faster when fewer CTAs share the GPU (about 1.8 us per tile
 // with 48 CTAs against 2.9 us with 148 on b8 L4096 H80), so the time won in the scan (~25 us)
 // goes to the state-to-output pass.
