@@ -905,36 +905,53 @@ __device__ __forceinline__ int hsw(int r, int c, int W) {
 // 16 bytes (8 fp16) for columns 8 c8 .. 8 c8 + 7 of row r.
 __device__ __forceinline__ __half* hsw8(__half* M, int r, int c8, int W) { return M + r * W + 8 * (c8 ^ (r & 7)); }
 
-// The pair (k, k + 1) at index `o` (the row of A / the column of B): ROWK = the tile holds k
-// along its rows (one word), else along its columns (two rows).
-template <bool ROWK>
-__device__ __forceinline__ uint32_t hpair(const __half* M, int W, int o, int k) {
-    if (ROWK) return *reinterpret_cast<const uint32_t*>(M + hsw(o, k, W));
-    const __half2 v = __halves2half2(M[hsw(k, o, W)], M[hsw(k + 1, o, W)]);
-    return *reinterpret_cast<const uint32_t*>(&v);
+// ldmatrix: four 8 x 8 fp16 matrices whose rows (16 bytes each) lanes 8 m .. 8 m + 7 address;
+// .trans delivers each transposed.  With the swizzle above a 16-byte row chunk stays contiguous
+// and eight consecutive rows of one chunk fall in eight different bank groups.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const __half* p) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const __half* p) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
 }
 
-// mma_tile for fp16 tiles: A(r, k) = A[r][k] (AROWK) or A[k][r]; Bm(k, n) = Bm[n][k] (BROWK) or Bm[k][n].
+// mma_tile for fp16 tiles: A(r, k) = A[r][k] (AROWK) or A[k][r]; Bm(k, n) = Bm[n][k] (BROWK) or
+// Bm[k][n]; fragments by ldmatrix (NT even).  Lane l addresses row l % 8 of matrix l / 8: for A
+// the matrices are (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
+// -- the m16n8k16 A registers in order; for B, (k 0-7) and (k 8-15) of columns n .. n + 7, then
+// of n + 8 .. n + 15 -- the B registers of two adjacent 8-column tiles.
 template <int MT, int NT, bool AROWK, bool BROWK>
 __device__ __forceinline__ void mma_tile_h(float (&acc)[MT][NT][4], const __half* A, int WA, const __half* Bm, int WB,
                                            int r0, int c0, int K) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    static_assert(NT % 2 == 0, "B fragments come two tiles at a time");
+    const int lane = threadIdx.x & 31, m = lane >> 3, rr = lane & 7;
 #pragma unroll 1
     for (int k = 0; k < K; k += 16) {
         uint32_t af[MT][4], bf[NT][2];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-            const int ra = r0 + 16 * mt + g;
-            af[mt][0] = hpair<AROWK>(A, WA, ra, k + 2 * t);
-            af[mt][1] = hpair<AROWK>(A, WA, ra + 8, k + 2 * t);
-            af[mt][2] = hpair<AROWK>(A, WA, ra, k + 2 * t + 8);
-            af[mt][3] = hpair<AROWK>(A, WA, ra + 8, k + 2 * t + 8);
+            const int r = r0 + 16 * mt;
+            if (AROWK)
+                ldsm_x4(af[mt], hsw8(const_cast<__half*>(A), r + rr + 8 * (m & 1), (k >> 3) + (m >> 1), WA));
+            else
+                ldsm_x4_t(af[mt], hsw8(const_cast<__half*>(A), k + rr + 8 * (m >> 1), (r >> 3) + (m & 1), WA));
         }
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int n = c0 + 8 * nt + g;
-            bf[nt][0] = hpair<BROWK>(Bm, WB, n, k + 2 * t);
-            bf[nt][1] = hpair<BROWK>(Bm, WB, n, k + 2 * t + 8);
+        for (int nt = 0; nt < NT; nt += 2) {
+            const int n = c0 + 8 * nt;
+            uint32_t t4[4];
+            if (BROWK)
+                ldsm_x4(t4, hsw8(const_cast<__half*>(Bm), n + rr + 8 * (m >> 1), (k >> 3) + (m & 1), WB));
+            else
+                ldsm_x4_t(t4, hsw8(const_cast<__half*>(Bm), k + rr + 8 * (m & 1), (n >> 3) + (m >> 1), WB));
+            bf[nt][0] = t4[0];
+            bf[nt][1] = t4[1];
+            bf[nt + 1][0] = t4[2];
+            bf[nt + 1][1] = t4[3];
         }
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
@@ -1085,7 +1102,8 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = frag_row(r64, 0, e), i = frag_col(c64, nt, e);
-                    const float L = (i <= j && j < q) ? expf(scs[j] - scs[i]) : 0.f;
+                    // the fast exponential: this path's operands are fp16 anyway
+                    const float L = (i <= j && j < q) ? __expf(scs[j] - scs[i]) : 0.f;
                     const float cb = sCB[j * Q + i], di = sd[i], dyx = acc[0][nt][e];
                     sW[hsw(j, i, Q)] = __float2half_rn(cb * L * di);
                     sK[hsw(j, i, Q)] = __float2half_rn(L * dyx * di);
