@@ -76,7 +76,7 @@ template <> struct Vec16<__nv_bfloat16> {
     }
 };
 
-template <typename T>
+template <typename T, int kCh>
 __global__ void k_group_norm_vec(const T* __restrict__ x, const float* __restrict__ gamma,
                                  const float* __restrict__ beta, float eps, int64_t rows, int C, int gs,
                                  T* __restrict__ out) {
@@ -88,10 +88,10 @@ __global__ void k_group_norm_vec(const T* __restrict__ x, const float* __restric
     const int64_t row = wid / ng;
     const int c0 = (int)(wid % ng) * gs;
     const T* xr = x + row * C + c0;
-    float v[kMaxChunks][VN];
+    float v[kCh][VN];
     float s = 0.f;
 #pragma unroll
-    for (int m = 0; m < kMaxChunks; ++m) {
+    for (int m = 0; m < kCh; ++m) {
         const int ch = lane + 32 * m;
         if (ch < nch) {
             Vec16<T>::load(xr + ch * VN, v[m]);
@@ -102,7 +102,7 @@ __global__ void k_group_norm_vec(const T* __restrict__ x, const float* __restric
     const float mean = warp_sum(s) / gs;
     float q = 0.f;
 #pragma unroll
-    for (int m = 0; m < kMaxChunks; ++m)
+    for (int m = 0; m < kCh; ++m)
         if (lane + 32 * m < nch) {
 #pragma unroll
             for (int i = 0; i < VN; ++i) {
@@ -113,7 +113,7 @@ __global__ void k_group_norm_vec(const T* __restrict__ x, const float* __restric
     const float rstd = rsqrtf(warp_sum(q) / gs + eps);
     T* orow = out + row * C + c0;
 #pragma unroll
-    for (int m = 0; m < kMaxChunks; ++m) {
+    for (int m = 0; m < kCh; ++m) {
         const int ch = lane + 32 * m;
         if (ch < nch) {
             float o[VN];
@@ -294,8 +294,18 @@ void group_norm_typed(const T* x, const float* gamma, const float* beta, float e
                      ((uintptr_t)out & 15u) == 0 && ((uintptr_t)gamma & 15u) == 0 && ((uintptr_t)beta & 15u) == 0 &&
                      gs / (int)(16 / sizeof(T)) <= 32 * kMaxChunks;
     const unsigned grid = warps_grid(rows * ngroups);
-    if (vec)
-        k_group_norm_vec<T><<<grid, 256, 0, st>>>(x, gamma, beta, eps, rows, (int)C, gs, out);
+    // chunks per lane: as few registers as the group size needs (occupancy)
+    const int ch = (gs / (int)(16 / sizeof(T)) + 31) / 32;
+    if (vec && ch <= 1)
+        k_group_norm_vec<T, 1><<<grid, 256, 0, st>>>(x, gamma, beta, eps, rows, (int)C, gs, out);
+    else if (vec && ch <= 2)
+        k_group_norm_vec<T, 2><<<grid, 256, 0, st>>>(x, gamma, beta, eps, rows, (int)C, gs, out);
+    else if (vec && ch <= 3)
+        k_group_norm_vec<T, 3><<<grid, 256, 0, st>>>(x, gamma, beta, eps, rows, (int)C, gs, out);
+    else if (vec && ch <= 4)
+        k_group_norm_vec<T, 4><<<grid, 256, 0, st>>>(x, gamma, beta, eps, rows, (int)C, gs, out);
+    else if (vec)
+        k_group_norm_vec<T, kMaxChunks><<<grid, 256, 0, st>>>(x, gamma, beta, eps, rows, (int)C, gs, out);
     else
         k_group_norm<T><<<grid, 256, 0, st>>>(x, gamma, beta, eps, rows, (int)C, gs, out);
 }

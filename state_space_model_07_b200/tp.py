@@ -198,12 +198,13 @@ def quant_allreduce(z, comm, ops_: Optional[TPOps] = None, dtype=torch.bfloat16)
 def mixer_fwd(u, s, comm, *, ngroups, dstate, headdim, chunk=256, quantized=True, ops_: Optional[TPOps] = None):
     """This rank's part of the layer: u (b, L, d_model) bf16, the rank's weights `s` (``shard``),
     ngroups = the layer's groups (G / Tp of them here).  Returns the layer output (b L, d_model):
-    bf16 through the quantised all-reduce, or float32 through an exact one."""
+    bf16 through the quantised all-reduce, or float32 through an exact one (float32 too with one
+    rank, which has nothing to reduce)."""
     o = ops_ or TPOps()
     n = o.local_output(u, s, ngroups=ngroups // comm.world, dstate=dstate, headdim=headdim, chunk=chunk)
     z = o.out_proj(n, s)
-    if comm.world == 1 and not quantized:
-        return z
+    if comm.world == 1:
+        return z          # one rank: its partial is the output, there is nothing to reduce
     return quant_allreduce(z, comm, o) if quantized else comm.all_reduce(z)
 
 
