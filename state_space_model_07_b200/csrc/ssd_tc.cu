@@ -206,6 +206,17 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 }
                 ++bc_issued;
             };
+            // x, B and C of a tile are pulled into L2 three tiles ahead of use, so that the loads on
+            // the critical path (the single B / C stage is refilled only once a tile's MMAs are done)
+            // read L2 rather than HBM
+            auto prefetch = [&](int t) {
+                const int tok = (int)(tok0 + (int64_t)t * kT);
+                tma_prefetch_l2_3d(&tm_x, 0, h, tok);
+                for (int k = 0; k < C::kBoxes; ++k) {
+                    tma_prefetch_l2_3d(&tm_b, 64 * k, g, tok);
+                    tma_prefetch_l2_3d(&tm_c, 64 * k, g, tok);
+                }
+            };
             const uint32_t id_cb = idesc_f16(128, 128, 0, 0);
             load_x(0);
             load_bc(0);
@@ -213,8 +224,10 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 load_x(1);
                 if (C::kBCStages == 2) load_bc(1);
             }
+            if (nt > 2) prefetch(2);
             bool ok = true;
             for (int t = 0; t < nt; ++t) {
+                if (t + 3 < nt) prefetch(t + 3);
                 const int bst = t % C::kBCStages;
                 const uint32_t bpar = (uint32_t)((t / C::kBCStages) & 1);
                 if (!(ok = wait_bar(ctl, &s.bcfull[bst], bpar, p.status))) break;
