@@ -27,9 +27,13 @@
 //   * k_tc_scan<N> (N = 256): the first design, in which the MMA accumulates
 //     the state in TMEM (the math warps scale it by the tile's total decay,
 //     then B^T (w o x) is added on the tensor core) and the epilogue combines
-//     two accumulators.  Warp roles (576 threads): P (warps 0-7) decay scan and
+//     two accumulators.  Warp roles (608 threads): P (warps 0-7) decay scan and
 //     the causal mask; E (warps 8-15) state hand-over, fp16 operands and the
-//     epilogue; W16 TMA loads and C B^T; W17 the other MMAs.
+//     epilogue; W16 TMA loads and C B^T; W17 C h_prev, then S x; W18
+//     B^T (w o x).  A single thread issues tcgen05.mma chains at roughly one
+//     instruction per 100-200 cycles whatever N is, so the three 16-instruction
+//     chains of a tile come from separate warps, and each starts on the first
+//     64-column box of B / C while the rest is still loading.
 //
 // A warp can reach only its quarter of the 128 TMEM lanes, so each math role
 // has two warps per lane quarter (thread j of a quarter owns token / state row
@@ -56,15 +60,14 @@ namespace {
 using namespace tc;
 
 constexpr int kRoleThreads = 256;   // P and E: two warps per TMEM lane quarter
-constexpr int kThreads = 576;
+constexpr int kThreads = 608;
 constexpr uint32_t kTmemCols = 512;
 
-// Layout constants for dstate N (128 or 256).
-//   N = 128: B and C tiles double-buffered; Yd, Yo double-buffered.
-//   N = 256: B and C tiles (64 KB each) single-buffered, reloaded once the
-//            tile's C h_prev and B^T (w o x) MMAs are done; Yd single-buffered
-//            (its MMA waits for the previous epilogue), Yo double-buffered; the
-//            state takes two 128-lane TMEM blocks.
+// Layout constants for dstate N (the kernel is instantiated for N = 256 only):
+// B and C tiles (64 KB each) single-buffered, reloaded once the tile's C B^T,
+// C h_prev and B^T (w o x) MMAs are done; Yd single-buffered (its MMA waits for
+// the previous epilogue), Yo double-buffered; the state takes two 128-lane TMEM
+// blocks.
 template <int N>
 struct Cfg {
     static constexpr int kBoxes = N / 64;                   // 64-column boxes per B / C tile
@@ -76,7 +79,6 @@ struct Cfg {
     static constexpr uint32_t kColYo = kColYd + 64 * kYdBufs;
     static constexpr uint32_t kColH = kColYo + 128;
     static_assert(kColH + 64 * kHBlocks <= kTmemCols, "TMEM columns");
-    static constexpr uint32_t kBCBytes = 2 * kBoxes * kBoxBytes;  // B and C of one tile
 };
 
 
@@ -93,16 +95,17 @@ struct __align__(1024) TcSmem {
     float wtot[2][4];
     // Every barrier's next phase depends on an action its waiters take after
     // waiting, so no waiter can ever see a barrier two phases ahead.
-    uint64_t xfull[2];        // TMA x -> E, W17          (per x stage)
-    uint64_t bcfull[2];       // TMA B, C -> W16, W17     (per B/C stage)
-    uint64_t scan_done[2];    // P -> E                   (per tile parity)
-    uint64_t e_done[2];       // E -> P (and W17 at N = 256)  (per tile parity)
-    uint64_t yd_par[2];       // W17 commit -> E, P, W16  (per tile parity)
-    uint64_t cb_done;         // W16 commit -> P
+    uint64_t xfull[2];        // TMA x -> E                    (per x stage)
+    uint64_t bcfull[4];       // TMA B, C box k -> W16, W17, W18  (per 64-column box)
+    uint64_t scan_done[2];    // P -> E                        (per tile parity)
+    uint64_t e_done[2];       // E -> P, W17                   (per tile parity)
+    uint64_t x_ready[2];      // E -> W17, W18                 (per tile parity)
+    uint64_t yd_par[2];       // W17 commit (S x) -> E, P, W16 (per tile parity)
+    uint64_t cb_done;         // W16 commit -> P, W16
     uint64_t s_ready;         // P -> W16, W17
-    uint64_t x_ready;         // E -> W17
-    uint64_t sc_done;         // W17 commit -> E (and W16 at N = 256)
-    uint64_t fin[2];          // W16, W17: own tcgen05 work drained before exit
+    uint64_t sc_done;         // W17 (C h_prev) and W18 (B^T (w o x)) commits -> E, W16
+    uint64_t b_zeroed;        // P -> W18, once: B rows past the sequence end zeroed
+    uint64_t fin[3];          // W16, W17, W18: own tcgen05 work drained before exit
     uint32_t tmem_base;
     TcCtl ctl;
 };
@@ -142,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
           const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
     using C = Cfg<N>;
+    static_assert(C::kBCStages == 1 && C::kYdBufs == 1, "the hand-off below is written for N = 256");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // Align to 1024 bytes (128-byte swizzle atoms) by pointer arithmetic on the
     // shared array, so that the compiler keeps every access in the shared state
@@ -163,16 +167,17 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.xfull[i], 1);
-            mbar_init(&s.bcfull[i], 1);
             mbar_init(&s.scan_done[i], kRoleThreads);
             mbar_init(&s.e_done[i], kRoleThreads);
+            mbar_init(&s.x_ready[i], kRoleThreads);
             mbar_init(&s.yd_par[i], 1);
-            mbar_init(&s.fin[i], 1);
         }
+        for (int i = 0; i < 4; ++i) mbar_init(&s.bcfull[i], 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&s.fin[i], 1);
         mbar_init(&s.cb_done, 1);
         mbar_init(&s.s_ready, kRoleThreads);
-        mbar_init(&s.x_ready, kRoleThreads);
-        mbar_init(&s.sc_done, 1);
+        mbar_init(&s.sc_done, 2);
+        mbar_init(&s.b_zeroed, kRoleThreads);
         ctl.abort = 0;
         fence_mbar_init();
     }
@@ -196,13 +201,14 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 tma_load_3d(s.x[st], &tm_x, &s.xfull[st], 0, h, (int)(tok0 + (int64_t)t * kT));
                 ++x_issued;
             };
+            // B and C land box by box, so that the MMAs of a tile start on the first 64 state
+            // columns while the rest is still in flight
             auto load_bc = [&](int t) {
-                const int st = t % C::kBCStages;
                 const int tok = (int)(tok0 + (int64_t)t * kT);
-                mbar_expect_tx(&s.bcfull[st], C::kBCBytes);
                 for (int k = 0; k < C::kBoxes; ++k) {
-                    tma_load_3d(s.b[st][k], &tm_b, &s.bcfull[st], 64 * k, g, tok);
-                    tma_load_3d(s.c[st][k], &tm_c, &s.bcfull[st], 64 * k, g, tok);
+                    mbar_expect_tx(&s.bcfull[k], 2 * kBoxBytes);
+                    tma_load_3d(s.b[0][k], &tm_b, &s.bcfull[k], 64 * k, g, tok);
+                    tma_load_3d(s.c[0][k], &tm_c, &s.bcfull[k], 64 * k, g, tok);
                 }
                 ++bc_issued;
             };
@@ -220,36 +226,34 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             const uint32_t id_cb = idesc_f16(128, 128, 0, 0);
             load_x(0);
             load_bc(0);
-            if (nt > 1) {
-                load_x(1);
-                if (C::kBCStages == 2) load_bc(1);
-            }
+            if (nt > 1) load_x(1);
             if (nt > 2) prefetch(2);
             bool ok = true;
             for (int t = 0; t < nt; ++t) {
                 if (t + 3 < nt) prefetch(t + 3);
-                const int bst = t % C::kBCStages;
-                const uint32_t bpar = (uint32_t)((t / C::kBCStages) & 1);
-                if (!(ok = wait_bar(ctl, &s.bcfull[bst], bpar, p.status))) break;
                 // P has finished reading C B^T of the previous tile
                 if (t > 0 && !(ok = wait_bar(ctl, &s.s_ready, (t - 1) & 1, p.status))) break;
-                tc_fence_after();
-                const uint32_t cb = smem_u32(s.c[bst][0]), bb = smem_u32(s.b[bst][0]);
+                const uint32_t cb = smem_u32(s.c[0][0]), bb = smem_u32(s.b[0][0]);
                 for (int k = 0; k < N / 16; ++k) {
+                    if ((k & 3) == 0) {
+                        if (!(ok = wait_bar(ctl, &s.bcfull[k >> 2], (uint32_t)(t & 1), p.status))) break;
+                        tc_fence_after();
+                    }
                     const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
                     mma_ss(tmem + C::kColCB, sdesc_sw128(cb + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024),
                            id_cb, k > 0);
                 }
+                if (!ok) break;
                 mma_commit(&s.cb_done);
                 if (t >= 1 && t + 1 < nt) {
-                    // x stage (t + 1) & 1 (and, double-buffered, that B/C stage) is free once
-                    // every MMA of tile t - 1 has completed
+                    // x stage (t + 1) & 1 is free once S x of tile t - 1 has completed
                     if (!(ok = wait_bar(ctl, &s.yd_par[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status))) break;
                     load_x(t + 1);
-                    if (C::kBCStages == 2) load_bc(t + 1);
                 }
-                if (C::kBCStages == 1 && t + 1 < nt) {
-                    // the single B/C stage is free once C h_prev and B^T (w o x) of tile t are done
+                if (t + 1 < nt) {
+                    // the single B/C stage is free once C B^T, C h_prev and B^T (w o x) of
+                    // tile t are done
+                    if (!(ok = wait_bar(ctl, &s.cb_done, t & 1, p.status))) break;
                     if (!(ok = wait_bar(ctl, &s.sc_done, t & 1, p.status))) break;
                     load_bc(t + 1);
                 }
@@ -258,7 +262,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 // Give up: let the copies already in flight land before the CTA exits.
                 for (int t = 0; t < x_issued; ++t) mbar_wait(&s.xfull[t & 1], (t >> 1) & 1, 400000000ll);
                 for (int t = 0; t < bc_issued; ++t)
-                    mbar_wait(&s.bcfull[t % C::kBCStages], (t / C::kBCStages) & 1, 400000000ll);
+                    for (int k = 0; k < C::kBoxes; ++k) mbar_wait(&s.bcfull[k], t & 1, 400000000ll);
             }
             // every C B^T issued has completed before TMEM is freed (on a timeout nobody else
             // waits for the last ones)
@@ -266,48 +270,72 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             mbar_wait(&s.fin[0], 0, 400000000ll);
         }
     } else if (warp == 17) {
-        // ----------------------------------- W17: C h_prev, B^T (w o x), S x
+        // -------------------------------------------------------- W17: C h_prev, S x
         if (lane == 0) {
             const uint32_t id_pn = idesc_f16(128, 64, 0, 1);   // K-major A, MN-major B
-            const uint32_t id_mn = idesc_f16(128, 64, 1, 1);   // MN-major A and B
-            for (int t = 0; t < nt; ++t) {
-                const int st = t & 1, bst = t % C::kBCStages;
-                if (!wait_bar(ctl, &s.x_ready, t & 1, p.status)) break;
-                // C h_prev reads the C tile: its TMA load must have landed (x_ready does not
-                // imply it: E waits only for x)
-                if (!wait_bar(ctl, &s.bcfull[bst], (uint32_t)((t / C::kBCStages) & 1), p.status)) break;
-                tc_fence_after();
-                const uint32_t cb = smem_u32(s.c[bst][0]), bb = smem_u32(s.b[bst][0]);
-                const uint32_t hsb = smem_u32(s.hs), wxb = smem_u32(s.wx), xb = smem_u32(s.x[st]);
-                // Yo = C h_prev
+            bool ok = true;
+            for (int t = 0; ok && t < nt; ++t) {
+                const int st = t & 1;
+                // E has written h_prev (fp16) and read out Yo[st] two tiles back
+                if (!(ok = wait_bar(ctl, &s.x_ready[st], (uint32_t)((t >> 1) & 1), p.status))) break;
+                const uint32_t cb = smem_u32(s.c[0][0]), hsb = smem_u32(s.hs);
+                // Yo = C h_prev, box by box as C lands
                 for (int k = 0; k < N / 16; ++k) {
+                    if ((k & 3) == 0) {
+                        if (!(ok = wait_bar(ctl, &s.bcfull[k >> 2], (uint32_t)(t & 1), p.status))) break;
+                        tc_fence_after();
+                    }
                     const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
                     mma_ss(tmem + C::kColYo + 64 * st, sdesc_sw128(cb + off, 16, 1024),
                            sdesc_sw128(hsb + k * 2048, kBoxBytes, 1024), id_pn, k > 0);
                 }
-                // H += B^T (w o x), one 128-row block of the state at a time: needs the B rows
-                // past the sequence end zeroed by P
-                if (!wait_bar(ctl, &s.s_ready, t & 1, p.status)) break;
-                tc_fence_after();
-                for (int mb = 0; mb < C::kHBlocks; ++mb)
-                    for (int k = 0; k < kT / 16; ++k)
-                        mma_ss(tmem + C::kColH + 64 * mb,
-                               sdesc_sw128(bb + 2 * mb * kBoxBytes + k * 2048, kBoxBytes, 1024),
-                               sdesc_sw128(wxb + k * 2048, kBoxBytes, 1024), id_mn, 1);
+                if (!ok) break;
                 mma_commit(&s.sc_done);
-                // Yd = S x  (S carries D on its diagonal); a single Yd buffer must first be
-                // read out by the previous epilogue
-                if (C::kYdBufs == 1 && t > 0 &&
-                    !wait_bar(ctl, &s.e_done[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status))
-                    break;
-                const uint32_t yd = tmem + C::kColYd + 64 * (C::kYdBufs == 2 ? st : 0);
+                // Yd = S x  (S carries D on its diagonal), issued after C h_prev so that it never
+                // delays the state chain: S must be written, and the single Yd buffer read out
+                // by the previous epilogue
+                if (!(ok = wait_bar(ctl, &s.s_ready, t & 1, p.status))) break;
+                if (t > 0 && !(ok = wait_bar(ctl, &s.e_done[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status))) break;
+                tc_fence_after();
+                const uint32_t xb = smem_u32(s.x[st]);
                 for (int k = 0; k < kT / 16; ++k)
-                    mma_ts(yd, tmem + C::kColS + k * 8, sdesc_sw128(xb + k * 2048, kBoxBytes, 1024), id_pn, k > 0);
+                    mma_ts(tmem + C::kColYd, tmem + C::kColS + k * 8, sdesc_sw128(xb + k * 2048, kBoxBytes, 1024),
+                           id_pn, k > 0);
                 mma_commit(&s.yd_par[st]);
             }
             if (nt > 0) {
                 mma_commit(&s.fin[1]);
                 mbar_wait(&s.fin[1], 0, 400000000ll);
+            }
+        }
+    } else if (warp == 18) {
+        // ------------------------------------------------- W18: H += B^T (w o x)
+        if (lane == 0) {
+            const uint32_t id_mn = idesc_f16(128, 64, 1, 1);   // MN-major A and B
+            const int qlast = (int)(len - (int64_t)(nt - 1) * kT);
+            bool ok = true;
+            for (int t = 0; ok && t < nt; ++t) {
+                // E has scaled the state in TMEM by the tile's total decay and written w o x
+                if (!(ok = wait_bar(ctl, &s.x_ready[t & 1], (uint32_t)((t >> 1) & 1), p.status))) break;
+                // on a partial last tile, the B rows past the sequence end must read as zeros
+                if (t == nt - 1 && qlast < kT && !(ok = wait_bar(ctl, &s.b_zeroed, 0, p.status))) break;
+                const uint32_t bb = smem_u32(s.b[0][0]), wxb = smem_u32(s.wx);
+                // one 128-row block of the state at a time: rows 128 mb .. 128 mb + 127 are the
+                // B columns of boxes 2 mb and 2 mb + 1
+                for (int mb = 0; ok && mb < C::kHBlocks; ++mb) {
+                    if (!(ok = wait_bar(ctl, &s.bcfull[2 * mb], (uint32_t)(t & 1), p.status))) break;
+                    if (!(ok = wait_bar(ctl, &s.bcfull[2 * mb + 1], (uint32_t)(t & 1), p.status))) break;
+                    tc_fence_after();
+                    for (int k = 0; k < kT / 16; ++k)
+                        mma_ss(tmem + C::kColH + 64 * mb,
+                               sdesc_sw128(bb + 2 * mb * kBoxBytes + k * 2048, kBoxBytes, 1024),
+                               sdesc_sw128(wxb + k * 2048, kBoxBytes, 1024), id_mn, 1);
+                }
+                if (ok) mma_commit(&s.sc_done);
+            }
+            if (nt > 0) {
+                mma_commit(&s.fin[2]);
+                mbar_wait(&s.fin[2], 0, 400000000ll);
             }
         }
     } else if (warp < 8) {
@@ -333,7 +361,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
         float dt_next = 0.f;
         if (nt > 0 && j < len) dt_next = __bfloat162float(p.dt[(tok0 + j) * H + h]);
         for (int t = 0; t < nt; ++t) {
-            const int buf = t & 1, bst = t % C::kBCStages;
+            const int buf = t & 1;
             const int q = (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT);
             // E is done with tile t - 2, whose decay arrays share this parity
             if (t >= 2 && !wait_bar_w(ctl, &s.e_done[buf], ((t - 2) >> 1) & 1, p.status))
@@ -344,8 +372,6 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 dj = softplus_f(dt_next + bias);
                 a = dj * A2;
             }
-            if (t + 1 < nt && (int64_t)(t + 1) * kT + j < len)
-                dt_next = __bfloat162float(p.dt[(tok0 + (int64_t)(t + 1) * kT + j) * H + h]);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float u = __shfl_up_sync(0xffffffffu, a, o);
@@ -364,16 +390,24 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 s.colfac[buf][j] = ex2(cs2_pivot - cs2j) * dj;
             }
             mbar_arrive(&s.scan_done[buf]);
+            // dt of the next tile: loaded only now, since an arrival (a release) waits for the
+            // thread's loads in flight; the next one (s_ready) comes after C B^T of this tile
+            if (t + 1 < nt && (int64_t)(t + 1) * kT + j < len)
+                dt_next = __bfloat162float(p.dt[(tok0 + (int64_t)(t + 1) * kT + j) * H + h]);
             p_bar();
             if (!wait_bar_w(ctl, &s.cb_done, t & 1, p.status)) break;
-            if (j >= q) {
-                // C B^T has read this tile's B: zero the rows past the sequence end
-                // so that B^T (w o x) sees exact zeros there (even for non-finite data)
-                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                for (int bx = half; bx < C::kBoxes; bx += 2)
+            if (q < kT) {
+                // (the last tile only) C B^T has read this tile's B: zero the rows past the
+                // sequence end so that B^T (w o x) sees exact zeros there (even for non-finite
+                // data), then let W18 issue it
+                if (j >= q) {
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                    for (int bx = half; bx < C::kBoxes; bx += 2)
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(s.b[bst][bx] + sw128_off(j, c)) = z;
-                fence_proxy_async_smem();
+                        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(s.b[0][bx] + sw128_off(j, c)) = z;
+                    fence_proxy_async_smem();
+                }
+                mbar_arrive(&s.b_zeroed);
             }
             // S of the previous tile has been consumed by its S x
             if (t > 0 &&
@@ -513,22 +547,21 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&s.x_ready);
+            mbar_arrive(&s.x_ready[st]);
             return true;
         };
         // Step k prepares tile k (once the state entering it is complete) and then
         // writes the output of tile k - 1.
         bool ok = true;
         for (int k = 0; ok && k <= nt; ++k) {
-            if (k < nt) {
-                // the state entering tile k is complete once B^T (w o x) of tile k - 1 has been
-                // added; that also frees hs and (w o x) for tile k
-                if (k > 0) {
-                    if (!(ok = wait_bar_w(ctl, &s.sc_done, (k - 1) & 1, p.status))) break;
-                    tc_fence_after();
-                }
-                if (!(ok = prepare(k, k == 0))) break;
+            // the state entering tile k is complete once B^T (w o x) of tile k - 1 has been
+            // added; that also frees hs and (w o x) for tile k, and C h_prev of tile k - 1
+            // (read by its epilogue below) is done
+            if (k > 0) {
+                if (!(ok = wait_bar_w(ctl, &s.sc_done, (k - 1) & 1, p.status))) break;
+                tc_fence_after();
             }
+            if (k < nt && !(ok = prepare(k, k == 0))) break;
             if (k == 0) continue;
             const int t = k - 1, st = t & 1;
             const int q = (int)(len - (int64_t)t * kT < kT ? len - (int64_t)t * kT : kT);
@@ -538,7 +571,7 @@ k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             {
                 const float ej = ex2(s.cs[st][j]);
                 __nv_bfloat16* yrow = p.y + (tok0 + (int64_t)t * kT + j) * H * kP + (int64_t)h * kP;
-                const uint32_t yd = tmem + lane_base + C::kColYd + 64 * (C::kYdBufs == 2 ? st : 0);
+                const uint32_t yd = tmem + lane_base + C::kColYd;
                 const uint32_t yo = tmem + lane_base + C::kColYo + 64 * st;
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {

@@ -725,27 +725,35 @@ def build_scan3_pair(nt: int, partial: bool = False, drop: frozenset = frozenset
     return m
 
 
-# The first-generation kernel (k_tc_scan<N>): state accumulated in TMEM.
-# n = 128: B/C double-buffered, two Yd buffers; n = 256: one B/C stage (its
-# reload waits for the tile's C h_prev and B^T (w o x)), one Yd buffer (its
-# S x waits for the previous epilogue).  `fin`: the two MMA-issuing threads
-# drain their tensor-core work before the CTA exits.
+# The first-generation kernel (k_tc_scan<N>, N = 256): state accumulated in TMEM.
+# One B/C stage, loaded as four 64-column boxes with a barrier each (its reload
+# waits for the tile's C B^T, C h_prev and B^T (w o x)); one Yd buffer (its S x
+# waits for the previous epilogue), Yo per tile parity.  Three MMA-issuing
+# threads: W16 (C B^T), W17 (C h_prev, then S x) and W18 (B^T (w o x), state
+# rows of boxes 0-1, then 2-3); sc_done completes once W17 and W18 have both
+# committed.  On a partial last tile, W18 waits for P to zero the B rows past
+# the sequence end (b_zeroed, used once).  `fin`: the MMA-issuing threads drain
+# their tensor-core work before the CTA exits.
 
-def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = frozenset(),
-                fin: bool = True) -> Machine:
-    bc_stages = 2 if n == 128 else 1
-    yd_bufs = 2 if n == 128 else 1
+BOXES = 4
+
+
+def build_scan1(nt: int, partial: bool = False, drop: frozenset = frozenset(), fin: bool = True) -> Machine:
     m = Machine()
     for i in range(2):
         m.barrier(f"xfull{i}", 1)
-        m.barrier(f"bcfull{i}", 1)
         m.barrier(f"scan_done{i}", 8)
         m.barrier(f"e_done{i}", 8)
+        m.barrier(f"x_ready{i}", 8)
         m.barrier(f"yd_par{i}", 1)
+    for k in range(BOXES):
+        m.barrier(f"bcfull{k}", 1)
+    for i in range(3):
         m.barrier(f"fin{i}", 1)
-    for name, count in (("cb_done", 1), ("s_ready", 8), ("x_ready", 8), ("sc_done", 1)):
+    for name, count in (("cb_done", 1), ("s_ready", 8), ("sc_done", 2), ("b_zeroed", 8)):
         m.barrier(name, count)
     last_partial = lambda t: partial and t == nt - 1
+    b_all = tuple(f"b{k}" for k in range(BOXES))
 
     def w16():      # TMA and C B^T
         if nt == 0:
@@ -757,77 +765,105 @@ def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = 
             yield ("tma_load", f"xfull{t & 1}", f"x{t & 1}")
             issued["x"] += 1
 
-        def load_bc(t):
-            st = t % bc_stages
-            yield ("arrive_tx", f"bcfull{st}", 2)
-            yield ("tma_load", f"bcfull{st}", f"b{st}")
-            yield ("tma_load", f"bcfull{st}", f"c{st}")
+        def load_bc():
+            for k in range(BOXES):
+                yield ("arrive_tx", f"bcfull{k}", 2)
+                yield ("tma_load", f"bcfull{k}", f"b{k}")
+                yield ("tma_load", f"bcfull{k}", f"c{k}")
             issued["bc"] += 1
 
         yield from load_x(0)
-        yield from load_bc(0)
+        yield from load_bc()
         if nt > 1:
             yield from load_x(1)
-            if bc_stages == 2:
-                yield from load_bc(1)
         ok = True
         for t in range(nt):
-            bst = t % bc_stages
-            if not (ok := (yield ("wait", f"bcfull{bst}", t // bc_stages))):
-                break
             if t > 0 and "w16_s_ready" not in drop:
                 if not (ok := (yield ("wait", "s_ready", t - 1))):
                     break
-            yield ("mma", (f"c{bst}", f"b{bst}"), ("tCB",))
+            for k in range(BOXES):
+                if not (ok := (yield ("wait", f"bcfull{k}", t))):
+                    break
+                yield ("mma", (f"c{k}", f"b{k}"), ("tCB",))
+            if not ok:
+                break
             yield ("commit", "cb_done")
             if t >= 1 and t + 1 < nt:
                 if "w16_yd_par" not in drop:
                     if not (ok := (yield ("wait", f"yd_par{(t - 1) & 1}", (t - 1) >> 1))):
                         break
                 yield from load_x(t + 1)
-                if bc_stages == 2:
-                    yield from load_bc(t + 1)
-            if bc_stages == 1 and t + 1 < nt:
+            if t + 1 < nt:
+                if "w16_cb_done" not in drop:
+                    if not (ok := (yield ("wait", "cb_done", t))):
+                        break
                 if "w16_sc_done" not in drop:
                     if not (ok := (yield ("wait", "sc_done", t))):
                         break
-                yield from load_bc(t + 1)
+                yield from load_bc()
         if not ok:
             for t in range(issued["x"]):
                 yield ("bwait", f"xfull{t & 1}", t >> 1)
             for t in range(issued["bc"]):
-                yield ("bwait", f"bcfull{t % bc_stages}", t // bc_stages)
+                for k in range(BOXES):
+                    yield ("bwait", f"bcfull{k}", t)
         if fin:
             yield ("commit", "fin0")
             yield ("bwait", "fin0", 0)
 
-    def w17():
+    def w17():      # C h_prev, box by box, then S x
+        ok = True
         for t in range(nt):
-            st, bst = t & 1, t % bc_stages
-            if not (yield ("wait", "x_ready", t)):
+            st = t & 1
+            if not (ok := (yield ("wait", f"x_ready{st}", t >> 1))):
                 break
-            if "w17_bcfull" not in drop:
-                if not (yield ("wait", f"bcfull{bst}", t // bc_stages)):
-                    break
-            yield ("mma", (f"c{bst}", "hs"), (f"tYo{st}",))
-            if not (yield ("wait", "s_ready", t)):
+            for k in range(BOXES):
+                if "w17_bcfull" not in drop:
+                    if not (ok := (yield ("wait", f"bcfull{k}", t))):
+                        break
+                yield ("mma", (f"c{k}", "hs"), (f"tYo{st}",))
+            if not ok:
                 break
-            yield ("mma", (f"b{bst}", "wx", "tH"), ("tH",))
             yield ("commit", "sc_done")
-            if yd_bufs == 1 and t > 0 and "w17_e_done" not in drop:
-                if not (yield ("wait", f"e_done{(t - 1) & 1}", (t - 1) >> 1)):
+            if "w17_s_ready" not in drop:
+                if not (ok := (yield ("wait", "s_ready", t))):
                     break
-            yd = f"tYd{st if yd_bufs == 2 else 0}"
-            yield ("mma", ("tS", f"x{st}"), (yd,))
+            if t > 0 and "w17_e_done" not in drop:
+                if not (ok := (yield ("wait", f"e_done{(t - 1) & 1}", (t - 1) >> 1))):
+                    break
+            yield ("mma", ("tS", f"x{st}"), ("tYd",))
             yield ("commit", f"yd_par{st}")
         if fin and nt > 0:
             yield ("commit", "fin1")
             yield ("bwait", "fin1", 0)
 
+    def w18():      # H += B^T (w o x), state rows of boxes 0-1, then 2-3
+        ok = True
+        for t in range(nt):
+            if not (ok := (yield ("wait", f"x_ready{t & 1}", t >> 1))):
+                break
+            if last_partial(t) and "w18_b_zeroed" not in drop:
+                if not (ok := (yield ("wait", "b_zeroed", 0))):
+                    break
+            for mb in range(BOXES // 2):
+                for k in (2 * mb, 2 * mb + 1):
+                    if "w18_bcfull" not in drop:
+                        if not (ok := (yield ("wait", f"bcfull{k}", t))):
+                            break
+                if not ok:
+                    break
+                yield ("mma", (f"b{2 * mb}", f"b{2 * mb + 1}", "wx", f"tH{mb}"), (f"tH{mb}",))
+            if not ok:
+                break
+            yield ("commit", "sc_done")
+        if fin and nt > 0:
+            yield ("commit", "fin2")
+            yield ("bwait", "fin2", 0)
+
     def p_role():
         yield ("write", "tS")
         for t in range(nt):
-            buf, bst = t & 1, t % bc_stages
+            buf = t & 1
             if t >= 2 and "p_e_done" not in drop:
                 if not (yield ("wait", f"e_done{buf}", (t - 2) >> 1)):
                     break
@@ -836,7 +872,8 @@ def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = 
             if not (yield ("wait", "cb_done", t)):
                 break
             if last_partial(t):
-                yield ("write", f"b{bst}")          # rows past the sequence end zeroed
+                yield ("write", *b_all)             # rows past the sequence end zeroed
+                yield ("arrive", "b_zeroed", 8)
             if t > 0 and "p_yd_par" not in drop:
                 if not (yield ("wait", f"yd_par{(t - 1) & 1}", (t - 1) >> 1)):
                     break
@@ -851,35 +888,36 @@ def build_scan1(nt: int, n: int = 128, partial: bool = False, drop: frozenset = 
                 return False
             yield ("read", f"ring{st}")
             if u > 0:
-                yield ("read", "tH")
-            yield ("write", "hs", "tH")
+                yield ("read", "tH0", "tH1")
+            yield ("write", "hs", "tH0", "tH1")
             if not (yield ("wait", f"xfull{st}", u >> 1)):
                 return False
             yield ("read", f"x{st}")
             yield ("write", f"x{st}", "wx")
-            yield ("arrive", "x_ready", 8)
+            yield ("arrive", f"x_ready{st}", 8)
             return True
 
         ok = True
         for k in range(nt + 1):
-            if k < nt:
-                if k > 0 and "e_sc_done" not in drop:
-                    if not (ok := (yield ("wait", "sc_done", k - 1))):
-                        break
-                if not (ok := (yield from prepare(k))):
+            # sc_done of tile k - 1: the state entering tile k is complete, hs and w o x are
+            # free, and C h_prev of tile k - 1 (read by its epilogue) is done
+            if k > 0 and not (k == nt and "e_last_sc_done" in drop) and not (k < nt and "e_sc_done" in drop):
+                if not (ok := (yield ("wait", "sc_done", k - 1))):
                     break
+            if k < nt and not (ok := (yield from prepare(k))):
+                break
             if k == 0:
                 continue
             t = k - 1
             st = t & 1
             if not (ok := (yield ("wait", f"yd_par{st}", t >> 1))):
                 break
-            yield ("read", f"ring{st}", f"tYd{st if yd_bufs == 2 else 0}", f"tYo{st}")
+            yield ("read", f"ring{st}", "tYd", f"tYo{st}")
             yield ("arrive", f"e_done{st}", 8)
         if nt > 0 and ok:
-            yield ("read", "tH")
+            yield ("read", "tH0", "tH1")               # the final state
 
-    for name, gen in (("W16", w16()), ("W17", w17()), ("P", p_role()), ("E", e_role())):
+    for name, gen in (("W16", w16()), ("W17", w17()), ("W18", w18()), ("P", p_role()), ("E", e_role())):
         m.role(name, gen)
     return m
 

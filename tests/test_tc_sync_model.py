@@ -115,15 +115,14 @@ def test_scan3_protocol_has_no_race_deadlock_or_aliasing(partial):
         check(build_scan3, 25, seed=100 + nt, nt=nt, partial=partial)
 
 
-@pytest.mark.parametrize("n", [128, 256])
 @pytest.mark.parametrize("partial", [False, True])
-def test_scan1_protocol_has_no_race_deadlock_or_aliasing(n, partial):
+def test_scan1_protocol_has_no_race_deadlock_or_aliasing(partial):
     for nt in TILES:
-        check(build_scan1, 25, seed=200 + nt, nt=nt, n=n, partial=partial)
+        check(build_scan1, 25, seed=200 + nt, nt=nt, partial=partial)
 
 
 def _caught(build, drop, **kw):
-    for nt in (3, 5, 8):
+    for nt in (1, 3, 5, 8):
         for partial in (False, True):
             try:
                 check(build, 40, seed=nt, nt=nt, partial=partial, drop=frozenset([drop]), **kw)
@@ -140,19 +139,23 @@ NEEDED = [
     (build_scan3, {}, "p_y_full", "tS"),
     (build_scan3, {}, "y_store_wait", "hs"),
     (build_scan3, {}, "e_stg_free", "hs"),
-    (build_scan1, {"n": 128}, "w16_s_ready", "tCB"),
-    (build_scan1, {"n": 128}, "w16_yd_par", "x"),
-    (build_scan1, {"n": 256}, "w16_sc_done", "b0"),
-    (build_scan1, {"n": 256}, "w17_e_done", "tYd0"),
-    (build_scan1, {"n": 128}, "w17_bcfull", "c0"),
-    (build_scan1, {"n": 256}, "w17_bcfull", "c0"),
-    (build_scan1, {"n": 256}, "p_e_done", "ring"),
-    (build_scan1, {"n": 256}, "p_yd_par", "tS"),
-    (build_scan1, {"n": 256}, "e_sc_done", ""),
+    (build_scan1, {}, "w16_s_ready", "tCB"),
+    (build_scan1, {}, "w16_yd_par", "x"),
+    (build_scan1, {}, "w16_sc_done", ""),
+    (build_scan1, {}, "w16_cb_done", ""),
+    (build_scan1, {}, "w17_bcfull", "c"),
+    (build_scan1, {}, "w18_bcfull", "b"),
+    (build_scan1, {}, "w18_b_zeroed", "b"),
+    (build_scan1, {}, "w17_s_ready", "tS"),
+    (build_scan1, {}, "w17_e_done", "tYd"),
+    (build_scan1, {}, "p_e_done", "ring"),
+    (build_scan1, {}, "p_yd_par", "tS"),
+    (build_scan1, {}, "e_sc_done", ""),
+    (build_scan1, {}, "e_last_sc_done", "tH"),
 ]
 
 
-@pytest.mark.parametrize("build,kw,drop,buf", NEEDED, ids=[f"{b.__name__}-{kw.get('n', 128)}-{d}" for b, kw, d, _ in NEEDED])
+@pytest.mark.parametrize("build,kw,drop,buf", NEEDED, ids=[f"{b.__name__}-{d}" for b, kw, d, _ in NEEDED])
 def test_removing_a_needed_wait_is_caught(build, kw, drop, buf):
     msg = _caught(build, drop, **kw)
     assert msg is not None and "race on " + buf in msg, msg
@@ -161,13 +164,10 @@ def test_removing_a_needed_wait_is_caught(build, kw, drop, buf):
 def test_waits_implied_by_other_waits():
     """Waits the kernels keep although another wait already implies them:
     k_tc_scan3's W18 y_full wait (its full-barrier wait follows W16's y_full wait), W17's
-    e_done wait (hs_ready follows E's stg_free wait, which follows Y's read of the Y buffer),
-    and, with one B/C stage, the first-generation W16's s_ready wait (the stage's reload
-    waited for sc_done, which follows s_ready).  The tensor-core drains before exit (fin)
-    matter only on the timeout path (tested below)."""
+    e_done wait (hs_ready follows E's stg_free wait, which follows Y's read of the Y buffer).
+    The tensor-core drains before exit (fin) matter only on the timeout path (tested below)."""
     for build, kw, drop in ((build_scan3, {}, "w18_y_full"), (build_scan3, {}, "w17_e_done"),
-                            (build_scan3, {}, "w17_fin"), (build_scan3, {}, "w18_fin"),
-                            (build_scan1, {"n": 256}, "w16_s_ready")):
+                            (build_scan3, {}, "w17_fin"), (build_scan3, {}, "w18_fin")):
         assert _caught(build, drop, **kw) is None, drop
 
 
@@ -196,12 +196,11 @@ def test_scan3_needs_each_of_its_drains(drain):
     assert "in flight" in (_faults(build_scan3, frozenset([drain])) or "")
 
 
-@pytest.mark.parametrize("n", [128, 256])
-def test_scan1_timeout_path_needs_its_mma_drains(n):
+def test_scan1_timeout_path_needs_its_mma_drains():
     """The first-generation kernel's MMA-issuing threads drain their tensor-core work before
     exit; without that, a timeout can leave MMAs writing TMEM after it is freed."""
-    assert _faults(build_scan1, n=n) is None
-    assert "in flight" in (_faults(build_scan1, n=n, fin=False) or "")
+    assert _faults(build_scan1) is None
+    assert "in flight" in (_faults(build_scan1, fin=False) or "")
 
 
 def test_planned_zeroing_of_b_rows_past_a_sequence_end():
