@@ -61,6 +61,9 @@ def parse():
                     help="with --mixer: an fp32 all-reduce instead of the quantised one")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (small cases for profiling; not a bench line)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count, a multiple of its groups (small cases for "
+                         "profiling; not a bench line)")
     return ap.parse_args()
 
 
@@ -69,6 +72,10 @@ def workload_of(args):
     w = inputs.WORKLOADS[args.workload]
     if args.batch is not None and not w.packed_nseqs:
         w = inputs.scaled(w, batch=args.batch)
+    if args.heads is not None:
+        if args.heads <= 0 or args.heads % w.ngroups:
+            raise SystemExit(f"--heads must be a positive multiple of the {w.ngroups} groups")
+        w = inputs.scaled(w, nheads=args.heads)
     return w
 
 
