@@ -242,12 +242,17 @@ SSD_API int ssd_dequant_chunks(int64_t T, int64_t D, int64_t ranks, int dtype, c
  *   dfinal    (S, H, N, P)  float32, NULL = zero
  * chunk is validated as in the forward; the result does not depend on it.
  * Every output is overwritten (none is read).  Gradient buffers must not
- * overlap the inputs or each other.  Computed on CUDA cores in fp32 with
- * checkpoints of the state every 64 tokens; workspace (stream-ordered, from
- * the library's pool) is 4 N P H (blocks + 64 S) + 8 b L G N bytes, blocks =
- * the number of 64-token blocks over all sequences.  Supported: headdim
- * dividing 256 and headdim * dstate in {256, 512, ..., 8192}; other shapes
- * return SSD_ERR_UNSUPPORTED.
+ * overlap the inputs or each other; dy is 16-byte aligned like x (both
+ * SSD_ERR_SHAPE otherwise).  blocks = the number of 64-token blocks over all
+ * sequences.  headdim 64 with dstate 64 or 128: the block decomposition over
+ * 64-token chunks (per-chunk terms, a sequential pass over chunk states,
+ * per-chunk gradients; for bf16 the matrix products on the tensor cores with
+ * fp16 operands and fp32 accumulation), workspace 8 N P H blocks + 4 H blocks
+ * bytes.  Other shapes: CUDA cores in fp32 with checkpoints of the state every
+ * 64 tokens, workspace 4 N P H (blocks + 64 S) + 8 b L G N bytes; supported
+ * there are headdim dividing 256 and headdim * dstate in {256, 512, ...,
+ * 8192}, other shapes return SSD_ERR_UNSUPPORTED.  Workspace is stream-ordered,
+ * from the library's pool (each piece rounded up to 256 bytes).
  */
 SSD_API int ssd_chunk_scan_bwd(const ssd_dims* dims, const void* x, const void* dt, const float* dt_bias,
                                const float* A, const void* B, const void* C, const float* D,

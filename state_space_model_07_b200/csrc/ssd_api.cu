@@ -539,6 +539,7 @@ extern "C" int ssd_chunk_scan_bwd(const ssd_dims* dims, const void* x, const voi
     const size_t es = a.dtype == SSD_BF16 ? 2 : 4;
     if (ntok > 0) {
         if (!dy || !ddt || !dB || !dC) return fail(SSD_ERR_NULL, "dy, ddt, dB and dC are required");
+        if (!aligned16(dy)) return fail(SSD_ERR_SHAPE, "dy must be 16-byte aligned");
         const size_t nx = (size_t)ntok * a.H * a.P * es, nbc = (size_t)ntok * a.G * a.N * es;
         const size_t ndt = (size_t)ntok * a.H * es;
         const void* outs[4] = {dx, ddt, dB, dC};

@@ -929,7 +929,7 @@ __device__ __forceinline__ void mma_tile_h(float (&acc)[MT][NT][4], const __half
                                            int r0, int c0, int K) {
     static_assert(NT % 2 == 0, "B fragments come two tiles at a time");
     const int lane = threadIdx.x & 31, m = lane >> 3, rr = lane & 7;
-#pragma unroll 1
+#pragma unroll 4
     for (int k = 0; k < K; k += 16) {
         uint32_t af[MT][4], bf[NT][2];
 #pragma unroll
@@ -981,6 +981,28 @@ __device__ __forceinline__ void load_rows_h(__half* dst, const __nv_bfloat16* sr
     }
 }
 
+// 16-byte asynchronous copy global -> shared (cached at L2 only), and the wait for all of this
+// thread's copies committed so far.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(a), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Layout of k_bwd_grads_h's dynamic shared memory: the fp16 tiles, the fp32 C B^T and per-token
+// arrays, then (16-byte aligned) the staging area of the next head's inputs.
+template <int N>
+constexpr size_t grads_h_stage_offset() {
+    return (2 * (2 * kQb * N + 2 * kQb * kPb + 2 * N * kPb + 2 * kQb * kQb) + sizeof(float) * (kQb * kQb + 9 * kQb + 4) +
+            15) & ~(size_t)15;
+}
+
+template <int N>
+constexpr size_t grads_h_smem() {
+    return grads_h_stage_offset<N>() + 2 * 2 * kQb * kPb + 2 * sizeof(float) * N * kPb;
+}
+
 // 512 threads (16 warps) per block: the 64 x 64 products in 16 x 16 warp tiles, the 64 x N
 // products in 16 x (N / 4) warp tiles.
 constexpr int kGradThreads = 512;
@@ -1010,6 +1032,13 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     float* rowZ = rowRd + Q;
     float* rowY = rowZ + Q;
     float* sred = rowY + Q;           // [0] <dh_end, h_prev>, [1] sum dy x, [2] last cs
+    // staging for the next head's inputs, filled by asynchronous copies while this head computes:
+    // x and dy as they are in memory (bf16 rows), the two fp32 states
+    uint8_t* stg = smraw + grads_h_stage_offset<N>();
+    T* stX = reinterpret_cast<T*>(stg);
+    T* stDY = stX + Q * P;
+    float* stHP = reinterpret_cast<float*>(stDY + Q * P);
+    float* stDH = stHP + N * P;
     const int H = p.H, G = p.G, HG = H / G;
     const int tid = threadIdx.x, lane = tid & 31;
     const int64_t f = blockIdx.x / G;
@@ -1019,6 +1048,27 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     const int q = (int)(r.t1 - r.t0);
     const int64_t tok0 = r.row * p.si.L + r.t0;
     const T* dtg = (const T*)p.dt;
+    // copies of head hh's x, dy rows (those inside the chunk) and states into the staging area
+    auto stage = [&](int hh) {
+        const int h = g * HG + hh;
+        const T* xs = (const T*)p.x + (tok0 * H + h) * P;
+        const T* dys = (const T*)p.dy + (tok0 * H + h) * P;
+        for (int e = tid; e < Q * P / 8; e += blockDim.x) {
+            const int r = e / (P / 8), c8 = e % (P / 8);
+            if (r < q) {
+                cp_async16(stX + r * P + 8 * c8, xs + (int64_t)r * H * P + 8 * c8);
+                cp_async16(stDY + r * P + 8 * c8, dys + (int64_t)r * H * P + 8 * c8);
+            }
+        }
+        const float* hp = p.S + ((int64_t)f * H + h) * N * P;
+        const float* dh = p.T + ((int64_t)f * H + h) * N * P;
+        for (int e = tid; e < N * P / 4; e += blockDim.x) {
+            cp_async16(stHP + 4 * e, hp + 4 * e);
+            cp_async16(stDH + 4 * e, dh + 4 * e);
+        }
+        cp_async_commit();
+    };
+    stage(0);
     load_rows_h(sB, (const T*)p.B + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
     load_rows_h(sC, (const T*)p.C + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
     __syncthreads();
@@ -1041,18 +1091,29 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     for (int hh = 0; hh < HG; ++hh) {
         const int h = g * HG + hh;
         const float bias = p.dt_bias ? p.dt_bias[h] : 0.f, Ah = p.A[h], Dh = p.D ? p.D[h] : 0.f;
-        load_rows_h(sX, (const T*)p.x + (tok0 * H + h) * P, (int64_t)H * P, q, Q, P);
-        load_rows_h(sDY, (const T*)p.dy + (tok0 * H + h) * P, (int64_t)H * P, q, Q, P);
+        // this head's inputs have landed in the staging area (every thread's copies)
+        cp_async_wait_all();
+        __syncthreads();
+        for (int e = tid; e < Q * P / 8; e += blockDim.x) {
+            const int r = e / (P / 8), c8 = e % (P / 8);
+            uint4 ox = make_uint4(0u, 0u, 0u, 0u), od = ox;
+            if (r < q) {
+                ox = bf16x8_to_f16x8_bwd(*reinterpret_cast<const uint4*>(stX + r * P + 8 * c8));
+                od = bf16x8_to_f16x8_bwd(*reinterpret_cast<const uint4*>(stDY + r * P + 8 * c8));
+            }
+            *reinterpret_cast<uint4*>(hsw8(sX, r, c8, P)) = ox;
+            *reinterpret_cast<uint4*>(hsw8(sDY, r, c8, P)) = od;
+        }
         float hpdh = 0.f;   // <h_prev, dh_end> in fp32 from the fp32 states
         {
-            const float* hp = p.S + ((int64_t)f * H + h) * N * P;
-            const float* dh = p.T + ((int64_t)f * H + h) * N * P;
+            const float* hp = stHP;
+            const float* dh = stDH;
             for (int e = tid; e < N * P / 8; e += blockDim.x) {
                 const int n = e / (P / 8), c8 = e % (P / 8);
-                const float4 a0 = *reinterpret_cast<const float4*>(hp + (int64_t)n * P + 8 * c8);
-                const float4 a1 = *reinterpret_cast<const float4*>(hp + (int64_t)n * P + 8 * c8 + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(dh + (int64_t)n * P + 8 * c8);
-                const float4 b1 = *reinterpret_cast<const float4*>(dh + (int64_t)n * P + 8 * c8 + 4);
+                const float4 a0 = *reinterpret_cast<const float4*>(hp + n * P + 8 * c8);
+                const float4 a1 = *reinterpret_cast<const float4*>(hp + n * P + 8 * c8 + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(dh + n * P + 8 * c8);
+                const float4 b1 = *reinterpret_cast<const float4*>(dh + n * P + 8 * c8 + 4);
                 *reinterpret_cast<uint4*>(hsw8(sHP, n, c8, P)) =
                     make_uint4(h2pack(a0.x, a0.y), h2pack(a0.z, a0.w), h2pack(a1.x, a1.y), h2pack(a1.z, a1.w));
                 *reinterpret_cast<uint4*>(hsw8(sDH, n, c8, P)) =
@@ -1077,6 +1138,9 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
             }
         }
         __syncthreads();
+        // every thread is done with the staging area: the next head's copies fly while this one
+        // computes
+        if (hh + 1 < HG) stage(hh + 1);
         {
             // x and dy share one swizzle, so element e is the same (row, column) in both
             float a1 = hpdh, a2 = 0.f;
@@ -1295,11 +1359,6 @@ __global__ void __launch_bounds__(256) k_bwd_terms_h(const ChunkedBwd p) {
         __syncthreads();
     }
     if (threadIdx.x == 0) p.E[f * H + h] = expf(slast);
-}
-
-template <int N>
-constexpr size_t grads_h_smem() {
-    return 2 * (2 * kQb * N + 2 * kQb * kPb + 2 * N * kPb + 2 * kQb * kQb) + sizeof(float) * (kQb * kQb + 9 * kQb + 4);
 }
 
 template <int N>
