@@ -286,13 +286,17 @@ bool bwd_chunked(const ScanArgs& a) { return a.P == kPb && (a.N == 64 || a.N == 
 // the chunk's last cs; tokens past q get d = 0.
 template <typename T>
 __device__ __forceinline__ void chunk_decay(const T* dt, int64_t tok0, int H, int h, int q, float bias, float Ah,
-                                            float* sd, float* sz, float* scs, float* slast) {
+                                            float* sd, float* sz, float* scs, float* slast);
+
+// The same from raw dt values already loaded (tokens 2 lane and 2 lane + 1; ignored past q).
+__device__ __forceinline__ void chunk_decay_raw(const float (&raw)[2], int q, float bias, float Ah, float* sd,
+                                                float* sz, float* scs, float* slast) {
     const int lane = threadIdx.x & 31;
     float dd[2], zz[2], cc[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         const int j = 2 * lane + k;
-        zz[k] = j < q ? to_f<T>(dt[(tok0 + j) * H + h]) + bias : 0.f;
+        zz[k] = j < q ? raw[k] + bias : 0.f;
         dd[k] = j < q ? softplus_f(zz[k]) : 0.f;
     }
     cc[0] = dd[0] * Ah;
@@ -311,6 +315,25 @@ __device__ __forceinline__ void chunk_decay(const T* dt, int64_t tok0, int H, in
         scs[2 * lane + k] = excl + cc[k];
     }
     if (lane == 31) *slast = incl;   // tokens past q add 0, so this is cs of token q - 1
+}
+
+// dt of tokens 2 lane and 2 lane + 1 of the chunk (0 past q).
+template <typename T>
+__device__ __forceinline__ void load_dt2(float (&raw)[2], const T* dt, int64_t tok0, int H, int h, int q) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int j = 2 * lane + k;
+        raw[k] = j < q ? to_f<T>(dt[(tok0 + j) * H + h]) : 0.f;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void chunk_decay(const T* dt, int64_t tok0, int H, int h, int q, float bias, float Ah,
+                                            float* sd, float* sz, float* scs, float* slast) {
+    float raw[2];
+    load_dt2<T>(raw, dt, tok0, H, h, q);
+    chunk_decay_raw(raw, q, bias, Ah, sd, sz, scs, slast);
 }
 
 // acc[i][j] += sum_k A(r0 + i, k) Bm(k, c0 + j), A(r, k) = A[r ar + k ak], Bm(k, c) = Bm[k bk + c bc],
@@ -1069,6 +1092,9 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         cp_async_commit();
     };
     stage(0);
+    // warp 0 holds the raw dt of the head it prepares next (loaded a head ahead)
+    float dt_raw[2] = {0.f, 0.f};
+    if (tid < 32) load_dt2<T>(dt_raw, dtg, tok0, H, g * HG, q);
     load_rows_h(sB, (const T*)p.B + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
     load_rows_h(sC, (const T*)p.C + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
     __syncthreads();
@@ -1127,7 +1153,8 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         }
         if (tid < 2) sred[tid] = 0.f;      // sred[2] is written by the decay scan below
         if (tid < 32) {
-            chunk_decay<T>(dtg, tok0, H, h, q, bias, Ah, sd, sz, scs, &sred[2]);
+            chunk_decay_raw(dt_raw, q, bias, Ah, sd, sz, scs, &sred[2]);
+            if (hh + 1 < HG) load_dt2<T>(dt_raw, dtg, tok0, H, h + 1, q);
             __syncwarp();
             const float last = sred[2];
 #pragma unroll
