@@ -397,6 +397,12 @@ __device__ __forceinline__ uint32_t h2pack(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// The fp16 pair of what the packed pair `hi` (the fp16 roundings of a and b) leaves of a and b.
+__device__ __forceinline__ uint32_t h2lo(uint32_t hi, float a, float b) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&hi);
+    return h2pack(a - __low2float(h), b - __high2float(h));
+}
+
 template <bool K1>
 __device__ __forceinline__ uint32_t pair_k(const float* M, int64_t at, int kstride) {
     if (K1) {
@@ -1017,7 +1023,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // arrays, then (16-byte aligned) the staging area of the next head's inputs.
 template <int N>
 constexpr size_t grads_h_stage_offset() {
-    return (2 * (2 * kQb * N + 2 * kQb * kPb + 2 * N * kPb + 2 * kQb * kQb) + sizeof(float) * (kQb * kQb + 9 * kQb + 4) +
+    return (2 * (2 * kQb * N + 2 * kQb * kPb + 3 * N * kPb + 3 * kQb * kQb) + sizeof(float) * (kQb * kQb + 9 * kQb + 4) +
             15) & ~(size_t)15;
 }
 
@@ -1044,7 +1050,12 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     __half* sDH = sHP + N * P;                       // [N][P] adjoint of the state leaving it
     __half* sW = sDH + N * P;                        // [Q][Q]
     __half* sK = sW + Q * Q;                         // [Q][Q]
-    float* sCB = reinterpret_cast<float*>(sK + Q * Q);   // [Q][Q] C_j . B_i in fp32 (it enters the decays)
+    // dx = D dy + W^T dy + u o (B dh_end): its last two terms can each be many times dx itself
+    // and cancel, so W and dh_end enter those products as fp16 pairs hi + lo (lo = the fp16
+    // rounding of what hi leaves), which makes them exact to about 2^-22
+    __half* sDHl = sK + Q * Q;                       // [N][P]
+    __half* sWl = sDHl + N * P;                      // [Q][Q]
+    float* sCB = reinterpret_cast<float*>(sWl + Q * Q);   // [Q][Q] C_j . B_i in fp32 (it enters the decays)
     float* sd = sCB + Q * Q;
     float* sz = sd + Q;
     float* scs = sz + Q;
@@ -1142,8 +1153,12 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                 const float4 b1 = *reinterpret_cast<const float4*>(dh + n * P + 8 * c8 + 4);
                 *reinterpret_cast<uint4*>(hsw8(sHP, n, c8, P)) =
                     make_uint4(h2pack(a0.x, a0.y), h2pack(a0.z, a0.w), h2pack(a1.x, a1.y), h2pack(a1.z, a1.w));
-                *reinterpret_cast<uint4*>(hsw8(sDH, n, c8, P)) =
+                const uint4 dhi =
                     make_uint4(h2pack(b0.x, b0.y), h2pack(b0.z, b0.w), h2pack(b1.x, b1.y), h2pack(b1.z, b1.w));
+                *reinterpret_cast<uint4*>(hsw8(sDH, n, c8, P)) = dhi;
+                *reinterpret_cast<uint4*>(hsw8(sDHl, n, c8, P)) =
+                    make_uint4(h2lo(dhi.x, b0.x, b0.y), h2lo(dhi.y, b0.z, b0.w), h2lo(dhi.z, b1.x, b1.y),
+                               h2lo(dhi.w, b1.z, b1.w));
                 hpdh += a0.x * b0.x + a0.y * b0.y + a0.z * b0.z + a0.w * b0.w + a1.x * b1.x + a1.y * b1.y +
                         a1.z * b1.z + a1.w * b1.w;
             }
@@ -1196,7 +1211,10 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                     // the fast exponential: this path's operands are fp16 anyway
                     const float L = (i <= j && j < q) ? __expf(scs[j] - scs[i]) : 0.f;
                     const float cb = sCB[j * Q + i], di = sd[i], dyx = acc[0][nt][e];
-                    sW[hsw(j, i, Q)] = __float2half_rn(cb * L * di);
+                    const float wv = cb * L * di;
+                    const __half whi = __float2half_rn(wv);
+                    sW[hsw(j, i, Q)] = whi;
+                    sWl[hsw(j, i, Q)] = __float2half_rn(wv - __half2float(whi));
                     sK[hsw(j, i, Q)] = __float2half_rn(L * dyx * di);
                     const float R = cb * dyx * L;
                     rrow[e >> 1] += R * di;
@@ -1216,7 +1234,9 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
             zero_frag(bd);
             zero_frag(wd);
             mma_tile_h<1, 2, true, false>(bd, sB, N, sDH, P, r64, c64, N);
+            mma_tile_h<1, 2, true, false>(bd, sB, N, sDHl, P, r64, c64, N);
             mma_tile_h<1, 2, false, false>(wd, sW, Q, sDY, P, r64, c64, Q);
+            mma_tile_h<1, 2, false, false>(wd, sWl, Q, sDY, P, r64, c64, Q);
             T* dxg = (T*)p.dx + (tok0 * H + h) * P;
             float z[2] = {0.f, 0.f};
 #pragma unroll

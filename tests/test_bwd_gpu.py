@@ -16,7 +16,7 @@ import torch
 import oracle
 import state_space_model_07_b200 as ssd
 from state_space_model_07_b200 import inputs
-from tests.helpers import TOL, assert_close, to_cpu
+from tests.helpers import TOL, assert_close, head_slice, to_cpu
 
 pytestmark = pytest.mark.gpu
 W = inputs.WORKLOADS
@@ -101,3 +101,36 @@ def test_backward_refuses_unsupported_shapes_before_launching():
     with pytest.raises(ssd.SsdError) as e:
         ssd.chunk_scan_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], dy, chunk=16)
     assert e.value.code == 5
+
+
+def test_backward_full_size_sampled_heads():
+    """The bench-shaped layer at full size (b8 L4096 H80 P64 N128, one group), in the launch
+    configuration the benchmark times.  Each head's recurrence is independent, so the oracle
+    recomputes sampled heads whole (all rows and tokens): their dx, ddt, d init_state and the
+    per-head sums dt_bias, A, D.  dB and dC sum all 80 heads and are checked as finite."""
+    w = W["mamba2_2.7b_layer"]
+    d = inputs.make_inputs(w, "cuda")
+    dy, dfinal = _upstream(d, w, 11)
+    got = ssd.chunk_scan_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], dy, dt_bias=d["dt_bias"], D=d["D"],
+                             init_state=d["init_state"], chunk=w.chunk, dfinal=dfinal)
+    torch.cuda.synchronize()
+    for k, v in got.items():
+        assert torch.isfinite(v.float()).all(), f"d{k} has non-finite entries"
+    tol = TOL[d["x"].dtype]
+    sums = {k: [] for k in ("dt_bias", "A", "D")}
+    heads = (0, 41, 79)
+    for h in heads:
+        hd = to_cpu(head_slice(d, h, w.nheads, w.ngroups))
+        ref = oracle.ssd_scan_bwd(hd["x"], hd["dt"], hd["A"], hd["B"], hd["C"], dy[:, :, h:h + 1].cpu(),
+                                  dt_bias=hd["dt_bias"], D=hd["D"], init_state=hd["init_state"],
+                                  dfinal=dfinal[:, h:h + 1].cpu())
+        assert_close(got["x"][:, :, h:h + 1], ref["x"], tol, f"dx head {h}")
+        assert_close(got["dt"][:, :, h:h + 1], ref["dt"], tol, f"ddt head {h}")
+        assert_close(got["init_state"][:, h:h + 1], ref["init_state"], tol, f"dinit head {h}")
+        for k in sums:
+            sums[k].append(float(ref[k][0]))
+    # sums over 32 768 tokens, relative to the largest of their kind (as in _check)
+    for k, refs in sums.items():
+        scale = 1.0 + max(abs(r) for r in refs)
+        err = max(abs(float(got[k][h]) - r) for h, r in zip(heads, refs)) / scale
+        assert err <= tol, f"d{k}: max |d| / (1 + max |ref|) = {err:.3e} > {tol:.1e}"
