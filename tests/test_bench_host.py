@@ -1,6 +1,8 @@
 """Host-side pieces of bench.py that need no GPU."""
 import json
 
+import pytest
+
 import bench
 
 
@@ -69,3 +71,17 @@ def test_scan_hash_covers_the_measured_kernel_not_the_d_state_256_one(tmp_path, 
     j = src.index("{", src.index("k_tc_scan3(const __grid_constant__"))
     f.write_text(src[:j + 1] + "\n    int unused_probe = 0;\n" + src[j + 1:])
     assert bench.kernel_source_sha("tc_scan") != h0
+
+
+def test_profiling_overrides_shrink_the_workload_and_reject_bad_heads():
+    import argparse
+    import bench
+    ns = lambda **kw: argparse.Namespace(**dict({"workload": "packed_varlen", "batch": None, "heads": None}, **kw))
+    w = bench.workload_of(ns(heads=16))
+    assert (w.nheads, w.ngroups, w.dstate, w.packed_nseqs) == (16, 4, 256, 16)
+    w = bench.workload_of(ns(workload="mamba2_2.7b_layer", batch=2))
+    assert (w.batch, w.seqlen, w.nheads) == (2, 4096, 80)
+    assert bench.workload_of(ns(batch=2)).batch == 1          # packed input has one row
+    for bad in (0, 6, -4):
+        with pytest.raises(SystemExit):
+            bench.workload_of(ns(heads=bad))
