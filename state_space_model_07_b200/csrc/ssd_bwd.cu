@@ -1359,8 +1359,12 @@ __global__ void __launch_bounds__(256) k_bwd_terms_h(const ChunkedBwd p) {
     using T = __nv_bfloat16;
     constexpr int P = kPb, Q = kQb;
     extern __shared__ __align__(16) uint8_t smraw[];
-    __half* sM = reinterpret_cast<__half*>(smraw);   // [Q][N]: B, then C
-    __half* sV = sM + Q * N;                         // [Q][P]: u_j x_j, then e_j dy_j
+    // both products' operands at once, so that every load of the block is in flight together:
+    // [0] B with u_j x_j -> S, [1] C with e_j dy_j -> T
+    __half* sM0 = reinterpret_cast<__half*>(smraw);  // [Q][N]
+    __half* sM1 = sM0 + Q * N;
+    __half* sV0 = sM1 + Q * N;                       // [Q][P]
+    __half* sV1 = sV0 + Q * P;
     __shared__ float sd[kQb], sz[kQb], scs[kQb], slast;
     const int H = p.H, G = p.G;
     const int64_t f = blockIdx.x / H;
@@ -1371,29 +1375,43 @@ __global__ void __launch_bounds__(256) k_bwd_terms_h(const ChunkedBwd p) {
     const int64_t tok0 = r.row * p.si.L + r.t0;
     if (threadIdx.x < 32)
         chunk_decay<T>((const T*)p.dt, tok0, H, h, q, p.dt_bias ? p.dt_bias[h] : 0.f, p.A[h], sd, sz, scs, &slast);
+    load_rows_h(sM0, (const T*)p.B + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
+    load_rows_h(sM1, (const T*)p.C + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
+    // x and dy rows as they are (bf16 -> fp16 exactly); their weights need the decay scan
+    const T* xv = (const T*)p.x + (tok0 * H + h) * P;
+    const T* dyv = (const T*)p.dy + (tok0 * H + h) * P;
+    uint4 vx[Q * (P / 8) / 256], vd[Q * (P / 8) / 256];
+#pragma unroll
+    for (int k = 0; k < Q * (P / 8) / 256; ++k) {
+        const int e = threadIdx.x + 256 * k, j = e / (P / 8), c8 = e % (P / 8);
+        vx[k] = vd[k] = make_uint4(0u, 0u, 0u, 0u);
+        if (j < q) {
+            vx[k] = *reinterpret_cast<const uint4*>(xv + (int64_t)j * H * P + 8 * c8);
+            vd[k] = *reinterpret_cast<const uint4*>(dyv + (int64_t)j * H * P + 8 * c8);
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < Q * (P / 8) / 256; ++k) {
+        const int e = threadIdx.x + 256 * k, j = e / (P / 8), c8 = e % (P / 8);
+        const float wu = j < q ? expf(slast - scs[j]) * sd[j] : 0.f, we = j < q ? expf(scs[j]) : 0.f;
+        auto cv = [](uint32_t u, float w) {
+            return h2pack(w * __uint_as_float(u << 16), w * __uint_as_float(u & 0xffff0000u));
+        };
+        *reinterpret_cast<uint4*>(hsw8(sV0, j, c8, P)) =
+            make_uint4(cv(vx[k].x, wu), cv(vx[k].y, wu), cv(vx[k].z, wu), cv(vx[k].w, wu));
+        *reinterpret_cast<uint4*>(hsw8(sV1, j, c8, P)) =
+            make_uint4(cv(vd[k].x, we), cv(vd[k].y, we), cv(vd[k].z, we), cv(vd[k].w, we));
+    }
     __syncthreads();
     constexpr int MT = N / 64;
     const int warp = threadIdx.x >> 5;
     const int n0 = 16 * MT * (warp >> 1), c0 = 32 * (warp & 1);
+#pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
-        // pass 0: B with u and x -> S; pass 1: C with e and dy -> T
-        load_rows_h(sM, (const T*)(pass == 0 ? p.B : p.C) + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
-        const T* vec = (const T*)(pass == 0 ? p.x : p.dy) + (tok0 * H + h) * P;
-        for (int e = threadIdx.x; e < Q * (P / 8); e += blockDim.x) {
-            const int j = e / (P / 8), c8 = e % (P / 8);
-            uint4 o = make_uint4(0u, 0u, 0u, 0u);
-            if (j < q) {
-                const float w = pass == 0 ? expf(slast - scs[j]) * sd[j] : expf(scs[j]);
-                const uint4 v = *reinterpret_cast<const uint4*>(vec + (int64_t)j * H * P + 8 * c8);
-                auto cv = [&](uint32_t u) { return h2pack(w * __uint_as_float(u << 16), w * __uint_as_float(u & 0xffff0000u)); };
-                o = make_uint4(cv(v.x), cv(v.y), cv(v.z), cv(v.w));
-            }
-            *reinterpret_cast<uint4*>(hsw8(sV, j, c8, P)) = o;
-        }
-        __syncthreads();
         float acc[MT][4][4];
         zero_frag(acc);
-        mma_tile_h<MT, 4, false, false>(acc, sM, N, sV, P, n0, c0, Q);
+        mma_tile_h<MT, 4, false, false>(acc, pass == 0 ? sM0 : sM1, N, pass == 0 ? sV0 : sV1, P, n0, c0, Q);
         float* out = (pass == 0 ? p.S : p.T) + ((int64_t)f * H + h) * N * P;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
@@ -1403,7 +1421,6 @@ __global__ void __launch_bounds__(256) k_bwd_terms_h(const ChunkedBwd p) {
                 for (int e = 0; e < 4; e += 2)
                     *reinterpret_cast<float2*>(out + (int64_t)frag_row(n0, mt, e) * P + frag_col(c0, nt, e)) =
                         make_float2(acc[mt][nt][e], acc[mt][nt][e + 1]);
-        __syncthreads();
     }
     if (threadIdx.x == 0) p.E[f * H + h] = expf(slast);
 }
@@ -1423,7 +1440,7 @@ void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
     {
         ProfScope ps(K_SCAN_BWD, st);
         if constexpr (sizeof(T) == 2) {
-            const size_t sm_h = 2 * (kQb * N + kQb * kPb);
+            const size_t sm_h = 2 * 2 * (kQb * N + kQb * kPb);
             cudaFuncSetAttribute(k_bwd_terms_h<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_h);
             k_bwd_terms_h<N><<<(unsigned)(chunks * p.H), 256, sm_h, st>>>(p);
         } else {
