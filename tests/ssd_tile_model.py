@@ -41,10 +41,38 @@ def _round(a, kind):
 _FP8 = {"e4m3": (torch.float8_e4m3fn, 448.0), "e5m2": (torch.float8_e5m2, 57344.0)}
 
 
+# Microscaled fp8 (the OCP MX formats that the sm_100 block-scaled MMAs take): one power-of-two
+# scale per 32 consecutive elements along the contracted dimension, 2^(floor(log2 amax) - emax)
+# with emax the element format's largest exponent (8 for e4m3, 15 for e5m2); elements that land
+# above the format's largest value saturate to it.
+_MX = {"mxe4m3": ("e4m3", 8), "mxe5m2": ("e5m2", 15)}
+
+
+def _round_mx(a, kind, axis):
+    fmt, emax = _MX[kind]
+    dt, top = _FP8[fmt]
+    m = np.moveaxis(np.asarray(a, dtype=np.float64), axis, -1)
+    k = m.shape[-1]
+    pad = (-k) % 32
+    if pad:
+        m = np.concatenate([m, np.zeros(m.shape[:-1] + (pad,))], axis=-1)
+    blk = m.reshape(m.shape[:-1] + (-1, 32))
+    amax = np.max(np.abs(blk), axis=-1, keepdims=True)
+    e = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - emax, 0.0)
+    scale = np.exp2(e)
+    q = np.clip(blk / scale, -top, top)
+    t = torch.from_numpy(np.ascontiguousarray(q, dtype=np.float32)).to(dt).to(torch.float64).numpy()
+    out = (t * scale).reshape(m.shape)[..., :k]
+    return np.moveaxis(out, -1, axis)
+
+
 def _round_op(a, kind, axis):
     """Rounds one GEMM operand.  fp8 kinds carry one scale per slice along `axis` (the
     contracted dimension: a row of A, a column of B), as a scaled fp8 MMA would: the scales
-    multiply back in its epilogue."""
+    multiply back in its epilogue.  mx kinds carry one power-of-two scale per 32 elements of
+    that slice (block scaling)."""
+    if kind in _MX:
+        return _round_mx(a, kind, axis)
     if kind not in _FP8:
         return _round(a, kind)
     dt, top = _FP8[kind]
@@ -82,7 +110,8 @@ def tile_form(x, dt, A, B, C, dt_bias=None, D=None, init_state=None, rounding=No
 
     `operands` (with rounding="kernel") overrides the operand type of single GEMMs: keys "cb"
     (C B^T), "state" (B^T (w o x)), "out" (C' h_prev), "diag" (S x); values "f16", "bf16",
-    "e4m3", "e5m2" (fp8 with one scale per row of A and per column of B).
+    "e4m3", "e5m2" (fp8 with one scale per row of A and per column of B), "mxe4m3", "mxe5m2" (fp8
+    with one power-of-two scale per 32 elements along the contracted dimension).
 
     `stats` (a dict) collects the largest magnitude of each thread-made tensor-core operand
     ("S", "h_prev", "wx", "Cp"), to check their fp16 range.
