@@ -1122,6 +1122,62 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
             for (int e = 0; e < 4; ++e)
                 sCB[frag_row(r64, 0, e) * Q + frag_col(c64, nt, e)] = acc[0][nt][e];
     }
+    // (5) the decays of head hh, on warp 0 (tokens 2 lane, 2 lane + 1): they read only the per-token
+    // arrays and sums of that head, so warp 0 runs them while the other warps convert the next
+    // head's operands
+    auto decays = [&](int hh) {
+        const int h = g * HG + hh;
+        const float Ah = p.A[h];
+        const float last = sred[2], E = expf(last);
+        float ddir[2], dcs[2], uz = 0.f;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int j = 2 * lane + k;
+            const bool in = j < q;
+            const float Z = rowZ[j];
+            ddir[k] = in ? colR[j] + expf(last - scs[j]) * Z : 0.f;
+            dcs[k] = in ? rowRd[j] - sd[j] * colR[j] + se[j] * rowY[j] - su[j] * Z : 0.f;
+            uz += in ? su[j] * Z : 0.f;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) uz += __shfl_xor_sync(0xffffffffu, uz, o);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            if (2 * lane + k == q - 1) dcs[k] += E * sred[0] + uz;
+        const float pair = dcs[0] + dcs[1];
+        float suf = pair;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float tt = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += tt;
+        }
+        const float above = suf - pair;
+        const float da[2] = {above + pair, above + dcs[1]};
+        float sdA = 0.f, sbias = 0.f;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int j = 2 * lane + k;
+            if (j < q) {
+                const float dd = ddir[k] + Ah * da[k];
+                const float z = sz[j];
+                const float sg = z >= 0.f ? 1.f / (1.f + expf(-z)) : expf(z) / (1.f + expf(z));
+                const float dz = dd * sg;
+                ((T*)p.ddt)[(tok0 + j) * H + h] = from_f<T>(dz);
+                sdA += sd[j] * da[k];
+                sbias += dz;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            sdA += __shfl_xor_sync(0xffffffffu, sdA, o);
+            sbias += __shfl_xor_sync(0xffffffffu, sbias, o);
+        }
+        if (lane == 0) {
+            atomicAdd(&p.dA[h], sdA);
+            atomicAdd(&p.ddt_bias[h], sbias);
+            atomicAdd(&p.dD[h], sred[1]);
+        }
+    };
     float dBa[1][NTN][4], dCa[1][NTN][4];
     zero_frag(dBa);
     zero_frag(dCa);
@@ -1131,7 +1187,10 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         // this head's inputs have landed in the staging area (every thread's copies)
         cp_async_wait_all();
         __syncthreads();
-        for (int e = tid; e < Q * P / 8; e += blockDim.x) {
+        // warp 0: the previous head's decays; warps 1-15: this head's operands
+        const int ct = tid - 32, cn = (int)blockDim.x - 32;
+        if (warp == 0 && hh > 0) decays(hh - 1);
+        for (int e = warp == 0 ? Q * P / 8 : ct; e < Q * P / 8; e += cn) {
             const int r = e / (P / 8), c8 = e % (P / 8);
             uint4 ox = make_uint4(0u, 0u, 0u, 0u), od = ox;
             if (r < q) {
@@ -1145,7 +1204,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         {
             const float* hp = stHP;
             const float* dh = stDH;
-            for (int e = tid; e < N * P / 8; e += blockDim.x) {
+            for (int e = warp == 0 ? N * P / 8 : ct; e < N * P / 8; e += cn) {
                 const int n = e / (P / 8), c8 = e % (P / 8);
                 const float4 a0 = *reinterpret_cast<const float4*>(hp + n * P + 8 * c8);
                 const float4 a1 = *reinterpret_cast<const float4*>(hp + n * P + 8 * c8 + 4);
@@ -1163,11 +1222,14 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                         a1.z * b1.z + a1.w * b1.w;
             }
         }
-        if (tid < Q) {
-            colR[tid] = 0.f; rowRd[tid] = 0.f; rowZ[tid] = 0.f; rowY[tid] = 0.f;
-        }
-        if (tid < 2) sred[tid] = 0.f;      // sred[2] is written by the decay scan below
         if (tid < 32) {
+            // (after the previous head's decays, which read them in other lanes)
+            __syncwarp();
+            for (int j = lane; j < Q; j += 32) {
+                colR[j] = 0.f; rowRd[j] = 0.f; rowZ[j] = 0.f; rowY[j] = 0.f;
+            }
+            if (lane < 2) sred[lane] = 0.f;   // sred[2] is written by the decay scan below
+            __syncwarp();
             chunk_decay_raw(dt_raw, q, bias, Ah, sd, sz, scs, &sred[2]);
             if (hh + 1 < HG) load_dt2<T>(dt_raw, dtg, tok0, H, h + 1, q);
             __syncwarp();
@@ -1284,61 +1346,10 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
 #pragma unroll
                 for (int e = 0; e < 4; ++e) dCa[0][nt][e] += se[frag_row(rN, 0, e)] * t[0][nt][e];
         }
-        __syncthreads();
-        // (5) the decays, on warp 0: tokens 2 lane, 2 lane + 1
-        if (tid < 32) {
-            const float last = sred[2], E = expf(last);
-            float ddir[2], dcs[2], uz = 0.f;
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int j = 2 * lane + k;
-                const bool in = j < q;
-                const float Z = rowZ[j];
-                ddir[k] = in ? colR[j] + expf(last - scs[j]) * Z : 0.f;
-                dcs[k] = in ? rowRd[j] - sd[j] * colR[j] + se[j] * rowY[j] - su[j] * Z : 0.f;
-                uz += in ? su[j] * Z : 0.f;
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) uz += __shfl_xor_sync(0xffffffffu, uz, o);
-#pragma unroll
-            for (int k = 0; k < 2; ++k)
-                if (2 * lane + k == q - 1) dcs[k] += E * sred[0] + uz;
-            const float pair = dcs[0] + dcs[1];
-            float suf = pair;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float tt = __shfl_down_sync(0xffffffffu, suf, o);
-                if (lane + o < 32) suf += tt;
-            }
-            const float above = suf - pair;
-            const float da[2] = {above + pair, above + dcs[1]};
-            float sdA = 0.f, sbias = 0.f;
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int j = 2 * lane + k;
-                if (j < q) {
-                    const float dd = ddir[k] + Ah * da[k];
-                    const float z = sz[j];
-                    const float sg = z >= 0.f ? 1.f / (1.f + expf(-z)) : expf(z) / (1.f + expf(z));
-                    const float dz = dd * sg;
-                    ((T*)p.ddt)[(tok0 + j) * H + h] = from_f<T>(dz);
-                    sdA += sd[j] * da[k];
-                    sbias += dz;
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                sdA += __shfl_xor_sync(0xffffffffu, sdA, o);
-                sbias += __shfl_xor_sync(0xffffffffu, sbias, o);
-            }
-            if (lane == 0) {
-                atomicAdd(&p.dA[h], sdA);
-                atomicAdd(&p.ddt_bias[h], sbias);
-                atomicAdd(&p.dD[h], sred[1]);
-            }
-        }
-        __syncthreads();
+        // (the barrier at the top of the next head orders these reads before its conversion)
     }
+    __syncthreads();
+    if (warp == 0) decays(HG - 1);
     T* dBg = (T*)p.dB + (tok0 * G + g) * N;
     T* dCg = (T*)p.dC + (tok0 * G + g) * N;
 #pragma unroll
