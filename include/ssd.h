@@ -248,7 +248,9 @@ SSD_API int ssd_dequant_chunks(int64_t T, int64_t D, int64_t ranks, int dtype, c
  * 64-token chunks (per-chunk terms, a sequential pass over chunk states,
  * per-chunk gradients; for bf16 the matrix products on the tensor cores with
  * fp16 operands and fp32 accumulation), workspace 8 N P H blocks + 4 H blocks
- * bytes.  Other shapes: CUDA cores in fp32 with checkpoints of the state every
+ * bytes, plus 8 K b L G N bytes of fp32 dB / dC partials when bf16 gradient
+ * blocks split each group's heads K ways (K = 2 or 4, chosen from the block
+ * count and the SM count to fill the last wave).  Other shapes: CUDA cores in fp32 with checkpoints of the state every
  * 64 tokens, workspace 4 N P H (blocks + 64 S) + 8 b L G N bytes; supported
  * there are headdim dividing 256 and headdim * dstate in {256, 512, ...,
  * 8192}, other shapes return SSD_ERR_UNSUPPORTED.  Workspace is stream-ordered,

@@ -26,6 +26,8 @@
 // it recomputes the block's per-token states into a per-(sequence, head)
 // scratch area and then runs the adjoint sweep over the block's tokens, last
 // to first.  Every quantity is fp32; inputs are read in their own dtype.
+#include <algorithm>
+#include <cmath>
 #include <cuda_fp16.h>
 #include <stdio.h>
 
@@ -514,6 +516,11 @@ struct ChunkedBwd {
     float *ddt_bias, *dA, *dD, *dinit;
     float *S, *T, *E;                  // (chunks, H, N P), (chunks, H, N P), (chunks, H)
     int H, N, G;
+    // k_bwd_grads_h only: the heads of a group split over hsplit blocks per chunk; each part's
+    // dB, dC go to fp32 partials (part p at dBp + p part_stride, laid out as dB), summed after
+    int hsplit = 1;
+    float *dBp = nullptr, *dCp = nullptr;
+    int64_t part_stride = 0;
 };
 
 // Loads rows [0, q) of a (tokens, stride) slab of T into shared fp32 (rows, cols) with row
@@ -1075,8 +1082,10 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     float* stDH = stHP + N * P;
     const int H = p.H, G = p.G, HG = H / G;
     const int tid = threadIdx.x, lane = tid & 31;
-    const int64_t f = blockIdx.x / G;
-    const int g = (int)(blockIdx.x % G);
+    const int64_t f = blockIdx.x / ((int64_t)G * p.hsplit);
+    const int g = (int)((blockIdx.x / p.hsplit) % G), part = (int)(blockIdx.x % p.hsplit);
+    // this block's heads of group g: hh0 .. hh1 - 1
+    const int hh0 = part * (HG / p.hsplit), hh1 = hh0 + HG / p.hsplit;
     ChunkRef r;
     if (!chunk_ref(p.si, f, r)) return;
     const int q = (int)(r.t1 - r.t0);
@@ -1102,10 +1111,10 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         }
         cp_async_commit();
     };
-    stage(0);
+    stage(hh0);
     // warp 0 holds the raw dt of the head it prepares next (loaded a head ahead)
     float dt_raw[2] = {0.f, 0.f};
-    if (tid < 32) load_dt2<T>(dt_raw, dtg, tok0, H, g * HG, q);
+    if (tid < 32) load_dt2<T>(dt_raw, dtg, tok0, H, g * HG + hh0, q);
     load_rows_h(sB, (const T*)p.B + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
     load_rows_h(sC, (const T*)p.C + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
     __syncthreads();
@@ -1181,7 +1190,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     float dBa[1][NTN][4], dCa[1][NTN][4];
     zero_frag(dBa);
     zero_frag(dCa);
-    for (int hh = 0; hh < HG; ++hh) {
+    for (int hh = hh0; hh < hh1; ++hh) {
         const int h = g * HG + hh;
         const float bias = p.dt_bias ? p.dt_bias[h] : 0.f, Ah = p.A[h], Dh = p.D ? p.D[h] : 0.f;
         // this head's inputs have landed in the staging area (every thread's copies)
@@ -1189,7 +1198,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         __syncthreads();
         // warp 0: the previous head's decays; warps 1-15: this head's operands
         const int ct = tid - 32, cn = (int)blockDim.x - 32;
-        if (warp == 0 && hh > 0) decays(hh - 1);
+        if (warp == 0 && hh > hh0) decays(hh - 1);
         for (int e = warp == 0 ? Q * P / 8 : ct; e < Q * P / 8; e += cn) {
             const int r = e / (P / 8), c8 = e % (P / 8);
             uint4 ox = make_uint4(0u, 0u, 0u, 0u), od = ox;
@@ -1231,7 +1240,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
             if (lane < 2) sred[lane] = 0.f;   // sred[2] is written by the decay scan below
             __syncwarp();
             chunk_decay_raw(dt_raw, q, bias, Ah, sd, sz, scs, &sred[2]);
-            if (hh + 1 < HG) load_dt2<T>(dt_raw, dtg, tok0, H, h + 1, q);
+            if (hh + 1 < hh1) load_dt2<T>(dt_raw, dtg, tok0, H, h + 1, q);
             __syncwarp();
             const float last = sred[2];
 #pragma unroll
@@ -1244,7 +1253,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         __syncthreads();
         // every thread is done with the staging area: the next head's copies fly while this one
         // computes
-        if (hh + 1 < HG) stage(hh + 1);
+        if (hh + 1 < hh1) stage(hh + 1);
         {
             // x and dy share one swizzle, so element e is the same (row, column) in both
             float a1 = hpdh, a2 = 0.f;
@@ -1349,7 +1358,23 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         // (the barrier at the top of the next head orders these reads before its conversion)
     }
     __syncthreads();
-    if (warp == 0) decays(HG - 1);
+    if (warp == 0) decays(hh1 - 1);
+    if (p.hsplit > 1) {
+        // this part's sums, in fp32, for k_bwd_sum_parts
+        float* dBg = p.dBp + part * p.part_stride + (tok0 * G + g) * N;
+        float* dCg = p.dCp + part * p.part_stride + (tok0 * G + g) * N;
+#pragma unroll
+        for (int nt = 0; nt < NTN; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                const int i = frag_row(rN, 0, e), n = frag_col(cN, nt, e);
+                if (i < q) {
+                    *reinterpret_cast<float2*>(dBg + (int64_t)i * G * N + n) = make_float2(dBa[0][nt][e], dBa[0][nt][e + 1]);
+                    *reinterpret_cast<float2*>(dCg + (int64_t)i * G * N + n) = make_float2(dCa[0][nt][e], dCa[0][nt][e + 1]);
+                }
+            }
+        return;
+    }
     T* dBg = (T*)p.dB + (tok0 * G + g) * N;
     T* dCg = (T*)p.dC + (tok0 * G + g) * N;
 #pragma unroll
@@ -1442,6 +1467,52 @@ constexpr size_t grads_smem() {
                             10 * kQb + 4);
 }
 
+// dB, dC = the sum of the gradient blocks' fp32 partials (parts in order), rounded once; 4 per step.
+__global__ void k_bwd_sum_parts(const float* __restrict__ pb, const float* __restrict__ pc,
+                                __nv_bfloat16* __restrict__ db, __nv_bfloat16* __restrict__ dc, int64_t n4, int parts,
+                                int64_t stride) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        float4 sb = reinterpret_cast<const float4*>(pb)[i], sc = reinterpret_cast<const float4*>(pc)[i];
+        for (int k = 1; k < parts; ++k) {
+            const float4 ob = reinterpret_cast<const float4*>(pb + k * stride)[i];
+            const float4 oc = reinterpret_cast<const float4*>(pc + k * stride)[i];
+            sb.x += ob.x; sb.y += ob.y; sb.z += ob.z; sb.w += ob.w;
+            sc.x += oc.x; sc.y += oc.y; sc.z += oc.z; sc.w += oc.w;
+        }
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(sb.x, sb.y), b1 = __floats2bfloat162_rn(sb.z, sb.w);
+        const __nv_bfloat162 c0 = __floats2bfloat162_rn(sc.x, sc.y), c1 = __floats2bfloat162_rn(sc.z, sc.w);
+        reinterpret_cast<__nv_bfloat162*>(db)[2 * i] = b0;
+        reinterpret_cast<__nv_bfloat162*>(db)[2 * i + 1] = b1;
+        reinterpret_cast<__nv_bfloat162*>(dc)[2 * i] = c0;
+        reinterpret_cast<__nv_bfloat162*>(dc)[2 * i + 1] = c1;
+    }
+}
+
+// Blocks per (chunk, group) of the bf16 gradient kernel, each taking an equal share of the
+// group's heads: 1, 2 or 4, whichever fills the last wave of the SMs best (by at least 3%, since
+// every extra part repeats C B^T and adds the pass summing dB, dC).  With one 512-thread block
+// per SM, 512 blocks on 148 SMs run as 3.46 waves (four, the last half empty); 1024 as 6.92.
+int grads_hsplit(const ScanArgs& a, int64_t chunks) {
+    if (a.dtype == 0 || !bwd_chunked(a)) return 1;
+    const int64_t HG = a.H / a.G;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = 148;
+    auto fill = [&](int S) {
+        const double w = (double)(chunks * a.G * S) / sms;
+        return w / std::ceil(w);
+    };
+    int best = 1;
+    double bf = fill(1);
+    for (int S = 2; S <= 4; S *= 2)
+        if (HG % S == 0 && fill(S) > bf + 0.03) {
+            best = S;
+            bf = fill(S);
+        }
+    return best;
+}
+
 template <typename T, int N>
 void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
     const size_t sm_terms = sizeof(float) * (kQb * N + kQb * kPb);
@@ -1468,7 +1539,13 @@ void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
         ProfScope ps(K_BWD_GRADS, st);
         if constexpr (sizeof(T) == 2) {
             cudaFuncSetAttribute(k_bwd_grads_h<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grads_h_smem<N>());
-            k_bwd_grads_h<N><<<(unsigned)(chunks * p.G), kGradThreads, grads_h_smem<N>(), st>>>(p);
+            k_bwd_grads_h<N><<<(unsigned)(chunks * p.G * p.hsplit), kGradThreads, grads_h_smem<N>(), st>>>(p);
+            if (p.hsplit > 1) {
+                const int64_t n4 = p.part_stride / 4;
+                const unsigned grid = (unsigned)std::min<int64_t>((n4 + 255) / 256, 148 * 8);
+                k_bwd_sum_parts<<<grid, 256, 0, st>>>(p.dBp, p.dCp, (__nv_bfloat16*)p.dB, (__nv_bfloat16*)p.dC, n4,
+                                                       p.hsplit, p.part_stride);
+            }
         } else {
             k_bwd_grads<T, N><<<(unsigned)(chunks * p.G), 256, grads_smem<N>(), st>>>(p);
         }
@@ -1513,7 +1590,11 @@ size_t bwd_workspace_bytes(const ScanArgs& a) {
                                      : a.b * ((a.L + kBwdBlock - 1) / kBwdBlock);
     const size_t NP = (size_t)a.N * a.P;
     auto r = [](size_t v) { return (v + 255) & ~(size_t)255; };
-    if (bwd_chunked(a)) return 2 * r(sizeof(float) * blocks * a.H * NP) + r(sizeof(float) * blocks * a.H);
+    if (bwd_chunked(a)) {
+        const int S = grads_hsplit(a, blocks);
+        const size_t parts = S > 1 ? 2 * r(sizeof(float) * S * (size_t)(a.b * a.L) * a.G * a.N) : 0;
+        return 2 * r(sizeof(float) * blocks * a.H * NP) + r(sizeof(float) * blocks * a.H) + parts;
+    }
     return r(sizeof(float) * blocks * a.H * NP) + r(sizeof(float) * a.S * a.H * kBwdBlock * NP) +
            2 * r(sizeof(float) * a.b * a.L * a.G * a.N);
 }
@@ -1533,8 +1614,14 @@ int launch_scan_bwd(const ScanArgs& a, const BwdArgs& g, const SeqInfo& si64, vo
         c.ddt_bias = g.ddt_bias; c.dA = g.dA; c.dD = g.dD; c.dinit = g.dinit;
         c.S = (float*)w; w += r(sizeof(float) * blocks * a.H * NP);
         c.T = (float*)w; w += r(sizeof(float) * blocks * a.H * NP);
-        c.E = (float*)w;
+        c.E = (float*)w; w += r(sizeof(float) * blocks * a.H);
         c.H = (int)a.H; c.N = (int)a.N; c.G = (int)a.G;
+        c.hsplit = grads_hsplit(a, blocks);
+        if (c.hsplit > 1) {
+            c.part_stride = a.b * a.L * a.G * a.N;
+            c.dBp = (float*)w; w += r(sizeof(float) * c.hsplit * c.part_stride);
+            c.dCp = (float*)w;
+        }
         cudaError_t e = cudaMemsetAsync(g.ddt_bias, 0, sizeof(float) * a.H, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(g.dA, 0, sizeof(float) * a.H, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(g.dD, 0, sizeof(float) * a.H, st);
