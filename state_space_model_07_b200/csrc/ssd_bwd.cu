@@ -1199,12 +1199,20 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         // warp 0: the previous head's decays; warps 1-15: this head's operands
         const int ct = tid - 32, cn = (int)blockDim.x - 32;
         if (warp == 0 && hh > hh0) decays(hh - 1);
+        float xdy = 0.f;   // this thread's part of sum dy . x (bf16 values, exact in fp32 products)
         for (int e = warp == 0 ? Q * P / 8 : ct; e < Q * P / 8; e += cn) {
             const int r = e / (P / 8), c8 = e % (P / 8);
             uint4 ox = make_uint4(0u, 0u, 0u, 0u), od = ox;
             if (r < q) {
-                ox = bf16x8_to_f16x8_bwd(*reinterpret_cast<const uint4*>(stX + r * P + 8 * c8));
-                od = bf16x8_to_f16x8_bwd(*reinterpret_cast<const uint4*>(stDY + r * P + 8 * c8));
+                const uint4 vx = *reinterpret_cast<const uint4*>(stX + r * P + 8 * c8);
+                const uint4 vd = *reinterpret_cast<const uint4*>(stDY + r * P + 8 * c8);
+                const uint32_t wx[4] = {vx.x, vx.y, vx.z, vx.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    xdy += __uint_as_float(wx[m] << 16) * __uint_as_float(wd[m] << 16) +
+                           __uint_as_float(wx[m] & 0xffff0000u) * __uint_as_float(wd[m] & 0xffff0000u);
+                ox = bf16x8_to_f16x8_bwd(vx);
+                od = bf16x8_to_f16x8_bwd(vd);
             }
             *reinterpret_cast<uint4*>(hsw8(sX, r, c8, P)) = ox;
             *reinterpret_cast<uint4*>(hsw8(sDY, r, c8, P)) = od;
@@ -1255,9 +1263,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         // computes
         if (hh + 1 < hh1) stage(hh + 1);
         {
-            // x and dy share one swizzle, so element e is the same (row, column) in both
-            float a1 = hpdh, a2 = 0.f;
-            for (int e = tid; e < Q * P; e += blockDim.x) a2 += __half2float(sDY[e]) * __half2float(sX[e]);
+            float a1 = hpdh, a2 = xdy;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 a1 += __shfl_xor_sync(0xffffffffu, a1, o);
@@ -1277,19 +1283,27 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
+                for (int e = 0; e < 4; e += 2) {
+                    // elements (j, i) and (j, i + 1), i even: one fp16 pair per tile
                     const int j = frag_row(r64, 0, e), i = frag_col(c64, nt, e);
+                    const float2 cb = *reinterpret_cast<const float2*>(&sCB[j * Q + i]);
+                    const float2 di = *reinterpret_cast<const float2*>(&sd[i]);
+                    const float2 ci = *reinterpret_cast<const float2*>(&scs[i]);
                     // the fast exponential: this path's operands are fp16 anyway
-                    const float L = (i <= j && j < q) ? __expf(scs[j] - scs[i]) : 0.f;
-                    const float cb = sCB[j * Q + i], di = sd[i], dyx = acc[0][nt][e];
-                    const float wv = cb * L * di;
-                    const __half whi = __float2half_rn(wv);
-                    sW[hsw(j, i, Q)] = whi;
-                    sWl[hsw(j, i, Q)] = __float2half_rn(wv - __half2float(whi));
-                    sK[hsw(j, i, Q)] = __float2half_rn(L * dyx * di);
-                    const float R = cb * dyx * L;
-                    rrow[e >> 1] += R * di;
-                    rcol[nt][e & 1] += R;
+                    const float L0 = (i <= j && j < q) ? __expf(scs[j] - ci.x) : 0.f;
+                    const float L1 = (i + 1 <= j && j < q) ? __expf(scs[j] - ci.y) : 0.f;
+                    const float dyx0 = acc[0][nt][e], dyx1 = acc[0][nt][e + 1];
+                    const float w0 = cb.x * L0 * di.x, w1 = cb.y * L1 * di.y;
+                    const __half2 whi = __floats2half2_rn(w0, w1);
+                    const int at = hsw(j, i, Q);
+                    *reinterpret_cast<__half2*>(&sW[at]) = whi;
+                    *reinterpret_cast<__half2*>(&sWl[at]) =
+                        __floats2half2_rn(w0 - __low2float(whi), w1 - __high2float(whi));
+                    *reinterpret_cast<__half2*>(&sK[at]) = __floats2half2_rn(L0 * dyx0 * di.x, L1 * dyx1 * di.y);
+                    const float R0 = cb.x * dyx0 * L0, R1 = cb.y * dyx1 * L1;
+                    rrow[e >> 1] += R0 * di.x + R1 * di.y;
+                    rcol[nt][0] += R0;
+                    rcol[nt][1] += R1;
                 }
 #pragma unroll
             for (int a = 0; a < 2; ++a) atomicAdd(&rowRd[frag_row(r64, 0, 2 * a)], rrow[a]);
