@@ -1327,12 +1327,18 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = frag_row(r64, 0, e), c = frag_col(c64, nt, e);
-                    z[e >> 1] += bd[0][nt][e] * __half2float(sX[hsw(i, c, P)]);
-                    if (i < q)
-                        dxg[(int64_t)i * H * P + c] =
-                            from_f<T>(Dh * __half2float(sDY[hsw(i, c, P)]) + wd[0][nt][e] + su[i] * bd[0][nt][e]);
+                for (int e = 0; e < 4; e += 2) {
+                    // columns c, c + 1 (c even) of row i: one fp16 pair of x and of dy, one bf16 pair out
+                    const int i = frag_row(r64, 0, e), c = frag_col(c64, nt, e), at = hsw(i, c, P);
+                    const float2 xv = __half22float2(*reinterpret_cast<const __half2*>(&sX[at]));
+                    const float2 dv = __half22float2(*reinterpret_cast<const __half2*>(&sDY[at]));
+                    z[e >> 1] += bd[0][nt][e] * xv.x + bd[0][nt][e + 1] * xv.y;
+                    if (i < q) {
+                        const float ui = su[i];
+                        *reinterpret_cast<__nv_bfloat162*>(dxg + (int64_t)i * H * P + c) =
+                            __floats2bfloat162_rn(Dh * dv.x + wd[0][nt][e] + ui * bd[0][nt][e],
+                                                  Dh * dv.y + wd[0][nt][e + 1] + ui * bd[0][nt][e + 1]);
+                    }
                 }
 #pragma unroll
             for (int a = 0; a < 2; ++a) atomicAdd(&rowZ[frag_row(r64, 0, 2 * a)], z[a]);
@@ -1346,8 +1352,11 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    y[e >> 1] += ch[0][nt][e] * __half2float(sDY[hsw(frag_row(r64, 0, e), frag_col(c64, nt, e), P)]);
+                for (int e = 0; e < 4; e += 2) {
+                    const float2 dv = __half22float2(
+                        *reinterpret_cast<const __half2*>(&sDY[hsw(frag_row(r64, 0, e), frag_col(c64, nt, e), P)]));
+                    y[e >> 1] += ch[0][nt][e] * dv.x + ch[0][nt][e + 1] * dv.y;
+                }
 #pragma unroll
             for (int a = 0; a < 2; ++a) atomicAdd(&rowY[frag_row(r64, 0, 2 * a)], y[a]);
         }
