@@ -1017,6 +1017,18 @@ __device__ __forceinline__ void load_rows_h(__half* dst, const __nv_bfloat16* sr
     }
 }
 
+// Sums over the lanes of an mma.sync fragment that hold one row (the four lanes of a quad) or one
+// column (the same lane of the eight quads); every lane gets the sum.
+__device__ __forceinline__ float quad_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    return v + __shfl_xor_sync(0xffffffffu, v, 2);
+}
+__device__ __forceinline__ float across_quads_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    return v + __shfl_xor_sync(0xffffffffu, v, 16);
+}
+
 // 16-byte asynchronous copy global -> shared (cached at L2 only), and the wait for all of this
 // thread's copies committed so far.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -1305,12 +1317,20 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                     rcol[nt][0] += R0;
                     rcol[nt][1] += R1;
                 }
+            // summed in the warp first (a row's values sit in one lane quad, a column's in the
+            // eight quads), then one shared atomic per row or column and warp
 #pragma unroll
-            for (int a = 0; a < 2; ++a) atomicAdd(&rowRd[frag_row(r64, 0, 2 * a)], rrow[a]);
+            for (int a = 0; a < 2; ++a) {
+                const float v = quad_sum(rrow[a]);
+                if ((lane & 3) == 0) atomicAdd(&rowRd[frag_row(r64, 0, 2 * a)], v);
+            }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int b = 0; b < 2; ++b) atomicAdd(&colR[frag_col(c64, nt, b)], rcol[nt][b]);
+                for (int b = 0; b < 2; ++b) {
+                    const float v = across_quads_sum(rcol[nt][b]);
+                    if (lane < 4) atomicAdd(&colR[frag_col(c64, nt, b)], v);
+                }
         }
         __syncthreads();
         // (2) dx = D dy + W^T dy + u o (B dh_end), and Z_i = B_i^T dh_end x_i
@@ -1341,7 +1361,10 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                     }
                 }
 #pragma unroll
-            for (int a = 0; a < 2; ++a) atomicAdd(&rowZ[frag_row(r64, 0, 2 * a)], z[a]);
+            for (int a = 0; a < 2; ++a) {
+                const float v = quad_sum(z[a]);
+                if ((lane & 3) == 0) atomicAdd(&rowZ[frag_row(r64, 0, 2 * a)], v);
+            }
         }
         // (3) Y_j = C_j^T h_prev dy_j
         {
@@ -1358,7 +1381,10 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                     y[e >> 1] += ch[0][nt][e] * dv.x + ch[0][nt][e + 1] * dv.y;
                 }
 #pragma unroll
-            for (int a = 0; a < 2; ++a) atomicAdd(&rowY[frag_row(r64, 0, 2 * a)], y[a]);
+            for (int a = 0; a < 2; ++a) {
+                const float v = quad_sum(y[a]);
+                if ((lane & 3) == 0) atomicAdd(&rowY[frag_row(r64, 0, 2 * a)], v);
+            }
         }
         // (4) dB += K^T C + u o (x dh_end^T),  dC += K B + e o (dy h_prev^T)
         {
