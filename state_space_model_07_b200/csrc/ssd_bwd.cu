@@ -490,6 +490,18 @@ __device__ __forceinline__ void prod(float (&acc)[MT][NT][4], const float* A, in
 __device__ __forceinline__ int frag_row(int r0, int mt, int e) { return r0 + 16 * mt + ((threadIdx.x & 31) >> 2) + 8 * (e >> 1); }
 __device__ __forceinline__ int frag_col(int c0, int nt, int e) { return c0 + 8 * nt + 2 * (threadIdx.x & 3) + (e & 1); }
 
+// Sums over the lanes of an mma.sync fragment that hold one row (the four lanes of a quad) or one
+// column (the same lane of the eight quads); every lane gets the sum.
+__device__ __forceinline__ float quad_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    return v + __shfl_xor_sync(0xffffffffu, v, 2);
+}
+__device__ __forceinline__ float across_quads_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    return v + __shfl_xor_sync(0xffffffffu, v, 16);
+}
+
 template <int MT, int NT>
 __device__ __forceinline__ void zero_frag(float (&acc)[MT][NT][4]) {
 #pragma unroll
@@ -784,11 +796,17 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads(const ChunkedBwd p) {
                     rcol[nt][e & 1] += R;
                 }
 #pragma unroll
-            for (int a = 0; a < 2; ++a) atomicAdd(&rowRd[frag_row(r64, 0, 2 * a)], rrow[a]);
+            for (int a = 0; a < 2; ++a) {
+                const float v = quad_sum(rrow[a]);
+                if ((threadIdx.x & 3) == 0) atomicAdd(&rowRd[frag_row(r64, 0, 2 * a)], v);
+            }
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                for (int b = 0; b < 2; ++b) atomicAdd(&colR[frag_col(c64, nt, b)], rcol[nt][b]);
+                for (int b = 0; b < 2; ++b) {
+                    const float v = across_quads_sum(rcol[nt][b]);
+                    if ((threadIdx.x & 31) < 4) atomicAdd(&colR[frag_col(c64, nt, b)], v);
+                }
         }
         __syncthreads();
         // (2) dx = D dy + W^T dy + u o (B dh_end), and Z_i = B_i^T dh_end x_i
@@ -810,7 +828,10 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads(const ChunkedBwd p) {
                         dxg[(int64_t)i * H * P + c] = from_f<T>(Dh * sDY[i * LP + c] + wd[0][nt][e] + su[i] * bd[0][nt][e]);
                 }
 #pragma unroll
-            for (int a = 0; a < 2; ++a) atomicAdd(&rowZ[frag_row(r64, 0, 2 * a)], z[a]);
+            for (int a = 0; a < 2; ++a) {
+                const float v = quad_sum(z[a]);
+                if ((threadIdx.x & 3) == 0) atomicAdd(&rowZ[frag_row(r64, 0, 2 * a)], v);
+            }
         }
         // (3) Y_j = C_j^T h_prev dy_j
         {
@@ -824,7 +845,10 @@ __global__ void __launch_bounds__(256, 1) k_bwd_grads(const ChunkedBwd p) {
                 for (int e = 0; e < 4; ++e)
                     y[e >> 1] += ch[0][nt][e] * sDY[frag_row(r64, 0, e) * LP + frag_col(c64, nt, e)];
 #pragma unroll
-            for (int a = 0; a < 2; ++a) atomicAdd(&rowY[frag_row(r64, 0, 2 * a)], y[a]);
+            for (int a = 0; a < 2; ++a) {
+                const float v = quad_sum(y[a]);
+                if ((threadIdx.x & 3) == 0) atomicAdd(&rowY[frag_row(r64, 0, 2 * a)], v);
+            }
         }
         // (4) dB += K^T C + u o (x dh_end^T),  dC += K B + e o (dy h_prev^T)
         {
@@ -1015,18 +1039,6 @@ __device__ __forceinline__ void load_rows_h(__half* dst, const __nv_bfloat16* sr
         }
         *reinterpret_cast<uint4*>(hsw8(dst, r, c8, W)) = o;
     }
-}
-
-// Sums over the lanes of an mma.sync fragment that hold one row (the four lanes of a quad) or one
-// column (the same lane of the eight quads); every lane gets the sum.
-__device__ __forceinline__ float quad_sum(float v) {
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    return v + __shfl_xor_sync(0xffffffffu, v, 2);
-}
-__device__ __forceinline__ float across_quads_sum(float v) {
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    return v + __shfl_xor_sync(0xffffffffu, v, 16);
 }
 
 // 16-byte asynchronous copy global -> shared (cached at L2 only), and the wait for all of this
