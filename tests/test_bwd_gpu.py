@@ -74,8 +74,12 @@ def test_backward_of_the_bench_shaped_layer_at_oracle_size():
     _check(inputs.make_inputs(w, "cuda"), w, seed=3)
 
 
-def test_backward_packed_sequences_and_no_dfinal():
-    w = inputs.scaled(W["packed_varlen"], nheads=4, dstate=64)
+@pytest.mark.parametrize("nheads,dstate", [(4, 64), (8, 128)])
+def test_backward_packed_sequences_and_no_dfinal(nheads, dstate):
+    """Packed sequences (chunks restart at every sequence start).  With 8 heads in 4 groups the
+    bf16 gradient blocks split each group's two heads over two blocks (few blocks for 148 SMs),
+    so the summed dB, dC partials are covered for packed input too."""
+    w = inputs.scaled(W["packed_varlen"], nheads=nheads, dstate=dstate)
     lens = [100, 1, 64, 65, 30]
     d = inputs.make_inputs(w, "cuda", lengths=lens)
     _check(d, w, seed=5)
