@@ -1450,6 +1450,149 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         }
 }
 
+// ---- k_bwd_pass_h: the chunk terms computed inside the sequential pass (bf16, P = Q = 64) ----
+//
+// One block per (sequence, head) walks the sequence's chunks forwards, then backwards, holding the
+// N x 64 state (then its adjoint) in mma.sync accumulator fragments: warp w owns 16 state rows and
+// P / NCB columns.  At every chunk it computes the chunk's own term on the tensor cores,
+// S = B^T (u o x) forwards and T = C^T (e o dy) backwards (u_j = exp(cs_last - cs_j) d_j,
+// e_j = exp(cs_j)), from operands staged by cp.async one chunk ahead, so no term goes through
+// HBM.  It writes the state entering every chunk (forwards, over S) and the adjoint of the state
+// leaving every chunk (backwards, over T) for k_bwd_grads_h, and d h0 at the end.
+template <int N>
+__global__ void __launch_bounds__(256) k_bwd_pass_h(const ChunkedBwd p) {
+    using T = __nv_bfloat16;
+    constexpr int P = kPb, Q = kQb;
+    constexpr int NRB = N / 16;          // 16-row blocks of the state
+    constexpr int NCB = 8 / NRB;         // column blocks per row block (eight warps)
+    constexpr int NT = P / NCB / 8;      // 8-column MMA tiles per warp
+    static_assert(NRB * NCB == 8 && NT % 2 == 0, "eight warps cover the N x 64 state");
+    extern __shared__ __align__(16) uint8_t smraw[];
+    __half* sM = reinterpret_cast<__half*>(smraw);   // [Q][N] B or C, fp16 swizzled
+    __half* sV = sM + Q * N;                         // [Q][P] u o x or e o dy
+    T* stM = reinterpret_cast<T*>(sV + Q * P);       // [Q][N] the next chunk's raw rows
+    T* stV = stM + Q * N;                            // [Q][P]
+    __shared__ float sd[kQb], sz[kQb], scs[kQb], sw[kQb], slast;
+    const int H = p.H, G = p.G;
+    const int s = (int)(blockIdx.x / H), h = (int)(blockIdx.x % H), g = h / (H / G);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nc = seq_nchunks(p.si, s);
+    const int64_t cf0 = seq_chunk0(p.si, s);
+    int64_t row, ts, te;
+    seq_span(p.si, s, row, ts, te);
+    const float bias = p.dt_bias ? p.dt_bias[h] : 0.f, Ah = p.A[h];
+    const int n0 = 16 * (warp % NRB), col0 = (P / NCB) * (warp / NRB);
+    const T* dtg = (const T*)p.dt;
+    auto chunk_q = [&](int c) {
+        const int64_t t0 = ts + (int64_t)c * Q;
+        return (int)(te - t0 < Q ? te - t0 : Q);
+    };
+    auto chunk_tok0 = [&](int c) { return row * p.si.L + ts + (int64_t)c * Q; };
+    const int64_t slab = (int64_t)N * P;
+    // raw rows (those inside the chunk) of M (B or C, per group) and V (x or dy, per head)
+    auto stage = [&](int c, const T* Mg, const T* Vg) {
+        const int q = chunk_q(c);
+        const int64_t tok0 = chunk_tok0(c);
+        for (int e = tid; e < Q * N / 8; e += blockDim.x) {
+            const int r = e / (N / 8), c8 = e % (N / 8);
+            if (r < q) cp_async16(stM + r * N + 8 * c8, Mg + ((tok0 + r) * G + g) * N + 8 * c8);
+        }
+        for (int e = tid; e < Q * P / 8; e += blockDim.x) {
+            const int r = e / (P / 8), c8 = e % (P / 8);
+            if (r < q) cp_async16(stV + r * P + 8 * c8, Vg + ((tok0 + r) * H + h) * P + 8 * c8);
+        }
+        cp_async_commit();
+    };
+    float acc[1][NT][4];
+    // (N, P) fp32 row-major <-> this warp's fragment (null source: zero)
+    auto load_frag = [&](const float* src) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                float2 v = make_float2(0.f, 0.f);
+                if (src) v = *reinterpret_cast<const float2*>(src + frag_row(n0, 0, e) * P + frag_col(col0, nt, e));
+                acc[0][nt][e] = v.x;
+                acc[0][nt][e + 1] = v.y;
+            }
+    };
+    auto store_frag = [&](float* dst) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; e += 2)
+                *reinterpret_cast<float2*>(dst + frag_row(n0, 0, e) * P + frag_col(col0, nt, e)) =
+                    make_float2(acc[0][nt][e], acc[0][nt][e + 1]);
+    };
+    auto sweep = [&](bool fwd) {
+        const T* Mg = (const T*)(fwd ? p.B : p.C);
+        const T* Vg = (const T*)(fwd ? p.x : p.dy);
+        float* slabs = fwd ? p.S : p.T;
+        const int cfirst = fwd ? 0 : nc - 1, step = fwd ? 1 : -1;
+        float dt_raw[2] = {0.f, 0.f};   // warp 0: raw dt of the chunk it prepares next
+        if (nc > 0) {
+            stage(cfirst, Mg, Vg);
+            if (tid < 32) load_dt2<T>(dt_raw, dtg, chunk_tok0(cfirst), H, h, chunk_q(cfirst));
+        }
+        for (int i = 0; i < nc; ++i) {
+            const int c = cfirst + step * i;
+            const int q = chunk_q(c);
+            // chunk c's rows have landed; every warp is done with the previous chunk's operands
+            cp_async_wait_all();
+            __syncthreads();
+            if (tid < 32) {
+                chunk_decay_raw(dt_raw, q, bias, Ah, sd, sz, scs, &slast);
+                __syncwarp();
+                const float last = slast;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int j = 2 * lane + k;
+                    sw[j] = j < q ? (fwd ? expf(last - scs[j]) * sd[j] : expf(scs[j])) : 0.f;
+                }
+                if (i + 1 < nc) load_dt2<T>(dt_raw, dtg, chunk_tok0(c + step), H, h, chunk_q(c + step));
+            } else {
+                for (int e = tid - 32; e < Q * N / 8; e += blockDim.x - 32) {
+                    const int r = e / (N / 8), c8 = e % (N / 8);
+                    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < q) o = bf16x8_to_f16x8_bwd(*reinterpret_cast<const uint4*>(stM + r * N + 8 * c8));
+                    *reinterpret_cast<uint4*>(hsw8(sM, r, c8, N)) = o;
+                }
+            }
+            __syncthreads();   // the weights are in sw
+            for (int e = tid; e < Q * P / 8; e += blockDim.x) {
+                const int r = e / (P / 8), c8 = e % (P / 8);
+                uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                if (r < q) {
+                    const float w = sw[r];
+                    const uint4 v = *reinterpret_cast<const uint4*>(stV + r * P + 8 * c8);
+                    auto cv = [w](uint32_t u) {
+                        return h2pack(w * __uint_as_float(u << 16), w * __uint_as_float(u & 0xffff0000u));
+                    };
+                    o = make_uint4(cv(v.x), cv(v.y), cv(v.z), cv(v.w));
+                }
+                *reinterpret_cast<uint4*>(hsw8(sV, r, c8, P)) = o;
+            }
+            const float E = expf(slast);
+            __syncthreads();   // operands ready; the staging area is free again
+            if (i + 1 < nc) stage(c + step, Mg, Vg);
+            // the state entering chunk c (forwards) / the adjoint of the state leaving it (backwards)
+            store_frag(slabs + ((cf0 + c) * H + h) * slab);
+            float t[1][NT][4];
+            zero_frag(t);
+            mma_tile_h<1, NT, false, false>(t, sM, N, sV, P, n0, col0, Q);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[0][nt][e] = fmaf(E, acc[0][nt][e], t[0][nt][e]);
+        }
+    };
+    load_frag(p.init_state ? p.init_state + ((int64_t)s * H + h) * slab : nullptr);
+    sweep(true);
+    load_frag(p.dfinal ? p.dfinal + ((int64_t)s * H + h) * slab : nullptr);
+    sweep(false);
+    if (p.dinit) store_frag(p.dinit + ((int64_t)s * H + h) * slab);
+}
+
 // k_bwd_terms for bf16 inputs with fp16 operand tiles (swizzled as for k_bwd_grads_h).
 template <int N>
 __global__ void __launch_bounds__(256) k_bwd_terms_h(const ChunkedBwd p) {
@@ -1580,17 +1723,17 @@ void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
     cudaFuncSetAttribute(k_bwd_terms<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_terms);
     if constexpr (sizeof(T) == 4)
         cudaFuncSetAttribute(k_bwd_grads<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grads_smem<N>());
-    {
-        ProfScope ps(K_SCAN_BWD, st);
-        if constexpr (sizeof(T) == 2) {
-            const size_t sm_h = 2 * 2 * (kQb * N + kQb * kPb);
-            cudaFuncSetAttribute(k_bwd_terms_h<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_h);
-            k_bwd_terms_h<N><<<(unsigned)(chunks * p.H), 256, sm_h, st>>>(p);
-        } else {
+    if constexpr (sizeof(T) == 2) {
+        // bf16: the chunk terms are computed inside the pass (k_bwd_pass_h)
+        ProfScope ps(K_BWD_PASS, st);
+        const size_t sm_p = 2 * 2 * (kQb * N + kQb * kPb);
+        cudaFuncSetAttribute(k_bwd_pass_h<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_p);
+        k_bwd_pass_h<N><<<(unsigned)((int64_t)p.si.S * p.H), 256, sm_p, st>>>(p);
+    } else {
+        {
+            ProfScope ps(K_SCAN_BWD, st);
             k_bwd_terms<T, N><<<(unsigned)(chunks * p.H), 256, sm_terms, st>>>(p);
         }
-    }
-    {
         ProfScope ps(K_BWD_PASS, st);
         constexpr int kVec = N * kPb / 4 / kPassThreads;
         k_bwd_pass<kVec><<<(unsigned)((int64_t)p.si.S * p.H), kPassThreads, 0, st>>>(p.S, p.T, p.E, p.init_state,
