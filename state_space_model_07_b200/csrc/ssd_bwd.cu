@@ -1452,8 +1452,8 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
 
 // ---- k_bwd_pass_h: the chunk terms computed inside the sequential pass (bf16, P = Q = 64) ----
 //
-// One block per (sequence, head) walks the sequence's chunks forwards, then backwards, holding the
-// N x 64 state (then its adjoint) in mma.sync accumulator fragments: warp w owns 16 state rows and
+// Two blocks per (sequence, head) walk the sequence's chunks, one forwards, one backwards, each
+// holding the N x 64 state (or its adjoint) in mma.sync accumulator fragments: warp w owns 16 state rows and
 // P / NCB columns.  At every chunk it computes the chunk's own term on the tensor cores,
 // S = B^T (u o x) forwards and T = C^T (e o dy) backwards (u_j = exp(cs_last - cs_j) d_j,
 // e_j = exp(cs_j)), from operands staged by cp.async one chunk ahead, so no term goes through
@@ -1474,7 +1474,10 @@ __global__ void __launch_bounds__(256) k_bwd_pass_h(const ChunkedBwd p) {
     T* stV = stM + Q * N;                            // [Q][P]
     __shared__ float sd[kQb], sz[kQb], scs[kQb], sw[kQb], slast;
     const int H = p.H, G = p.G;
-    const int s = (int)(blockIdx.x / H), h = (int)(blockIdx.x % H), g = h / (H / G);
+    // blocks [0, S H) run the forward sweep, [S H, 2 S H) the backward one: they are independent
+    const bool fwd_block = blockIdx.x < (unsigned)(p.si.S * H);
+    const int sh = (int)(fwd_block ? blockIdx.x : blockIdx.x - p.si.S * H);
+    const int s = sh / H, h = sh % H, g = h / (H / G);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nc = seq_nchunks(p.si, s);
     const int64_t cf0 = seq_chunk0(p.si, s);
@@ -1586,11 +1589,14 @@ __global__ void __launch_bounds__(256) k_bwd_pass_h(const ChunkedBwd p) {
                 for (int e = 0; e < 4; ++e) acc[0][nt][e] = fmaf(E, acc[0][nt][e], t[0][nt][e]);
         }
     };
-    load_frag(p.init_state ? p.init_state + ((int64_t)s * H + h) * slab : nullptr);
-    sweep(true);
-    load_frag(p.dfinal ? p.dfinal + ((int64_t)s * H + h) * slab : nullptr);
-    sweep(false);
-    if (p.dinit) store_frag(p.dinit + ((int64_t)s * H + h) * slab);
+    if (fwd_block) {
+        load_frag(p.init_state ? p.init_state + ((int64_t)s * H + h) * slab : nullptr);
+        sweep(true);
+    } else {
+        load_frag(p.dfinal ? p.dfinal + ((int64_t)s * H + h) * slab : nullptr);
+        sweep(false);
+        if (p.dinit) store_frag(p.dinit + ((int64_t)s * H + h) * slab);
+    }
 }
 
 // k_bwd_terms for bf16 inputs with fp16 operand tiles (swizzled as for k_bwd_grads_h).
@@ -1728,7 +1734,7 @@ void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
         ProfScope ps(K_BWD_PASS, st);
         const size_t sm_p = 2 * 2 * (kQb * N + kQb * kPb);
         cudaFuncSetAttribute(k_bwd_pass_h<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_p);
-        k_bwd_pass_h<N><<<(unsigned)((int64_t)p.si.S * p.H), 256, sm_p, st>>>(p);
+        k_bwd_pass_h<N><<<(unsigned)(2 * (int64_t)p.si.S * p.H), 256, sm_p, st>>>(p);
     } else {
         {
             ProfScope ps(K_SCAN_BWD, st);
