@@ -1460,7 +1460,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
 // HBM.  It writes the state entering every chunk (forwards, over S) and the adjoint of the state
 // leaving every chunk (backwards, over T) for k_bwd_grads_h, and d h0 at the end.
 template <int N>
-__global__ void __launch_bounds__(256) k_bwd_pass_h(const ChunkedBwd p) {
+__global__ void __launch_bounds__(256, N == 64 ? 3 : 2) k_bwd_pass_h(const ChunkedBwd p) {
     using T = __nv_bfloat16;
     constexpr int P = kPb, Q = kQb;
     constexpr int NRB = N / 16;          // 16-row blocks of the state
@@ -1580,13 +1580,12 @@ __global__ void __launch_bounds__(256) k_bwd_pass_h(const ChunkedBwd p) {
             if (i + 1 < nc) stage(c + step, Mg, Vg);
             // the state entering chunk c (forwards) / the adjoint of the state leaving it (backwards)
             store_frag(slabs + ((cf0 + c) * H + h) * slab);
-            float t[1][NT][4];
-            zero_frag(t);
-            mma_tile_h<1, NT, false, false>(t, sM, N, sV, P, n0, col0, Q);
+            // h <- E h + (the chunk's term): scale, then let the MMA add the term in place
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) acc[0][nt][e] = fmaf(E, acc[0][nt][e], t[0][nt][e]);
+                for (int e = 0; e < 4; ++e) acc[0][nt][e] *= E;
+            mma_tile_h<1, NT, false, false>(acc, sM, N, sV, P, n0, col0, Q);
         }
     };
     if (fwd_block) {
