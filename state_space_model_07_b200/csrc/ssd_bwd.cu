@@ -273,11 +273,13 @@ k_scan_bwd(const BwdParams p) {
 //   dJ/dcs_k = sum_i R[k,i] d_i - sum_j R[j,k] d_k + e_k Y_k - u_k Z_k
 //              (+ E <dh_end, h_prev> + sum_i u_i Z_i at k = last)
 //   dJ/da_m = sum_{k>=m} dJ/dcs_k,  dd = direct + A dJ/da,  dA += d dJ/da,  dz = dd sigmoid(z).
-// Three kernels: k_bwd_terms (per chunk and head: the chunk's own state term S = sum_i u_i B_i
-// x_i^T and adjoint term T = sum_j e_j C_j dy_j^T, and E), k_bwd_pass (per state element: the
-// state entering every chunk, forwards, and the adjoint leaving every chunk, backwards), and
-// k_bwd_grads (per chunk and group: every gradient of the chunk's tokens; C B^T is shared by the
-// group's heads, and dB, dC are summed over them in registers, so no atomics touch them).
+// fp32 inputs, three kernels: k_bwd_terms (per chunk and head: the chunk's own state term
+// S = sum_i u_i B_i x_i^T and adjoint term T = sum_j e_j C_j dy_j^T, and E), k_bwd_pass (per
+// state element: the state entering every chunk, forwards, and the adjoint leaving every chunk,
+// backwards), and k_bwd_grads (per chunk and group: every gradient of the chunk's tokens; C B^T
+// is shared by the group's heads, and dB, dC are summed over them in registers, so no atomics
+// touch them).  bf16 inputs, two: k_bwd_pass_h (the pass with each chunk's term computed on the
+// tensor cores as it goes, so the terms never reach HBM) and k_bwd_grads_h.
 
 constexpr int kQb = 64;   // tokens per chunk of the chunked backward
 constexpr int kPb = 64;   // headdim of the chunked backward
@@ -1598,78 +1600,6 @@ __global__ void __launch_bounds__(256, N == 64 ? 3 : 2) k_bwd_pass_h(const Chunk
     }
 }
 
-// k_bwd_terms for bf16 inputs with fp16 operand tiles (swizzled as for k_bwd_grads_h).
-template <int N>
-__global__ void __launch_bounds__(256) k_bwd_terms_h(const ChunkedBwd p) {
-    using T = __nv_bfloat16;
-    constexpr int P = kPb, Q = kQb;
-    extern __shared__ __align__(16) uint8_t smraw[];
-    // both products' operands at once, so that every load of the block is in flight together:
-    // [0] B with u_j x_j -> S, [1] C with e_j dy_j -> T
-    __half* sM0 = reinterpret_cast<__half*>(smraw);  // [Q][N]
-    __half* sM1 = sM0 + Q * N;
-    __half* sV0 = sM1 + Q * N;                       // [Q][P]
-    __half* sV1 = sV0 + Q * P;
-    __shared__ float sd[kQb], sz[kQb], scs[kQb], slast;
-    const int H = p.H, G = p.G;
-    const int64_t f = blockIdx.x / H;
-    const int h = (int)(blockIdx.x % H), g = h / (H / G);
-    ChunkRef r;
-    if (!chunk_ref(p.si, f, r)) return;
-    const int q = (int)(r.t1 - r.t0);
-    const int64_t tok0 = r.row * p.si.L + r.t0;
-    if (threadIdx.x < 32)
-        chunk_decay<T>((const T*)p.dt, tok0, H, h, q, p.dt_bias ? p.dt_bias[h] : 0.f, p.A[h], sd, sz, scs, &slast);
-    load_rows_h(sM0, (const T*)p.B + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
-    load_rows_h(sM1, (const T*)p.C + (tok0 * G + g) * N, (int64_t)G * N, q, Q, N);
-    // x and dy rows as they are (bf16 -> fp16 exactly); their weights need the decay scan
-    const T* xv = (const T*)p.x + (tok0 * H + h) * P;
-    const T* dyv = (const T*)p.dy + (tok0 * H + h) * P;
-    uint4 vx[Q * (P / 8) / 256], vd[Q * (P / 8) / 256];
-#pragma unroll
-    for (int k = 0; k < Q * (P / 8) / 256; ++k) {
-        const int e = threadIdx.x + 256 * k, j = e / (P / 8), c8 = e % (P / 8);
-        vx[k] = vd[k] = make_uint4(0u, 0u, 0u, 0u);
-        if (j < q) {
-            vx[k] = *reinterpret_cast<const uint4*>(xv + (int64_t)j * H * P + 8 * c8);
-            vd[k] = *reinterpret_cast<const uint4*>(dyv + (int64_t)j * H * P + 8 * c8);
-        }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < Q * (P / 8) / 256; ++k) {
-        const int e = threadIdx.x + 256 * k, j = e / (P / 8), c8 = e % (P / 8);
-        const float wu = j < q ? expf(slast - scs[j]) * sd[j] : 0.f, we = j < q ? expf(scs[j]) : 0.f;
-        auto cv = [](uint32_t u, float w) {
-            return h2pack(w * __uint_as_float(u << 16), w * __uint_as_float(u & 0xffff0000u));
-        };
-        *reinterpret_cast<uint4*>(hsw8(sV0, j, c8, P)) =
-            make_uint4(cv(vx[k].x, wu), cv(vx[k].y, wu), cv(vx[k].z, wu), cv(vx[k].w, wu));
-        *reinterpret_cast<uint4*>(hsw8(sV1, j, c8, P)) =
-            make_uint4(cv(vd[k].x, we), cv(vd[k].y, we), cv(vd[k].z, we), cv(vd[k].w, we));
-    }
-    __syncthreads();
-    constexpr int MT = N / 64;
-    const int warp = threadIdx.x >> 5;
-    const int n0 = 16 * MT * (warp >> 1), c0 = 32 * (warp & 1);
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-        float acc[MT][4][4];
-        zero_frag(acc);
-        mma_tile_h<MT, 4, false, false>(acc, pass == 0 ? sM0 : sM1, N, pass == 0 ? sV0 : sV1, P, n0, c0, Q);
-        float* out = (pass == 0 ? p.S : p.T) + ((int64_t)f * H + h) * N * P;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; e += 2)
-                    *reinterpret_cast<float2*>(out + (int64_t)frag_row(n0, mt, e) * P + frag_col(c0, nt, e)) =
-                        make_float2(acc[mt][nt][e], acc[mt][nt][e + 1]);
-    }
-    if (threadIdx.x == 0) p.E[f * H + h] = expf(slast);
-}
-
 template <int N>
 constexpr size_t grads_smem() {
     return sizeof(float) * (2 * kQb * (N + 4) + 3 * kQb * kQb + 2 * kQb * (kPb + 4) + 2 * N * (kPb + 4) +
@@ -1725,9 +1655,10 @@ int grads_hsplit(const ScanArgs& a, int64_t chunks) {
 template <typename T, int N>
 void launch_chunked_t(const ChunkedBwd& p, int64_t chunks, cudaStream_t st) {
     const size_t sm_terms = sizeof(float) * (kQb * N + kQb * kPb);
-    cudaFuncSetAttribute(k_bwd_terms<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_terms);
-    if constexpr (sizeof(T) == 4)
+    if constexpr (sizeof(T) == 4) {
+        cudaFuncSetAttribute(k_bwd_terms<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_terms);
         cudaFuncSetAttribute(k_bwd_grads<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grads_smem<N>());
+    }
     if constexpr (sizeof(T) == 2) {
         // bf16: the chunk terms are computed inside the pass (k_bwd_pass_h)
         ProfScope ps(K_BWD_PASS, st);
