@@ -1474,7 +1474,8 @@ __global__ void __launch_bounds__(256, N == 64 ? 3 : 2) k_bwd_pass_h(const Chunk
     __half* sV = sM + Q * N;                         // [Q][P] u o x or e o dy
     T* stM = reinterpret_cast<T*>(sV + Q * P);       // [Q][N] the next chunk's raw rows
     T* stV = stM + Q * N;                            // [Q][P]
-    __shared__ float sd[kQb], sz[kQb], scs[kQb], sw[kQb], slast;
+    // decay quantities of a chunk, double-buffered: warp 0 prepares chunk i + 1 while chunk i runs
+    __shared__ float sd[2][kQb], sz[2][kQb], scs[2][kQb], sw[2][kQb], slast[2];
     const int H = p.H, G = p.G;
     // blocks [0, S H) run the forward sweep, [S H, 2 S H) the backward one: they are independent
     const bool fwd_block = blockIdx.x < (unsigned)(p.si.S * H);
@@ -1534,27 +1535,39 @@ __global__ void __launch_bounds__(256, N == 64 ? 3 : 2) k_bwd_pass_h(const Chunk
         const T* Vg = (const T*)(fwd ? p.x : p.dy);
         float* slabs = fwd ? p.S : p.T;
         const int cfirst = fwd ? 0 : nc - 1, step = fwd ? 1 : -1;
-        float dt_raw[2] = {0.f, 0.f};   // warp 0: raw dt of the chunk it prepares next
+        float dt_raw[2] = {0.f, 0.f};   // warp 0: raw dt of the next chunk to prepare
+        // warp 0: d, z, cs and the operand weights (u forwards, e backwards) of chunk c into buffer b
+        auto decay = [&](int c, int b) {
+            const int q = chunk_q(c);
+            chunk_decay_raw(dt_raw, q, bias, Ah, sd[b], sz[b], scs[b], &slast[b]);
+            __syncwarp();
+            const float last = slast[b];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int j = 2 * lane + k;
+                sw[b][j] = j < q ? (fwd ? expf(last - scs[b][j]) * sd[b][j] : expf(scs[b][j])) : 0.f;
+            }
+        };
         if (nc > 0) {
             stage(cfirst, Mg, Vg);
-            if (tid < 32) load_dt2<T>(dt_raw, dtg, chunk_tok0(cfirst), H, h, chunk_q(cfirst));
+            if (tid < 32) {
+                load_dt2<T>(dt_raw, dtg, chunk_tok0(cfirst), H, h, chunk_q(cfirst));
+                decay(cfirst, 0);
+                if (nc > 1) load_dt2<T>(dt_raw, dtg, chunk_tok0(cfirst + step), H, h, chunk_q(cfirst + step));
+            }
         }
         for (int i = 0; i < nc; ++i) {
-            const int c = cfirst + step * i;
+            const int c = cfirst + step * i, b = i & 1;
             const int q = chunk_q(c);
-            // chunk c's rows have landed; every warp is done with the previous chunk's operands
+            // chunk c's rows have landed and its decay is in buffer b; every warp is done with the
+            // previous chunk's operands and with buffer b ^ 1
             cp_async_wait_all();
             __syncthreads();
             if (tid < 32) {
-                chunk_decay_raw(dt_raw, q, bias, Ah, sd, sz, scs, &slast);
-                __syncwarp();
-                const float last = slast;
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const int j = 2 * lane + k;
-                    sw[j] = j < q ? (fwd ? expf(last - scs[j]) * sd[j] : expf(scs[j])) : 0.f;
+                if (i + 1 < nc) {
+                    decay(c + step, b ^ 1);
+                    if (i + 2 < nc) load_dt2<T>(dt_raw, dtg, chunk_tok0(c + 2 * step), H, h, chunk_q(c + 2 * step));
                 }
-                if (i + 1 < nc) load_dt2<T>(dt_raw, dtg, chunk_tok0(c + step), H, h, chunk_q(c + step));
             } else {
                 for (int e = tid - 32; e < Q * N / 8; e += blockDim.x - 32) {
                     const int r = e / (N / 8), c8 = e % (N / 8);
@@ -1562,22 +1575,21 @@ __global__ void __launch_bounds__(256, N == 64 ? 3 : 2) k_bwd_pass_h(const Chunk
                     if (r < q) o = bf16x8_to_f16x8_bwd(*reinterpret_cast<const uint4*>(stM + r * N + 8 * c8));
                     *reinterpret_cast<uint4*>(hsw8(sM, r, c8, N)) = o;
                 }
-            }
-            __syncthreads();   // the weights are in sw
-            for (int e = tid; e < Q * P / 8; e += blockDim.x) {
-                const int r = e / (P / 8), c8 = e % (P / 8);
-                uint4 o = make_uint4(0u, 0u, 0u, 0u);
-                if (r < q) {
-                    const float w = sw[r];
-                    const uint4 v = *reinterpret_cast<const uint4*>(stV + r * P + 8 * c8);
-                    auto cv = [w](uint32_t u) {
-                        return h2pack(w * __uint_as_float(u << 16), w * __uint_as_float(u & 0xffff0000u));
-                    };
-                    o = make_uint4(cv(v.x), cv(v.y), cv(v.z), cv(v.w));
+                for (int e = tid - 32; e < Q * P / 8; e += blockDim.x - 32) {
+                    const int r = e / (P / 8), c8 = e % (P / 8);
+                    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < q) {
+                        const float w = sw[b][r];
+                        const uint4 v = *reinterpret_cast<const uint4*>(stV + r * P + 8 * c8);
+                        auto cv = [w](uint32_t u) {
+                            return h2pack(w * __uint_as_float(u << 16), w * __uint_as_float(u & 0xffff0000u));
+                        };
+                        o = make_uint4(cv(v.x), cv(v.y), cv(v.z), cv(v.w));
+                    }
+                    *reinterpret_cast<uint4*>(hsw8(sV, r, c8, P)) = o;
                 }
-                *reinterpret_cast<uint4*>(hsw8(sV, r, c8, P)) = o;
             }
-            const float E = expf(slast);
+            const float E = expf(slast[b]);
             __syncthreads();   // operands ready; the staging area is free again
             if (i + 1 < nc) stage(c + step, Mg, Vg);
             // the state entering chunk c (forwards) / the adjoint of the state leaving it (backwards)
