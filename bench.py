@@ -292,10 +292,12 @@ def config_of(w):
 
 # Definitions in a source file that belong only to kernels other than the one a
 # capture measured: removed before hashing.  ssd_tc.cu also holds the
-# first-generation k_tc_scan<N> (the d_state 256 kernel) and its shared-memory
-# layout TcSmem<N>, neither of which the measured k_tc_scan3 uses.
+# first-generation k_tc_scan<N> (the d_state 256 kernel), its shared-memory
+# layout TcSmem<N> and its constants Cfg<N>, none of which the measured
+# k_tc_scan3 uses.
 _NOT_MEASURED = {"tc_scan": (("template <int N>", "k_tc_scan(const __grid_constant__"),
-                             ("template <int N>", "struct __align__(1024) TcSmem {"))}
+                             ("template <int N>", "struct __align__(1024) TcSmem {"),
+                             ("template <int N>", "struct Cfg {"))}
 
 
 def _drop_definition(code, head, signature):

@@ -60,7 +60,6 @@ namespace {
 using namespace tc;
 
 constexpr int kRoleThreads = 256;   // P and E: two warps per TMEM lane quarter
-constexpr int kThreads = 608;
 constexpr uint32_t kTmemCols = 512;
 
 // Layout constants for dstate N (the kernel is instantiated for N = 256 only):
@@ -70,6 +69,7 @@ constexpr uint32_t kTmemCols = 512;
 // blocks.
 template <int N>
 struct Cfg {
+    static constexpr int kThreads = 608;                    // P 0-7, E 8-15, W16, W17, W18
     static constexpr int kBoxes = N / 64;                   // 64-column boxes per B / C tile
     static constexpr int kBCStages = N == 128 ? 2 : 1;
     static constexpr int kYdBufs = N == 128 ? 2 : 1;
@@ -141,7 +141,7 @@ __device__ __forceinline__ void p_bar() { asm volatile("bar.sync 1, 256;" ::: "m
 
 
 template <int N>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<N>::kThreads, 1)
 k_tc_scan(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
           const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
     using C = Cfg<N>;
@@ -1496,7 +1496,7 @@ int launch_tc_scan(const ScanArgs& a, const SeqInfo& si, int64_t, void* ws, int3
     } else {
         const size_t smem = sizeof(TcSmem<256>) + 1024;
         cudaFuncSetAttribute(k_tc_scan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_tc_scan<256><<<(unsigned)(a.S * a.H), kThreads, smem, st>>>(tm_x, tm_b, tm_c, p);
+        k_tc_scan<256><<<(unsigned)(a.S * a.H), Cfg<256>::kThreads, smem, st>>>(tm_x, tm_b, tm_c, p);
     }
     return 0;
 }
