@@ -1028,6 +1028,66 @@ __device__ __forceinline__ void mma_tile_h(float (&acc)[MT][NT][4], const __half
     }
 }
 
+// acc += A Bm + A2 Bm (kSecondA) or A Bm + A Bm2: the two products of an operand split into an fp16
+// pair hi + lo, with the shared operand's fragments read once per k step.  Layouts as in mma_tile_h.
+template <int MT, int NT, bool AROWK, bool BROWK, bool kSecondA>
+__device__ __forceinline__ void mma_tile_h_pair(float (&acc)[MT][NT][4], const __half* A, const __half* A2, int WA,
+                                                const __half* Bm, const __half* Bm2, int WB, int r0, int c0, int K) {
+    static_assert(NT % 2 == 0, "B fragments come two tiles at a time");
+    const int lane = threadIdx.x & 31, m = lane >> 3, rr = lane & 7;
+    auto load_a = [&](uint32_t (&af)[MT][4], const __half* M, int k) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int r = r0 + 16 * mt;
+            if (AROWK)
+                ldsm_x4(af[mt], hsw8(const_cast<__half*>(M), r + rr + 8 * (m & 1), (k >> 3) + (m >> 1), WA));
+            else
+                ldsm_x4_t(af[mt], hsw8(const_cast<__half*>(M), k + rr + 8 * (m >> 1), (r >> 3) + (m & 1), WA));
+        }
+    };
+    auto load_b = [&](uint32_t (&bf)[NT][2], const __half* M, int k) {
+#pragma unroll
+        for (int nt = 0; nt < NT; nt += 2) {
+            const int n = c0 + 8 * nt;
+            uint32_t t4[4];
+            if (BROWK)
+                ldsm_x4(t4, hsw8(const_cast<__half*>(M), n + rr + 8 * (m >> 1), (k >> 3) + (m & 1), WB));
+            else
+                ldsm_x4_t(t4, hsw8(const_cast<__half*>(M), k + rr + 8 * (m & 1), (n >> 3) + (m >> 1), WB));
+            bf[nt][0] = t4[0];
+            bf[nt][1] = t4[1];
+            bf[nt + 1][0] = t4[2];
+            bf[nt + 1][1] = t4[3];
+        }
+    };
+    auto mma = [&](const uint32_t (&af)[MT][4], const uint32_t (&bf)[NT][2]) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                asm volatile(
+                    "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                    "{%8, %9}, {%0, %1, %2, %3};"
+                    : "+f"(acc[mt][nt][0]), "+f"(acc[mt][nt][1]), "+f"(acc[mt][nt][2]), "+f"(acc[mt][nt][3])
+                    : "r"(af[mt][0]), "r"(af[mt][1]), "r"(af[mt][2]), "r"(af[mt][3]), "r"(bf[nt][0]),
+                      "r"(bf[nt][1]));
+    };
+#pragma unroll 2
+    for (int k = 0; k < K; k += 16) {
+        uint32_t af[MT][4], bf[NT][2];
+        load_a(af, A, k);
+        load_b(bf, Bm, k);
+        mma(af, bf);
+        if (kSecondA) {
+            load_a(af, A2, k);
+            mma(af, bf);
+        } else {
+            load_b(bf, Bm2, k);
+            mma(af, bf);
+        }
+    }
+}
+
 // Rows [0, q) of a bf16 (tokens, stride) slab -> fp16 tile [rows][W] (swizzled), zero past q.
 __device__ __forceinline__ void load_rows_h(__half* dst, const __nv_bfloat16* src, int64_t stride, int q, int rows,
                                             int W) {
@@ -1352,10 +1412,8 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
             float bd[1][2][4], wd[1][2][4];
             zero_frag(bd);
             zero_frag(wd);
-            mma_tile_h<1, 2, true, false>(bd, sB, N, sDH, P, r64, c64, N);
-            mma_tile_h<1, 2, true, false>(bd, sB, N, sDHl, P, r64, c64, N);
-            mma_tile_h<1, 2, false, false>(wd, sW, Q, sDY, P, r64, c64, Q);
-            mma_tile_h<1, 2, false, false>(wd, sWl, Q, sDY, P, r64, c64, Q);
+            mma_tile_h_pair<1, 2, true, false, false>(bd, sB, nullptr, N, sDH, sDHl, P, r64, c64, N);
+            mma_tile_h_pair<1, 2, false, false, true>(wd, sW, sWl, Q, sDY, nullptr, P, r64, c64, Q);
             T* dxg = (T*)p.dx + (tok0 * H + h) * P;
             float z[2] = {0.f, 0.f};
 #pragma unroll
