@@ -986,12 +986,12 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const __half* p) {
 // the matrices are (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
 // -- the m16n8k16 A registers in order; for B, (k 0-7) and (k 8-15) of columns n .. n + 7, then
 // of n + 8 .. n + 15 -- the B registers of two adjacent 8-column tiles.
-template <int MT, int NT, bool AROWK, bool BROWK>
+template <int MT, int NT, bool AROWK, bool BROWK, int kUnroll = 4>
 __device__ __forceinline__ void mma_tile_h(float (&acc)[MT][NT][4], const __half* A, int WA, const __half* Bm, int WB,
                                            int r0, int c0, int K) {
     static_assert(NT % 2 == 0, "B fragments come two tiles at a time");
     const int lane = threadIdx.x & 31, m = lane >> 3, rr = lane & 7;
-#pragma unroll 4
+#pragma unroll kUnroll
     for (int k = 0; k < K; k += 16) {
         uint32_t af[MT][4], bf[NT][2];
 #pragma unroll
@@ -1520,7 +1520,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
 // HBM.  It writes the state entering every chunk (forwards, over S) and the adjoint of the state
 // leaving every chunk (backwards, over T) for k_bwd_grads_h, and d h0 at the end.
 template <int N>
-__global__ void __launch_bounds__(256, N == 64 ? 3 : 2) k_bwd_pass_h(const ChunkedBwd p) {
+__global__ void __launch_bounds__(256, 3) k_bwd_pass_h(const ChunkedBwd p) {
     using T = __nv_bfloat16;
     constexpr int P = kPb, Q = kQb;
     constexpr int NRB = N / 16;          // 16-row blocks of the state
@@ -1657,7 +1657,7 @@ __global__ void __launch_bounds__(256, N == 64 ? 3 : 2) k_bwd_pass_h(const Chunk
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[0][nt][e] *= E;
-            mma_tile_h<1, NT, false, false>(acc, sM, N, sV, P, n0, col0, Q);
+            mma_tile_h<1, NT, false, false, 1>(acc, sM, N, sV, P, n0, col0, Q);
         }
     };
     if (fwd_block) {
