@@ -1276,6 +1276,10 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     float dBa[1][NTN][4], dCa[1][NTN][4];
     zero_frag(dBa);
     zero_frag(dCa);
+    // K = L o (dy x^T) o d summed over this block's heads (this thread's fragment of the 64 x 64
+    // product (1)): the terms K^T C of dB and K B of dC share C and B across the group's heads,
+    // so they are one product each of the sum, after the last head
+    float ksum[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     for (int hh = hh0; hh < hh1; ++hh) {
         const int h = g * HG + hh;
         const float bias = p.dt_bias ? p.dt_bias[h] : 0.f, Ah = p.A[h], Dh = p.D ? p.D[h] : 0.f;
@@ -1385,7 +1389,8 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                     *reinterpret_cast<__half2*>(&sW[at]) = whi;
                     *reinterpret_cast<__half2*>(&sWl[at]) =
                         __floats2half2_rn(w0 - __low2float(whi), w1 - __high2float(whi));
-                    *reinterpret_cast<__half2*>(&sK[at]) = __floats2half2_rn(L0 * dyx0 * di.x, L1 * dyx1 * di.y);
+                    ksum[nt][e] += L0 * dyx0 * di.x;
+                    ksum[nt][e + 1] += L1 * dyx1 * di.y;
                     const float R0 = cb.x * dyx0 * L0, R1 = cb.y * dyx1 * L1;
                     rrow[e >> 1] += R0 * di.x + R1 * di.y;
                     rcol[nt][0] += R0;
@@ -1458,17 +1463,15 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                 if ((lane & 3) == 0) atomicAdd(&rowY[frag_row(r64, 0, 2 * a)], v);
             }
         }
-        // (4) dB += K^T C + u o (x dh_end^T),  dC += K B + e o (dy h_prev^T)
+        // (4) dB += u o (x dh_end^T),  dC += e o (dy h_prev^T)  (K^T C and K B after the last head)
         {
             float t[1][NTN][4];
-            mma_tile_h<1, NTN, false, false>(dBa, sK, Q, sC, N, rN, cN, Q);
             zero_frag(t);
             mma_tile_h<1, NTN, true, true>(t, sX, P, sDH, P, rN, cN, P);
 #pragma unroll
             for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) dBa[0][nt][e] += su[frag_row(rN, 0, e)] * t[0][nt][e];
-            mma_tile_h<1, NTN, true, false>(dCa, sK, Q, sB, N, rN, cN, Q);
             zero_frag(t);
             mma_tile_h<1, NTN, true, true>(t, sDY, P, sHP, P, rN, cN, P);
 #pragma unroll
@@ -1480,6 +1483,23 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     }
     __syncthreads();
     if (warp == 0) decays(hh1 - 1);
+    // dB += (sum K)^T C, dC += (sum K) B, the sum as an fp16 pair hi + lo (lo over W's last tile)
+    {
+        __half* sKl = sWl;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                const int at = hsw(frag_row(r64, 0, e), frag_col(c64, nt, e), Q);
+                const __half2 hi = __floats2half2_rn(ksum[nt][e], ksum[nt][e + 1]);
+                *reinterpret_cast<__half2*>(&sK[at]) = hi;
+                *reinterpret_cast<__half2*>(&sKl[at]) =
+                    __floats2half2_rn(ksum[nt][e] - __low2float(hi), ksum[nt][e + 1] - __high2float(hi));
+            }
+        __syncthreads();
+        mma_tile_h_pair<1, NTN, false, false, true>(dBa, sK, sKl, Q, sC, nullptr, N, rN, cN, Q);
+        mma_tile_h_pair<1, NTN, true, false, true>(dCa, sK, sKl, Q, sB, nullptr, N, rN, cN, Q);
+    }
     if (p.hsplit > 1) {
         // this part's sums, in fp32, for k_bwd_sum_parts
         float* dBg = p.dBp + part * p.part_stride + (tok0 * G + g) * N;
