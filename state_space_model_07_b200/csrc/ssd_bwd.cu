@@ -1443,27 +1443,8 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                 if ((lane & 3) == 0) atomicAdd(&rowZ[frag_row(r64, 0, 2 * a)], v);
             }
         }
-        // (3) Y_j = C_j^T h_prev dy_j
-        {
-            float ch[1][2][4];
-            zero_frag(ch);
-            mma_tile_h<1, 2, true, false>(ch, sC, N, sHP, P, r64, c64, N);
-            float y[2] = {0.f, 0.f};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; e += 2) {
-                    const float2 dv = __half22float2(
-                        *reinterpret_cast<const __half2*>(&sDY[hsw(frag_row(r64, 0, e), frag_col(c64, nt, e), P)]));
-                    y[e >> 1] += ch[0][nt][e] * dv.x + ch[0][nt][e + 1] * dv.y;
-                }
-#pragma unroll
-            for (int a = 0; a < 2; ++a) {
-                const float v = quad_sum(y[a]);
-                if ((lane & 3) == 0) atomicAdd(&rowY[frag_row(r64, 0, 2 * a)], v);
-            }
-        }
-        // (4) dB += u o (x dh_end^T),  dC += e o (dy h_prev^T)  (K^T C and K B after the last head)
+        // (4) dB += u o (x dh_end^T),  dC += e o (dy h_prev^T)  (K^T C and K B after the last head),
+        // and Y_j = C_j^T h_prev dy_j = sum_n C_jn (dy h_prev^T)_jn from the second product
         {
             float t[1][NTN][4];
             zero_frag(t);
@@ -1474,10 +1455,23 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                 for (int e = 0; e < 4; ++e) dBa[0][nt][e] += su[frag_row(rN, 0, e)] * t[0][nt][e];
             zero_frag(t);
             mma_tile_h<1, NTN, true, true>(t, sDY, P, sHP, P, rN, cN, P);
+            float y[2] = {0.f, 0.f};
 #pragma unroll
             for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) dCa[0][nt][e] += se[frag_row(rN, 0, e)] * t[0][nt][e];
+                for (int e = 0; e < 4; e += 2) {
+                    const int j = frag_row(rN, 0, e), n = frag_col(cN, nt, e);
+                    const float2 cv = __half22float2(*reinterpret_cast<const __half2*>(&sC[hsw(j, n, N)]));
+                    y[e >> 1] += cv.x * t[0][nt][e] + cv.y * t[0][nt][e + 1];
+                    const float ej = se[j];
+                    dCa[0][nt][e] += ej * t[0][nt][e];
+                    dCa[0][nt][e + 1] += ej * t[0][nt][e + 1];
+                }
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+                const float v = quad_sum(y[a]);
+                if ((lane & 3) == 0) atomicAdd(&rowY[frag_row(rN, 0, 2 * a)], v);
+            }
         }
         // (the barrier at the top of the next head orders these reads before its conversion)
     }
