@@ -1142,7 +1142,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     __half* sHP = sDY + Q * P;                       // [N][P] state entering the chunk
     __half* sDH = sHP + N * P;                       // [N][P] adjoint of the state leaving it
     __half* sW = sDH + N * P;                        // [Q][Q]
-    __half* sK = sW + Q * Q;                         // [Q][Q]
+    __half* sK = sW + Q * Q;                         // [Q][Q] K summed over the heads (hi), at the end
     // dx = D dy + W^T dy + u o (B dh_end): its last two terms can each be many times dx itself
     // and cancel, so W and dh_end enter those products as fp16 pairs hi + lo (lo = the fp16
     // rounding of what hi leaves), which makes them exact to about 2^-22
