@@ -31,9 +31,14 @@ def _sigmoid(z):
     return np.where(z >= 0, 1.0 / (1.0 + np.exp(-np.abs(z))), np.exp(-np.abs(z)) / (1.0 + np.exp(-np.abs(z))))
 
 
-def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfinal=None, Q=16, operands=None):
+def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfinal=None, Q=16, operands=None,
+                grouped=False):
     """x, dy (b,L,H,P); dt (b,L,H); B, C (b,L,G,N); A, dt_bias, D (H,); init_state, dfinal
     (b,H,N,P) or None.  Returns the same dict of gradients as the oracle.
+
+    `grouped` takes two terms the way the tensor-core gradient kernel does: K^T C of dB and K B of
+    dC once per (chunk, group) from K summed over the group's heads (C and B are the group's), and
+    Y_j = C_j^T h_prev dy_j as sum_n C_jn (dy h_prev^T)_jn, the product dC's state term uses.
 
     `operands` ("f16" or "bf16") rounds both operands of every matrix product (the work a
     tensor-core kernel would do) to that type, with products and sums kept in fp32; the
@@ -58,6 +63,7 @@ def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfina
     out = {"x": np.zeros_like(x), "dt": np.zeros((b, L, H)), "dt_bias": np.zeros(H), "A": np.zeros(H),
            "B": np.zeros_like(B), "C": np.zeros_like(C), "D": np.zeros(H), "init_state": np.zeros((b, H, N, P))}
     starts = list(range(0, L, Q))
+    ksum = {}   # grouped: (batch row, chunk, group) -> K summed over the group's heads
     for bb in range(b):
         for h in range(H):
             g = h // (H // G)
@@ -90,8 +96,14 @@ def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfina
                 # x, B, C, D
                 dx = Dv[h] * dyc + mm(W.T, dyc) + u[:, None] * mm(Bc, dh_end)
                 K = Lm * dyx * dc[None, :]                       # [j, i]
-                dB = mm(K.T, Cc) + u[:, None] * mm(xc, dh_end.T)
-                dC = mm(K, Bc) + e[:, None] * mm(dyc, hp.T)
+                dyhp = mm(dyc, hp.T)                             # [j, n] = dy_j . h_prev[n]
+                if grouped:
+                    ksum[(bb, c, g)] = ksum.get((bb, c, g), 0.0) + K
+                    dB = u[:, None] * mm(xc, dh_end.T)
+                    dC = e[:, None] * dyhp
+                else:
+                    dB = mm(K.T, Cc) + u[:, None] * mm(xc, dh_end.T)
+                    dC = mm(K, Bc) + e[:, None] * dyhp
                 out["x"][bb, t0:t1, h] += dx
                 out["B"][bb, t0:t1, g] += dB
                 out["C"][bb, t0:t1, g] += dC
@@ -99,7 +111,10 @@ def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfina
                 # decays: direct d_i terms and dJ/dcs_k
                 R = CB * dyx * Lm                                # [j, i] = (C_j.B_i)(dy_j.x_i) exp(cs_j - cs_i)
                 Z = np.einsum("in,np,ip->i", Bc, dh_end, xc)     # B_i^T dh_end x_i
-                Yoff = np.einsum("jn,np,jp->j", Cc, hp, dyc)     # C_j^T h_prev dy_j
+                if grouped:
+                    Yoff = np.sum(Cc * dyhp, axis=1)             # C_j^T h_prev dy_j
+                else:
+                    Yoff = np.einsum("jn,np,jp->j", Cc, hp, dyc)
                 ddir = R.sum(axis=0) + np.exp(cs[-1] - cs) * Z
                 Rd = R * dc[None, :]
                 dcs = Rd.sum(axis=1) - Rd.sum(axis=0) + e * Yoff
@@ -114,4 +129,9 @@ def chunked_bwd(x, dt, A, B, C, dy, dt_bias=None, D=None, init_state=None, dfina
                 # reverse state passing
                 dh_end = E * dh_end + mm((Cc * e[:, None]).T, dyc)
             out["init_state"][bb, h] = dh_end
+    for (bb, c, g), Ks in ksum.items():
+        t0 = starts[c]
+        t1 = min(t0 + Q, L)
+        out["B"][bb, t0:t1, g] += mm(Ks.T, C[bb, t0:t1, g])
+        out["C"][bb, t0:t1, g] += mm(Ks, B[bb, t0:t1, g])
     return out

@@ -159,16 +159,19 @@ def test_packed_equals_separate_sequences():
         assert np.allclose(packed[k], shared[k], rtol=1e-12, atol=1e-14), k
 
 
+@pytest.mark.parametrize("grouped", [False, True])
 @pytest.mark.parametrize("Q", [1, 4, 16, 64])
-def test_chunked_backward_matches_the_oracle(Q):
+def test_chunked_backward_matches_the_oracle(Q, grouped):
     """The chunked backward (per chunk: quadratic terms, state terms, decay gradients by a reverse
     cumulative sum; reverse state passing between chunks) equals the token-by-token gradient
-    oracle, with a ragged last chunk, groups, an initial state and dfinal."""
+    oracle, with a ragged last chunk, groups, an initial state and dfinal.  `grouped` is the form
+    the tensor-core gradient kernel takes: K^T C and K B once per (chunk, group) from K summed over
+    the group's heads, Y from the dy h_prev^T product."""
     from tests.ssd_blocks_bwd_ref import chunked_bwd
     args, dy, dfinal = _case(b=2, L=23, H=4, P=3, N=5, G=2, seed=17)
     g = _grads(args, dy, dfinal)
     c = chunked_bwd(args["x"], args["dt"], args["A"], args["B"], args["C"], dy, dt_bias=args["dt_bias"],
-                    D=args["D"], init_state=args["init_state"], dfinal=dfinal, Q=Q)
+                    D=args["D"], init_state=args["init_state"], dfinal=dfinal, Q=Q, grouped=grouped)
     for k in KEYS:
         assert np.max(np.abs(c[k] - g[k]) / (1 + np.abs(g[k]))) < 1e-12, (Q, k)
 
