@@ -1113,10 +1113,13 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Layout of k_bwd_grads_h's dynamic shared memory: the fp16 tiles, the fp32 C B^T and per-token
-// arrays, then (16-byte aligned) the staging area of the next head's inputs.
+// arrays, then (16-byte aligned) the staging area of the next head's inputs.  C B^T rows are
+// kCBW = Q + 8 floats apart: a fragment's eight rows then start 8 banks apart, so its float2
+// reads (four lanes per row) take the two wavefronts 256 bytes need instead of eight.
+constexpr int kCBW = kQb + 8;
 template <int N>
 constexpr size_t grads_h_stage_offset() {
-    return (2 * (2 * kQb * N + 2 * kQb * kPb + 3 * N * kPb + 3 * kQb * kQb) + sizeof(float) * (kQb * kQb + 9 * kQb + 4) +
+    return (2 * (2 * kQb * N + 2 * kQb * kPb + 3 * N * kPb + 3 * kQb * kQb) + sizeof(float) * (kQb * kCBW + 9 * kQb + 4) +
             15) & ~(size_t)15;
 }
 
@@ -1148,8 +1151,8 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
     // rounding of what hi leaves), which makes them exact to about 2^-22
     __half* sDHl = sK + Q * Q;                       // [N][P]
     __half* sWl = sDHl + N * P;                      // [Q][Q]
-    float* sCB = reinterpret_cast<float*>(sWl + Q * Q);   // [Q][Q] C_j . B_i in fp32 (it enters the decays)
-    float* sd = sCB + Q * Q;
+    float* sCB = reinterpret_cast<float*>(sWl + Q * Q);   // [Q][kCBW] C_j . B_i in fp32 (it enters the decays)
+    float* sd = sCB + Q * kCBW;
     float* sz = sd + Q;
     float* scs = sz + Q;
     float* se = scs + Q;
@@ -1215,7 +1218,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                sCB[frag_row(r64, 0, e) * Q + frag_col(c64, nt, e)] = acc[0][nt][e];
+                sCB[frag_row(r64, 0, e) * kCBW + frag_col(c64, nt, e)] = acc[0][nt][e];
     }
     // (5) the decays of head hh, on warp 0 (tokens 2 lane, 2 lane + 1): they read only the per-token
     // arrays and sums of that head, so warp 0 runs them while the other warps convert the next
@@ -1376,7 +1379,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) k_bwd_grads_h(const ChunkedBw
                 for (int e = 0; e < 4; e += 2) {
                     // elements (j, i) and (j, i + 1), i even: one fp16 pair per tile
                     const int j = frag_row(r64, 0, e), i = frag_col(c64, nt, e);
-                    const float2 cb = *reinterpret_cast<const float2*>(&sCB[j * Q + i]);
+                    const float2 cb = *reinterpret_cast<const float2*>(&sCB[j * kCBW + i]);
                     const float2 di = *reinterpret_cast<const float2*>(&sd[i]);
                     const float2 ci = *reinterpret_cast<const float2*>(&scs[i]);
                     // the fast exponential: this path's operands are fp16 anyway
