@@ -225,8 +225,9 @@ def test_backward_operand_precision():
     """Design input for a tensor-core backward: with the operands of every matrix product of the
     chunked backward rounded to fp16 (fp32 accumulation, 128-token chunks), every gradient stays
     within 1e-2 (1 + |ref|) of the oracle on the long-context distributions (seeded: <= 0.005);
-    with bf16 operands x, B and the initial-state gradients miss it (0.03).  The pages give no
-    tolerance for gradients; the forward's form is used as a yardstick."""
+    with bf16 operands x, B and the initial-state gradients miss it (0.03).  The grouped form (K
+    summed over a group's heads before K^T C and K B, fp16 operands there too) stays within it as
+    well.  The pages give no tolerance for gradients; the forward's form is used as a yardstick."""
     from tests.ssd_blocks_bwd_ref import chunked_bwd
     w = inputs.scaled(inputs.WORKLOADS["long_context"], seqlen=640, nheads=4, ngroups=2)
     d = inputs.make_inputs(w, "cpu")
@@ -242,4 +243,7 @@ def test_backward_operand_precision():
                         init_state=a["init_state"], dfinal=dfinal, Q=128, operands=ops)
         err[ops] = {k: float(np.max(np.abs(c[k] - g[k]) / (1 + np.abs(g[k])))) for k in KEYS}
     assert max(err["f16"].values()) < 1e-2
+    c = chunked_bwd(a["x"], a["dt"], a["A"], a["B"], a["C"], dy, dt_bias=a["dt_bias"], D=a["D"],
+                    init_state=a["init_state"], dfinal=dfinal, Q=128, operands="f16", grouped=True)
+    assert max(float(np.max(np.abs(c[k] - g[k]) / (1 + np.abs(g[k])))) for k in KEYS) < 1e-2
     assert err["bf16"]["x"] > 1e-2 and err["bf16"]["B"] > 1e-2 and err["bf16"]["init_state"] > 1e-2
