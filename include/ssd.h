@@ -58,7 +58,7 @@ typedef enum {
     SSD_ERR_SHAPE = 2,       /* sizes out of the supported range or inconsistent    */
     SSD_ERR_DTYPE = 3,       /* dtype is not an ssd_dtype value                     */
     SSD_ERR_CHUNK = 4,       /* chunk is not a power of two in [16, 256]            */
-    SSD_ERR_UNSUPPORTED = 5, /* valid request this build does not implement         */
+    SSD_ERR_UNSUPPORTED = 5, /* valid request the library does not implement       */
     SSD_ERR_CUDA = 6,        /* a CUDA call failed; see ssd_last_error()            */
     SSD_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up (debug check)     */
     SSD_ERR_SEQIDX = 8,      /* seq_idx breaks its contract (debug check only)       */

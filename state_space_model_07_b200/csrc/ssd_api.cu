@@ -249,7 +249,7 @@ const char* ssd_status_string(int s) {
         case SSD_ERR_SHAPE: return "sizes out of range, inconsistent, overlapping or misaligned buffers";
         case SSD_ERR_DTYPE: return "unknown dtype";
         case SSD_ERR_CHUNK: return "chunk must be a power of two in [16, 256]";
-        case SSD_ERR_UNSUPPORTED: return "request not supported by this build";
+        case SSD_ERR_UNSUPPORTED: return "request not supported by this library";
         case SSD_ERR_CUDA: return "CUDA error";
         case SSD_ERR_TIMEOUT: return "bounded device wait timed out";
         case SSD_ERR_SEQIDX: return "seq_idx breaks its contract";
