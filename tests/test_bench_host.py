@@ -54,6 +54,18 @@ def test_algorithmic_bytes_of_the_bench_workload():
     assert bench.workload_bytes(w, w.batch, tokens, 2) == tokens * per_tok + 8 * 80 * 128 * 64 * 4 == 714080256
 
 
+def test_algorithmic_flops_count_the_causal_pairs_once():
+    """The chunked form's multiply-adds counted by enumeration on a small case: per chunk and head
+    every causal pair (i <= j) once for S x (P each) and per group once for C B^T (N each), every
+    token's B x^T and C h_prev (N P each), and one N x P state update per chunk."""
+    from state_space_model_07_b200 import inputs
+    w = inputs.Workload("f", 2, 24, 3, 8, 16, 1, 8, "bf16", 0, False)
+    L_tot, Q, H, P, N, G = w.batch * w.seqlen, w.chunk, w.nheads, w.headdim, w.dstate, w.ngroups
+    pairs = sum(1 for _ in range(L_tot // Q) for j in range(Q) for i in range(j + 1))
+    macs = H * (pairs * P + L_tot * N * P * 2 + (L_tot // Q) * N * P) + G * pairs * N
+    assert bench.workload_flops(w, L_tot, Q) == pytest.approx(2 * macs, rel=1e-12)
+
+
 def test_scan_hash_covers_the_measured_kernel_not_the_d_state_256_one(tmp_path, monkeypatch):
     src = open(bench.os.path.join(bench.ROOT, "state_space_model_07_b200", "csrc", "ssd_tc.cu")).read()
     csrc = tmp_path / "state_space_model_07_b200" / "csrc"
