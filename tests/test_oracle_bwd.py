@@ -193,6 +193,19 @@ MUTANTS = {
 }
 
 
+@pytest.mark.parametrize("Q", [64, 128])
+def test_grouped_chunked_backward_over_several_long_chunks(Q):
+    """The grouped form at the chunk lengths a tensor-core backward takes (64 and 128 tokens), over
+    several chunks with a ragged last one, equals the gradient oracle."""
+    from tests.ssd_blocks_bwd_ref import chunked_bwd
+    args, dy, dfinal = _case(b=1, L=300, H=4, P=3, N=5, G=2, seed=23)
+    g = _grads(args, dy, dfinal)
+    c = chunked_bwd(args["x"], args["dt"], args["A"], args["B"], args["C"], dy, dt_bias=args["dt_bias"],
+                    D=args["D"], init_state=args["init_state"], dfinal=dfinal, Q=Q, grouped=True)
+    for k in KEYS:
+        assert np.max(np.abs(c[k] - g[k]) / (1 + np.abs(g[k]))) < 1e-12, (Q, k)
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(tmp_path, monkeypatch, name):
     import ctypes
